@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of the rasterizer's hot path: one step = preprocess -> bin/sort
+-> render forward -> render backward -> preprocess backward for one frame of
+the 1M-Gaussian 1920x1080 synthetic scene (16x16 tiles), fp32.
+
+Prints one JSON line.  ``value`` is Gaussian-pixel evaluations per second for
+the whole job (all ranks), where a frame's evaluations are the (pixel,
+Gaussian) terms inside each pixel's contributor prefix, counted once for the
+forward and once for the backward: 2 * sum(n_contrib).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Under torchrun each rank renders its own frame (replicas, no collective on
+the data path); the timed region is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("rasterizer fwd+bwd ms/frame and Gaussian·pixel evals/s; bwd HBM GB/s vs B200 peak")
+UNIT = "Gaussian·pixel evals/s"
+
+# Algorithmic FP32 operations per evaluated term (each add, mul, min, div or
+# exp counts one): forward = 15 to evaluate alpha + 9 to blend; backward = 15
+# to re-evaluate alpha + 45 for the gradient formulas.
+OPS_FWD_EVAL = 24
+OPS_BWD_EVAL = 60
+# Algorithmic bytes: per (tile, Gaussian) pair visited, id + mean2d +
+# conic/opacity + colour = 40 B read; the backward adds 36 B of gradient
+# atomics per pair; per pixel the forward writes 20 B (image, T, n_contrib)
+# and the backward reads 20 B (T, n_contrib, dL/dpixel).
+BYTES_PAIR_READ = 40
+BYTES_PAIR_ATOMIC = 36
+BYTES_PIXEL = 20
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)), src="measured")
+    return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"gs_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=mx, reasons=sorted(reasons), samples=len(sm))
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _scene(cfg: int):
+    from differentiable_gaussian_splatting_preprocess_b200 import scenes
+    return scenes.preset(cfg)
+
+
+def cpu_oracle_sample(sc, tile_stride: int, max_seconds: float = 25.0):
+    """Time the oracle on a bounded sample of the workload: full preprocess
+    and binning, then compositing forward (fp32) and backward (fp64) on every
+    ``tile_stride``-th tile."""
+    import oracle
+    cam = sc.cameras[0]
+    t0 = time.perf_counter()
+    pre = oracle.preprocess(cam, sc.means, sc.scales, sc.quats, sc.opacity, "f32")
+    b = oracle.bin_pairs(cam, pre["depth"], pre["rect"], pre["tiles_touched"], "f32")
+    tiles = np.arange(0, cam.num_tiles, tile_stride, dtype=np.int32)
+    r = oracle.render_fwd(cam, b["ranges"], b["ids"], pre["mean2d"], pre["conic_opacity"], sc.colors, "f32",
+                          tiles=tiles)
+    g = oracle.render_bwd(cam, sc.N, b["ranges"], b["ids"], pre["mean2d"], pre["conic_opacity"], sc.colors,
+                          sc.dL_dimage[0], "f64", tiles=tiles)
+    oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, pre["radius"], g["dL_dmean2d"],
+                          g["dL_dconic_opacity"], g["dL_dcolor"], "f64")
+    dt = time.perf_counter() - t0
+    evals = 2 * int(r["n_contrib"].astype(np.int64).sum())
+    return dict(value=evals / dt, unit=UNIT, cores=oracle.num_threads(), kind="oracle",
+                sample=(f"full preprocess + binning of the {sc.name} scene, compositing fwd (fp32) + bwd "
+                        f"(fp64) on every {tile_stride}th tile ({tiles.size} of {cam.num_tiles}), "
+                        f"{dt:.2f} s"), seconds=dt, evals=evals)
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    sc = _scene(args.config)
+    stride = 16 if args.config >= 4 else 1
+    import oracle
+    for _ in range(args.warmup):
+        cpu_oracle_sample(sc, stride * 4)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = cpu_oracle_sample(sc, stride)
+        vals.append(r["evals"])
+        secs.append(r["seconds"])
+    value = sum(vals) / sum(secs)
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=ws, steps=args.steps, warmup=args.warmup,
+                ms_per_step=1e3 * sum(secs) / len(secs), higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f32 fwd / f64 bwd", data="synthetic", impl="reference",
+                config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {sc.cameras[0].width}x{sc.cameras[0].height},"
+                                     " 16x16 tiles (bounded tile sample per step)"),
+                cpu_baseline=dict(kind="oracle", cores=oracle.num_threads(), value=value, unit=UNIT,
+                                  sample=r["sample"]),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from differentiable_gaussian_splatting_preprocess_b200 import binding as B
+    from differentiable_gaussian_splatting_preprocess_b200 import rasterizer as RZ
+
+    world, rank, local = _dist()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    B.lib()
+
+    sc = _scene(args.config)
+    cam = sc.cameras[0]
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    means, scales, quats, opacity, colors = (t(x) for x in (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors))
+    dL = t(sc.dL_dimage[0])
+    rz = RZ.Rasterizer(cam, dev)
+    # size the pair buffers once (host read of P), then run in capacity mode
+    fr = rz.forward(means, scales, quats, opacity, colors)
+    P = fr.capacity
+    capacity = P
+    grads = RZ.zero_grads(sc.N, dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stages = ["preprocess_fwd", "bin_sort", "render_fwd", "render_bwd", "preprocess_bwd"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        pre = rz.preprocess(means, scales, quats, opacity)
+        mark(1)
+        ws = rz.workspace(sc.N, capacity)
+        B.gs_bin_sort(cam, pre["depth"], pre["rect"], pre["tiles_touched"], pre["num_pairs"], capacity,
+                      rz._bufs["ids"], rz._bufs["ranges"], None, ws)
+        mark(2)
+        B.gs_render_fwd(cam, rz._bufs["ranges"], rz._bufs["ids"], pre["mean2d"], pre["conic_opacity"], colors,
+                        rz._bufs["image"], rz._bufs["final_T"], rz._bufs["n_contrib"])
+        mark(3)
+        B.gs_render_bwd(cam, rz._bufs["ranges"], rz._bufs["ids"], pre["mean2d"], pre["conic_opacity"], colors,
+                        rz._bufs["final_T"], rz._bufs["n_contrib"], dL, rz._bufs["dL_dmean2d"],
+                        rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"])
+        mark(4)
+        B.gs_preprocess_bwd(cam, means, scales, quats, pre["radius"], pre["conic_opacity"], rz._bufs["dL_dmean2d"],
+                            rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"], grads["dL_dmeans"],
+                            grads["dL_dscales"], grads["dL_dquats"], grads["dL_dopacity"], grads["dL_dcolors"])
+        mark(5)
+
+    rz.backward(fr, means, scales, quats, colors, dL)  # allocate the 2D gradient buffers
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = rz.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+    n_contrib = rz._bufs["n_contrib"].view(torch.int32).to(torch.int64).sum().item()
+    evals_per_frame = 2 * int(n_contrib)
+
+    sampler = ClockSampler(local)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    for k in range(args.steps):
+        flush.zero_()  # L2 flush outside the timed interval
+        step(events[k])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    clocks = sampler.stop()
+    stage_ms = {s: [] for s in stages}
+    step_ms = []
+    for ev in events:
+        for i, s in enumerate(stages):
+            stage_ms[s].append(ev[i].elapsed_time(ev[i + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[5]))
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    value = world * evals_per_frame * args.steps / (total_ms / 1e3)
+    st = rz.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+
+    # launches of this library's kernels per step
+    T = B.num_tiles(cam)
+    tile_bits = max(0, (T - 1).bit_length())
+    tpasses = (tile_bits + 7) // 8
+    launches = 1 + (1 + 4 * 3 + 3 + 1 + 3 * tpasses + 1) + 1 + 2 + 1
+
+    # roofline of the dominant kernel (render backward: FP32 ALU bound)
+    peaks = _peaks()
+    mean = {s: statistics.mean(v) for s, v in stage_ms.items()}
+    dominant = max(mean, key=mean.get)
+    bwd_ops = (evals_per_frame // 2) * OPS_BWD_EVAL
+    fwd_ops = (evals_per_frame // 2) * OPS_FWD_EVAL
+    alu_peak = SMS * FP32_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12  # T lane-ops/s
+    rb_ach = bwd_ops / (mean["render_bwd"] / 1e3) / 1e12
+    roofline = dict(kernel="k_render_bwd", bound="alu", achieved=rb_ach, peak=alu_peak, unit="Tops/s",
+                    frac=rb_ach / alu_peak, traffic=None,
+                    ops_per_launch=bwd_ops, peak_src=f"148 SMs x 128 FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz")
+    # HBM view of render fwd + bwd, as asked
+    pix = cam.width * cam.height
+    pairs = evals_per_frame // 2  # visited pairs are bounded below by the contributor prefixes
+    fwd_bytes = P * BYTES_PAIR_READ + pix * BYTES_PIXEL
+    bwd_bytes = P * (BYTES_PAIR_READ + BYTES_PAIR_ATOMIC) + pix * BYTES_PIXEL
+    rfb_s = (mean["render_fwd"] + mean["render_bwd"]) / 1e3
+    render_hbm = dict(achieved_gbs=(fwd_bytes + bwd_bytes) / rfb_s / 1e9, peak_gbs=peaks["hbm_gbs"],
+                      frac=(fwd_bytes + bwd_bytes) / rfb_s / 1e9 / peaks["hbm_gbs"],
+                      bytes_per_frame=fwd_bytes + bwd_bytes, peak_src=peaks["src"])
+    fwd_alu = fwd_ops / (mean["render_fwd"] / 1e3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device ->
+    # forward (host read of P) + backward -> 3D gradients back to the host
+    e2e = None
+    if not args.no_e2e:
+        host_in = [torch.from_numpy(np.ascontiguousarray(x)).pin_memory()
+                   for x in (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0])]
+        h2d = sum(x.numel() * x.element_size() for x in host_in)
+        rz2 = RZ.Rasterizer(cam, dev)
+        host_out = None
+        e2e_times = []
+        for k in range(args.warmup + args.steps):
+            flush.zero_()
+            torch.cuda.synchronize(dev)
+            t0 = time.perf_counter()
+            d = [x.to(dev, non_blocking=True) for x in host_in]
+            f2 = rz2.forward(d[0], d[1], d[2], d[3], d[4])
+            g2 = rz2.backward(f2, d[0], d[1], d[2], d[4], d[5])
+            outs = [g2[k2] for k2 in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors")]
+            if host_out is None:
+                host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+            for ho, o in zip(host_out, outs):
+                ho.copy_(o, non_blocking=True)
+            torch.cuda.synchronize(dev)
+            if k >= args.warmup:
+                e2e_times.append(time.perf_counter() - t0)
+        d2h = sum(o.numel() * o.element_size() for o in host_out)
+        e2e_s = sum(e2e_times)
+        if world > 1:
+            tt = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_s = float(tt.item())
+        e2e = dict(value=world * evals_per_frame * args.steps / e2e_s, unit=UNIT, h2d_bytes_per_step=h2d,
+                   d2h_bytes_per_step=d2h, ms_per_step=1e3 * e2e_s / args.steps)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_oracle_sample(sc, tile_stride=16 if args.config >= 4 else 1)
+        for k in ("seconds", "evals"):
+            cpu.pop(k)
+
+    if rank == 0:
+        line = dict(
+            metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+            ms_per_step=total_ms / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,
+            dtype="f32", data="synthetic",
+            config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam.width}x{cam.height}, 16x16 tiles, fp32",
+                        num_pairs=P, evals_per_frame=evals_per_frame, l2="flushed between steps (256 MiB write)",
+                        parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+            fwd_ms_per_frame=mean["preprocess_fwd"] + mean["bin_sort"] + mean["render_fwd"],
+            bwd_ms_per_frame=mean["render_bwd"] + mean["preprocess_bwd"],
+            stage_ms={s: round(v, 4) for s, v in mean.items()}, dominant_stage=dominant,
+            roofline=roofline, render_fwd_alu=dict(achieved=fwd_alu, peak=alu_peak, unit="Tops/s",
+                                                   frac=fwd_alu / alu_peak),
+            render_hbm=render_hbm, cpu_baseline=cpu, e2e=e2e, gpu_launches=launches * args.steps,
+            clocks=clocks)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

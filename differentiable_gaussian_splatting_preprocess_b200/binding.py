@@ -1,0 +1,265 @@
+"""Thin Python binding of ``libgs.so`` (the C ABI declared in ``include/gs.h``).
+
+Argument marshalling only: every function here checks the tensors it is given
+(device, dtype, shape, contiguity), passes raw device pointers and the current
+CUDA stream to the C entry point of the same name, and raises on a non-zero
+status.  All arithmetic runs in the library's CUDA kernels.  There is no CPU
+path: if ``libgs.so`` is missing or no CUDA device is present, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgs.so")
+
+GS_OK = 0
+GS_ERR_INVALID_ARG = 1
+GS_ERR_CAPACITY = 2
+GS_ERR_TIMEOUT = 4
+GS_ERR_CUDA = 8
+GS_ERR_UNIMPLEMENTED = 16
+GS_ERR_OVERFLOW = 32
+GS_STAGE_PREPROCESS_FWD = 0
+GS_STAGE_BIN_SORT = 1
+TILE = 16
+
+# Every symbol include/gs.h declares.
+EXPORTED = ("gs_version", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
+            "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd")
+
+
+class GsCamera(ctypes.Structure):
+    """Mirror of ``gs_camera`` in include/gs.h."""
+    _fields_ = [
+        ("width", ctypes.c_int), ("height", ctypes.c_int), ("tile", ctypes.c_int),
+        ("fx", ctypes.c_float), ("fy", ctypes.c_float), ("cx", ctypes.c_float), ("cy", ctypes.c_float),
+        ("R", ctypes.c_float * 9), ("t", ctypes.c_float * 3),
+        ("z_near", ctypes.c_float), ("eps2d", ctypes.c_float), ("alpha_max", ctypes.c_float),
+        ("alpha_min", ctypes.c_float), ("T_min", ctypes.c_float), ("sigma_mult", ctypes.c_float),
+        ("bg", ctypes.c_float * 3),
+    ]
+
+
+class GsError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgs.so; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "differentiable_gaussian_splatting_preprocess_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, U, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
+        cam = ctypes.POINTER(GsCamera)
+        L.gs_version.restype = I
+        L.gs_version.argtypes = []
+        L.gs_status_string.restype = ctypes.c_char_p
+        L.gs_status_string.argtypes = [I]
+        L.gs_workspace_bytes.restype = S
+        L.gs_workspace_bytes.argtypes = [I, I, U, I, I]
+        L.gs_read_status.restype = I
+        L.gs_read_status.argtypes = [P, ctypes.POINTER(I), P]
+        L.gs_clear_status.restype = I
+        L.gs_clear_status.argtypes = [P, P]
+        L.gs_preprocess_fwd.restype = I
+        L.gs_preprocess_fwd.argtypes = [cam, I] + [P] * 11 + [P, S, P]
+        L.gs_bin_sort.restype = I
+        L.gs_bin_sort.argtypes = [cam, I, P, P, P, P, U, P, P, P, P, S, P]
+        L.gs_render_fwd.restype = I
+        L.gs_render_fwd.argtypes = [cam] + [P] * 8 + [P]
+        L.gs_render_bwd.restype = I
+        L.gs_render_bwd.argtypes = [cam, I] + [P] * 11 + [P]
+        L.gs_preprocess_bwd.restype = I
+        L.gs_preprocess_bwd.argtypes = [cam, I] + [P] * 13 + [P]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gs_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(lib().gs_version())
+
+
+def camera_struct(cam) -> GsCamera:
+    """Build the C camera record from any object with the gs_camera fields."""
+    c = GsCamera()
+    c.width, c.height, c.tile = int(cam.width), int(cam.height), int(getattr(cam, "tile", TILE))
+    c.fx, c.fy, c.cx, c.cy = float(cam.fx), float(cam.fy), float(cam.cx), float(cam.cy)
+    for k in range(9):
+        c.R[k] = float(cam.R[k])
+    for k in range(3):
+        c.t[k] = float(cam.t[k])
+        c.bg[k] = float(cam.bg[k])
+    c.z_near, c.eps2d, c.alpha_max = float(cam.z_near), float(cam.eps2d), float(cam.alpha_max)
+    c.alpha_min, c.T_min, c.sigma_mult = float(cam.alpha_min), float(cam.T_min), float(cam.sigma_mult)
+    return c
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[ctypes.c_void_p]:
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype, shape=None, optional: bool = False) -> None:
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _ok(fn: str, status: int) -> None:
+    if status != GS_OK:
+        raise GsError(fn, status)
+
+
+def num_tiles(cam) -> int:
+    return ((cam.width + TILE - 1) // TILE) * ((cam.height + TILE - 1) // TILE)
+
+
+def gs_workspace_bytes(stage: int, N: int, capacity: int, width: int, height: int) -> int:
+    return int(lib().gs_workspace_bytes(int(stage), int(N), int(capacity), int(width), int(height)))
+
+
+def gs_read_status(ws: torch.Tensor, stream=None) -> int:
+    st = ctypes.c_int(0)
+    _ok("gs_read_status", lib().gs_read_status(_ptr(ws), ctypes.byref(st), _stream(stream)))
+    return int(st.value)
+
+
+def gs_clear_status(ws: torch.Tensor, stream=None) -> None:
+    _ok("gs_clear_status", lib().gs_clear_status(_ptr(ws), _stream(stream)))
+
+
+def gs_preprocess_fwd(cam, means, scales, quats, opacity, mean2d, depth, conic_opacity, radius, rect,
+                      tiles_touched, d_num_pairs, ws, stream=None) -> None:
+    N = means.shape[0]
+    f32, i32, u32 = torch.float32, torch.int32, torch.uint32
+    _check(means, "means", f32, (N, 3))
+    _check(scales, "scales", f32, (N, 3))
+    _check(quats, "quats", f32, (N, 4))
+    _check(opacity, "opacity", f32, (N,))
+    _check(mean2d, "mean2d", f32, (N, 2))
+    _check(depth, "depth", f32, (N,))
+    _check(conic_opacity, "conic_opacity", f32, (N, 4))
+    _check(radius, "radius", i32, (N,))
+    _check(rect, "rect", i32, (N, 4))
+    _check(tiles_touched, "tiles_touched", u32, (N,))
+    _check(d_num_pairs, "d_num_pairs", u32)
+    _check(ws, "ws", torch.uint8)
+    c = camera_struct(cam)
+    _ok("gs_preprocess_fwd", lib().gs_preprocess_fwd(
+        ctypes.byref(c), int(N), _ptr(means), _ptr(scales), _ptr(quats), _ptr(opacity), _ptr(mean2d), _ptr(depth),
+        _ptr(conic_opacity), _ptr(radius), _ptr(rect), _ptr(tiles_touched), _ptr(d_num_pairs), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def gs_bin_sort(cam, depth, rect, tiles_touched, d_num_pairs, capacity: int, ids, ranges, keys, ws,
+                stream=None) -> None:
+    N = depth.shape[0]
+    _check(depth, "depth", torch.float32, (N,))
+    _check(rect, "rect", torch.int32, (N, 4))
+    _check(tiles_touched, "tiles_touched", torch.uint32, (N,))
+    _check(d_num_pairs, "d_num_pairs", torch.uint32)
+    _check(ids, "ids", torch.uint32)
+    if ids.numel() < capacity:
+        raise ValueError("ids holds fewer elements than capacity")
+    _check(ranges, "ranges", torch.uint32, (num_tiles(cam), 2))
+    _check(keys, "keys", torch.uint64, optional=True)
+    if keys is not None and keys.numel() < capacity:
+        raise ValueError("keys holds fewer elements than capacity")
+    _check(ws, "ws", torch.uint8)
+    c = camera_struct(cam)
+    _ok("gs_bin_sort", lib().gs_bin_sort(
+        ctypes.byref(c), int(N), _ptr(depth), _ptr(rect), _ptr(tiles_touched), _ptr(d_num_pairs), int(capacity),
+        _ptr(ids), _ptr(ranges), _ptr(keys), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def gs_render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_T, n_contrib, stream=None) -> None:
+    N = mean2d.shape[0]
+    H, W = cam.height, cam.width
+    _check(ranges, "ranges", torch.uint32, (num_tiles(cam), 2))
+    _check(ids, "ids", torch.uint32)
+    _check(mean2d, "mean2d", torch.float32, (N, 2))
+    _check(conic_opacity, "conic_opacity", torch.float32, (N, 4))
+    _check(colors, "colors", torch.float32, (N, 3))
+    _check(image, "image", torch.float32, (3, H, W))
+    _check(final_T, "final_T", torch.float32, (H, W))
+    _check(n_contrib, "n_contrib", torch.uint32, (H, W))
+    c = camera_struct(cam)
+    _ok("gs_render_fwd", lib().gs_render_fwd(
+        ctypes.byref(c), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(colors), _ptr(image),
+        _ptr(final_T), _ptr(n_contrib), _stream(stream)))
+
+
+def gs_render_bwd(cam, ranges, ids, mean2d, conic_opacity, colors, final_T, n_contrib, dL_dimage, dL_dmean2d,
+                  dL_dconic_opacity, dL_dcolor, stream=None) -> None:
+    N = mean2d.shape[0]
+    H, W = cam.height, cam.width
+    _check(ranges, "ranges", torch.uint32, (num_tiles(cam), 2))
+    _check(ids, "ids", torch.uint32)
+    _check(mean2d, "mean2d", torch.float32, (N, 2))
+    _check(conic_opacity, "conic_opacity", torch.float32, (N, 4))
+    _check(colors, "colors", torch.float32, (N, 3))
+    _check(final_T, "final_T", torch.float32, (H, W))
+    _check(n_contrib, "n_contrib", torch.uint32, (H, W))
+    _check(dL_dimage, "dL_dimage", torch.float32, (3, H, W))
+    _check(dL_dmean2d, "dL_dmean2d", torch.float32, (N, 2))
+    _check(dL_dconic_opacity, "dL_dconic_opacity", torch.float32, (N, 4))
+    _check(dL_dcolor, "dL_dcolor", torch.float32, (N, 3))
+    c = camera_struct(cam)
+    _ok("gs_render_bwd", lib().gs_render_bwd(
+        ctypes.byref(c), int(N), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(colors),
+        _ptr(final_T), _ptr(n_contrib), _ptr(dL_dimage), _ptr(dL_dmean2d), _ptr(dL_dconic_opacity),
+        _ptr(dL_dcolor), _stream(stream)))
+
+
+def gs_preprocess_bwd(cam, means, scales, quats, radius, conic_opacity, dL_dmean2d, dL_dconic_opacity,
+                      dL_dcolor2d, dL_dmeans, dL_dscales, dL_dquats, dL_dopacity, dL_dcolors, stream=None) -> None:
+    N = means.shape[0]
+    f32 = torch.float32
+    _check(means, "means", f32, (N, 3))
+    _check(scales, "scales", f32, (N, 3))
+    _check(quats, "quats", f32, (N, 4))
+    _check(radius, "radius", torch.int32, (N,))
+    _check(conic_opacity, "conic_opacity", f32, (N, 4))
+    _check(dL_dmean2d, "dL_dmean2d", f32, (N, 2))
+    _check(dL_dconic_opacity, "dL_dconic_opacity", f32, (N, 4))
+    _check(dL_dcolor2d, "dL_dcolor2d", f32, (N, 3))
+    _check(dL_dmeans, "dL_dmeans", f32, (N, 3))
+    _check(dL_dscales, "dL_dscales", f32, (N, 3))
+    _check(dL_dquats, "dL_dquats", f32, (N, 4))
+    _check(dL_dopacity, "dL_dopacity", f32, (N,))
+    _check(dL_dcolors, "dL_dcolors", f32, (N, 3))
+    c = camera_struct(cam)
+    _ok("gs_preprocess_bwd", lib().gs_preprocess_bwd(
+        ctypes.byref(c), int(N), _ptr(means), _ptr(scales), _ptr(quats), _ptr(radius), _ptr(conic_opacity),
+        _ptr(dL_dmean2d), _ptr(dL_dconic_opacity), _ptr(dL_dcolor2d), _ptr(dL_dmeans), _ptr(dL_dscales),
+        _ptr(dL_dquats), _ptr(dL_dopacity), _ptr(dL_dcolors), _stream(stream)))

@@ -1,0 +1,60 @@
+// Library-level entry points: version, status text, workspace sizing and the
+// sticky device status word.
+
+#include <cuda_runtime.h>
+
+#include "gs_internal.cuh"
+
+extern "C" size_t gs_preprocess_ws_bytes(int N);
+extern "C" size_t gs_bin_sort_ws_bytes(int N, unsigned capacity);
+
+namespace {
+__global__ void k_clear_status(gs::WsHeader* h) { h->status = 0u; }
+}  // namespace
+
+extern "C" int gs_version(void) { return (1 << 16) | 0; }
+
+extern "C" const char* gs_status_string(int status) {
+    switch (status) {
+        case GS_OK: return "ok";
+        case GS_ERR_INVALID_ARG: return "invalid argument";
+        case GS_ERR_CAPACITY: return "pair count exceeds the caller's capacity";
+        case GS_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case GS_ERR_CUDA: return "CUDA launch or copy failed";
+        case GS_ERR_UNIMPLEMENTED: return "not implemented";
+        case GS_ERR_OVERFLOW: return "pair count does not fit in 32 bits";
+        default: return "several error flags are set";
+    }
+}
+
+extern "C" size_t gs_workspace_bytes(int stage, int N, unsigned capacity, int width, int height) {
+    if (N < 0 || width < 1 || height < 1) return 0;
+    switch (stage) {
+        case GS_STAGE_PREPROCESS_FWD: return gs_preprocess_ws_bytes(N);
+        case GS_STAGE_BIN_SORT: return gs_bin_sort_ws_bytes(N, capacity);
+        default: return 0;
+    }
+}
+
+extern "C" int gs_read_status(const void* ws, int* status, void* stream) {
+    if (!ws || !status) return GS_ERR_INVALID_ARG;
+    unsigned v = 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&v, ws, sizeof(unsigned), cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GS_ERR_CUDA;
+    }
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GS_ERR_CUDA;
+    }
+    *status = (int)v;
+    return GS_OK;
+}
+
+extern "C" int gs_clear_status(void* ws, void* stream) {
+    if (!ws) return GS_ERR_INVALID_ARG;
+    k_clear_status<<<1, 1, 0, (cudaStream_t)stream>>>(reinterpret_cast<gs::WsHeader*>(ws));
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+}

@@ -1,0 +1,510 @@
+// Tile binning and (tile, depth) ordering.
+//
+// "4-3DGS训练与优化" section E.3: each projected Gaussian's AABB selects the
+// tiles it may touch; the Gaussians of each tile are sorted by depth and
+// splatted in that order; tiles are independent.  "Gaussian Splatting反向传播的
+// CUDA实现" section 1: the sorted list and the per-tile ranges are kept and
+// reused by the backward.
+//
+// The order produced is that of a sort of 64-bit keys (tile << 32 |
+// float_bits(depth)) with ties broken by Gaussian id.  It is reached in two
+// sorts instead of one wide one:
+//   1. the N Gaussians are sorted by depth bits (stable LSD radix sort, 8-bit
+//      digits, ids in increasing order initially, culled ones last), which
+//      gives every visible Gaussian its (depth, id) rank;
+//   2. the (tile, Gaussian) pairs are emitted in rank order and stably sorted
+//      by tile id alone (ceil(log2 T) bits, at most 8 per pass).
+// A stable sort by tile of a list already in (depth, id) order yields the
+// (tile, depth, id) order, so the result is the same as the 64-bit sort while
+// the pair-sized passes only move the tile bits.
+//
+// Every kernel is a plain grid over its data; there are no inter-block waits.
+
+#include <cuda_runtime.h>
+
+#include "gs_internal.cuh"
+
+namespace gs {
+namespace {
+
+constexpr int kSortBlock = 256;
+constexpr int kSortMaxGrid = 148 * 4;  // CTAs per radix pass: a multiple of the SM count
+constexpr int kRadixMax = 256;
+constexpr int kMaxPasses = 8;          // 4 depth passes + up to 3 tile passes (+1 spare)
+constexpr int kScanItems = 8;          // items per thread in the rank-order scan
+constexpr int kScanTile = kSortBlock * kScanItems;
+
+struct SortMisc {
+    unsigned n_gauss;    // N
+    unsigned p_eff;      // P if it fits the capacity, else 0
+    unsigned pad[62];
+};
+
+struct BinWs {
+    WsHeader* hdr;
+    SortMisc* misc;
+    unsigned *dkeys0, *dvals0, *dkeys1, *dvals1;  // depth sort, N each
+    unsigned* pair_off;                            // N + 1
+    unsigned* scan_part;                           // ceil(N / kScanTile) + 1
+    unsigned *tkeys0, *tvals0, *tkeys1, *tvals1;   // pair sort, capacity each
+    unsigned* hist;                                // kMaxPasses * kRadixMax * kSortMaxGrid
+    unsigned* totals;                              // kMaxPasses * kRadixMax
+};
+
+size_t carve(void* base, int N, unsigned capacity, BinWs* w) {
+    size_t off = sizeof(WsHeader);
+    char* b = reinterpret_cast<char*>(base);
+    auto take = [&](size_t bytes) -> void* {
+        void* p = b ? b + off : nullptr;
+        off += align_up(bytes, 256);
+        return p;
+    };
+    const size_t n = (size_t)N, cap = (size_t)capacity;
+    BinWs t;
+    t.hdr = reinterpret_cast<WsHeader*>(base);
+    t.misc = (SortMisc*)take(sizeof(SortMisc));
+    t.dkeys0 = (unsigned*)take(n * 4);
+    t.dvals0 = (unsigned*)take(n * 4);
+    t.dkeys1 = (unsigned*)take(n * 4);
+    t.dvals1 = (unsigned*)take(n * 4);
+    t.pair_off = (unsigned*)take((n + 1) * 4);
+    t.scan_part = (unsigned*)take(((n + kScanTile - 1) / kScanTile + 1) * 4);
+    t.tkeys0 = (unsigned*)take(cap * 4);
+    t.tvals0 = (unsigned*)take(cap * 4);
+    t.tkeys1 = (unsigned*)take(cap * 4);
+    t.tvals1 = (unsigned*)take(cap * 4);
+    t.hist = (unsigned*)take((size_t)kMaxPasses * kRadixMax * kSortMaxGrid * 4);
+    t.totals = (unsigned*)take((size_t)kMaxPasses * kRadixMax * 4);
+    if (w) *w = t;
+    return off;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Zero the ranges and the per-pass digit totals, build the depth keys, check
+// the pair count against the capacity.
+__global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const unsigned* __restrict__ tiles_touched,
+                           const unsigned* __restrict__ d_num_pairs, unsigned capacity, BinWs w,
+                           unsigned* __restrict__ ranges) {
+    const int stride = gridDim.x * blockDim.x;
+    const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int i = tid; i < 2 * T; i += stride) ranges[i] = 0u;
+    for (int i = tid; i < kMaxPasses * kRadixMax; i += stride) w.totals[i] = 0u;
+    for (int i = tid; i < N; i += stride) {
+        w.dkeys0[i] = tiles_touched[i] > 0 ? __float_as_uint(depth[i]) : 0xFFFFFFFFu;
+        w.dvals0[i] = (unsigned)i;
+    }
+    if (tid == 0) {
+        const unsigned P = *d_num_pairs;
+        w.misc->n_gauss = (unsigned)N;
+        if (P > capacity) {
+            raise_status(w.hdr, GS_ERR_CAPACITY);
+            w.misc->p_eff = 0;
+        } else {
+            w.misc->p_eff = P;
+        }
+    }
+}
+
+__device__ __forceinline__ void chunk_of(unsigned n, unsigned& lo, unsigned& hi) {
+    const unsigned G = gridDim.x;
+    unsigned chunk = (n + G - 1) / G;
+    chunk = (chunk + 31u) & ~31u;
+    lo = min(n, blockIdx.x * chunk);
+    hi = min(n, lo + chunk);
+}
+
+// Per-CTA digit histogram of its contiguous chunk, stored digit-major:
+// hist[d * G + cta]; digit totals accumulate into totals[d].
+__global__ void __launch_bounds__(kSortBlock)
+k_radix_hist(const unsigned* __restrict__ keys, const unsigned* __restrict__ n_ptr, int shift, int bits,
+             unsigned* __restrict__ hist, unsigned* __restrict__ totals) {
+    __shared__ unsigned s_h[kRadixMax];
+    const int radix = 1 << bits;
+    const unsigned mask = radix - 1;
+    for (int d = threadIdx.x; d < radix; d += kSortBlock) s_h[d] = 0;
+    __syncthreads();
+    unsigned lo, hi;
+    chunk_of(*n_ptr, lo, hi);
+    const int lane = threadIdx.x & 31;
+    for (unsigned base = lo; base < hi; base += kSortBlock) {
+        const unsigned i = base + threadIdx.x;
+        const bool valid = i < hi;
+        const unsigned d = valid ? (keys[i] >> shift) & mask : (unsigned)kRadixMax;
+        const unsigned peers = __match_any_sync(0xffffffffu, d);
+        if (valid && lane == __ffs(peers) - 1) atomicAdd(&s_h[d], (unsigned)__popc(peers));
+    }
+    __syncthreads();
+    const unsigned G = gridDim.x;
+    for (int d = threadIdx.x; d < radix; d += kSortBlock) {
+        const unsigned c = s_h[d];
+        hist[(size_t)d * G + blockIdx.x] = c;
+        if (c) atomicAdd(&totals[d], c);
+    }
+}
+
+// One CTA per digit d: offsets[d][c] = (sum of totals below d) + exclusive
+// prefix over CTAs of hist[d][.], in place.
+__global__ void __launch_bounds__(kSortBlock)
+k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, int G) {
+    const int d = blockIdx.x;
+    __shared__ unsigned s_w[kSortBlock / 32];
+    __shared__ unsigned s_base;
+    // base of digit d
+    unsigned b = 0;
+    for (int e = threadIdx.x; e < d; e += kSortBlock) b += totals[e];
+    b = __reduce_add_sync(0xffffffffu, b);
+    if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = b;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned s = 0;
+        for (int k = 0; k < kSortBlock / 32; ++k) s += s_w[k];
+        s_base = s;
+    }
+    __syncthreads();
+    // exclusive scan of hist[d][0..G) with each thread owning a contiguous run
+    const int per = (G + kSortBlock - 1) / kSortBlock;
+    unsigned* row = hist + (size_t)d * G;
+    const int c0 = threadIdx.x * per;
+    unsigned local = 0;
+    for (int k = 0; k < per; ++k)
+        if (c0 + k < G) local += row[c0 + k];
+    // block exclusive scan of `local`
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    __syncthreads();
+    if (lane == 31) s_w[warp] = incl;
+    __syncthreads();
+    unsigned wbase = 0;
+    for (int k = 0; k < warp; ++k) wbase += s_w[k];
+    unsigned run = s_base + wbase + incl - local;
+    for (int k = 0; k < per; ++k)
+        if (c0 + k < G) {
+            const unsigned c = row[c0 + k];
+            row[c0 + k] = run;
+            run += c;
+        }
+}
+
+// Stable scatter: each CTA walks its chunk in order, 256 items at a time;
+// items with equal digits keep their order (warp, then lane, then step).
+__global__ void __launch_bounds__(kSortBlock)
+k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict__ vals_in,
+                unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out,
+                const unsigned* __restrict__ n_ptr, int shift, int bits, const unsigned* __restrict__ offsets) {
+    constexpr int kWarps = kSortBlock / 32;
+    __shared__ unsigned s_base[kRadixMax];
+    __shared__ unsigned s_cnt[kWarps][kRadixMax];
+    __shared__ unsigned s_off[kWarps][kRadixMax];
+    const int radix = 1 << bits;
+    const unsigned mask = radix - 1;
+    const unsigned G = gridDim.x;
+    for (int d = threadIdx.x; d < radix; d += kSortBlock) {
+        s_base[d] = offsets[(size_t)d * G + blockIdx.x];
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s_cnt[w][d] = 0;
+    }
+    __syncthreads();
+    unsigned lo, hi;
+    chunk_of(*n_ptr, lo, hi);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt = lanemask_lt();
+    for (unsigned base = lo; base < hi; base += kSortBlock) {
+        const unsigned i = base + threadIdx.x;
+        const bool valid = i < hi;
+        const unsigned key = valid ? keys_in[i] : 0u;
+        const unsigned val = valid ? vals_in[i] : 0u;
+        const unsigned d = valid ? (key >> shift) & mask : (unsigned)kRadixMax;
+        const unsigned peers = __match_any_sync(0xffffffffu, d);
+        const unsigned rank = __popc(peers & lt);
+        if (valid && lane == __ffs(peers) - 1) s_cnt[warp][d] = __popc(peers);
+        __syncthreads();
+        for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
+            unsigned run = s_base[dd];
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const unsigned c = s_cnt[w][dd];
+                s_cnt[w][dd] = 0;
+                s_off[w][dd] = run;
+                run += c;
+            }
+            s_base[dd] = run;
+        }
+        __syncthreads();
+        if (valid) {
+            const unsigned pos = s_off[warp][d] + rank;
+            keys_out[pos] = key;
+            vals_out[pos] = val;
+        }
+    }
+}
+
+// Exclusive scan, in depth-rank order, of the pair counts:
+// pair_off[r] = sum over ranks r' < r of tiles_touched[order[r']].
+__global__ void __launch_bounds__(kSortBlock)
+k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ tiles_touched,
+                unsigned* __restrict__ part) {
+    const int base = blockIdx.x * kScanTile;
+    unsigned s = 0;
+#pragma unroll
+    for (int k = 0; k < kScanItems; ++k) {
+        const int r = base + k * kSortBlock + threadIdx.x;
+        if (r < N) s += tiles_touched[order[r]];
+    }
+    s = __reduce_add_sync(0xffffffffu, s);
+    __shared__ unsigned s_w[kSortBlock / 32];
+    if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned t = 0;
+        for (int k = 0; k < kSortBlock / 32; ++k) t += s_w[k];
+        part[blockIdx.x] = t;
+    }
+}
+
+__global__ void __launch_bounds__(1024) k_scan_top(unsigned* __restrict__ part, int nb) {
+    // exclusive scan of nb partial sums by one CTA, each thread a contiguous run
+    __shared__ unsigned s_w[32];
+    const int per = (nb + 1023) / 1024;
+    const int c0 = threadIdx.x * per;
+    unsigned local = 0;
+    for (int k = 0; k < per; ++k)
+        if (c0 + k < nb) local += part[c0 + k];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_w[warp] = incl;
+    __syncthreads();
+    unsigned wbase = 0;
+    for (int k = 0; k < warp; ++k) wbase += s_w[k];
+    unsigned run = wbase + incl - local;
+    for (int k = 0; k < per; ++k)
+        if (c0 + k < nb) {
+            const unsigned c = part[c0 + k];
+            part[c0 + k] = run;
+            run += c;
+        }
+}
+
+__global__ void __launch_bounds__(kSortBlock)
+k_scan_down(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ tiles_touched,
+            const unsigned* __restrict__ part, unsigned* __restrict__ pair_off) {
+    // each thread owns kScanItems consecutive ranks
+    const int base = blockIdx.x * kScanTile + threadIdx.x * kScanItems;
+    unsigned v[kScanItems];
+    unsigned local = 0;
+#pragma unroll
+    for (int k = 0; k < kScanItems; ++k) {
+        const int r = base + k;
+        v[k] = r < N ? tiles_touched[order[r]] : 0u;
+        local += v[k];
+    }
+    __shared__ unsigned s_w[kSortBlock / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_w[warp] = incl;
+    __syncthreads();
+    unsigned wbase = 0;
+    for (int k = 0; k < warp; ++k) wbase += s_w[k];
+    unsigned run = part[blockIdx.x] + wbase + incl - local;
+#pragma unroll
+    for (int k = 0; k < kScanItems; ++k) {
+        const int r = base + k;
+        if (r < N) pair_off[r] = run;
+        run += v[k];
+    }
+}
+
+// Emit the (tile, Gaussian) pairs in depth-rank order.  A warp takes 32
+// consecutive ranks and writes each Gaussian's tiles with all 32 lanes
+// (row-major over its rectangle), so stores are coalesced and a Gaussian
+// covering thousands of tiles does not stall one lane.
+__global__ void __launch_bounds__(kSortBlock)
+k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
+       const int4* __restrict__ rect, const unsigned* __restrict__ tiles_touched, const SortMisc* __restrict__ misc,
+       unsigned* __restrict__ tkeys, unsigned* __restrict__ tvals) {
+    const unsigned P = misc->p_eff;
+    if (P == 0) return;  // nothing to emit, or over capacity
+    const int lane = threadIdx.x & 31;
+    const int warp_global = (blockIdx.x * kSortBlock + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * kSortBlock) >> 5;
+    for (int r0 = warp_global * 32; r0 < N; r0 += nwarps * 32) {
+        const int r = r0 + lane;
+        unsigned g = 0, off = 0, cnt = 0;
+        int4 rc = make_int4(0, 0, 0, 0);
+        if (r < N) {
+            g = order[r];
+            cnt = tiles_touched[g];
+            if (cnt) {
+                off = pair_off[r];
+                rc = rect[g];
+            }
+        }
+        unsigned todo = __ballot_sync(0xffffffffu, cnt != 0);
+        while (todo) {
+            const int src = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const unsigned gg = __shfl_sync(0xffffffffu, g, src);
+            const unsigned oo = __shfl_sync(0xffffffffu, off, src);
+            const unsigned cc = __shfl_sync(0xffffffffu, cnt, src);
+            const int x0 = __shfl_sync(0xffffffffu, rc.x, src);
+            const int y0 = __shfl_sync(0xffffffffu, rc.y, src);
+            const int x1 = __shfl_sync(0xffffffffu, rc.z, src);
+            const unsigned wdt = (unsigned)(x1 - x0);
+            // never write past P, even if the caller's counts disagree
+            const unsigned lim = oo < P ? min(cc, P - oo) : 0u;
+            for (unsigned k = lane; k < lim; k += 32) {
+                const unsigned ty = (unsigned)y0 + k / wdt;
+                const unsigned tx = (unsigned)x0 + k % wdt;
+                tkeys[oo + k] = ty * (unsigned)TX + tx;
+                tvals[oo + k] = gg;
+            }
+        }
+    }
+}
+
+// ranges[t] = [first, last + 1) of tile t in the sorted list, found by
+// comparing neighbours; optional 64-bit keys for callers that want them.
+__global__ void k_ranges(const unsigned* __restrict__ tkeys, const unsigned* __restrict__ ids,
+                         const float* __restrict__ depth, const SortMisc* __restrict__ misc, unsigned* __restrict__ ranges,
+                         unsigned long long* __restrict__ keys) {
+    const unsigned P = misc->p_eff;
+    const unsigned stride = gridDim.x * blockDim.x;
+    for (unsigned k = blockIdx.x * blockDim.x + threadIdx.x; k < P; k += stride) {
+        const unsigned t = tkeys[k];
+        if (k == 0 || tkeys[k - 1] != t) ranges[2 * t] = k;
+        if (k + 1 == P || tkeys[k + 1] != t) ranges[2 * t + 1] = k + 1;
+        if (keys) keys[k] = ((unsigned long long)t << 32) | __float_as_uint(depth[ids[k]]);
+    }
+}
+
+int ceil_log2(unsigned x) {
+    int b = 0;
+    while ((1ull << b) < x) ++b;
+    return b;
+}
+
+// One stable LSD radix sort of (keys, vals) over bits [0, total_bits), with
+// at most 8 bits per pass.  The final pass writes to (final_keys, final_vals)
+// when they are given.  Returns the number of passes.
+int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, unsigned* k0, unsigned* v0,
+               unsigned* k1, unsigned* v1, unsigned* final_vals, unsigned** out_keys, unsigned* hist,
+               unsigned* totals, int pass_base) {
+    const int passes = (total_bits + 7) / 8;
+    if (passes == 0) {
+        *out_keys = k0;
+        return 0;
+    }
+    const int bits = (total_bits + passes - 1) / passes;
+    unsigned *ki = k0, *vi = v0, *ko = k1, *vo = v1;
+    for (int p = 0; p < passes; ++p) {
+        const bool last = p == passes - 1;
+        unsigned* vdst = (last && final_vals) ? final_vals : vo;
+        unsigned* h = hist + (size_t)(pass_base + p) * kRadixMax * kSortMaxGrid;
+        unsigned* tot = totals + (size_t)(pass_base + p) * kRadixMax;
+        k_radix_hist<<<G, kSortBlock, 0, st>>>(ki, n_ptr, p * bits, bits, h, tot);
+        k_radix_scan<<<1 << bits, kSortBlock, 0, st>>>(h, tot, G);
+        k_radix_scatter<<<G, kSortBlock, 0, st>>>(ki, vi, ko, vdst, n_ptr, p * bits, bits, h);
+        unsigned* tk = ki;
+        ki = ko;
+        ko = tk;
+        unsigned* tv = vi;
+        vi = vdst;
+        vo = tv;
+    }
+    *out_keys = ki;
+    return passes;
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" size_t gs_bin_sort_ws_bytes(int N, unsigned capacity) {
+    if (N < 0) return 0;
+    return carve(nullptr, N, capacity, nullptr);
+}
+
+extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, const int* rect,
+                           const unsigned* tiles_touched, const unsigned* d_num_pairs, unsigned capacity,
+                           unsigned* ids, unsigned* ranges, unsigned long long* keys, void* ws, size_t ws_bytes,
+                           void* stream) {
+    if (!camera_ok(cam) || N < 0 || !d_num_pairs || !ranges || !ws) return GS_ERR_INVALID_ARG;
+    if (N > 0 && (!depth || !rect || !tiles_touched)) return GS_ERR_INVALID_ARG;
+    if (capacity > 0 && !ids) return GS_ERR_INVALID_ARG;
+    if (!aligned(ws, 256) || ws_bytes < gs_bin_sort_ws_bytes(N, capacity)) return GS_ERR_INVALID_ARG;
+    if (rect && !aligned(rect, 16)) return GS_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    BinWs w;
+    carve(ws, N, capacity, &w);
+    const int TX = tiles_x(*cam), TY = tiles_y(*cam), T = TX * TY;
+
+    {
+        int work = N > 2 * T ? N : 2 * T;
+        int blocks = (work + 255) / 256;
+        if (blocks < 1) blocks = 1;
+        if (blocks > 148 * 8) blocks = 148 * 8;
+        k_bin_init<<<blocks, 256, 0, st>>>(N, T, depth, tiles_touched, d_num_pairs, capacity, w, ranges);
+        GS_LAUNCH_CHECK();
+    }
+    if (N == 0) return GS_OK;
+
+    // 1. depth ranks of the Gaussians (32-bit keys, culled ones last)
+    const int Gd = (N + 2047) / 2048 < kSortMaxGrid ? (N + 2047) / 2048 : kSortMaxGrid;
+    unsigned* dkeys_sorted = nullptr;
+    const int dpasses = radix_sort(st, Gd, &w.misc->n_gauss, 32, w.dkeys0, w.dvals0, w.dkeys1, w.dvals1, nullptr,
+                                   &dkeys_sorted, w.hist, w.totals, 0);
+    const unsigned* order = (dpasses % 2 == 0) ? w.dvals0 : w.dvals1;
+    GS_LAUNCH_CHECK();
+
+    // 2. pair offsets in rank order
+    const int nb = (N + kScanTile - 1) / kScanTile;
+    k_scan_partials<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, w.scan_part);
+    k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb);
+    k_scan_down<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, w.scan_part, w.pair_off);
+    GS_LAUNCH_CHECK();
+    if (capacity == 0) return GS_OK;
+
+    // 3. emit pairs in rank order, then a stable sort by tile id
+    const int tile_bits = ceil_log2((unsigned)T);
+    const int tpasses = (tile_bits + 7) / 8;
+    {
+        int blocks = (N + kSortBlock - 1) / kSortBlock;
+        if (blocks > 148 * 16) blocks = 148 * 16;
+        unsigned* emit_vals = tpasses == 0 ? ids : w.tvals0;
+        k_emit<<<blocks, kSortBlock, 0, st>>>(N, TX, order, w.pair_off, reinterpret_cast<const int4*>(rect),
+                                              tiles_touched, w.misc, w.tkeys0, emit_vals);
+        GS_LAUNCH_CHECK();
+    }
+    const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
+    unsigned* tkeys_sorted = nullptr;
+    radix_sort(st, Gp, &w.misc->p_eff, tile_bits, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, ids, &tkeys_sorted,
+               w.hist, w.totals, 4);
+    GS_LAUNCH_CHECK();
+
+    // 4. tile ranges (and optional 64-bit keys)
+    {
+        int blocks = (int)((capacity + 255u) / 256u);
+        if (blocks > 148 * 8) blocks = 148 * 8;
+        if (blocks < 1) blocks = 1;
+        k_ranges<<<blocks, 256, 0, st>>>(tkeys_sorted, ids, depth, w.misc, ranges, keys);
+        GS_LAUNCH_CHECK();
+    }
+    return GS_OK;
+}

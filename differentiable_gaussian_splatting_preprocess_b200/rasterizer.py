@@ -1,0 +1,138 @@
+"""A frame-level driver over the C ABI: allocates device buffers with torch,
+calls the five stages in order on the current stream, and keeps the forward's
+buffers (sorted ids, tile ranges, final transmittance, contributor counts) for
+the backward, as the backward of "Gaussian Splatting反向传播的CUDA实现"
+(section 1) reuses them.  All arithmetic runs in libgs.so.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import torch
+
+from . import binding as B
+
+
+@dataclasses.dataclass
+class Frame:
+    """Buffers of one forward pass (device tensors)."""
+    N: int
+    capacity: int
+    mean2d: torch.Tensor
+    depth: torch.Tensor
+    conic_opacity: torch.Tensor
+    radius: torch.Tensor
+    rect: torch.Tensor
+    tiles_touched: torch.Tensor
+    num_pairs: torch.Tensor      # [1] uint32, on the device
+    ids: torch.Tensor
+    ranges: torch.Tensor
+    keys: Optional[torch.Tensor]
+    image: torch.Tensor
+    final_T: torch.Tensor
+    n_contrib: torch.Tensor
+
+
+class Rasterizer:
+    """One camera's rasterizer with cached device buffers.
+
+    Buffers are reused across calls while N, the capacity and the image size
+    stay the same, so repeated frames allocate nothing.  The workspace is
+    zero-filled when it is (re)allocated, as the C ABI requires.
+    """
+
+    def __init__(self, cam, device: Optional[torch.device] = None):
+        self.cam = cam
+        self.device = torch.device("cuda") if device is None else torch.device(device)
+        self._bufs: Dict[str, torch.Tensor] = {}
+        self.ws: Optional[torch.Tensor] = None
+
+    # -- buffers ----------------------------------------------------------
+    def _buf(self, name: str, shape, dtype, zero: bool = False) -> torch.Tensor:
+        t = self._bufs.get(name)
+        if t is None or tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+            t = (torch.zeros if zero else torch.empty)(tuple(shape), dtype=dtype, device=self.device)
+            self._bufs[name] = t
+        return t
+
+    def workspace(self, N: int, capacity: int) -> torch.Tensor:
+        W, H = self.cam.width, self.cam.height
+        need = max(B.gs_workspace_bytes(B.GS_STAGE_PREPROCESS_FWD, N, 0, W, H),
+                   B.gs_workspace_bytes(B.GS_STAGE_BIN_SORT, N, capacity, W, H))
+        if self.ws is None or self.ws.numel() < need:
+            self.ws = torch.zeros(need + (need >> 4), dtype=torch.uint8, device=self.device)
+        return self.ws
+
+    # -- stages -----------------------------------------------------------
+    def preprocess(self, means, scales, quats, opacity, stream=None):
+        N = means.shape[0]
+        ws = self.workspace(N, 0)
+        out = dict(mean2d=self._buf("mean2d", (N, 2), torch.float32),
+                   depth=self._buf("depth", (N,), torch.float32),
+                   conic_opacity=self._buf("conic_opacity", (N, 4), torch.float32),
+                   radius=self._buf("radius", (N,), torch.int32),
+                   rect=self._buf("rect", (N, 4), torch.int32),
+                   tiles_touched=self._buf("tiles_touched", (N,), torch.uint32),
+                   num_pairs=self._buf("num_pairs", (1,), torch.uint32))
+        B.gs_preprocess_fwd(self.cam, means, scales, quats, opacity, out["mean2d"], out["depth"],
+                            out["conic_opacity"], out["radius"], out["rect"], out["tiles_touched"],
+                            out["num_pairs"], ws, stream)
+        return out
+
+    def forward(self, means, scales, quats, opacity, colors, capacity: Optional[int] = None,
+                want_keys: bool = False, stream=None) -> Frame:
+        """Preprocess, bin/sort and composite one frame.
+
+        With ``capacity=None`` the pair count is read back to size the sort
+        buffers (one device-to-host copy).  With a capacity the call makes no
+        host round trip; if the frame needs more pairs, the status word of
+        the workspace reports GS_ERR_CAPACITY and every tile range is empty.
+        """
+        N = means.shape[0]
+        pre = self.preprocess(means, scales, quats, opacity, stream)
+        if capacity is None:
+            capacity = int(pre["num_pairs"].to("cpu").view(torch.int32).item()) & 0xFFFFFFFF
+        ws = self.workspace(N, capacity)
+        ids = self._buf("ids", (max(capacity, 1),), torch.uint32)
+        ranges = self._buf("ranges", (B.num_tiles(self.cam), 2), torch.uint32)
+        keys = self._buf("keys", (max(capacity, 1),), torch.uint64) if want_keys else None
+        B.gs_bin_sort(self.cam, pre["depth"], pre["rect"], pre["tiles_touched"], pre["num_pairs"], capacity, ids,
+                      ranges, keys, ws, stream)
+        H, W = self.cam.height, self.cam.width
+        image = self._buf("image", (3, H, W), torch.float32)
+        final_T = self._buf("final_T", (H, W), torch.float32)
+        n_contrib = self._buf("n_contrib", (H, W), torch.uint32)
+        B.gs_render_fwd(self.cam, ranges, ids, pre["mean2d"], pre["conic_opacity"], colors, image, final_T,
+                        n_contrib, stream)
+        return Frame(N=N, capacity=capacity, ids=ids, ranges=ranges, keys=keys, image=image, final_T=final_T,
+                     n_contrib=n_contrib, **pre)
+
+    def backward(self, frame: Frame, means, scales, quats, colors, dL_dimage,
+                 grads: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
+        """Render backward then preprocess backward.  3D gradients are
+        accumulated into ``grads`` (zeros are allocated when it is None)."""
+        N = frame.N
+        g2 = dict(dL_dmean2d=self._buf("dL_dmean2d", (N, 2), torch.float32),
+                  dL_dconic_opacity=self._buf("dL_dconic_opacity", (N, 4), torch.float32),
+                  dL_dcolor=self._buf("dL_dcolor", (N, 3), torch.float32))
+        B.gs_render_bwd(self.cam, frame.ranges, frame.ids, frame.mean2d, frame.conic_opacity, colors, frame.final_T,
+                        frame.n_contrib, dL_dimage, g2["dL_dmean2d"], g2["dL_dconic_opacity"], g2["dL_dcolor"],
+                        stream)
+        if grads is None:
+            grads = zero_grads(N, self.device)
+        B.gs_preprocess_bwd(self.cam, means, scales, quats, frame.radius, frame.conic_opacity, g2["dL_dmean2d"],
+                            g2["dL_dconic_opacity"], g2["dL_dcolor"], grads["dL_dmeans"], grads["dL_dscales"],
+                            grads["dL_dquats"], grads["dL_dopacity"], grads["dL_dcolors"], stream)
+        grads.update(g2)
+        return grads
+
+    def status(self, stream=None) -> int:
+        return 0 if self.ws is None else B.gs_read_status(self.ws, stream)
+
+
+def zero_grads(N: int, device) -> Dict[str, torch.Tensor]:
+    f = dict(dtype=torch.float32, device=device)
+    return dict(dL_dmeans=torch.zeros((N, 3), **f), dL_dscales=torch.zeros((N, 3), **f),
+                dL_dquats=torch.zeros((N, 4), **f), dL_dopacity=torch.zeros((N,), **f),
+                dL_dcolors=torch.zeros((N, 3), **f))

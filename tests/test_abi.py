@@ -1,0 +1,69 @@
+"""The C-ABI library loads and exports every symbol include/gs.h declares, and
+its host-side helpers behave; no compute call is made (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from differentiable_gaussian_splatting_preprocess_b200 import binding as B
+from differentiable_gaussian_splatting_preprocess_b200 import build as BUILD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.lib()
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"GS_API\s+[\w\s\*]+?\b(gs_\w+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert declared == set(B.EXPORTED)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_camera_struct_layout_matches_header():
+    # int width, height, tile; float fx, fy, cx, cy, R[9], t[3], 6 scalars, bg[3]
+    assert ctypes.sizeof(B.GsCamera) == 4 * (3 + 4 + 9 + 3 + 6 + 3)
+
+
+def test_version_and_status_strings(lib):
+    assert B.version() >> 16 == 1
+    assert B.status_string(B.GS_OK) == "ok"
+    assert "capacity" in B.status_string(B.GS_ERR_CAPACITY)
+    assert "several" in B.status_string(B.GS_ERR_CAPACITY | B.GS_ERR_TIMEOUT)
+
+
+def test_workspace_sizes(lib):
+    a = B.gs_workspace_bytes(B.GS_STAGE_PREPROCESS_FWD, 1000, 0, 64, 64)
+    b = B.gs_workspace_bytes(B.GS_STAGE_PREPROCESS_FWD, 100000, 0, 64, 64)
+    assert 256 < a < b
+    c = B.gs_workspace_bytes(B.GS_STAGE_BIN_SORT, 1000, 10000, 64, 64)
+    d = B.gs_workspace_bytes(B.GS_STAGE_BIN_SORT, 1000, 20000, 64, 64)
+    assert d - c >= 4 * 4 * 10000 - 4 * 256  # four pair-sized buffers, each 256-byte aligned
+    assert B.gs_workspace_bytes(7, 10, 10, 64, 64) == 0
+    assert B.gs_workspace_bytes(B.GS_STAGE_BIN_SORT, -1, 10, 64, 64) == 0
+
+
+def test_host_argument_checks_need_no_device(lib):
+    cam = B.GsCamera()
+    cam.width, cam.height, cam.tile = 64, 64, 8  # tile must be 16
+    rc = lib.gs_preprocess_fwd(ctypes.byref(cam), 0, *([None] * 11), None, 0, None)
+    assert rc == B.GS_ERR_INVALID_ARG
+    cam.tile = 16
+    rc = lib.gs_render_fwd(ctypes.byref(cam), *([None] * 8), None)
+    assert rc == B.GS_ERR_INVALID_ARG
+    rc = lib.gs_bin_sort(ctypes.byref(cam), -1, None, None, None, None, 0, None, None, None, None, 0, None)
+    assert rc == B.GS_ERR_INVALID_ARG

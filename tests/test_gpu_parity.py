@@ -1,0 +1,291 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars: bit-exact preprocess integers, depth bits, tile ranges, sorted ids and
+64-bit keys; contributor counts equal on >= 99.99% of pixels; image absolute
+error <= 1e-4; per-tensor gradient relative L2 error <= 1e-3 (fp32 kernels
+against the float64 oracle).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from differentiable_gaussian_splatting_preprocess_b200 import binding as B
+from differentiable_gaussian_splatting_preprocess_b200 import scenes
+
+from _gpu_pipeline import (GRAD_REL_L2, IMAGE_ATOL, N_CONTRIB_MATCH, GpuScene, frame_np, rel_l2, run_gpu, to_dev,
+                           to_np)
+
+pytestmark = pytest.mark.gpu
+
+_CACHE = {}
+
+
+def _scene(cfg):
+    if cfg not in _CACHE:
+        _CACHE.clear()
+        _CACHE[cfg] = scenes.preset(cfg)
+    return _CACHE[cfg]
+
+
+def _check_preprocess(sc, cam, g):
+    o = oracle.preprocess(cam, sc.means, sc.scales, sc.quats, sc.opacity, "f32")
+    for k in ("radius", "rect", "tiles_touched"):
+        np.testing.assert_array_equal(g[k], o[k], err_msg=k)
+    for k in ("depth", "mean2d", "conic_opacity"):
+        np.testing.assert_array_equal(g[k].view(np.uint32), o[k].view(np.uint32), err_msg=k)
+    assert g["num_pairs"] == int(o["tiles_touched"].astype(np.uint64).sum())
+    return o
+
+
+def _check_bins(cam, g, pre):
+    b = oracle.bin_pairs(cam, pre["depth"], pre["rect"], pre["tiles_touched"], "f32")
+    assert b["num_pairs"] == g["num_pairs"]
+    np.testing.assert_array_equal(g["ranges"], b["ranges"])
+    np.testing.assert_array_equal(g["ids"], b["ids"])
+    np.testing.assert_array_equal(g["keys"], b["keys"])
+    return b
+
+
+def _check_render_fwd(cam, sc, g, tiles=None):
+    o = oracle.render_fwd(cam, g["ranges"], g["ids"], g["mean2d"], g["conic_opacity"], sc.colors, "f32", tiles=tiles)
+    if tiles is None:
+        mask = np.ones((cam.height, cam.width), bool)
+    else:
+        mask = np.zeros((cam.height, cam.width), bool)
+        TX = cam.tiles_x
+        for t in tiles:
+            tx, ty = t % TX, t // TX
+            mask[ty * 16:(ty + 1) * 16, tx * 16:(tx + 1) * 16] = True
+    err = np.abs(g["image"] - o["image"])[:, mask].max()
+    assert err <= IMAGE_ATOL, f"image abs err {err}"
+    match = (g["n_contrib"][mask] == o["n_contrib"][mask]).mean()
+    assert match >= N_CONTRIB_MATCH, f"n_contrib match {match}"
+    assert np.abs(g["final_T"] - o["final_T"])[mask].max() <= IMAGE_ATOL
+    return o
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_forward_parity(cfg):
+    sc = _scene(cfg)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    r = run_gpu(gs, cam)
+    g = frame_np(r["frame"])
+    assert r["rz"].status() == 0
+    pre = _check_preprocess(sc, cam, g)
+    _check_bins(cam, g, pre)          # isolated == end to end: preprocess is bit-exact
+    _check_render_fwd(cam, sc, g)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_backward_parity(cfg):
+    sc = _scene(cfg)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    r = run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0])
+    g = frame_np(r["frame"])
+    gr = {k: to_np(v) for k, v in r["grads"].items()}
+    # 2D gradients on identical inputs (isolated)
+    o2 = oracle.render_bwd(cam, sc.N, g["ranges"], g["ids"], g["mean2d"], g["conic_opacity"], sc.colors,
+                           sc.dL_dimage[0], "f64")
+    assert rel_l2(gr["dL_dmean2d"], o2["dL_dmean2d"]) <= GRAD_REL_L2
+    assert rel_l2(gr["dL_dconic_opacity"][:, :3], o2["dL_dconic_opacity"][:, :3]) <= GRAD_REL_L2
+    assert rel_l2(gr["dL_dconic_opacity"][:, 3], o2["dL_dconic_opacity"][:, 3]) <= GRAD_REL_L2
+    assert rel_l2(gr["dL_dcolor"], o2["dL_dcolor"]) <= GRAD_REL_L2
+    # 3D gradients from the same 2D gradients (isolated chain rule)
+    o3 = oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, g["radius"], gr["dL_dmean2d"],
+                               gr["dL_dconic_opacity"], gr["dL_dcolor"], "f64")
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+        e = rel_l2(gr[k], o3[k])
+        assert e <= 1e-5, (k, e)
+    # end to end: the float64 oracle's own forward and backward
+    if cfg <= 3:
+        f = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0],
+                                    "f64")
+        for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+            e = rel_l2(gr[k], f[k])
+            assert e <= GRAD_REL_L2, (k, e)
+        assert np.abs(g["image"] - f["image"]).max() <= IMAGE_ATOL
+
+
+def _sample_tiles(cam, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(cam.num_tiles, size=min(n, cam.num_tiles), replace=False)).astype(np.int32)
+
+
+@pytest.mark.slow
+def test_config5_four_cameras_sampled():
+    """3M Gaussians, four cameras rendered back to back with 3D gradients
+    accumulated: preprocess bit-exact per camera, sampled tile lists against
+    brute force, sampled tiles' compositing and gradients against the oracle
+    (the upstream gradient is restricted to the sampled tiles, so the oracle
+    only has to run those)."""
+    sc = _scene(5)
+    gs = GpuScene(sc)
+    grads = None
+    o3 = None
+    for ci, cam in enumerate(sc.cameras):
+        tiles = _sample_tiles(cam, 12, ci)
+        mask = np.zeros((cam.height, cam.width), bool)
+        for t in tiles:
+            tx, ty = t % cam.tiles_x, t // cam.tiles_x
+            mask[ty * 16:(ty + 1) * 16, tx * 16:(tx + 1) * 16] = True
+        dl = np.where(mask[None], sc.dL_dimage[ci], 0.0).astype(np.float32)
+        r = run_gpu(gs, cam, dL_dimage=dl, want_keys=False, grads=grads)
+        grads = {k: r["grads"][k] for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors")}
+        g = frame_np(r["frame"])
+        pre = _check_preprocess(sc, cam, g)
+        for t in tiles[:6]:
+            s, e = g["ranges"][t]
+            np.testing.assert_array_equal(g["ids"][s:e], oracle.tile_list(cam, pre["depth"], pre["rect"],
+                                                                          pre["tiles_touched"], int(t)))
+        _check_render_fwd(cam, sc, g, tiles=tiles)
+        o2 = oracle.render_bwd(cam, sc.N, g["ranges"], g["ids"], g["mean2d"], g["conic_opacity"], sc.colors, dl,
+                               "f64", tiles=tiles)
+        gr = {k: to_np(r["grads"][k]) for k in ("dL_dmean2d", "dL_dconic_opacity", "dL_dcolor")}
+        assert rel_l2(gr["dL_dmean2d"], o2["dL_dmean2d"]) <= GRAD_REL_L2
+        assert rel_l2(gr["dL_dconic_opacity"], o2["dL_dconic_opacity"]) <= GRAD_REL_L2
+        assert rel_l2(gr["dL_dcolor"], o2["dL_dcolor"]) <= GRAD_REL_L2
+        o3 = oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, g["radius"], o2["dL_dmean2d"],
+                                   o2["dL_dconic_opacity"], o2["dL_dcolor"], "f64", accumulate_into=o3)
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+        e = rel_l2(to_np(grads[k]), o3[k])
+        assert e <= GRAD_REL_L2, (k, e)
+
+
+# --------------------------------------------------------------------------
+# Edge cases
+# --------------------------------------------------------------------------
+
+def _tiny(**kw):
+    return scenes.random_tiny(**kw)
+
+
+def test_empty_scene():
+    cam = scenes.Camera(40, 24, 40.0, 40.0, 20.0, 12.0, bg=(0.25, 0.5, 0.75))
+    e = np.zeros((0, 3), np.float32)
+    sc = scenes.Scene("empty", e, e, np.zeros((0, 4), np.float32), np.zeros(0, np.float32), e, [cam],
+                      [np.ones((3, 24, 40), np.float32)])
+    gs = GpuScene(sc)
+    r = run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0], want_keys=True)
+    g = frame_np(r["frame"])
+    assert g["num_pairs"] == 0 and not g["ranges"].any()
+    np.testing.assert_array_equal(g["image"], np.broadcast_to(np.array([0.25, 0.5, 0.75], np.float32)[:, None, None],
+                                                              (3, 24, 40)))
+    assert np.all(g["final_T"] == 1.0) and not g["n_contrib"].any()
+
+
+def test_all_culled():
+    sc = _tiny(n=20, seed=3)
+    sc.means[:, 2] = -1.0
+    gs = GpuScene(sc)
+    r = run_gpu(gs, sc.cameras[0], dL_dimage=sc.dL_dimage[0])
+    g = frame_np(r["frame"])
+    assert g["num_pairs"] == 0 and not g["radius"].any()
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+        assert not to_np(r["grads"][k]).any()
+
+
+@pytest.mark.parametrize("W,H", [(37, 23), (16, 16), (1, 1), (300, 17)])
+def test_ragged_and_tiny_images(W, H):
+    sc = _tiny(n=40, width=W, height=H, seed=W + H, z_range=(1.5, 6.0))
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    dl = np.random.default_rng(0).normal(size=(3, H, W)).astype(np.float32)
+    r = run_gpu(gs, cam, dL_dimage=dl)
+    g = frame_np(r["frame"])
+    pre = _check_preprocess(sc, cam, g)
+    _check_bins(cam, g, pre)
+    _check_render_fwd(cam, sc, g)
+    f = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, dl, "f64")
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+        assert rel_l2(to_np(r["grads"][k]), f[k]) <= GRAD_REL_L2, k
+
+
+def test_no_thresholds_and_large_support():
+    """alpha_min = T_min = 0 and a support radius covering the whole image."""
+    sc = _tiny(n=24, width=64, height=48, seed=11, sigma_mult=1e3, alpha_min=0.0, T_min=0.0)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    r = run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0])
+    g = frame_np(r["frame"])
+    pre = _check_preprocess(sc, cam, g)
+    assert np.all(pre["tiles_touched"] == cam.num_tiles)
+    _check_bins(cam, g, pre)
+    _check_render_fwd(cam, sc, g)
+    f = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0], "f64")
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+        assert rel_l2(to_np(r["grads"][k]), f[k]) <= GRAD_REL_L2, k
+
+
+def test_capacity_overflow_is_reported_and_recoverable():
+    sc = _scene(2)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    r = run_gpu(gs, cam, capacity=1000)
+    rz = r["rz"]
+    assert rz.status() & B.GS_ERR_CAPACITY
+    assert not to_np(r["frame"].ranges).any()
+    B.gs_clear_status(rz.ws)
+    assert rz.status() == 0
+    fr = rz.forward(gs.means, gs.scales, gs.quats, gs.opacity, gs.colors)
+    torch.cuda.synchronize()
+    assert rz.status() == 0 and int(to_np(fr.num_pairs)[0]) > 1000
+
+
+def test_capacity_mode_matches_host_sized():
+    sc = _scene(2)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    a = frame_np(run_gpu(gs, cam)["frame"])
+    b = frame_np(run_gpu(gs, cam, capacity=a["num_pairs"] + 12345)["frame"])
+    for k in ("ranges", "ids", "keys", "image", "n_contrib"):
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_degenerate_inputs_are_culled():
+    sc = _tiny(n=8, seed=5)
+    sc.means[0] = np.nan
+    sc.quats[1] = 0.0
+    sc.scales[2] = 0.0  # zero covariance: dilation keeps the determinant positive
+    sc.means[3, 2] = 0.1  # nearer than z_near
+    gs = GpuScene(sc)
+    r = run_gpu(gs, sc.cameras[0], dL_dimage=sc.dL_dimage[0])
+    g = frame_np(r["frame"])
+    pre = _check_preprocess(sc, sc.cameras[0], g)
+    assert list(pre["radius"][[0, 1, 3]]) == [0, 0, 0]
+    assert pre["radius"][2] > 0
+    _check_render_fwd(sc.cameras[0], sc, g)
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats"):
+        v = to_np(r["grads"][k])
+        assert np.all(np.isfinite(v)) and not v[[0, 1, 3]].any()
+
+
+def test_invalid_arguments_raise_without_launch():
+    sc = _tiny(n=4)
+    gs = GpuScene(sc)
+    cam = sc.cameras[0]
+    bad = cam.replace(tile=8)
+    from differentiable_gaussian_splatting_preprocess_b200 import rasterizer as RZ
+    with pytest.raises(B.GsError):
+        RZ.Rasterizer(bad).forward(gs.means, gs.scales, gs.quats, gs.opacity, gs.colors)
+    rz = RZ.Rasterizer(cam)
+    small_ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    out = rz.preprocess(gs.means, gs.scales, gs.quats, gs.opacity)
+    with pytest.raises(B.GsError):
+        B.gs_preprocess_fwd(cam, gs.means, gs.scales, gs.quats, gs.opacity, out["mean2d"], out["depth"],
+                            out["conic_opacity"], out["radius"], out["rect"], out["tiles_touched"],
+                            out["num_pairs"], small_ws)
+
+
+def test_preprocess_backward_accumulates():
+    sc = _tiny(n=16, seed=9)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    r1 = run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0])
+    once = {k: to_np(v).copy() for k, v in r1["grads"].items()}
+    r2 = run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0], grads={k: v.clone() for k, v in r1["grads"].items()
+                                                              if k.startswith("dL_d") and v.shape[0] == sc.N})
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+        np.testing.assert_allclose(to_np(r2["grads"][k]), 2 * once[k], rtol=1e-5, atol=1e-7)
