@@ -30,7 +30,8 @@ TILE = 16
 
 # Every symbol include/gs.h declares.
 EXPORTED = ("gs_version", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
-            "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd")
+            "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd",
+            "gs_preprocess_fwd_noalloc")
 
 
 class GsCamera(ctypes.Structure):
@@ -263,3 +264,35 @@ def gs_preprocess_bwd(cam, means, scales, quats, radius, conic_opacity, dL_dmean
         ctypes.byref(c), int(N), _ptr(means), _ptr(scales), _ptr(quats), _ptr(radius), _ptr(conic_opacity),
         _ptr(dL_dmean2d), _ptr(dL_dconic_opacity), _ptr(dL_dcolor2d), _ptr(dL_dmeans), _ptr(dL_dscales),
         _ptr(dL_dquats), _ptr(dL_dopacity), _ptr(dL_dcolors), _stream(stream)))
+
+
+NOALLOC_MAX_GAUSSIANS = 1 << 24
+
+
+def gs_preprocess_fwd_noalloc(cam, means, scales, quats, opacity, mean2d, depth, conic_opacity, radius, rect,
+                              tiles_touched, d_num_pairs, stream=None) -> None:
+    """gs_preprocess_fwd without a workspace, for callers that cannot
+    allocate device memory: the scratch is a fixed array inside libgs.so
+    (N up to NOALLOC_MAX_GAUSSIANS; calls on one device must not overlap)."""
+    L = lib()
+    fn = L.gs_preprocess_fwd_noalloc
+    if fn.argtypes is None:
+        fn.restype = ctypes.c_int
+        fn.argtypes = [ctypes.POINTER(GsCamera), ctypes.c_int] + [ctypes.c_void_p] * 11 + [ctypes.c_void_p]
+    N = means.shape[0]
+    f32, i32, u32 = torch.float32, torch.int32, torch.uint32
+    _check(means, "means", f32, (N, 3))
+    _check(scales, "scales", f32, (N, 3))
+    _check(quats, "quats", f32, (N, 4))
+    _check(opacity, "opacity", f32, (N,))
+    _check(mean2d, "mean2d", f32, (N, 2))
+    _check(depth, "depth", f32, (N,))
+    _check(conic_opacity, "conic_opacity", f32, (N, 4))
+    _check(radius, "radius", i32, (N,))
+    _check(rect, "rect", i32, (N, 4))
+    _check(tiles_touched, "tiles_touched", u32, (N,))
+    _check(d_num_pairs, "d_num_pairs", u32)
+    c = camera_struct(cam)
+    _ok("gs_preprocess_fwd_noalloc", fn(
+        ctypes.byref(c), int(N), _ptr(means), _ptr(scales), _ptr(quats), _ptr(opacity), _ptr(mean2d), _ptr(depth),
+        _ptr(conic_opacity), _ptr(radius), _ptr(rect), _ptr(tiles_touched), _ptr(d_num_pairs), _stream(stream)))

@@ -392,3 +392,86 @@ extern "C" int gs_preprocess_bwd(const gs_camera* cam, int N, const float* means
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
+
+// ---------------------------------------------------------------------------
+// gs_preprocess_fwd_noalloc: the same projection for callers that may not
+// allocate device memory at all - a plug-in living inside a host application
+// whose allocator owns every device byte, or a per-frame loop where a
+// cudaMalloc would synchronise the device and stall the frame.  Such callers
+// cannot provide the workspace gs_preprocess_fwd asks for, so this variant
+// keeps its scratch (the status/ticket header and one 64-bit partial sum per
+// 256 Gaussians) in a fixed array compiled into the library.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace gs {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes =
+    sizeof(WsHeader) + (size_t)(GS_NOALLOC_MAX_GAUSSIANS / kPreBlock) * sizeof(unsigned long long);
+
+// One copy per device that loads the library, resident until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 256;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_device_addr[kNoAllocMaxDevices];  // device address of the array, per device
+
+// The array's name is only a host-side handle; the device address must be
+// looked up with the device current.  Done once per device, on first use.
+int noalloc_scratch_address(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GS_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return GS_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_device_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            (void)cudaGetLastError();
+            return GS_ERR_CUDA;
+        }
+        g_noalloc_device_addr[dev] = p;
+    }
+    *out = g_noalloc_device_addr[dev];
+    return GS_OK;
+}
+
+}  // namespace
+}  // namespace gs
+
+extern "C" int gs_preprocess_fwd_noalloc(const gs_camera* cam, int N, const float* means, const float* scales,
+                                         const float* quats, const float* opacity, float* mean2d, float* depth,
+                                         float* conic_opacity, int* radius, int* rect, unsigned* tiles_touched,
+                                         unsigned* d_num_pairs, void* stream) {
+    if (N < 0 || N > GS_NOALLOC_MAX_GAUSSIANS) return GS_ERR_INVALID_ARG;
+    if (!camera_ok(cam) || !d_num_pairs) return GS_ERR_INVALID_ARG;
+    if (N > 0) {
+        if (!means || !scales || !quats || !opacity || !mean2d || !depth || !conic_opacity || !radius || !rect ||
+            !tiles_touched)
+            return GS_ERR_INVALID_ARG;
+        if (!aligned(quats, 16) || !aligned(conic_opacity, 16) || !aligned(rect, 16) || !aligned(mean2d, 8))
+            return GS_ERR_INVALID_ARG;
+    }
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch_address(&scratch);
+    if (rc != GS_OK) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the header (status word and last-block ticket) must start at zero
+    if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GS_ERR_CUDA;
+    }
+    const int blocks = (N + kPreBlock - 1) / kPreBlock;
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(scratch);
+    unsigned long long* partials =
+        reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(scratch) + sizeof(WsHeader));
+    k_preprocess_fwd<<<blocks > 0 ? blocks : 1, kPreBlock, 0, st>>>(
+        *cam, N, tiles_x(*cam), tiles_y(*cam), means, scales, reinterpret_cast<const float4*>(quats), opacity,
+        reinterpret_cast<float2*>(mean2d), depth, reinterpret_cast<float4*>(conic_opacity), radius,
+        reinterpret_cast<int4*>(rect), tiles_touched, d_num_pairs, hdr, partials);
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+}

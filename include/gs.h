@@ -135,6 +135,36 @@ GS_API int gs_preprocess_fwd(const gs_camera* cam, int N, const float* means, co
                       unsigned* d_num_pairs, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * gs_preprocess_fwd_noalloc - gs_preprocess_fwd for callers that cannot
+ *   allocate device memory (no counterpart on the pages: it is a packaging
+ *   variant, not a step of the method).  Examples: a plug-in inside a host
+ *   application whose allocator owns all device memory, or a per-frame loop
+ *   where a cudaMalloc would synchronise the device.  Same arguments, outputs
+ *   and arithmetic as gs_preprocess_fwd, without `ws`: the scratch lives in a
+ *   fixed array inside the library (256 bytes + 8 bytes per 256 Gaussians,
+ *   about 512 KiB), held on every device that loads the library until the
+ *   process exits.
+ * Limits and behaviour:
+ *   - N > GS_NOALLOC_MAX_GAUSSIANS (or N < 0) returns GS_ERR_INVALID_ARG and
+ *     enqueues nothing.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (once per device); make that first call before any
+ *     stream capture.
+ *   - Calls allocate nothing (no cudaMalloc, cudaFree or allocating library
+ *     routine).  Each call clears the scratch header on `stream` first.
+ *   - Every call on a device shares the one array: calls that overlap on the
+ *     GPU (e.g. on two streams at once) race and give wrong pair counts.
+ *     Serialise them, or use gs_preprocess_fwd with one workspace each.
+ *   - A pair count that does not fit in 32 bits is reported only through
+ *     *d_num_pairs = 0xFFFFFFFF (there is no caller-visible status word).
+ */
+#define GS_NOALLOC_MAX_GAUSSIANS (1 << 24)
+GS_API int gs_preprocess_fwd_noalloc(const gs_camera* cam, int N, const float* means, const float* scales,
+                      const float* quats, const float* opacity, float* mean2d, float* depth,
+                      float* conic_opacity, int* radius, int* rect, unsigned* tiles_touched,
+                      unsigned* d_num_pairs, void* stream);
+
+/*
  * gs_bin_sort - tile binning and (tile, depth) sort ([TR] E.3; [CB] 1, 3).
  *   Produces, for every tile, the ids of the Gaussians whose rectangle
  *   contains it, in increasing (depth, id) order, concatenated in tile
