@@ -46,29 +46,110 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 __device__ __forceinline__ void raise_status(WsHeader* h, unsigned flag) { atomicOr(&h->status, flag); }
 
-// One (pixel, Gaussian) term of the compositing sum.  Every operation is an
-// explicit round-to-nearest intrinsic so that the forward and the backward
-// kernels, compiled separately, take bit-identical skip decisions and alphas.
-//   d = p - mean; power = -1/2 (a dx^2 + c dy^2) - b dx dy;
+// exp(x) in fp32 as a fixed sequence of IEEE operations, so that any IEEE
+// machine with a correctly rounded fused multiply-add reproduces every bit
+// (the library's expf does not promise that, and a one-ulp difference can
+// flip an alpha_min or T_min decision).  x is clamped to >= -87 (exp(-87) is
+// still a normal float); x log2(e) = n + f with n = rint(x log2(e)) taken
+// with the 1.5 * 2^23 shifter and |f| <= 1/2, f computed with log2(e) split
+// into a high and a low part (argument reduction after Cody and Waite); 2^f = exp(f ln 2) is the degree-7 Taylor polynomial
+// sum_k (ln 2)^k f^k / k! by Horner's rule with fused multiply-adds
+// (truncation below 6e-9 relative); n is added to the result's exponent bits.
+#define GS_EXP_LOG2E 0x1.715476p+0f
+#define GS_EXP_LOG2E_LO 0x1.4ae0c0p-26f
+#define GS_EXP_SHIFT 0x1.8p+23f
+#define GS_EXP_C7 0x1.ffcbfcp-17f
+#define GS_EXP_C6 0x1.430912p-13f
+#define GS_EXP_C5 0x1.5d87fep-10f
+#define GS_EXP_C4 0x1.3b2ab6p-7f
+#define GS_EXP_C3 0x1.c6b08ep-5f
+#define GS_EXP_C2 0x1.ebfbe0p-3f
+#define GS_EXP_C1 0x1.62e430p-1f
+
+__device__ __forceinline__ float2 exp_pair(float2 x) {
+    x = make_float2(fmaxf(x.x, -87.0f), fmaxf(x.y, -87.0f));
+    const float2 l2e = make_float2(GS_EXP_LOG2E, GS_EXP_LOG2E);
+    const float2 t = __ffma2_rn(x, l2e, make_float2(GS_EXP_SHIFT, GS_EXP_SHIFT));
+    const float2 n = __fadd2_rn(t, make_float2(-GS_EXP_SHIFT, -GS_EXP_SHIFT));
+    float2 f = __ffma2_rn(x, l2e, make_float2(-n.x, -n.y));
+    f = __ffma2_rn(x, make_float2(GS_EXP_LOG2E_LO, GS_EXP_LOG2E_LO), f);
+    float2 p = make_float2(GS_EXP_C7, GS_EXP_C7);
+    p = __ffma2_rn(p, f, make_float2(GS_EXP_C6, GS_EXP_C6));
+    p = __ffma2_rn(p, f, make_float2(GS_EXP_C5, GS_EXP_C5));
+    p = __ffma2_rn(p, f, make_float2(GS_EXP_C4, GS_EXP_C4));
+    p = __ffma2_rn(p, f, make_float2(GS_EXP_C3, GS_EXP_C3));
+    p = __ffma2_rn(p, f, make_float2(GS_EXP_C2, GS_EXP_C2));
+    p = __ffma2_rn(p, f, make_float2(GS_EXP_C1, GS_EXP_C1));
+    p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
+    const unsigned sb = __float_as_uint(GS_EXP_SHIFT);
+    const unsigned e0 = __float_as_uint(t.x) - sb, e1 = __float_as_uint(t.y) - sb;
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (e0 << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (e1 << 23)));
+}
+
+// One (pixel, Gaussian) term of the compositing sum, for two pixels of one
+// row (px.x, px.y share py), with packed fp32x2 operations:
+//   d = p - mean; power = -1/2 d^T A d = -1/2 (a dx^2 + 2 b dx dy + c dy^2);
 //   alpha = min(alpha_max, opacity exp(power)).
-// Returns false when the term is skipped (power > 0 or alpha < alpha_min).
-struct Term {
-    float dx, dy, G, at, alpha;
+// Every operation is an explicit round-to-nearest one in a fixed order (each
+// lane of a packed operation rounds like the scalar one), so the forward and
+// the backward kernels take bit-identical skip decisions and alphas, and an
+// IEEE fp32 implementation of the same steps reproduces them.
+// ok0 / ok1 are false when the term is skipped (power > 0 or alpha < alpha_min).
+struct TermPair {
+    float2 dx, G, at, alpha;
+    float dy;
+    bool ok0, ok1;
 };
 
-__device__ __forceinline__ bool eval_term(float px, float py, float2 xy, float4 co, float alpha_max,
-                                          float alpha_min, Term& e) {
-    e.dx = __fsub_rn(px, xy.x);
+__device__ __forceinline__ void eval_pair(float2 px, float py, float2 xy, float4 co, float alpha_max,
+                                          float alpha_min, TermPair& e) {
+    e.dx = __fadd2_rn(px, make_float2(-xy.x, -xy.x));
     e.dy = __fsub_rn(py, xy.y);
-    const float qa = __fmul_rn(__fmul_rn(co.x, e.dx), e.dx);
+    // q = a dx^2 + 2 b dx dy + c dy^2 with explicit fused multiply-adds: no
+    // product feeds an addition, so the compiler has no contraction left to
+    // choose (it does fuse packed multiplies into following packed adds).
     const float qc = __fmul_rn(__fmul_rn(co.z, e.dy), e.dy);
-    const float qb = __fmul_rn(__fmul_rn(co.y, e.dx), e.dy);
-    const float power = __fsub_rn(__fmul_rn(-0.5f, __fadd_rn(qa, qc)), qb);
-    if (power > 0.0f) return false;
-    e.G = expf(power);
-    e.at = __fmul_rn(co.w, e.G);
-    e.alpha = fminf(alpha_max, e.at);
-    return !(e.alpha < alpha_min);
+    const float2 adx = __fmul2_rn(make_float2(co.x, co.x), e.dx);
+    const float2 bdx2 = __fmul2_rn(make_float2(2.0f * co.y, 2.0f * co.y), e.dx);
+    float2 q = __ffma2_rn(adx, e.dx, make_float2(qc, qc));
+    q = __ffma2_rn(bdx2, make_float2(e.dy, e.dy), q);
+    const float2 power = __fmul2_rn(make_float2(-0.5f, -0.5f), q);
+    e.G = exp_pair(power);
+    e.at = __fmul2_rn(make_float2(co.w, co.w), e.G);
+    e.alpha = make_float2(fminf(alpha_max, e.at.x), fminf(alpha_max, e.at.y));
+    e.ok0 = !(power.x > 0.0f) && !(e.alpha.x < alpha_min);
+    e.ok1 = !(power.y > 0.0f) && !(e.alpha.y < alpha_min);
+}
+
+// Axis-aligned box (pixel coordinates: xmin, xmax, ymin, ymax) outside of
+// which a Gaussian cannot reach alpha >= alpha_min, so a warp whose pixels
+// all lie outside may skip it without changing any result.  The region is
+// the ellipse d^T A d <= 2 ln(opacity / alpha_min); its extents are
+// sqrt(k (A^-1)_xx) and sqrt(k (A^-1)_yy).  k is inflated to cover the fp32
+// rounding of `power` in eval_term, whose error grows with the conic's
+// condition number (bounded by (a + c)^2 / det), and of exp.  A non-finite
+// or undefined bound gives the infinite box (never skipped).
+__device__ __forceinline__ float4 contrib_box(float2 xy, float4 co, float alpha_min) {
+    const float inf = __int_as_float(0x7f800000);
+    const float4 all = make_float4(-inf, inf, -inf, inf);
+    if (!(alpha_min > 0.0f)) return all;
+    if (co.w < alpha_min) return make_float4(inf, -inf, inf, -inf);  // alpha <= opacity < alpha_min
+    const float det = co.x * co.z - co.y * co.y;
+    if (!(det > 0.0f)) return all;
+    const float tr = co.x + co.z;
+    const float k = 2.0f * logf(co.w / alpha_min);
+    const float ki = k * (1.001f + 1e-6f * (tr * tr / det)) + 1e-5f;
+    const float ex = sqrtf(ki * co.z / det) + 0.01f;
+    const float ey = sqrtf(ki * co.x / det) + 0.01f;
+    const float4 b = make_float4(xy.x - ex, xy.x + ex, xy.y - ey, xy.y + ey);
+    if (!(isfinite(b.x) && isfinite(b.y) && isfinite(b.z) && isfinite(b.w))) return all;
+    return b;
+}
+
+// True when the box misses the rectangle of pixel centres [x0, x1] x [y0, y1].
+__device__ __forceinline__ bool box_misses(float4 b, float x0, float x1, float y0, float y1) {
+    return b.y < x0 || b.x > x1 || b.w < y0 || b.z > y1;
 }
 
 }  // namespace gs

@@ -22,65 +22,124 @@
 namespace gs {
 namespace {
 
-constexpr int kBlock = kTilePixels;  // one thread per pixel of a 16x16 tile
+// One CTA per 16x16 tile with 128 threads: each thread owns two horizontally
+// adjacent pixels, evaluated together with packed fp32x2 arithmetic; warp w
+// owns the 16x4 strip of rows 4w..4w+3.  Gaussians are staged 128 at a time.
+// Before a warp walks a batch it builds a ballot mask of the staged
+// Gaussians whose contribution box (contrib_box) meets its strip, and walks
+// only those: a skipped Gaussian would have been rejected by the alpha_min
+// test at every pixel of the strip, so results are unchanged.
+constexpr int kThreads = 128;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 128;
+constexpr int kWords = kBatch / 32;
+static_assert(kThreads * 2 == kTilePixels, "two pixels per thread");
 
-__global__ void __launch_bounds__(kBlock)
+struct PixelPair {
+    int x0, y;
+    bool in0, in1;
+    float2 px;
+    float py;
+    float sx0, sx1, sy0, sy1;  // pixel-centre rectangle of this warp's strip
+};
+
+__device__ __forceinline__ PixelPair pixel_pair(const gs_camera& cam, int TX) {
+    PixelPair q;
+    const int tile = blockIdx.x;
+    const int tx0 = (tile % TX) * kTile, ty0 = (tile / TX) * kTile;
+    q.x0 = tx0 + 2 * (threadIdx.x & 7);
+    q.y = ty0 + (threadIdx.x >> 3);
+    q.in0 = q.x0 < cam.width && q.y < cam.height;
+    q.in1 = q.x0 + 1 < cam.width && q.y < cam.height;
+    q.px = make_float2((float)q.x0 + 0.5f, (float)q.x0 + 1.5f);
+    q.py = (float)q.y + 0.5f;
+    const int warp = threadIdx.x >> 5;
+    q.sx0 = (float)tx0 + 0.5f;
+    q.sx1 = (float)tx0 + 15.5f;
+    q.sy0 = (float)(ty0 + 4 * warp) + 0.5f;
+    q.sy1 = q.sy0 + 3.0f;
+    return q;
+}
+
+__global__ void __launch_bounds__(kThreads)
 k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
              const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
              const float* __restrict__ colors, float* __restrict__ image, float* __restrict__ final_T,
              unsigned* __restrict__ n_contrib) {
-    __shared__ float2 s_xy[kBlock];
-    __shared__ float4 s_co[kBlock];
-    __shared__ float4 s_col[kBlock];
-    const int tile = blockIdx.x;
-    const int x = (tile % TX) * kTile + (threadIdx.x & (kTile - 1));
-    const int y = (tile / TX) * kTile + (threadIdx.x / kTile);
-    const bool inside = x < cam.width && y < cam.height;
-    const float px = (float)x + 0.5f, py = (float)y + 0.5f;
-    const uint2 rg = ranges[tile];
+    __shared__ float2 s_xy[kBatch];
+    __shared__ float4 s_co[kBatch];
+    __shared__ float4 s_col[kBatch];
+    __shared__ float4 s_box[kBatch];
+    const PixelPair q = pixel_pair(cam, TX);
+    const int lane = threadIdx.x & 31;
+    const uint2 rg = ranges[blockIdx.x];
     const float amax = cam.alpha_max, amin = cam.alpha_min, tmin = cam.T_min;
 
-    float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
-    unsigned last = 0;
-    bool done = !inside;
-    for (unsigned b = rg.x; b < rg.y; b += kBlock) {
-        if (__syncthreads_count(done) == kBlock) break;
+    float2 T = make_float2(1.0f, 1.0f);
+    float2 C0 = make_float2(0.0f, 0.0f), C1 = C0, C2 = C0;
+    unsigned last0 = 0, last1 = 0;
+    bool done0 = !q.in0, done1 = !q.in1;
+    for (unsigned b = rg.x; b < rg.y; b += kBatch) {
+        if (__syncthreads_count(done0 && done1) == kThreads) break;
         const unsigned k = b + threadIdx.x;
         if (k < rg.y) {
             const unsigned j = ids[k];
-            s_xy[threadIdx.x] = mean2d[j];
-            s_co[threadIdx.x] = conic_opacity[j];
+            const float2 xy = mean2d[j];
+            const float4 co = conic_opacity[j];
+            s_xy[threadIdx.x] = xy;
+            s_co[threadIdx.x] = co;
             s_col[threadIdx.x] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+            s_box[threadIdx.x] = contrib_box(xy, co, amin);
         }
         __syncthreads();
-        const int n = min((unsigned)kBlock, rg.y - b);
-        if (!done) {
-            for (int jj = 0; jj < n; ++jj) {
-                Term e;
-                if (!eval_term(px, py, s_xy[jj], s_co[jj], amax, amin, e)) continue;
-                const float Tn = __fmul_rn(T, __fsub_rn(1.0f, e.alpha));
-                if (Tn < tmin) {
-                    done = true;
+        const int n = min((unsigned)kBatch, rg.y - b);
+        bool warp_done = __all_sync(0xffffffffu, done0 && done1);
+        for (int w = 0; w < kWords && !warp_done; ++w) {
+            const int jl = w * 32 + lane;
+            const bool keep = jl < n && !box_misses(s_box[jl], q.sx0, q.sx1, q.sy0, q.sy1);
+            unsigned m = __ballot_sync(0xffffffffu, keep);
+            while (m) {
+                const int jj = w * 32 + __ffs(m) - 1;
+                m &= m - 1;
+                TermPair e;
+                eval_pair(q.px, q.py, s_xy[jj], s_co[jj], amax, amin, e);
+                const float2 Tn = __fmul2_rn(T, __fadd2_rn(make_float2(1.0f, 1.0f),
+                                                           make_float2(-e.alpha.x, -e.alpha.y)));
+                const bool use0 = !done0 && e.ok0, use1 = !done1 && e.ok1;
+                const bool stop0 = use0 && Tn.x < tmin, stop1 = use1 && Tn.y < tmin;
+                const bool blend0 = use0 && !stop0, blend1 = use1 && !stop1;
+                done0 = done0 || stop0;
+                done1 = done1 || stop1;
+                const float2 wgt = make_float2(blend0 ? e.alpha.x * T.x : 0.0f, blend1 ? e.alpha.y * T.y : 0.0f);
+                const float4 c = s_col[jj];
+                C0 = __ffma2_rn(wgt, make_float2(c.x, c.x), C0);
+                C1 = __ffma2_rn(wgt, make_float2(c.y, c.y), C1);
+                C2 = __ffma2_rn(wgt, make_float2(c.z, c.z), C2);
+                const unsigned pos = b - rg.x + (unsigned)jj + 1u;
+                if (blend0) { T.x = Tn.x; last0 = pos; }
+                if (blend1) { T.y = Tn.y; last1 = pos; }
+                if (__all_sync(0xffffffffu, done0 && done1)) {
+                    warp_done = true;
                     break;
                 }
-                const float w = e.alpha * T;
-                const float4 c = s_col[jj];
-                C0 = fmaf(c.x, w, C0);
-                C1 = fmaf(c.y, w, C1);
-                C2 = fmaf(c.z, w, C2);
-                T = Tn;
-                last = b - rg.x + jj + 1;
             }
         }
     }
-    if (inside) {
-        const size_t pix = (size_t)y * cam.width + x;
-        const size_t plane = (size_t)cam.width * cam.height;
-        image[pix] = fmaf(T, cam.bg[0], C0);
-        image[plane + pix] = fmaf(T, cam.bg[1], C1);
-        image[2 * plane + pix] = fmaf(T, cam.bg[2], C2);
-        final_T[pix] = T;
-        n_contrib[pix] = last;
+    const size_t plane = (size_t)cam.width * cam.height;
+    const size_t pix = (size_t)q.y * cam.width + q.x0;
+    if (q.in0) {
+        image[pix] = fmaf(T.x, cam.bg[0], C0.x);
+        image[plane + pix] = fmaf(T.x, cam.bg[1], C1.x);
+        image[2 * plane + pix] = fmaf(T.x, cam.bg[2], C2.x);
+        final_T[pix] = T.x;
+        n_contrib[pix] = last0;
+    }
+    if (q.in1) {
+        image[pix + 1] = fmaf(T.y, cam.bg[0], C0.y);
+        image[plane + pix + 1] = fmaf(T.y, cam.bg[1], C1.y);
+        image[2 * plane + pix + 1] = fmaf(T.y, cam.bg[2], C2.y);
+        final_T[pix + 1] = T.y;
+        n_contrib[pix + 1] = last1;
     }
 }
 
@@ -114,110 +173,143 @@ __device__ __forceinline__ float reduce8(float v[8], int lane) {
 
 constexpr int kGradStride = 9;  // floats per staged Gaussian in shared memory
 
-__global__ void __launch_bounds__(kBlock)
+__global__ void __launch_bounds__(kThreads)
 k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
              const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
              const float* __restrict__ colors, const float* __restrict__ final_T,
              const unsigned* __restrict__ n_contrib, const float* __restrict__ dL_dimage,
              float2* __restrict__ dL_dmean2d, float4* __restrict__ dL_dconic_opacity,
              float* __restrict__ dL_dcolor) {
-    __shared__ unsigned s_id[kBlock];
-    __shared__ float2 s_xy[kBlock];
-    __shared__ float4 s_co[kBlock];
-    __shared__ float4 s_col[kBlock];
-    __shared__ float s_grad[kBlock * kGradStride];
-    __shared__ unsigned s_max[kBlock / 32];
+    __shared__ unsigned s_id[kBatch];
+    __shared__ float2 s_xy[kBatch];
+    __shared__ float4 s_co[kBatch];
+    __shared__ float4 s_col[kBatch];
+    __shared__ float4 s_box[kBatch];
+    __shared__ float s_grad[kBatch * kGradStride];
+    __shared__ unsigned s_max[kWarps];
 
-    const int tile = blockIdx.x;
+    const PixelPair q = pixel_pair(cam, TX);
     const int lane = threadIdx.x & 31;
-    const int x = (tile % TX) * kTile + (threadIdx.x & (kTile - 1));
-    const int y = (tile / TX) * kTile + (threadIdx.x / kTile);
-    const bool inside = x < cam.width && y < cam.height;
-    const float px = (float)x + 0.5f, py = (float)y + 0.5f;
-    const uint2 rg = ranges[tile];
+    const uint2 rg = ranges[blockIdx.x];
     const float amax = cam.alpha_max, amin = cam.alpha_min;
-
-    const size_t pix = (size_t)y * cam.width + x;
     const size_t plane = (size_t)cam.width * cam.height;
-    float T = 0.0f, g0 = 0.0f, g1 = 0.0f, g2 = 0.0f;
-    unsigned last = 0;
-    if (inside) {
-        T = final_T[pix];
-        last = n_contrib[pix];
-        g0 = dL_dimage[pix];
-        g1 = dL_dimage[plane + pix];
-        g2 = dL_dimage[2 * plane + pix];
-    }
-    float S0 = cam.bg[0], S1 = cam.bg[1], S2 = cam.bg[2];
+    const size_t pix = (size_t)q.y * cam.width + q.x0;
 
-    // furthest list position any pixel of the tile blended
-    const unsigned wmax = __reduce_max_sync(0xffffffffu, last);
-    if (lane == 0) s_max[threadIdx.x >> 5] = wmax;
-    for (int i = threadIdx.x; i < kBlock * kGradStride; i += kBlock) s_grad[i] = 0.0f;
+    float2 T = make_float2(0.0f, 0.0f), g0 = T, g1 = T, g2 = T;
+    unsigned last0 = 0, last1 = 0;
+    if (q.in0) {
+        T.x = final_T[pix];
+        last0 = n_contrib[pix];
+        g0.x = dL_dimage[pix];
+        g1.x = dL_dimage[plane + pix];
+        g2.x = dL_dimage[2 * plane + pix];
+    }
+    if (q.in1) {
+        T.y = final_T[pix + 1];
+        last1 = n_contrib[pix + 1];
+        g0.y = dL_dimage[pix + 1];
+        g1.y = dL_dimage[plane + pix + 1];
+        g2.y = dL_dimage[2 * plane + pix + 1];
+    }
+    float2 S0 = make_float2(cam.bg[0], cam.bg[0]), S1 = make_float2(cam.bg[1], cam.bg[1]);
+    float2 S2 = make_float2(cam.bg[2], cam.bg[2]);
+
+    // furthest list position any pixel of the warp / of the tile blended
+    const unsigned wlast = __reduce_max_sync(0xffffffffu, max(last0, last1));
+    if (lane == 0) s_max[threadIdx.x >> 5] = wlast;
+    for (int i = threadIdx.x; i < kBatch * kGradStride; i += kThreads) s_grad[i] = 0.0f;
     __syncthreads();
     unsigned max_last = 0;
 #pragma unroll
-    for (int w = 0; w < kBlock / 32; ++w) max_last = max(max_last, s_max[w]);
+    for (int w = 0; w < kWarps; ++w) max_last = max(max_last, s_max[w]);
     max_last = min(max_last, rg.y - rg.x);  // stay inside the tile's list
 
-    for (int top = (int)max_last; top > 0; top -= kBlock) {
+    for (int top = (int)max_last; top > 0; top -= kBatch) {
+        // stage positions top-1, top-2, ... so that staged order is back to front
         const int pos = top - 1 - (int)threadIdx.x;
         if (pos >= 0) {
             const unsigned j = ids[rg.x + pos];
+            const float2 xy = mean2d[j];
+            const float4 co = conic_opacity[j];
             s_id[threadIdx.x] = j;
-            s_xy[threadIdx.x] = mean2d[j];
-            s_co[threadIdx.x] = conic_opacity[j];
+            s_xy[threadIdx.x] = xy;
+            s_co[threadIdx.x] = co;
             s_col[threadIdx.x] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+            s_box[threadIdx.x] = contrib_box(xy, co, amin);
         }
         __syncthreads();
-        const int n = min(kBlock, top);
-        for (int jj = 0; jj < n; ++jj) {
-            const int p = top - 1 - jj;
-            Term e;
-            const float4 co = s_co[jj];
-            bool contrib = p < (int)last;
-            if (contrib) contrib = eval_term(px, py, s_xy[jj], co, amax, amin, e);
-            if (!__any_sync(0xffffffffu, contrib)) continue;
-            float v[8];
-            float vcol2 = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-            if (contrib) {
-                T = __fdividef(T, 1.0f - e.alpha);
+        const int n = min(kBatch, top);
+        for (int w = 0; w < kWords; ++w) {
+            const int jl = w * 32 + lane;
+            const bool keep = jl < n && top - 1 - jl < (int)wlast &&
+                              !box_misses(s_box[jl], q.sx0, q.sx1, q.sy0, q.sy1);
+            unsigned m = __ballot_sync(0xffffffffu, keep);
+            while (m) {
+                const int jj = w * 32 + __ffs(m) - 1;
+                m &= m - 1;
+                const int p = top - 1 - jj;
+                const float4 co = s_co[jj];
+                TermPair e;
+                eval_pair(q.px, q.py, s_xy[jj], co, amax, amin, e);
+                const bool c0 = p < (int)last0 && e.ok0;
+                const bool c1 = p < (int)last1 && e.ok1;
+                if (!__any_sync(0xffffffffu, c0 || c1)) continue;
+                // terms the forward did not blend contribute nothing
+                const float2 G = make_float2(c0 ? e.G.x : 0.0f, c1 ? e.G.y : 0.0f);
+                const float2 al = make_float2(c0 ? e.alpha.x : 0.0f, c1 ? e.alpha.y : 0.0f);
+                if (c0) T.x = __fdividef(T.x, 1.0f - al.x);
+                if (c1) T.y = __fdividef(T.y, 1.0f - al.y);
                 const float4 c = s_col[jj];
-                const float wgt = e.alpha * T;
-                v[5] = wgt * g0;  // dL/dcolor
-                v[6] = wgt * g1;
-                vcol2 = wgt * g2;
-                const float dLda = ((c.x - S0) * g0 + (c.y - S1) * g1 + (c.z - S2) * g2) * T;
-                const float om = 1.0f - e.alpha;
-                S0 = e.alpha * c.x + om * S0;
-                S1 = e.alpha * c.y + om * S1;
-                S2 = e.alpha * c.z + om * S2;
-                // exact derivative of min(alpha_max, sigma G): zero while capped
-                const bool free = e.at <= amax;
-                const float dLdsig = free ? e.G * dLda : 0.0f;
-                const float h = free ? e.G * co.w * dLda : 0.0f;  // dL/dpower
-                const float dx = e.dx, dy = e.dy;
-                v[0] = (co.x * dx + co.y * dy) * h;  // dL/du
-                v[1] = (co.y * dx + co.z * dy) * h;  // dL/dv
-                v[2] = -0.5f * dx * dx * h;          // dL/da
-                v[3] = -dx * dy * h;                 // dL/db
-                v[4] = -0.5f * dy * dy * h;          // dL/dc
-                v[7] = dLdsig;                       // dL/dopacity
-            }
-            const float r8 = reduce8(v, lane);
-            float r9 = vcol2;
+                const float2 wgt = __fmul2_rn(al, T);
+                const float2 d0 = __fadd2_rn(make_float2(c.x, c.x), make_float2(-S0.x, -S0.y));
+                const float2 d1 = __fadd2_rn(make_float2(c.y, c.y), make_float2(-S1.x, -S1.y));
+                const float2 d2 = __fadd2_rn(make_float2(c.z, c.z), make_float2(-S2.x, -S2.y));
+                float2 dLda = __fmul2_rn(d0, g0);
+                dLda = __ffma2_rn(d1, g1, dLda);
+                dLda = __ffma2_rn(d2, g2, dLda);
+                dLda = __fmul2_rn(dLda, T);
+                // colour behind the next term towards the front: S <- alpha c + (1 - alpha) S
+                S0 = __ffma2_rn(al, d0, S0);
+                S1 = __ffma2_rn(al, d1, S1);
+                S2 = __ffma2_rn(al, d2, S2);
+                // exact derivative of min(alpha_max, opacity G): zero while capped
+                const float2 Gf = make_float2(e.at.x <= amax ? G.x : 0.0f, e.at.y <= amax ? G.y : 0.0f);
+                const float2 dsig = __fmul2_rn(Gf, dLda);                       // dL/dopacity
+                const float2 h = __fmul2_rn(dsig, make_float2(co.w, co.w));     // dL/dpower
+                const float2 hdx = __fmul2_rn(h, e.dx);
+                const float hdy_s = e.dy;
+                const float2 hdy = __fmul2_rn(h, make_float2(hdy_s, hdy_s));
+                float v[8];
+                float2 t2;
+                t2 = __ffma2_rn(make_float2(co.x, co.x), hdx, __fmul2_rn(make_float2(co.y, co.y), hdy));
+                v[0] = t2.x + t2.y;  // dL/du
+                t2 = __ffma2_rn(make_float2(co.y, co.y), hdx, __fmul2_rn(make_float2(co.z, co.z), hdy));
+                v[1] = t2.x + t2.y;  // dL/dv
+                t2 = __fmul2_rn(hdx, e.dx);
+                v[2] = -0.5f * (t2.x + t2.y);  // dL/da
+                t2 = __fmul2_rn(hdx, make_float2(e.dy, e.dy));
+                v[3] = -(t2.x + t2.y);  // dL/db
+                t2 = __fmul2_rn(hdy, make_float2(e.dy, e.dy));
+                v[4] = -0.5f * (t2.x + t2.y);  // dL/dc
+                t2 = __fmul2_rn(wgt, g0);
+                v[5] = t2.x + t2.y;  // dL/dcolor r
+                t2 = __fmul2_rn(wgt, g1);
+                v[6] = t2.x + t2.y;  // dL/dcolor g
+                v[7] = dsig.x + dsig.y;  // dL/dopacity
+                t2 = __fmul2_rn(wgt, g2);
+                float r9 = t2.x + t2.y;  // dL/dcolor b
+                const float r8 = reduce8(v, lane);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
-            // lanes 4i hold value i (i < 8); lane 1 holds the ninth
-            float* sg = s_grad + jj * kGradStride;
-            if ((lane & 3) == 0) atomicAdd(sg + (lane >> 2), r8);
-            if (lane == 1) atomicAdd(sg + 8, r9);
+                for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
+                // lanes 4i hold value i (i < 8); lane 1 holds the ninth
+                float* sg = s_grad + jj * kGradStride;
+                if ((lane & 3) == 0) atomicAdd(sg + (lane >> 2), r8);
+                if (lane == 1) atomicAdd(sg + 8, r9);
+            }
         }
         __syncthreads();
         // flush this batch: one set of global atomics per (tile, Gaussian)
-        if (threadIdx.x < n) {
+        if ((int)threadIdx.x < n) {
             float* sg = s_grad + threadIdx.x * kGradStride;
             const float a0 = sg[0], a1 = sg[1], a2 = sg[2], a3 = sg[3], a4 = sg[4];
             const float a5 = sg[5], a6 = sg[6], a7 = sg[7], a8 = sg[8];
@@ -230,9 +322,9 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 atomicAdd(&dL_dcolor[3 * j + 0], a5);
                 atomicAdd(&dL_dcolor[3 * j + 1], a6);
                 atomicAdd(&dL_dcolor[3 * j + 2], a8);
-            }
 #pragma unroll
-            for (int i = 0; i < kGradStride; ++i) sg[i] = 0.0f;
+                for (int i = 0; i < kGradStride; ++i) sg[i] = 0.0f;
+            }
         }
         __syncthreads();
     }
@@ -258,7 +350,7 @@ extern "C" int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const
     if (!aligned(ranges, 8) || (conic_opacity && !aligned(conic_opacity, 16)) || (mean2d && !aligned(mean2d, 8)))
         return GS_ERR_INVALID_ARG;
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
-    k_render_fwd<<<T, kBlock, 0, (cudaStream_t)stream>>>(
+    k_render_fwd<<<T, kThreads, 0, (cudaStream_t)stream>>>(
         *cam, TX, reinterpret_cast<const uint2*>(ranges), ids, reinterpret_cast<const float2*>(mean2d),
         reinterpret_cast<const float4*>(conic_opacity), colors, image, final_T, n_contrib);
     GS_LAUNCH_CHECK();
@@ -284,7 +376,7 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
         GS_LAUNCH_CHECK();
     }
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
-    k_render_bwd<<<T, kBlock, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
+    k_render_bwd<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
                                        reinterpret_cast<const float2*>(mean2d),
                                        reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
                                        dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),

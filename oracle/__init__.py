@@ -78,10 +78,20 @@ def lib():
             getattr(L, f"oracle_render_bwd_{suf}").restype = None
             getattr(L, f"oracle_preprocess_bwd_{suf}").argtypes = [cam, I] + [P] * 12
             getattr(L, f"oracle_preprocess_bwd_{suf}").restype = None
+        L.oracle_exp_f32.argtypes = [P, P, ctypes.c_longlong]
+        L.oracle_exp_f32.restype = None
         L.oracle_num_threads.restype = I
         L.oracle_set_threads.argtypes = [I]
         _lib = L
     return _lib
+
+
+def exp_f32(x) -> np.ndarray:
+    """The fp32 mirror's exp (the one its compositing uses)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    y = np.empty_like(x)
+    lib().oracle_exp_f32(_p(x), _p(y), x.size)
+    return y
 
 
 def num_threads() -> int:

@@ -285,6 +285,42 @@ long long tile_list(const oracle_camera* cam, int N, const Real* depth, const in
     return (long long)v.size();
 }
 
+// exp for the fp32 mirror: the float result must be the one the kernels
+// compute, because a one-ulp difference in exp can flip an alpha_min or T_min
+// decision.  A fixed sequence of IEEE operations that any machine with a
+// correctly rounded fma reproduces: clamp x to >= -87; n = rint(x log2 e)
+// through the 1.5 * 2^23 shifter; f = x log2 e - n with log2 e split into a
+// high and a low part (two fused multiply-adds);
+// 2^f = sum_{k<=7} (ln 2)^k f^k / k! (Taylor series of exp(f ln 2), Horner
+// with fused multiply-adds); scale by 2^n through the exponent bits.
+// Argument reduction after Cody and Waite.  Pinned against float64 exp.
+inline float exp_mirror(float x) {
+    x = std::fmax(x, -87.0f);
+    const float t = std::fma(x, 0x1.715476p+0f, 0x1.8p+23f);
+    const float n = t - 0x1.8p+23f;
+    float f = std::fma(x, 0x1.715476p+0f, -n);
+    f = std::fma(x, 0x1.4ae0c0p-26f, f);
+    float p = 0x1.ffcbfcp-17f;
+    p = std::fma(p, f, 0x1.430912p-13f);
+    p = std::fma(p, f, 0x1.5d87fep-10f);
+    p = std::fma(p, f, 0x1.3b2ab6p-7f);
+    p = std::fma(p, f, 0x1.c6b08ep-5f);
+    p = std::fma(p, f, 0x1.ebfbe0p-3f);
+    p = std::fma(p, f, 0x1.62e430p-1f);
+    p = std::fma(p, f, 1.0f);
+    uint32_t tb, sb, pb;
+    const float shift = 0x1.8p+23f;
+    std::memcpy(&tb, &t, 4);
+    std::memcpy(&sb, &shift, 4);
+    std::memcpy(&pb, &p, 4);
+    pb += (tb - sb) << 23;
+    float r;
+    std::memcpy(&r, &pb, 4);
+    return r;
+}
+inline float oexp(float x) { return exp_mirror(x); }
+inline double oexp(double x) { return std::exp(x); }
+
 // Evaluation of one (pixel, Gaussian) term of the compositing sum.
 template <typename Real>
 struct Term {
@@ -297,11 +333,16 @@ inline Term<Real> eval_term(const oracle_camera& cam, Real px, Real py, const Re
     Term<Real> e;
     e.dx = px - xy[0];
     e.dy = py - xy[1];
-    const Real power = Real(-0.5) * (co[0] * e.dx * e.dx + co[2] * e.dy * e.dy) - co[1] * e.dx * e.dy;
+    // power = -1/2 d^T A d, with d^T A d = a dx^2 + 2 b dx dy + c dy^2 taken as
+    // fma(2 b dx, dy, fma(a dx, dx, c dy dy)): in fp32 this fixes every
+    // rounding, so the alpha_min / T_min decisions match the kernels'.
+    const Real qc = (co[2] * e.dy) * e.dy;
+    const Real q = std::fma(Real(2) * co[1] * e.dx, e.dy, std::fma(co[0] * e.dx, e.dx, qc));
+    const Real power = Real(-0.5) * q;
     e.used = false;
     e.G = e.at = e.alpha = Real(0);
     if (power > Real(0)) return e;  // only for a non positive-definite conic
-    e.G = std::exp(power);
+    e.G = oexp(power);
     e.at = co[3] * e.G;
     e.alpha = std::min(Real(cam.alpha_max), e.at);
     if (e.alpha < Real(cam.alpha_min)) return e;  // reading: alpha_min = 1/255
@@ -596,6 +637,10 @@ void preprocess_bwd(const oracle_camera* cam, int N, const Real* means, const Re
 }  // namespace
 
 extern "C" {
+
+void oracle_exp_f32(const float* x, float* y, long long n) {
+    for (long long i = 0; i < n; ++i) y[i] = exp_mirror(x[i]);
+}
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP

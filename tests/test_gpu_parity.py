@@ -62,6 +62,12 @@ def _check_render_fwd(cam, sc, g, tiles=None):
     match = (g["n_contrib"][mask] == o["n_contrib"][mask]).mean()
     assert match >= N_CONTRIB_MATCH, f"n_contrib match {match}"
     assert np.abs(g["final_T"] - o["final_T"])[mask].max() <= IMAGE_ATOL
+    # Stronger than the bar: alpha, the skip and stop decisions and T are
+    # computed by the same fixed IEEE steps on both sides (the quadratic form
+    # with explicit fused multiply-adds and the shared exp sequence), so the
+    # contributor counts and the final transmittance agree bit for bit.
+    np.testing.assert_array_equal(g["n_contrib"][mask], o["n_contrib"][mask])
+    np.testing.assert_array_equal(g["final_T"][mask].view(np.uint32), o["final_T"][mask].view(np.uint32))
     return o
 
 

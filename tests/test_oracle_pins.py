@@ -477,3 +477,17 @@ def test_backward_is_deterministic_across_thread_counts():
         oracle.set_threads(n0)
     for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
         np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_mirror_exp_error_bound():
+    """The fp32 mirror's exp (a fixed IEEE sequence that the kernels repeat
+    bit for bit) is within 2 ulp of exp over the range compositing uses."""
+    x = np.concatenate([np.linspace(-87.0, 0.0, 2_000_001, dtype=np.float32),
+                        np.float32(-np.logspace(-8, 1.9, 200_001)),
+                        np.array([0.0, -0.0, -1e-30, -87.0, -100.0, -np.inf], np.float32)])
+    y = oracle.exp_f32(x)
+    ref = np.exp(np.maximum(x.astype(np.float64), -87.0))
+    ulp = np.spacing(ref.astype(np.float32)).astype(np.float64)
+    err = np.abs(y.astype(np.float64) - ref) / ulp
+    assert err.max() <= 2.0, err.max()
+    assert oracle.exp_f32(np.zeros(1))[0] == 1.0
