@@ -4,9 +4,10 @@
 the 1M-Gaussian 1920x1080 synthetic scene (16x16 tiles), fp32.
 
 Prints one JSON line.  ``value`` is Gaussian-pixel evaluations per second for
-the whole job (all ranks), where a frame's evaluations are the (pixel,
-Gaussian) terms inside each pixel's contributor prefix, counted once for the
-forward and once for the backward: 2 * sum(n_contrib).
+the whole job (all ranks).  A frame's evaluations are, per pixel, the list
+entries the forward evaluated before the pixel stopped plus the entries of
+its contributor prefix that the backward walks: sum(n_evaluated) +
+sum(n_contrib), counted by the library's gs_render_stats.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4]
   python bench.py --impl reference ...   # the CPU oracle on the host cores
@@ -33,11 +34,16 @@ if ROOT not in sys.path:
 METRIC = ("rasterizer fwd+bwd ms/frame and Gaussian·pixel evals/s; bwd HBM GB/s vs B200 peak")
 UNIT = "Gaussian·pixel evals/s"
 
-# Algorithmic FP32 operations per evaluated term (each add, mul, min, div or
+# Algorithmic FP32 operations per blended term (each add, mul, min, div or
 # exp counts one): forward = 15 to evaluate alpha + 9 to blend; backward = 15
-# to re-evaluate alpha + 45 for the gradient formulas.
+# to re-evaluate alpha + 45 for the gradient formulas.  Only blended terms
+# count: any other term provably contributes nothing and may be skipped.
 OPS_FWD_EVAL = 24
 OPS_BWD_EVAL = 60
+# DRAM bytes per launch from the committed ncu capture of k_render_bwd
+# (dram__bytes_read.sum + dram__bytes_write.sum) and the SHA-1 of the render
+# sources it was taken on; reported only while the sources are unchanged.
+RECORDED_TRAFFIC = {"k_render_bwd": dict(bytes=None, sources_sha1=None)}
 # Algorithmic bytes: per (tile, Gaussian) pair visited, id + mean2d +
 # conic/opacity + colour = 40 B read; the backward adds 36 B of gradient
 # atomics per pair; per pixel the forward writes 20 B (image, T, n_contrib)
@@ -106,6 +112,15 @@ class ClockSampler:
         return dict(sm_mhz=statistics.median(sm), sm_max_mhz=mx, reasons=sorted(reasons), samples=len(sm))
 
 
+def _render_sources_sha1() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for name in ("render.cu", "gs_internal.cuh"):
+        with open(os.path.join(ROOT, "differentiable_gaussian_splatting_preprocess_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -135,7 +150,7 @@ def cpu_oracle_sample(sc, tile_stride: int, max_seconds: float = 25.0):
     oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, pre["radius"], g["dL_dmean2d"],
                           g["dL_dconic_opacity"], g["dL_dcolor"], "f64")
     dt = time.perf_counter() - t0
-    evals = 2 * int(r["n_contrib"].astype(np.int64).sum())
+    evals = int(r["n_eval"].astype(np.int64).sum()) + int(r["n_contrib"].astype(np.int64).sum())
     return dict(value=evals / dt, unit=UNIT, cores=oracle.num_threads(), kind="oracle",
                 sample=(f"full preprocess + binning of the {sc.name} scene, compositing fwd (fp32) + bwd "
                         f"(fp64) on every {tile_stride}th tile ({tiles.size} of {cam.num_tiles}), "
@@ -231,8 +246,14 @@ def run_ours(args):
     st = rz.status()
     if st != 0:
         raise RuntimeError(f"device status {st}: {B.status_string(st)}")
-    n_contrib = rz._bufs["n_contrib"].view(torch.int32).to(torch.int64).sum().item()
-    evals_per_frame = 2 * int(n_contrib)
+    n_contrib = int(rz._bufs["n_contrib"].view(torch.int32).to(torch.int64).sum().item())
+    n_eval_t = torch.empty((cam.height, cam.width), dtype=torch.uint32, device=dev)
+    n_blend_t = torch.empty_like(n_eval_t)
+    pre0 = rz._bufs
+    B.gs_render_stats(cam, pre0["ranges"], pre0["ids"], pre0["mean2d"], pre0["conic_opacity"], n_eval_t, n_blend_t)
+    n_evaluated = int(n_eval_t.view(torch.int32).to(torch.int64).sum().item())
+    n_blended = int(n_blend_t.view(torch.int32).to(torch.int64).sum().item())
+    evals_per_frame = n_evaluated + n_contrib
 
     sampler = ClockSampler(local)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
@@ -275,16 +296,18 @@ def run_ours(args):
     peaks = _peaks()
     mean = {s: statistics.mean(v) for s, v in stage_ms.items()}
     dominant = max(mean, key=mean.get)
-    bwd_ops = (evals_per_frame // 2) * OPS_BWD_EVAL
-    fwd_ops = (evals_per_frame // 2) * OPS_FWD_EVAL
+    bwd_ops = n_blended * OPS_BWD_EVAL
+    fwd_ops = n_blended * OPS_FWD_EVAL
     alu_peak = SMS * FP32_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12  # T lane-ops/s
     rb_ach = bwd_ops / (mean["render_bwd"] / 1e3) / 1e12
+    rec = RECORDED_TRAFFIC["k_render_bwd"]
+    traffic = rec["bytes"] if rec["sources_sha1"] == _render_sources_sha1() else None
     roofline = dict(kernel="k_render_bwd", bound="alu", achieved=rb_ach, peak=alu_peak, unit="Tops/s",
-                    frac=rb_ach / alu_peak, traffic=None,
-                    ops_per_launch=bwd_ops, peak_src=f"148 SMs x 128 FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz")
+                    frac=rb_ach / alu_peak, traffic=traffic, ops_per_launch=bwd_ops,
+                    ops_basis=f"{OPS_BWD_EVAL} FP32 ops x {n_blended} blended terms",
+                    peak_src=f"148 SMs x 128 FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz (sm_max_mhz)")
     # HBM view of render fwd + bwd, as asked
     pix = cam.width * cam.height
-    pairs = evals_per_frame // 2  # visited pairs are bounded below by the contributor prefixes
     fwd_bytes = P * BYTES_PAIR_READ + pix * BYTES_PIXEL
     bwd_bytes = P * (BYTES_PAIR_READ + BYTES_PAIR_ATOMIC) + pix * BYTES_PIXEL
     rfb_s = (mean["render_fwd"] + mean["render_bwd"]) / 1e3
@@ -329,9 +352,16 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_oracle_sample(sc, tile_stride=16 if args.config >= 4 else 1)
-        for k in ("seconds", "evals"):
-            cpu.pop(k)
+        # repeat the bounded sample until about 10 s of host work has been timed
+        stride = 4 if args.config >= 4 else 1
+        tot_s, tot_e, reps = 0.0, 0, 0
+        while tot_s < 10.0 and reps < 50:
+            c = cpu_oracle_sample(sc, tile_stride=stride)
+            tot_s += c["seconds"]
+            tot_e += c["evals"]
+            reps += 1
+        cpu = dict(value=tot_e / tot_s, unit=UNIT, cores=c["cores"], kind="oracle",
+                   sample=f"{reps} x ({c['sample']}); {tot_s:.1f} s in total")
 
     if rank == 0:
         line = dict(
@@ -339,7 +369,9 @@ def run_ours(args):
             ms_per_step=total_ms / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,
             dtype="f32", data="synthetic",
             config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam.width}x{cam.height}, 16x16 tiles, fp32",
-                        num_pairs=P, evals_per_frame=evals_per_frame, l2="flushed between steps (256 MiB write)",
+                        num_pairs=P, evals_per_frame=evals_per_frame, evaluated_fwd=n_evaluated,
+                        contributor_prefix_bwd=n_contrib, blended=n_blended,
+                        l2="flushed between steps (256 MiB write)",
                         parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
             fwd_ms_per_frame=mean["preprocess_fwd"] + mean["bin_sort"] + mean["render_fwd"],
             bwd_ms_per_frame=mean["render_bwd"] + mean["preprocess_bwd"],

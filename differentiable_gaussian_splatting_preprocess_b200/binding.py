@@ -31,7 +31,7 @@ TILE = 16
 # Every symbol include/gs.h declares.
 EXPORTED = ("gs_version", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
             "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd",
-            "gs_preprocess_fwd_noalloc")
+            "gs_preprocess_fwd_noalloc", "gs_render_stats")
 
 
 class GsCamera(ctypes.Structure):
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.gs_bin_sort.argtypes = [cam, I, P, P, P, P, U, P, P, P, P, S, P]
         L.gs_render_fwd.restype = I
         L.gs_render_fwd.argtypes = [cam] + [P] * 8 + [P]
+        L.gs_render_stats.restype = I
+        L.gs_render_stats.argtypes = [cam] + [P] * 6 + [P]
         L.gs_render_bwd.restype = I
         L.gs_render_bwd.argtypes = [cam, I] + [P] * 11 + [P]
         L.gs_preprocess_bwd.restype = I
@@ -218,6 +220,21 @@ def gs_render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_
     _ok("gs_render_fwd", lib().gs_render_fwd(
         ctypes.byref(c), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(colors), _ptr(image),
         _ptr(final_T), _ptr(n_contrib), _stream(stream)))
+
+
+def gs_render_stats(cam, ranges, ids, mean2d, conic_opacity, n_evaluated, n_blended, stream=None) -> None:
+    N = mean2d.shape[0]
+    H, W = cam.height, cam.width
+    _check(ranges, "ranges", torch.uint32, (num_tiles(cam), 2))
+    _check(ids, "ids", torch.uint32)
+    _check(mean2d, "mean2d", torch.float32, (N, 2))
+    _check(conic_opacity, "conic_opacity", torch.float32, (N, 4))
+    _check(n_evaluated, "n_evaluated", torch.uint32, (H, W))
+    _check(n_blended, "n_blended", torch.uint32, (H, W))
+    c = camera_struct(cam)
+    _ok("gs_render_stats", lib().gs_render_stats(
+        ctypes.byref(c), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(n_evaluated),
+        _ptr(n_blended), _stream(stream)))
 
 
 def gs_render_bwd(cam, ranges, ids, mean2d, conic_opacity, colors, final_T, n_contrib, dL_dimage, dL_dmean2d,

@@ -110,40 +110,93 @@ __global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const 
     }
 }
 
+// Radix passes.  A pass over n keys runs on G CTAs, each owning one
+// contiguous chunk of the input (a multiple of its tile of ITEMS x 256
+// keys), so that equal digits keep their input order: chunk, then tile,
+// then item slot j, then warp, then lane.  MAXB is the widest digit the
+// kernel instance handles; `bits` <= MAXB is the width of this pass.
+template <int MAXB>
+struct RadixCfg {
+    static constexpr int kRadix = 1 << MAXB;
+    static constexpr int kItems = MAXB >= 8 ? 4 : 8;
+    static constexpr int kTileKeys = kItems * kSortBlock;
+    static constexpr int kWarps = kSortBlock / 32;
+    static constexpr int kSlots = kItems * kWarps;  // (item, warp) groups per tile, in input order
+    // scatter shared memory: 16-bit per-(slot, digit) counts and tile-local
+    // offsets, 32-bit per-digit running bases / tile starts / tile bases,
+    // and the tile's keys and values regrouped by digit.
+    static constexpr size_t kScatterSmem = (size_t)2 * kSlots * kRadix * sizeof(unsigned short) +
+                                           (size_t)4 * kRadix * sizeof(unsigned) +
+                                           (size_t)2 * kTileKeys * sizeof(unsigned);
+};
+
+template <int MAXB>
 __device__ __forceinline__ void chunk_of(unsigned n, unsigned& lo, unsigned& hi) {
+    constexpr unsigned tile = RadixCfg<MAXB>::kTileKeys;
     const unsigned G = gridDim.x;
     unsigned chunk = (n + G - 1) / G;
-    chunk = (chunk + 31u) & ~31u;
-    lo = min(n, blockIdx.x * chunk);
+    chunk = (chunk + tile - 1) / tile * tile;
+    const unsigned long long l = (unsigned long long)blockIdx.x * chunk;
+    lo = l < n ? (unsigned)l : n;
     hi = min(n, lo + chunk);
 }
 
-// Per-CTA digit histogram of its contiguous chunk, stored digit-major:
-// hist[d * G + cta]; digit totals accumulate into totals[d].
+constexpr unsigned kNoDigit = 0xFFFFFFFFu;
+
+// Lanes of the warp holding the same digit as this lane, from one ballot per
+// digit bit (a warp-level multi-split); lanes without a key form their own
+// group.  Cheaper than __match_any_sync, whose throughput limited the passes.
+template <int MAXB>
+__device__ __forceinline__ unsigned digit_peers(unsigned d, int bits) {
+    const bool valid = d != kNoDigit;
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    unsigned m = valid ? vmask : ~vmask;
+#pragma unroll
+    for (int b = 0; b < MAXB; ++b) {
+        if (b < bits) {
+            const bool bit = (d >> b) & 1u;
+            const unsigned v = __ballot_sync(0xffffffffu, bit);
+            m &= bit ? v : ~v;
+        }
+    }
+    return m;
+}
+
+// Per-CTA digit histogram of its chunk, stored digit-major (hist[d * G + cta]);
+// digit totals accumulate into totals[d].  Each warp counts into its own
+// shared-memory histogram.
+template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_radix_hist(const unsigned* __restrict__ keys, const unsigned* __restrict__ n_ptr, int shift, int bits,
              unsigned* __restrict__ hist, unsigned* __restrict__ totals) {
-    __shared__ unsigned s_h[kRadixMax];
+    using C = RadixCfg<MAXB>;
+    __shared__ unsigned s_h[C::kWarps][C::kRadix];
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
-    for (int d = threadIdx.x; d < radix; d += kSortBlock) s_h[d] = 0;
+    for (int i = threadIdx.x; i < C::kWarps * C::kRadix; i += kSortBlock) (&s_h[0][0])[i] = 0;
     __syncthreads();
     unsigned lo, hi;
-    chunk_of(*n_ptr, lo, hi);
-    const int lane = threadIdx.x & 31;
-    for (unsigned base = lo; base < hi; base += kSortBlock) {
-        const unsigned i = base + threadIdx.x;
-        const bool valid = i < hi;
-        const unsigned d = valid ? (keys[i] >> shift) & mask : (unsigned)kRadixMax;
-        const unsigned peers = __match_any_sync(0xffffffffu, d);
-        if (valid && lane == __ffs(peers) - 1) atomicAdd(&s_h[d], (unsigned)__popc(peers));
+    chunk_of<MAXB>(*n_ptr, lo, hi);
+    const int warp = threadIdx.x >> 5;
+    for (unsigned base = lo; base < hi; base += C::kTileKeys) {
+        unsigned d[C::kItems];
+#pragma unroll
+        for (int j = 0; j < C::kItems; ++j) {
+            const unsigned i = base + j * kSortBlock + threadIdx.x;
+            d[j] = i < hi ? (keys[i] >> shift) & mask : kNoDigit;
+        }
+#pragma unroll
+        for (int j = 0; j < C::kItems; ++j)
+            if (d[j] != kNoDigit) atomicAdd(&s_h[warp][d[j]], 1u);
     }
     __syncthreads();
     const unsigned G = gridDim.x;
-    for (int d = threadIdx.x; d < radix; d += kSortBlock) {
-        const unsigned c = s_h[d];
-        hist[(size_t)d * G + blockIdx.x] = c;
-        if (c) atomicAdd(&totals[d], c);
+    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
+        unsigned c = 0;
+#pragma unroll
+        for (int w = 0; w < C::kWarps; ++w) c += s_h[w][dd];
+        hist[(size_t)dd * G + blockIdx.x] = c;
+        if (c) atomicAdd(&totals[dd], c);
     }
 }
 
@@ -154,26 +207,23 @@ k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, i
     const int d = blockIdx.x;
     __shared__ unsigned s_w[kSortBlock / 32];
     __shared__ unsigned s_base;
-    // base of digit d
     unsigned b = 0;
     for (int e = threadIdx.x; e < d; e += kSortBlock) b += totals[e];
     b = __reduce_add_sync(0xffffffffu, b);
     if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = b;
     __syncthreads();
     if (threadIdx.x == 0) {
-        unsigned s = 0;
-        for (int k = 0; k < kSortBlock / 32; ++k) s += s_w[k];
-        s_base = s;
+        unsigned s2 = 0;
+        for (int k = 0; k < kSortBlock / 32; ++k) s2 += s_w[k];
+        s_base = s2;
     }
     __syncthreads();
-    // exclusive scan of hist[d][0..G) with each thread owning a contiguous run
     const int per = (G + kSortBlock - 1) / kSortBlock;
     unsigned* row = hist + (size_t)d * G;
     const int c0 = threadIdx.x * per;
     unsigned local = 0;
     for (int k = 0; k < per; ++k)
         if (c0 + k < G) local += row[c0 + k];
-    // block exclusive scan of `local`
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned incl = local;
     for (int o = 1; o < 32; o <<= 1) {
@@ -194,56 +244,123 @@ k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, i
         }
 }
 
-// Stable scatter: each CTA walks its chunk in order, 256 items at a time;
-// items with equal digits keep their order (warp, then lane, then step).
+// Stable scatter.  Per tile of ITEMS x 256 keys:
+//   1. every warp ranks each of its item slots among its lanes (digit_peers)
+//      and records the group sizes per (slot, digit);
+//   2. one thread per digit turns those counts into tile-local offsets in
+//      input order (slot-major: item slot j, then warp), giving the tile's
+//      count per digit; the digit counts are scanned into tile-local starts;
+//   3. every key is placed in shared memory at its tile-local sorted
+//      position (keys regrouped by digit, input order kept within a digit);
+//   4. the regrouped tile is written out in order, so consecutive lanes write
+//      consecutive addresses of one digit's run (coalesced stores).
+template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict__ vals_in,
                 unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out,
                 const unsigned* __restrict__ n_ptr, int shift, int bits, const unsigned* __restrict__ offsets) {
-    constexpr int kWarps = kSortBlock / 32;
-    __shared__ unsigned s_base[kRadixMax];
-    __shared__ unsigned s_cnt[kWarps][kRadixMax];
-    __shared__ unsigned s_off[kWarps][kRadixMax];
+    using C = RadixCfg<MAXB>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned* s_base = reinterpret_cast<unsigned*>(smem_raw);   // [radix] running global base
+    unsigned* s_tcnt = s_base + C::kRadix;                      // [radix] this tile's count per digit
+    unsigned* s_tstart = s_tcnt + C::kRadix;                    // [radix] tile-local start per digit
+    unsigned* s_tbase = s_tstart + C::kRadix;                   // [radix] global base for this tile
+    unsigned* s_keys = s_tbase + C::kRadix;                     // [tile] regrouped keys
+    unsigned* s_vals = s_keys + C::kTileKeys;                   // [tile] regrouped values
+    unsigned short* s_cnt = reinterpret_cast<unsigned short*>(s_vals + C::kTileKeys);  // [slots][radix]
+    unsigned short* s_off = s_cnt + C::kSlots * C::kRadix;                              // [slots][radix]
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
     const unsigned G = gridDim.x;
-    for (int d = threadIdx.x; d < radix; d += kSortBlock) {
-        s_base[d] = offsets[(size_t)d * G + blockIdx.x];
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) s_cnt[w][d] = 0;
-    }
+    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) s_base[dd] = offsets[(size_t)dd * G + blockIdx.x];
+    for (int i = threadIdx.x; i < C::kSlots * C::kRadix; i += kSortBlock) s_cnt[i] = 0;
     __syncthreads();
     unsigned lo, hi;
-    chunk_of(*n_ptr, lo, hi);
+    chunk_of<MAXB>(*n_ptr, lo, hi);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned lt = lanemask_lt();
-    for (unsigned base = lo; base < hi; base += kSortBlock) {
-        const unsigned i = base + threadIdx.x;
-        const bool valid = i < hi;
-        const unsigned key = valid ? keys_in[i] : 0u;
-        const unsigned val = valid ? vals_in[i] : 0u;
-        const unsigned d = valid ? (key >> shift) & mask : (unsigned)kRadixMax;
-        const unsigned peers = __match_any_sync(0xffffffffu, d);
-        const unsigned rank = __popc(peers & lt);
-        if (valid && lane == __ffs(peers) - 1) s_cnt[warp][d] = __popc(peers);
-        __syncthreads();
-        for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
-            unsigned run = s_base[dd];
+    for (unsigned base = lo; base < hi; base += C::kTileKeys) {
+        const unsigned tile_n = min((unsigned)C::kTileKeys, hi - base);
+        unsigned key[C::kItems], val[C::kItems], d[C::kItems], rank[C::kItems];
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-                const unsigned c = s_cnt[w][dd];
-                s_cnt[w][dd] = 0;
-                s_off[w][dd] = run;
+        for (int j = 0; j < C::kItems; ++j) {
+            const unsigned i = base + j * kSortBlock + threadIdx.x;
+            const bool valid = i < hi;
+            key[j] = valid ? keys_in[i] : 0u;
+            val[j] = valid ? vals_in[i] : 0u;
+            d[j] = valid ? (key[j] >> shift) & mask : kNoDigit;
+        }
+        // 1. ranks within each warp's slot
+#pragma unroll
+        for (int j = 0; j < C::kItems; ++j) {
+            const unsigned peers = digit_peers<MAXB>(d[j], bits);
+            rank[j] = __popc(peers & lt);
+            if (d[j] != kNoDigit && lane == __ffs(peers) - 1)
+                s_cnt[(j * C::kWarps + warp) * C::kRadix + d[j]] = (unsigned short)__popc(peers);
+        }
+        __syncthreads();
+        // 2. per digit: tile-local offsets in input order, and the tile count
+        for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
+            unsigned run = 0;
+#pragma unroll 8
+            for (int e = 0; e < C::kSlots; ++e) {
+                const unsigned c = s_cnt[e * C::kRadix + dd];
+                s_cnt[e * C::kRadix + dd] = 0;
+                s_off[e * C::kRadix + dd] = (unsigned short)run;
                 run += c;
             }
-            s_base[dd] = run;
+            s_tcnt[dd] = run;
         }
         __syncthreads();
-        if (valid) {
-            const unsigned pos = s_off[warp][d] + rank;
-            keys_out[pos] = key;
-            vals_out[pos] = val;
+        // exclusive scan of the digit counts (one warp), bases for this tile
+        if (warp == 0) {
+            constexpr int per = (C::kRadix + 31) / 32;
+            unsigned v[per], sum = 0;
+#pragma unroll
+            for (int k = 0; k < per; ++k) {
+                const int dd = lane * per + k;
+                v[k] = dd < radix ? s_tcnt[dd] : 0u;
+                sum += v[k];
+            }
+            unsigned incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            unsigned run = incl - sum;
+#pragma unroll
+            for (int k = 0; k < per; ++k) {
+                const int dd = lane * per + k;
+                if (dd < radix) {
+                    s_tstart[dd] = run;
+                    s_tbase[dd] = s_base[dd];
+                    s_base[dd] += v[k];
+                }
+                run += v[k];
+            }
         }
+        __syncthreads();
+        // 3. regroup the tile by digit in shared memory
+#pragma unroll
+        for (int j = 0; j < C::kItems; ++j) {
+            if (d[j] != kNoDigit) {
+                const unsigned loc = s_tstart[d[j]] + s_off[(j * C::kWarps + warp) * C::kRadix + d[j]] + rank[j];
+                s_keys[loc] = key[j];
+                s_vals[loc] = val[j];
+            }
+        }
+        __syncthreads();
+        // 4. write the regrouped tile: consecutive q of one digit go to
+        //    consecutive output positions
+        for (unsigned q = threadIdx.x; q < tile_n; q += kSortBlock) {
+            const unsigned k2 = s_keys[q];
+            const unsigned dq = (k2 >> shift) & mask;
+            const unsigned pos = s_tbase[dq] + (q - s_tstart[dq]);
+            keys_out[pos] = k2;
+            vals_out[pos] = s_vals[q];
+        }
+        // the next tile's first barrier orders these reads before its writes
     }
 }
 
@@ -331,9 +448,11 @@ k_scan_down(int N, const unsigned* __restrict__ order, const unsigned* __restric
 }
 
 // Emit the (tile, Gaussian) pairs in depth-rank order.  A warp takes 32
-// consecutive ranks and writes each Gaussian's tiles with all 32 lanes
-// (row-major over its rectangle), so stores are coalesced and a Gaussian
-// covering thousands of tiles does not stall one lane.
+// consecutive ranks, whose pairs are contiguous in the output; each lane
+// writes every 32nd of those pairs, finding the Gaussian it belongs to by a
+// binary search over the warp's inclusive scan of pair counts (held in
+// registers, read with shuffles).  Stores are coalesced and the work per
+// lane is balanced however many tiles each Gaussian covers.
 __global__ void __launch_bounds__(kSortBlock)
 k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
        const int4* __restrict__ rect, const unsigned* __restrict__ tiles_touched, const SortMisc* __restrict__ misc,
@@ -345,34 +464,49 @@ k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __rest
     const int nwarps = (gridDim.x * kSortBlock) >> 5;
     for (int r0 = warp_global * 32; r0 < N; r0 += nwarps * 32) {
         const int r = r0 + lane;
-        unsigned g = 0, off = 0, cnt = 0;
-        int4 rc = make_int4(0, 0, 0, 0);
+        unsigned g = 0, cnt = 0, off = 0;
+        int x0 = 0, y0 = 0, wdt = 1;
         if (r < N) {
             g = order[r];
             cnt = tiles_touched[g];
+            off = pair_off[r];
             if (cnt) {
-                off = pair_off[r];
-                rc = rect[g];
+                const int4 rc = rect[g];
+                x0 = rc.x;
+                y0 = rc.y;
+                wdt = rc.z - rc.x;
             }
         }
-        unsigned todo = __ballot_sync(0xffffffffu, cnt != 0);
-        while (todo) {
-            const int src = __ffs(todo) - 1;
-            todo &= todo - 1;
-            const unsigned gg = __shfl_sync(0xffffffffu, g, src);
-            const unsigned oo = __shfl_sync(0xffffffffu, off, src);
-            const unsigned cc = __shfl_sync(0xffffffffu, cnt, src);
-            const int x0 = __shfl_sync(0xffffffffu, rc.x, src);
-            const int y0 = __shfl_sync(0xffffffffu, rc.y, src);
-            const int x1 = __shfl_sync(0xffffffffu, rc.z, src);
-            const unsigned wdt = (unsigned)(x1 - x0);
-            // never write past P, even if the caller's counts disagree
-            const unsigned lim = oo < P ? min(cc, P - oo) : 0u;
-            for (unsigned k = lane; k < lim; k += 32) {
-                const unsigned ty = (unsigned)y0 + k / wdt;
-                const unsigned tx = (unsigned)x0 + k % wdt;
-                tkeys[oo + k] = ty * (unsigned)TX + tx;
-                tvals[oo + k] = gg;
+        unsigned incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const unsigned total = __shfl_sync(0xffffffffu, incl, 31);
+        const unsigned off0 = __shfl_sync(0xffffffffu, off, 0);
+        const unsigned excl = incl - cnt;
+        // warp-uniform loop: every lane takes part in every shuffle
+        for (unsigned kb = 0; kb < total; kb += 32) {
+            const unsigned k = kb + lane;
+            // owner: the first lane whose inclusive count exceeds k
+            int sidx = 0;
+#pragma unroll
+            for (int b = 16; b >= 1; b >>= 1) {
+                const unsigned v = __shfl_sync(0xffffffffu, incl, sidx + b - 1);
+                if (v <= k) sidx += b;
+            }
+            sidx = min(sidx, 31);
+            const unsigned local = k - __shfl_sync(0xffffffffu, excl, sidx);
+            const unsigned gg = __shfl_sync(0xffffffffu, g, sidx);
+            const int ox = __shfl_sync(0xffffffffu, x0, sidx);
+            const int oy = __shfl_sync(0xffffffffu, y0, sidx);
+            const int ow = __shfl_sync(0xffffffffu, wdt, sidx);
+            const unsigned pos = off0 + k;
+            if (k < total && pos < P) {  // never write past P, even if the caller's counts disagree
+                tkeys[pos] = (unsigned)(oy + (int)(local / (unsigned)ow)) * (unsigned)TX +
+                             (unsigned)(ox + (int)(local % (unsigned)ow));
+                tvals[pos] = gg;
             }
         }
     }
@@ -399,6 +533,24 @@ int ceil_log2(unsigned x) {
     return b;
 }
 
+// The scatter needs more than the default 48 KiB of dynamic shared memory;
+// the attribute belongs to the current device, so it is set before each use.
+template <int MAXB>
+void enable_scatter_smem() {
+    cudaFuncSetAttribute(k_radix_scatter<MAXB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)RadixCfg<MAXB>::kScatterSmem);
+}
+
+template <int MAXB>
+void radix_pass(cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
+                const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals) {
+    enable_scatter_smem<MAXB>();
+    k_radix_hist<MAXB><<<G, kSortBlock, 0, st>>>(ki, n_ptr, shift, bits, hist, totals);
+    k_radix_scan<<<1 << bits, kSortBlock, 0, st>>>(hist, totals, G);
+    k_radix_scatter<MAXB><<<G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st>>>(ki, vi, ko, vo, n_ptr, shift, bits,
+                                                                                hist);
+}
+
 // One stable LSD radix sort of (keys, vals) over bits [0, total_bits), with
 // at most 8 bits per pass.  The final pass writes to (final_keys, final_vals)
 // when they are given.  Returns the number of passes.
@@ -417,9 +569,10 @@ int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, un
         unsigned* vdst = (last && final_vals) ? final_vals : vo;
         unsigned* h = hist + (size_t)(pass_base + p) * kRadixMax * kSortMaxGrid;
         unsigned* tot = totals + (size_t)(pass_base + p) * kRadixMax;
-        k_radix_hist<<<G, kSortBlock, 0, st>>>(ki, n_ptr, p * bits, bits, h, tot);
-        k_radix_scan<<<1 << bits, kSortBlock, 0, st>>>(h, tot, G);
-        k_radix_scatter<<<G, kSortBlock, 0, st>>>(ki, vi, ko, vdst, n_ptr, p * bits, bits, h);
+        if (bits <= 7)
+            radix_pass<7>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
+        else
+            radix_pass<8>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
         unsigned* tk = ki;
         ki = ko;
         ko = tk;

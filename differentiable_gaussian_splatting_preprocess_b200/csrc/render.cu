@@ -330,6 +330,40 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     }
 }
 
+// Work counts of the forward, per pixel: list entries evaluated before the
+// pixel stopped (the stopping entry included) and terms blended.  One thread
+// per pixel walking its tile's list in order with the same term evaluation as
+// the forward (pixel duplicated in both lanes), so the counts are those of the
+// compositing above.  A diagnostic for measurement, not part of the hot path.
+__global__ void __launch_bounds__(kTilePixels)
+k_render_stats(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
+               const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
+               unsigned* __restrict__ n_evaluated, unsigned* __restrict__ n_blended) {
+    const int tile = blockIdx.x;
+    const int x = (tile % TX) * kTile + (threadIdx.x & (kTile - 1));
+    const int y = (tile / TX) * kTile + (threadIdx.x / kTile);
+    if (x >= cam.width || y >= cam.height) return;
+    const uint2 rg = ranges[tile];
+    const float2 px = make_float2((float)x + 0.5f, (float)x + 0.5f);
+    const float py = (float)y + 0.5f;
+    float T = 1.0f;
+    unsigned ev = 0, bl = 0;
+    for (unsigned k = rg.x; k < rg.y; ++k) {
+        const unsigned j = ids[k];
+        ++ev;
+        TermPair e;
+        eval_pair(px, py, mean2d[j], conic_opacity[j], cam.alpha_max, cam.alpha_min, e);
+        if (!e.ok0) continue;
+        const float Tn = __fmul_rn(T, __fsub_rn(1.0f, e.alpha.x));
+        if (Tn < cam.T_min) break;
+        T = Tn;
+        ++bl;
+    }
+    const size_t pix = (size_t)y * cam.width + x;
+    n_evaluated[pix] = ev;
+    n_blended[pix] = bl;
+}
+
 __global__ void k_zero(float* __restrict__ a, size_t na, float* __restrict__ b, size_t nb, float* __restrict__ c,
                        size_t nc) {
     const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -381,6 +415,19 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
                                        reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
                                        dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),
                                        reinterpret_cast<float4*>(dL_dconic_opacity), dL_dcolor);
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+}
+
+extern "C" int gs_render_stats(const gs_camera* cam, const unsigned* ranges, const unsigned* ids, const float* mean2d,
+                               const float* conic_opacity, unsigned* n_evaluated, unsigned* n_blended, void* stream) {
+    if (!camera_ok(cam) || !ranges || !n_evaluated || !n_blended) return GS_ERR_INVALID_ARG;
+    if (!aligned(ranges, 8) || (conic_opacity && !aligned(conic_opacity, 16)) || (mean2d && !aligned(mean2d, 8)))
+        return GS_ERR_INVALID_ARG;
+    const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
+    k_render_stats<<<T, kTilePixels, 0, (cudaStream_t)stream>>>(
+        *cam, TX, reinterpret_cast<const uint2*>(ranges), ids, reinterpret_cast<const float2*>(mean2d),
+        reinterpret_cast<const float4*>(conic_opacity), n_evaluated, n_blended);
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

@@ -203,6 +203,17 @@ GS_API int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const uns
                   unsigned* n_contrib, void* stream);
 
 /*
+ * gs_render_stats - work counts of gs_render_fwd, per pixel (the derived
+ *   measures "evaluated" and "blended" terms; a diagnostic, not a stage of
+ *   the method).  n_evaluated [H,W]: list entries the pixel evaluated before
+ *   it stopped (the stopping entry included), or the tile's list length;
+ *   n_blended [H,W]: terms composited.  Same inputs and decisions as
+ *   gs_render_fwd.
+ */
+GS_API int gs_render_stats(const gs_camera* cam, const unsigned* ranges, const unsigned* ids, const float* mean2d,
+                           const float* conic_opacity, unsigned* n_evaluated, unsigned* n_blended, void* stream);
+
+/*
  * gs_render_bwd - reverse per-pixel traversal ([CB] 2, 3).  From T = final_T
  *   and the colour behind S = bg, for list positions n_contrib-1 down to 0
  *   (the terms the forward blended): T <- T / (1 - alpha);

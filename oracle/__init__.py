@@ -72,7 +72,7 @@ def lib():
             getattr(L, f"oracle_bin_{suf}").restype = ctypes.c_longlong
             getattr(L, f"oracle_tile_list_{suf}").argtypes = [cam, I, P, P, P, I, P]
             getattr(L, f"oracle_tile_list_{suf}").restype = ctypes.c_longlong
-            getattr(L, f"oracle_render_fwd_{suf}").argtypes = [cam] + [P] * 10 + [I]
+            getattr(L, f"oracle_render_fwd_{suf}").argtypes = [cam] + [P] * 11 + [I]
             getattr(L, f"oracle_render_fwd_{suf}").restype = None
             getattr(L, f"oracle_render_bwd_{suf}").argtypes = [cam, I] + [P] * 10 + [I]
             getattr(L, f"oracle_render_bwd_{suf}").restype = None
@@ -171,12 +171,14 @@ def render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, mode: str = "f32
     mean2d, conic_opacity, colors = (_a(x, dt) for x in (mean2d, conic_opacity, colors))
     H, W = cam.height, cam.width
     out = dict(image=np.zeros((3, H, W), dt), final_T=np.zeros((H, W), dt),
-               n_contrib=np.zeros((H, W), np.uint32), n_eval=np.zeros((H, W), np.uint32))
+               n_contrib=np.zeros((H, W), np.uint32), n_eval=np.zeros((H, W), np.uint32),
+               n_blended=np.zeros((H, W), np.uint32))
     sub = None if tiles is None else _a(tiles, np.int32)
     oc = camera(cam)
     getattr(lib(), f"oracle_render_fwd_{mode}")(
         ctypes.byref(oc), _p(ranges), _p(ids), _p(mean2d), _p(conic_opacity), _p(colors), _p(out["image"]),
-        _p(out["final_T"]), _p(out["n_contrib"]), _p(out["n_eval"]), _p(sub), 0 if sub is None else sub.size)
+        _p(out["final_T"]), _p(out["n_contrib"]), _p(out["n_eval"]), _p(out["n_blended"]), _p(sub),
+        0 if sub is None else sub.size)
     return out
 
 

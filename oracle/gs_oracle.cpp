@@ -368,7 +368,7 @@ void tiles_of(const oracle_camera* cam, const int* subset, int n_subset, std::ve
 template <typename Real>
 void render_fwd(const oracle_camera* cam, const unsigned* ranges, const unsigned* ids, const Real* mean2d,
                 const Real* conic_opacity, const Real* colors, Real* image, Real* final_T, unsigned* n_contrib,
-                unsigned* n_eval, const int* subset, int n_subset) {
+                unsigned* n_eval, unsigned* n_blend, const int* subset, int n_subset) {
     const int W = cam->width, H = cam->height, TS = cam->tile;
     const int TX = (W + TS - 1) / TS;
     std::vector<int> tiles;
@@ -382,7 +382,7 @@ void render_fwd(const oracle_camera* cam, const unsigned* ranges, const unsigned
             for (int x = tx * TS; x < std::min(W, tx * TS + TS); ++x) {
                 const Real px = Real(x) + Real(0.5), py = Real(y) + Real(0.5);
                 Real T = Real(1), C[3] = {Real(0), Real(0), Real(0)};
-                unsigned last = 0, evals = 0;
+                unsigned last = 0, evals = 0, blended = 0;
                 for (unsigned k = r0; k < r1; ++k) {
                     const unsigned j = ids[k];
                     ++evals;
@@ -393,12 +393,14 @@ void render_fwd(const oracle_camera* cam, const unsigned* ranges, const unsigned
                     for (int ch = 0; ch < 3; ++ch) C[ch] += colors[3 * j + ch] * e.alpha * T;
                     T = Tn;
                     last = k - r0 + 1;
+                    ++blended;
                 }
                 const size_t pix = (size_t)y * W + x;
                 for (int ch = 0; ch < 3; ++ch) image[(size_t)ch * H * W + pix] = C[ch] + T * Real(cam->bg[ch]);
                 final_T[pix] = T;
                 n_contrib[pix] = last;
                 if (n_eval) n_eval[pix] = evals;
+                if (n_blend) n_blend[pix] = blended;
             }
         }
     }
@@ -678,10 +680,10 @@ void oracle_set_threads(int n) {
     }                                                                                                        \
     void oracle_render_fwd_##SUF(const oracle_camera* cam, const unsigned* ranges, const unsigned* ids,      \
                                  const R* mean2d, const R* conic_opacity, const R* colors, R* image,         \
-                                 R* final_T, unsigned* n_contrib, unsigned* n_eval, const int* subset,       \
-                                 int n_subset) {                                                             \
+                                 R* final_T, unsigned* n_contrib, unsigned* n_eval, unsigned* n_blend,       \
+                                 const int* subset, int n_subset) {                                          \
         render_fwd<R>(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_T, n_contrib, n_eval,    \
-                      subset, n_subset);                                                                     \
+                      n_blend, subset, n_subset);                                                            \
     }                                                                                                        \
     void oracle_render_bwd_##SUF(const oracle_camera* cam, int N, const unsigned* ranges, const unsigned* ids, \
                                  const R* mean2d, const R* conic_opacity, const R* colors,                   \

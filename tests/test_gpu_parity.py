@@ -299,3 +299,22 @@ def test_preprocess_backward_accumulates():
                                                               if k.startswith("dL_d") and v.shape[0] == sc.N})
     for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
         np.testing.assert_allclose(to_np(r2["grads"][k]), 2 * once[k], rtol=1e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_render_stats_match_oracle_counts(cfg):
+    """The work counts behind the throughput figures (entries evaluated and
+    terms blended per pixel) equal the oracle's, bit for bit."""
+    sc = _scene(cfg)
+    cam = sc.cameras[0]
+    r = run_gpu(GpuScene(sc), cam, want_keys=False)
+    fr = r["frame"]
+    ne = torch.empty((cam.height, cam.width), dtype=torch.uint32, device="cuda")
+    nb = torch.empty_like(ne)
+    B.gs_render_stats(cam, fr.ranges, fr.ids, fr.mean2d, fr.conic_opacity, ne, nb)
+    torch.cuda.synchronize()
+    g = frame_np(fr)
+    o = oracle.render_fwd(cam, g["ranges"], g["ids"], g["mean2d"], g["conic_opacity"], sc.colors, "f32")
+    np.testing.assert_array_equal(to_np(ne), o["n_eval"])
+    np.testing.assert_array_equal(to_np(nb), o["n_blended"])
+    assert np.all(to_np(nb) <= g["n_contrib"])

@@ -262,6 +262,7 @@ def test_golden_compositing(mode):
         np.testing.assert_allclose(f["image"][:, py, px], exp["color"], atol=tol, err_msg=case["name"])
         assert f["final_T"][py, px] == pytest.approx(exp["final_T"], abs=tol), case["name"]
         assert f["n_contrib"][py, px] == exp["n_contrib"], case["name"]
+        assert f["n_blended"][py, px] == exp["n_blended"], case["name"]
 
 
 def test_single_gaussian_closed_form():
