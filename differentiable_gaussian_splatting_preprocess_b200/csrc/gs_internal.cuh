@@ -122,6 +122,52 @@ __device__ __forceinline__ void eval_pair(float2 px, float py, float2 xy, float4
     e.ok1 = !(power.y > 0.0f) && !(e.alpha.y < alpha_min);
 }
 
+// Inflated threshold k on q = d^T A d: a pixel can reach alpha >= alpha_min
+// only where q <= k (see contrib_box).  +inf when no bound is available
+// (never culled), -1 when the Gaussian can never reach alpha_min.
+__device__ __forceinline__ float contrib_threshold(float4 co, float alpha_min) {
+    const float inf = __int_as_float(0x7f800000);
+    if (!(alpha_min > 0.0f)) return inf;
+    if (co.w < alpha_min) return -1.0f;
+    const float det = co.x * co.z - co.y * co.y;
+    if (!(det > 0.0f)) return inf;
+    const float tr = co.x + co.z;
+    const float k = 2.0f * logf(co.w / alpha_min) * (1.001f + 1e-6f * (tr * tr / det)) + 1e-5f;
+    return isfinite(k) ? k : inf;
+}
+
+// True when q = a dx^2 + 2 b dx dy + c dy^2 exceeds `thr` at every point of
+// the rectangle [x0, x1] x [y0, y1] around the Gaussian's mean xy, i.e. when
+// no pixel centre inside can reach alpha >= alpha_min.  The minimum of the
+// positive-definite q over the rectangle is 0 when the mean is inside, else
+// it lies on an edge, where q is a quadratic in one variable minimised in
+// closed form and clamped to the edge.  Any undefined value keeps the
+// Gaussian (the comparison is false).
+__device__ __forceinline__ bool ellipse_misses(float2 xy, float4 co, float thr, float x0, float x1, float y0,
+                                               float y1) {
+    if (xy.x >= x0 && xy.x <= x1 && xy.y >= y0 && xy.y <= y1) return false;
+    const float a = co.x, b = co.y, c = co.z;
+    if (!(a > 0.0f && c > 0.0f)) return false;
+    const float ex0 = x0 - xy.x, ex1 = x1 - xy.x, ey0 = y0 - xy.y, ey1 = y1 - xy.y;
+    const float boc = b / c, boa = b / a;
+    float best = __int_as_float(0x7f800000);
+    // edges x = x0 and x = x1: minimise over dy in [ey0, ey1]; dy* = -b dx / c
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const float dx = e ? ex1 : ex0;
+        const float dy = fminf(fmaxf(-boc * dx, ey0), ey1);
+        best = fminf(best, a * dx * dx + 2.0f * b * dx * dy + c * dy * dy);
+    }
+    // edges y = y0 and y = y1: minimise over dx in [ex0, ex1]; dx* = -b dy / a
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const float dy = e ? ey1 : ey0;
+        const float dx = fminf(fmaxf(-boa * dy, ex0), ex1);
+        best = fminf(best, a * dx * dx + 2.0f * b * dx * dy + c * dy * dy);
+    }
+    return best > thr;
+}
+
 // Axis-aligned box (pixel coordinates: xmin, xmax, ymin, ymax) outside of
 // which a Gaussian cannot reach alpha >= alpha_min, so a warp whose pixels
 // all lie outside may skip it without changing any result.  The region is

@@ -24,14 +24,16 @@ namespace {
 
 // One CTA per 16x16 tile with 128 threads: each thread owns two horizontally
 // adjacent pixels, evaluated together with packed fp32x2 arithmetic; warp w
-// owns the 16x4 strip of rows 4w..4w+3.  Gaussians are staged 128 at a time.
+// owns one 8x8 quadrant of the tile.  Gaussians are staged 256 at a time.
 // Before a warp walks a batch it builds a ballot mask of the staged
-// Gaussians whose contribution box (contrib_box) meets its strip, and walks
-// only those: a skipped Gaussian would have been rejected by the alpha_min
-// test at every pixel of the strip, so results are unchanged.
+// Gaussians that can reach alpha >= alpha_min somewhere in its quadrant (a
+// box test, then an exact ellipse-versus-rectangle test, both inflated for
+// fp32 rounding) and walks only those: a skipped Gaussian would have been
+// rejected by the alpha_min test at every pixel of the quadrant, so results
+// are unchanged.
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 128;
+constexpr int kBatch = 256;
 constexpr int kWords = kBatch / 32;
 static_assert(kThreads * 2 == kTilePixels, "two pixels per thread");
 
@@ -40,25 +42,32 @@ struct PixelPair {
     bool in0, in1;
     float2 px;
     float py;
-    float sx0, sx1, sy0, sy1;  // pixel-centre rectangle of this warp's strip
+    float sx0, sx1, sy0, sy1;  // pixel-centre rectangle of this warp's quadrant
 };
 
 __device__ __forceinline__ PixelPair pixel_pair(const gs_camera& cam, int TX) {
     PixelPair q;
     const int tile = blockIdx.x;
-    const int tx0 = (tile % TX) * kTile, ty0 = (tile / TX) * kTile;
-    q.x0 = tx0 + 2 * (threadIdx.x & 7);
-    q.y = ty0 + (threadIdx.x >> 3);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bx = (tile % TX) * kTile + (warp & 1) * 8;
+    const int by = (tile / TX) * kTile + (warp >> 1) * 8;
+    q.x0 = bx + 2 * (lane & 3);
+    q.y = by + (lane >> 2);
     q.in0 = q.x0 < cam.width && q.y < cam.height;
     q.in1 = q.x0 + 1 < cam.width && q.y < cam.height;
     q.px = make_float2((float)q.x0 + 0.5f, (float)q.x0 + 1.5f);
     q.py = (float)q.y + 0.5f;
-    const int warp = threadIdx.x >> 5;
-    q.sx0 = (float)tx0 + 0.5f;
-    q.sx1 = (float)tx0 + 15.5f;
-    q.sy0 = (float)(ty0 + 4 * warp) + 0.5f;
-    q.sy1 = q.sy0 + 3.0f;
+    q.sx0 = (float)bx + 0.5f;
+    q.sx1 = q.sx0 + 7.0f;
+    q.sy0 = (float)by + 0.5f;
+    q.sy1 = q.sy0 + 7.0f;
     return q;
+}
+
+// Can the staged Gaussian reach alpha >= alpha_min in this warp's quadrant?
+__device__ __forceinline__ bool may_contribute(float4 box, float thr, float2 xy, float4 co, const PixelPair& q) {
+    if (box_misses(box, q.sx0, q.sx1, q.sy0, q.sy1)) return false;
+    return !ellipse_misses(xy, co, thr, q.sx0, q.sx1, q.sy0, q.sy1);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -70,6 +79,7 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     __shared__ float4 s_co[kBatch];
     __shared__ float4 s_col[kBatch];
     __shared__ float4 s_box[kBatch];
+    __shared__ float s_thr[kBatch];
     const PixelPair q = pixel_pair(cam, TX);
     const int lane = threadIdx.x & 31;
     const uint2 rg = ranges[blockIdx.x];
@@ -81,22 +91,25 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     bool done0 = !q.in0, done1 = !q.in1;
     for (unsigned b = rg.x; b < rg.y; b += kBatch) {
         if (__syncthreads_count(done0 && done1) == kThreads) break;
-        const unsigned k = b + threadIdx.x;
-        if (k < rg.y) {
-            const unsigned j = ids[k];
-            const float2 xy = mean2d[j];
-            const float4 co = conic_opacity[j];
-            s_xy[threadIdx.x] = xy;
-            s_co[threadIdx.x] = co;
-            s_col[threadIdx.x] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
-            s_box[threadIdx.x] = contrib_box(xy, co, amin);
+        for (int r = threadIdx.x; r < kBatch; r += kThreads) {
+            const unsigned k = b + r;
+            if (k < rg.y) {
+                const unsigned j = ids[k];
+                const float2 xy = mean2d[j];
+                const float4 co = conic_opacity[j];
+                s_xy[r] = xy;
+                s_co[r] = co;
+                s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+                s_box[r] = contrib_box(xy, co, amin);
+                s_thr[r] = contrib_threshold(co, amin);
+            }
         }
         __syncthreads();
         const int n = min((unsigned)kBatch, rg.y - b);
         bool warp_done = __all_sync(0xffffffffu, done0 && done1);
         for (int w = 0; w < kWords && !warp_done; ++w) {
             const int jl = w * 32 + lane;
-            const bool keep = jl < n && !box_misses(s_box[jl], q.sx0, q.sx1, q.sy0, q.sy1);
+            const bool keep = jl < n && may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], q);
             unsigned m = __ballot_sync(0xffffffffu, keep);
             while (m) {
                 const int jj = w * 32 + __ffs(m) - 1;
@@ -185,6 +198,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     __shared__ float4 s_co[kBatch];
     __shared__ float4 s_col[kBatch];
     __shared__ float4 s_box[kBatch];
+    __shared__ float s_thr[kBatch];
     __shared__ float s_grad[kBatch * kGradStride];
     __shared__ unsigned s_max[kWarps];
 
@@ -226,23 +240,26 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
 
     for (int top = (int)max_last; top > 0; top -= kBatch) {
         // stage positions top-1, top-2, ... so that staged order is back to front
-        const int pos = top - 1 - (int)threadIdx.x;
-        if (pos >= 0) {
-            const unsigned j = ids[rg.x + pos];
-            const float2 xy = mean2d[j];
-            const float4 co = conic_opacity[j];
-            s_id[threadIdx.x] = j;
-            s_xy[threadIdx.x] = xy;
-            s_co[threadIdx.x] = co;
-            s_col[threadIdx.x] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
-            s_box[threadIdx.x] = contrib_box(xy, co, amin);
+        for (int r = threadIdx.x; r < kBatch; r += kThreads) {
+            const int pos = top - 1 - r;
+            if (pos >= 0) {
+                const unsigned j = ids[rg.x + pos];
+                const float2 xy = mean2d[j];
+                const float4 co = conic_opacity[j];
+                s_id[r] = j;
+                s_xy[r] = xy;
+                s_co[r] = co;
+                s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+                s_box[r] = contrib_box(xy, co, amin);
+                s_thr[r] = contrib_threshold(co, amin);
+            }
         }
         __syncthreads();
         const int n = min(kBatch, top);
         for (int w = 0; w < kWords; ++w) {
             const int jl = w * 32 + lane;
             const bool keep = jl < n && top - 1 - jl < (int)wlast &&
-                              !box_misses(s_box[jl], q.sx0, q.sx1, q.sy0, q.sy1);
+                              may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], q);
             unsigned m = __ballot_sync(0xffffffffu, keep);
             while (m) {
                 const int jj = w * 32 + __ffs(m) - 1;
@@ -309,14 +326,14 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
         }
         __syncthreads();
         // flush this batch: one set of global atomics per (tile, Gaussian)
-        if ((int)threadIdx.x < n) {
-            float* sg = s_grad + threadIdx.x * kGradStride;
+        for (int r = threadIdx.x; r < n; r += kThreads) {
+            float* sg = s_grad + r * kGradStride;
             const float a0 = sg[0], a1 = sg[1], a2 = sg[2], a3 = sg[3], a4 = sg[4];
             const float a5 = sg[5], a6 = sg[6], a7 = sg[7], a8 = sg[8];
             const bool any = (a0 != 0.f) | (a1 != 0.f) | (a2 != 0.f) | (a3 != 0.f) | (a4 != 0.f) | (a5 != 0.f) |
                              (a6 != 0.f) | (a7 != 0.f) | (a8 != 0.f);
             if (any) {
-                const unsigned j = s_id[threadIdx.x];
+                const unsigned j = s_id[r];
                 atomicAdd(&dL_dmean2d[j], make_float2(a0, a1));
                 atomicAdd(&dL_dconic_opacity[j], make_float4(a2, a3, a4, a7));
                 atomicAdd(&dL_dcolor[3 * j + 0], a5);
