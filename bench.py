@@ -227,11 +227,11 @@ def run_ours(args):
                       rz._bufs["ids"], rz._bufs["ranges"], None, ws)
         mark(2)
         B.gs_render_fwd(cam, rz._bufs["ranges"], rz._bufs["ids"], pre["mean2d"], pre["conic_opacity"], colors,
-                        rz._bufs["image"], rz._bufs["final_T"], rz._bufs["n_contrib"])
+                        rz._bufs["image"], rz._bufs["final_T"], rz._bufs["n_contrib"], rz._bufs["contrib_mask"])
         mark(3)
         B.gs_render_bwd(cam, rz._bufs["ranges"], rz._bufs["ids"], pre["mean2d"], pre["conic_opacity"], colors,
                         rz._bufs["final_T"], rz._bufs["n_contrib"], dL, rz._bufs["dL_dmean2d"],
-                        rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"])
+                        rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"], rz._bufs["contrib_mask"])
         mark(4)
         B.gs_preprocess_bwd(cam, means, scales, quats, pre["radius"], pre["conic_opacity"], rz._bufs["dL_dmean2d"],
                             rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"], grads["dL_dmeans"],
@@ -290,7 +290,7 @@ def run_ours(args):
     T = B.num_tiles(cam)
     tile_bits = max(0, (T - 1).bit_length())
     tpasses = (tile_bits + 7) // 8
-    launches = 1 + (1 + 4 * 3 + 3 + 1 + 3 * tpasses + 1) + 1 + 2 + 1
+    launches = 1 + (1 + 4 * 3 + 3 + 1 + 3 * tpasses + 1) + 2 + 2 + 1
 
     # roofline of the dominant kernel (render backward: FP32 ALU bound)
     peaks = _peaks()

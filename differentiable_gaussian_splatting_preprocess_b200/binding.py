@@ -80,11 +80,11 @@ def lib() -> ctypes.CDLL:
         L.gs_bin_sort.restype = I
         L.gs_bin_sort.argtypes = [cam, I, P, P, P, P, U, P, P, P, P, S, P]
         L.gs_render_fwd.restype = I
-        L.gs_render_fwd.argtypes = [cam] + [P] * 8 + [P]
+        L.gs_render_fwd.argtypes = [cam] + [P] * 9 + [U, P]
         L.gs_render_stats.restype = I
         L.gs_render_stats.argtypes = [cam] + [P] * 6 + [P]
         L.gs_render_bwd.restype = I
-        L.gs_render_bwd.argtypes = [cam, I] + [P] * 11 + [P]
+        L.gs_render_bwd.argtypes = [cam, I] + [P] * 8 + [U] + [P] * 4 + [P]
         L.gs_preprocess_bwd.restype = I
         L.gs_preprocess_bwd.argtypes = [cam, I] + [P] * 13 + [P]
         _lib = L
@@ -205,7 +205,13 @@ def gs_bin_sort(cam, depth, rect, tiles_touched, d_num_pairs, capacity: int, ids
         _ptr(ids), _ptr(ranges), _ptr(keys), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def gs_render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_T, n_contrib, stream=None) -> None:
+def mask_words(capacity: int) -> int:
+    """Words of the contribution mask for `capacity` sorted pairs."""
+    return 4 * ((int(capacity) + 31) // 32)
+
+
+def gs_render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_T, n_contrib, contrib_mask=None,
+                  stream=None) -> None:
     N = mean2d.shape[0]
     H, W = cam.height, cam.width
     _check(ranges, "ranges", torch.uint32, (num_tiles(cam), 2))
@@ -216,10 +222,12 @@ def gs_render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_
     _check(image, "image", torch.float32, (3, H, W))
     _check(final_T, "final_T", torch.float32, (H, W))
     _check(n_contrib, "n_contrib", torch.uint32, (H, W))
+    _check(contrib_mask, "contrib_mask", torch.uint32, optional=True)
     c = camera_struct(cam)
     _ok("gs_render_fwd", lib().gs_render_fwd(
         ctypes.byref(c), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(colors), _ptr(image),
-        _ptr(final_T), _ptr(n_contrib), _stream(stream)))
+        _ptr(final_T), _ptr(n_contrib), _ptr(contrib_mask), 0 if contrib_mask is None else contrib_mask.numel(),
+        _stream(stream)))
 
 
 def gs_render_stats(cam, ranges, ids, mean2d, conic_opacity, n_evaluated, n_blended, stream=None) -> None:
@@ -238,7 +246,7 @@ def gs_render_stats(cam, ranges, ids, mean2d, conic_opacity, n_evaluated, n_blen
 
 
 def gs_render_bwd(cam, ranges, ids, mean2d, conic_opacity, colors, final_T, n_contrib, dL_dimage, dL_dmean2d,
-                  dL_dconic_opacity, dL_dcolor, stream=None) -> None:
+                  dL_dconic_opacity, dL_dcolor, contrib_mask=None, stream=None) -> None:
     N = mean2d.shape[0]
     H, W = cam.height, cam.width
     _check(ranges, "ranges", torch.uint32, (num_tiles(cam), 2))
@@ -252,11 +260,12 @@ def gs_render_bwd(cam, ranges, ids, mean2d, conic_opacity, colors, final_T, n_co
     _check(dL_dmean2d, "dL_dmean2d", torch.float32, (N, 2))
     _check(dL_dconic_opacity, "dL_dconic_opacity", torch.float32, (N, 4))
     _check(dL_dcolor, "dL_dcolor", torch.float32, (N, 3))
+    _check(contrib_mask, "contrib_mask", torch.uint32, optional=True)
     c = camera_struct(cam)
     _ok("gs_render_bwd", lib().gs_render_bwd(
         ctypes.byref(c), int(N), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(colors),
-        _ptr(final_T), _ptr(n_contrib), _ptr(dL_dimage), _ptr(dL_dmean2d), _ptr(dL_dconic_opacity),
-        _ptr(dL_dcolor), _stream(stream)))
+        _ptr(final_T), _ptr(n_contrib), _ptr(contrib_mask), 0 if contrib_mask is None else contrib_mask.numel(),
+        _ptr(dL_dimage), _ptr(dL_dmean2d), _ptr(dL_dconic_opacity), _ptr(dL_dcolor), _stream(stream)))
 
 
 def gs_preprocess_bwd(cam, means, scales, quats, radius, conic_opacity, dL_dmean2d, dL_dconic_opacity,

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kThreads)
 k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
              const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
              const float* __restrict__ colors, float* __restrict__ image, float* __restrict__ final_T,
-             unsigned* __restrict__ n_contrib) {
+             unsigned* __restrict__ n_contrib, unsigned* __restrict__ cmask, unsigned cmask_words) {
     __shared__ float2 s_xy[kBatch];
     __shared__ float4 s_co[kBatch];
     __shared__ float4 s_col[kBatch];
@@ -107,10 +107,25 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
         __syncthreads();
         const int n = min((unsigned)kBatch, rg.y - b);
         bool warp_done = __all_sync(0xffffffffu, done0 && done1);
+        // cull against the pixels of this warp that are still compositing
+        PixelPair qa = q;
+        if (!warp_done) {
+            const int ax0 = done0 ? 0x7fffffff : q.x0, ax1 = done1 ? -1 : q.x0 + 1;
+            const int axmin = __reduce_min_sync(0xffffffffu, min(ax0, done1 ? 0x7fffffff : q.x0 + 1));
+            const int axmax = __reduce_max_sync(0xffffffffu, max(ax1, done0 ? -1 : q.x0));
+            const int ay = (done0 && done1) ? -1 : q.y;
+            const int aymin = __reduce_min_sync(0xffffffffu, ay < 0 ? 0x7fffffff : ay);
+            const int aymax = __reduce_max_sync(0xffffffffu, ay);
+            qa.sx0 = (float)axmin + 0.5f;
+            qa.sx1 = (float)axmax + 0.5f;
+            qa.sy0 = (float)aymin + 0.5f;
+            qa.sy1 = (float)aymax + 0.5f;
+        }
         for (int w = 0; w < kWords && !warp_done; ++w) {
             const int jl = w * 32 + lane;
-            const bool keep = jl < n && may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], q);
+            const bool keep = jl < n && may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], qa);
             unsigned m = __ballot_sync(0xffffffffu, keep);
+            unsigned blended_word = 0;  // bit l: staged Gaussian w*32+l blended some pixel of this warp
             while (m) {
                 const int jj = w * 32 + __ffs(m) - 1;
                 m &= m - 1;
@@ -131,10 +146,20 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 const unsigned pos = b - rg.x + (unsigned)jj + 1u;
                 if (blend0) { T.x = Tn.x; last0 = pos; }
                 if (blend1) { T.y = Tn.y; last1 = pos; }
+                if (__any_sync(0xffffffffu, blend0 || blend1)) blended_word |= 1u << (jj & 31);
                 if (__all_sync(0xffffffffu, done0 && done1)) {
                     warp_done = true;
                     break;
                 }
+            }
+            // record the word at global list positions b + w*32 .. b + w*32 + 31
+            // (bit for position k: word (k >> 5) * 4 + warp, bit k & 31)
+            if (cmask && blended_word && lane == 0) {
+                const unsigned k0 = b + (unsigned)(w * 32);
+                const unsigned o = k0 & 31u;
+                const unsigned wi = (k0 >> 5) * kWarps + (threadIdx.x >> 5);
+                if (wi < cmask_words) atomicOr(&cmask[wi], blended_word << o);
+                if (o && wi + kWarps < cmask_words) atomicOr(&cmask[wi + kWarps], blended_word >> (32u - o));
             }
         }
     }
@@ -190,9 +215,9 @@ __global__ void __launch_bounds__(kThreads)
 k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
              const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
              const float* __restrict__ colors, const float* __restrict__ final_T,
-             const unsigned* __restrict__ n_contrib, const float* __restrict__ dL_dimage,
-             float2* __restrict__ dL_dmean2d, float4* __restrict__ dL_dconic_opacity,
-             float* __restrict__ dL_dcolor) {
+             const unsigned* __restrict__ n_contrib, const unsigned* __restrict__ cmask, unsigned cmask_words,
+             const float* __restrict__ dL_dimage, float2* __restrict__ dL_dmean2d,
+             float4* __restrict__ dL_dconic_opacity, float* __restrict__ dL_dcolor) {
     __shared__ unsigned s_id[kBatch];
     __shared__ float2 s_xy[kBatch];
     __shared__ float4 s_co[kBatch];
@@ -238,7 +263,23 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     for (int w = 0; w < kWarps; ++w) max_last = max(max_last, s_max[w]);
     max_last = min(max_last, rg.y - rg.x);  // stay inside the tile's list
 
+    const int warp = threadIdx.x >> 5;
     for (int top = (int)max_last; top > 0; top -= kBatch) {
+        // the forward's contribution bits for this batch, loaded early so that
+        // their latency overlaps the staging below
+        unsigned mbits = 0;  // bit w: staged Gaussian w * 32 + lane blended a pixel of this warp
+        if (cmask) {
+#pragma unroll
+            for (int w = 0; w < kWords; ++w) {
+                const int p = top - 1 - (w * 32 + lane);
+                if (p >= 0) {
+                    const unsigned k = rg.x + (unsigned)p;
+                    const unsigned wi = (k >> 5) * kWarps + warp;
+                    const unsigned bit = wi >= cmask_words || ((cmask[wi] >> (k & 31u)) & 1u);
+                    mbits |= bit << w;
+                }
+            }
+        }
         // stage positions top-1, top-2, ... so that staged order is back to front
         for (int r = threadIdx.x; r < kBatch; r += kThreads) {
             const int pos = top - 1 - r;
@@ -258,8 +299,13 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
         const int n = min(kBatch, top);
         for (int w = 0; w < kWords; ++w) {
             const int jl = w * 32 + lane;
-            const bool keep = jl < n && top - 1 - jl < (int)wlast &&
-                              may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], q);
+            const int p = top - 1 - jl;
+            bool keep = jl < n && p < (int)wlast;
+            if (cmask) {
+                keep = keep && ((mbits >> w) & 1u);
+            } else {
+                keep = keep && may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], q);
+            }
             unsigned m = __ballot_sync(0xffffffffu, keep);
             while (m) {
                 const int jj = w * 32 + __ffs(m) - 1;
@@ -396,22 +442,32 @@ using namespace gs;
 
 extern "C" int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const unsigned* ids, const float* mean2d,
                              const float* conic_opacity, const float* colors, float* image, float* final_T,
-                             unsigned* n_contrib, void* stream) {
+                             unsigned* n_contrib, unsigned* contrib_mask, unsigned mask_words, void* stream) {
     if (!camera_ok(cam) || !ranges || !image || !final_T || !n_contrib) return GS_ERR_INVALID_ARG;
+    if (contrib_mask && (mask_words == 0 || mask_words % kWarps != 0)) return GS_ERR_INVALID_ARG;
     if (!aligned(ranges, 8) || (conic_opacity && !aligned(conic_opacity, 16)) || (mean2d && !aligned(mean2d, 8)))
         return GS_ERR_INVALID_ARG;
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
-    k_render_fwd<<<T, kThreads, 0, (cudaStream_t)stream>>>(
+    cudaStream_t st = (cudaStream_t)stream;
+    if (contrib_mask) {
+        int blocks = (int)((mask_words + 255u) / 256u);
+        if (blocks > 148 * 8) blocks = 148 * 8;
+        k_zero<<<blocks, 256, 0, st>>>(reinterpret_cast<float*>(contrib_mask), mask_words, nullptr, 0, nullptr, 0);
+        GS_LAUNCH_CHECK();
+    }
+    k_render_fwd<<<T, kThreads, 0, st>>>(
         *cam, TX, reinterpret_cast<const uint2*>(ranges), ids, reinterpret_cast<const float2*>(mean2d),
-        reinterpret_cast<const float4*>(conic_opacity), colors, image, final_T, n_contrib);
+        reinterpret_cast<const float4*>(conic_opacity), colors, image, final_T, n_contrib, contrib_mask,
+        contrib_mask ? mask_words : 0u);
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
 
 extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges, const unsigned* ids,
                              const float* mean2d, const float* conic_opacity, const float* colors,
-                             const float* final_T, const unsigned* n_contrib, const float* dL_dimage,
-                             float* dL_dmean2d, float* dL_dconic_opacity, float* dL_dcolor, void* stream) {
+                             const float* final_T, const unsigned* n_contrib, const unsigned* contrib_mask,
+                             unsigned mask_words, const float* dL_dimage, float* dL_dmean2d,
+                             float* dL_dconic_opacity, float* dL_dcolor, void* stream) {
     if (!camera_ok(cam) || N < 0 || !ranges || !final_T || !n_contrib || !dL_dimage) return GS_ERR_INVALID_ARG;
     if (N > 0 && (!dL_dmean2d || !dL_dconic_opacity || !dL_dcolor)) return GS_ERR_INVALID_ARG;
     if (!aligned(ranges, 8) || (conic_opacity && !aligned(conic_opacity, 16)) || (mean2d && !aligned(mean2d, 8)) ||
@@ -430,7 +486,7 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
     k_render_bwd<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
                                        reinterpret_cast<const float2*>(mean2d),
                                        reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
-                                       dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),
+                                       contrib_mask, contrib_mask ? mask_words : 0u, dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),
                                        reinterpret_cast<float4*>(dL_dconic_opacity), dL_dcolor);
     GS_LAUNCH_CHECK();
     return GS_OK;

@@ -32,6 +32,7 @@ class Frame:
     image: torch.Tensor
     final_T: torch.Tensor
     n_contrib: torch.Tensor
+    contrib_mask: Optional[torch.Tensor]
 
 
 class Rasterizer:
@@ -81,7 +82,7 @@ class Rasterizer:
         return out
 
     def forward(self, means, scales, quats, opacity, colors, capacity: Optional[int] = None,
-                want_keys: bool = False, stream=None) -> Frame:
+                want_keys: bool = False, use_mask: bool = True, stream=None) -> Frame:
         """Preprocess, bin/sort and composite one frame.
 
         With ``capacity=None`` the pair count is read back to size the sort
@@ -103,10 +104,11 @@ class Rasterizer:
         image = self._buf("image", (3, H, W), torch.float32)
         final_T = self._buf("final_T", (H, W), torch.float32)
         n_contrib = self._buf("n_contrib", (H, W), torch.uint32)
+        cmask = self._buf("contrib_mask", (B.mask_words(max(capacity, 1)),), torch.uint32) if use_mask else None
         B.gs_render_fwd(self.cam, ranges, ids, pre["mean2d"], pre["conic_opacity"], colors, image, final_T,
-                        n_contrib, stream)
+                        n_contrib, cmask, stream)
         return Frame(N=N, capacity=capacity, ids=ids, ranges=ranges, keys=keys, image=image, final_T=final_T,
-                     n_contrib=n_contrib, **pre)
+                     n_contrib=n_contrib, contrib_mask=cmask, **pre)
 
     def backward(self, frame: Frame, means, scales, quats, colors, dL_dimage,
                  grads: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
@@ -118,7 +120,7 @@ class Rasterizer:
                   dL_dcolor=self._buf("dL_dcolor", (N, 3), torch.float32))
         B.gs_render_bwd(self.cam, frame.ranges, frame.ids, frame.mean2d, frame.conic_opacity, colors, frame.final_T,
                         frame.n_contrib, dL_dimage, g2["dL_dmean2d"], g2["dL_dconic_opacity"], g2["dL_dcolor"],
-                        stream)
+                        frame.contrib_mask, stream)
         if grads is None:
             grads = zero_grads(N, self.device)
         B.gs_preprocess_bwd(self.cam, means, scales, quats, frame.radius, frame.conic_opacity, g2["dL_dmean2d"],

@@ -197,10 +197,20 @@ GS_API int gs_bin_sort(const gs_camera* cam, int N, const float* depth, const in
  * Outputs: image [3,H,W]; final_T [H,W]; n_contrib [H,W] uint32 = list
  *   position (within the tile) of the last blended term plus one.
  * colors [N,3] are indexed by the ids in `ids`.
+ * contrib_mask (optional, may be NULL) receives, for every sorted position k
+ *   and every 8x8 quadrant q of k's tile (row-major: top-left, top-right,
+ *   bottom-left, bottom-right), bit (k & 31) of word (k >> 5) * 4 + q set when
+ *   that Gaussian was blended into at least one pixel of the quadrant.  The
+ *   call zeroes the first `mask_words` words, which must be a multiple of 4 and
+ *   at least GS_MASK_WORDS(number of sorted pairs).  gs_render_bwd uses it to
+ *   walk only the terms that contribute.
  */
+/* Words of the optional contribution mask for `capacity` sorted pairs. */
+#define GS_MASK_WORDS(capacity) (4u * (((unsigned)(capacity) + 31u) / 32u))
+
 GS_API int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const unsigned* ids, const float* mean2d,
                   const float* conic_opacity, const float* colors, float* image, float* final_T,
-                  unsigned* n_contrib, void* stream);
+                  unsigned* n_contrib, unsigned* contrib_mask, unsigned mask_words, void* stream);
 
 /*
  * gs_render_stats - work counts of gs_render_fwd, per pixel (the derived
@@ -222,6 +232,9 @@ GS_API int gs_render_stats(const gs_camera* cam, const unsigned* ranges, const u
  *   the alpha_max cap is active) to dL/dopacity and dL/dG, then
  *   dL/d(a, b, c) = G dL/dG (-dx^2/2, -dx dy, -dy^2/2) and
  *   dL/d(u, v) = G dL/dG (a dx + b dy, b dx + c dy).
+ * contrib_mask / mask_words: the forward's mask (see gs_render_fwd), or NULL
+ *   to let the backward find the contributing terms itself (slower; same
+ *   results up to the order of floating-point sums).
  * Outputs (OVERWRITTEN; the call zeroes them first): dL_dmean2d [N,2];
  *   dL_dconic_opacity [N,4] = (dL/da, dL/db, dL/dc, dL/dopacity);
  *   dL_dcolor [N,3].  Summation order across pixels is unspecified
@@ -229,8 +242,9 @@ GS_API int gs_render_stats(const gs_camera* cam, const unsigned* ranges, const u
  */
 GS_API int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges, const unsigned* ids,
                   const float* mean2d, const float* conic_opacity, const float* colors,
-                  const float* final_T, const unsigned* n_contrib, const float* dL_dimage,
-                  float* dL_dmean2d, float* dL_dconic_opacity, float* dL_dcolor, void* stream);
+                  const float* final_T, const unsigned* n_contrib, const unsigned* contrib_mask,
+                  unsigned mask_words, const float* dL_dimage, float* dL_dmean2d, float* dL_dconic_opacity,
+                  float* dL_dcolor, void* stream);
 
 /*
  * gs_preprocess_bwd - 2D gradients to 3D parameters by the chain rule

@@ -72,7 +72,7 @@ def lib():
             getattr(L, f"oracle_bin_{suf}").restype = ctypes.c_longlong
             getattr(L, f"oracle_tile_list_{suf}").argtypes = [cam, I, P, P, P, I, P]
             getattr(L, f"oracle_tile_list_{suf}").restype = ctypes.c_longlong
-            getattr(L, f"oracle_render_fwd_{suf}").argtypes = [cam] + [P] * 11 + [I]
+            getattr(L, f"oracle_render_fwd_{suf}").argtypes = [cam] + [P] * 12 + [I]
             getattr(L, f"oracle_render_fwd_{suf}").restype = None
             getattr(L, f"oracle_render_bwd_{suf}").argtypes = [cam, I] + [P] * 10 + [I]
             getattr(L, f"oracle_render_bwd_{suf}").restype = None
@@ -164,7 +164,11 @@ def tile_list(cam, depth, rect, tiles_touched, tile: int, mode: str = "f32") -> 
 
 
 def render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, mode: str = "f32",
-               tiles: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray]:
+               tiles: Optional[Sequence[int]] = None, blend_mask: bool = False) -> Dict[str, np.ndarray]:
+    """Compositing forward.  With ``blend_mask``, also the per-quadrant mask:
+    for sorted position k and 8x8 quadrant q of k's tile, bit (k & 31) of
+    word (k >> 5) * 4 + q is set when that term was blended into a pixel of
+    the quadrant."""
     dt = _dt(mode)
     ranges = _a(ranges, np.uint32)
     ids = _a(ids, np.uint32)
@@ -173,12 +177,14 @@ def render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, mode: str = "f32
     out = dict(image=np.zeros((3, H, W), dt), final_T=np.zeros((H, W), dt),
                n_contrib=np.zeros((H, W), np.uint32), n_eval=np.zeros((H, W), np.uint32),
                n_blended=np.zeros((H, W), np.uint32))
+    if blend_mask:
+        out["blend_mask"] = np.zeros(4 * ((ids.size + 31) // 32), np.uint32)
     sub = None if tiles is None else _a(tiles, np.int32)
     oc = camera(cam)
     getattr(lib(), f"oracle_render_fwd_{mode}")(
         ctypes.byref(oc), _p(ranges), _p(ids), _p(mean2d), _p(conic_opacity), _p(colors), _p(out["image"]),
-        _p(out["final_T"]), _p(out["n_contrib"]), _p(out["n_eval"]), _p(out["n_blended"]), _p(sub),
-        0 if sub is None else sub.size)
+        _p(out["final_T"]), _p(out["n_contrib"]), _p(out["n_eval"]), _p(out["n_blended"]),
+        _p(out.get("blend_mask")), _p(sub), 0 if sub is None else sub.size)
     return out
 
 

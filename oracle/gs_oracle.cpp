@@ -368,7 +368,7 @@ void tiles_of(const oracle_camera* cam, const int* subset, int n_subset, std::ve
 template <typename Real>
 void render_fwd(const oracle_camera* cam, const unsigned* ranges, const unsigned* ids, const Real* mean2d,
                 const Real* conic_opacity, const Real* colors, Real* image, Real* final_T, unsigned* n_contrib,
-                unsigned* n_eval, unsigned* n_blend, const int* subset, int n_subset) {
+                unsigned* n_eval, unsigned* n_blend, unsigned* blend_mask, const int* subset, int n_subset) {
     const int W = cam->width, H = cam->height, TS = cam->tile;
     const int TX = (W + TS - 1) / TS;
     std::vector<int> tiles;
@@ -394,6 +394,14 @@ void render_fwd(const oracle_camera* cam, const unsigned* ranges, const unsigned
                     T = Tn;
                     last = k - r0 + 1;
                     ++blended;
+                    if (blend_mask) {
+                        // bit k of the 8x8 quadrant of the tile this pixel lies in
+                        const unsigned quad = (unsigned)(((y % TS) / 8) * 2 + ((x % TS) / 8));
+                        unsigned* word = blend_mask + (size_t)(k >> 5) * 4 + quad;
+                        const unsigned bit = 1u << (k & 31u);
+#pragma omp atomic
+                        *word |= bit;
+                    }
                 }
                 const size_t pix = (size_t)y * W + x;
                 for (int ch = 0; ch < 3; ++ch) image[(size_t)ch * H * W + pix] = C[ch] + T * Real(cam->bg[ch]);
@@ -681,9 +689,9 @@ void oracle_set_threads(int n) {
     void oracle_render_fwd_##SUF(const oracle_camera* cam, const unsigned* ranges, const unsigned* ids,      \
                                  const R* mean2d, const R* conic_opacity, const R* colors, R* image,         \
                                  R* final_T, unsigned* n_contrib, unsigned* n_eval, unsigned* n_blend,       \
-                                 const int* subset, int n_subset) {                                          \
+                                 unsigned* blend_mask, const int* subset, int n_subset) {                    \
         render_fwd<R>(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_T, n_contrib, n_eval,    \
-                      n_blend, subset, n_subset);                                                            \
+                      n_blend, blend_mask, subset, n_subset);                                                \
     }                                                                                                        \
     void oracle_render_bwd_##SUF(const oracle_camera* cam, int N, const unsigned* ranges, const unsigned* ids, \
                                  const R* mean2d, const R* conic_opacity, const R* colors,                   \

@@ -63,7 +63,7 @@ def test_host_argument_checks_need_no_device(lib):
     rc = lib.gs_preprocess_fwd(ctypes.byref(cam), 0, *([None] * 11), None, 0, None)
     assert rc == B.GS_ERR_INVALID_ARG
     cam.tile = 16
-    rc = lib.gs_render_fwd(ctypes.byref(cam), *([None] * 8), None)
+    rc = lib.gs_render_fwd(ctypes.byref(cam), *([None] * 9), 0, None)
     assert rc == B.GS_ERR_INVALID_ARG
     rc = lib.gs_bin_sort(ctypes.byref(cam), -1, None, None, None, None, 0, None, None, None, None, 0, None)
     assert rc == B.GS_ERR_INVALID_ARG

@@ -318,3 +318,27 @@ def test_render_stats_match_oracle_counts(cfg):
     np.testing.assert_array_equal(to_np(ne), o["n_eval"])
     np.testing.assert_array_equal(to_np(nb), o["n_blended"])
     assert np.all(to_np(nb) <= g["n_contrib"])
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_contribution_mask_and_backward_without_it(cfg):
+    """The forward's per-quadrant contribution mask equals the oracle's bit for
+    bit, and the backward gives the same gradients with and without it."""
+    sc = _scene(cfg)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    r = run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0], want_keys=False)
+    fr = r["frame"]
+    g = frame_np(fr)
+    P = g["num_pairs"]
+    o = oracle.render_fwd(cam, g["ranges"], g["ids"], g["mean2d"], g["conic_opacity"], sc.colors, "f32",
+                          blend_mask=True)
+    words = 4 * ((P + 31) // 32)
+    np.testing.assert_array_equal(to_np(fr.contrib_mask)[:words], o["blend_mask"][:words])
+    with_mask = {k: to_np(r["grads"][k]).copy() for k in ("dL_dmean2d", "dL_dconic_opacity", "dL_dcolor")}
+    outs = {k: torch.empty_like(r["grads"][k]) for k in with_mask}
+    B.gs_render_bwd(cam, fr.ranges, fr.ids, fr.mean2d, fr.conic_opacity, gs.colors, fr.final_T, fr.n_contrib,
+                    to_dev(sc.dL_dimage[0]), outs["dL_dmean2d"], outs["dL_dconic_opacity"], outs["dL_dcolor"], None)
+    torch.cuda.synchronize()
+    for k in with_mask:
+        assert rel_l2(to_np(outs[k]), with_mask[k]) <= 1e-5, k
