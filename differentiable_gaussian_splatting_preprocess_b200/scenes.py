@@ -234,3 +234,13 @@ def random_tiny(n: int = 6, width: int = 32, height: int = 32, seed: int = 0,
                  quats=quats.astype(np.float32), opacity=opacity.astype(np.float32),
                  colors=colors.astype(np.float32), cameras=[cam],
                  dL_dimage=[dl.astype(np.float32)])
+
+
+def random_sh(n: int, degree: int, seed: int = 0, dc_max: float = 3.0, rest_std: float = 0.2) -> np.ndarray:
+    """Seeded spherical-harmonics coefficients [n, (degree+1)^2, 3] (float32):
+    the constant band uniform in [0, dc_max), the others normal(0, rest_std)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    K = (degree + 1) ** 2
+    sh = rng.normal(0.0, rest_std, size=(n, K, 3))
+    sh[:, 0, :] = rng.uniform(0.0, dc_max, size=(n, 3))
+    return np.ascontiguousarray(sh, dtype=np.float32)

@@ -78,6 +78,13 @@ def lib():
             getattr(L, f"oracle_render_bwd_{suf}").restype = None
             getattr(L, f"oracle_preprocess_bwd_{suf}").argtypes = [cam, I] + [P] * 12
             getattr(L, f"oracle_preprocess_bwd_{suf}").restype = None
+        for suf, R in (("f32", ctypes.c_float), ("f64", ctypes.c_double)):
+            getattr(L, f"oracle_sh_fwd_{suf}").argtypes = [cam, I, I, I, P, P, R, P]
+            getattr(L, f"oracle_sh_fwd_{suf}").restype = None
+            getattr(L, f"oracle_sh_bwd_{suf}").argtypes = [cam, I, I, I, P, P, R, P, P, P]
+            getattr(L, f"oracle_sh_bwd_{suf}").restype = None
+            getattr(L, f"oracle_sh_basis_{suf}").argtypes = [I, P, P]
+            getattr(L, f"oracle_sh_basis_{suf}").restype = None
         L.oracle_exp_f32.argtypes = [P, P, ctypes.c_longlong]
         L.oracle_exp_f32.restype = None
         L.oracle_num_threads.restype = I
@@ -245,3 +252,39 @@ def forward_backward(cam, means, scales, quats, opacity, colors, dL_dimage, mode
     f.update(g2)
     f.update(g3)
     return f
+
+
+# --------------------------------------------------------------------------
+# Spherical-harmonics colour
+# --------------------------------------------------------------------------
+
+def sh_basis(dirs, mode: str = "f64") -> np.ndarray:
+    """The 16 real SH basis values (degree <= 3) at unit directions [n, 3]."""
+    dt = _dt(mode)
+    d = _a(dirs, dt).reshape(-1, 3)
+    out = np.zeros((d.shape[0], 16), dt)
+    getattr(lib(), f"oracle_sh_basis_{mode}")(d.shape[0], _p(d), _p(out))
+    return out
+
+
+def sh_fwd(cam, means, sh, degree: int, offset: float = 0.0, mode: str = "f64") -> np.ndarray:
+    dt = _dt(mode)
+    means, sh = _a(means, dt), _a(sh, dt)
+    n, K = means.shape[0], sh.shape[1]
+    out = np.zeros((n, 3), dt)
+    oc = camera(cam)
+    getattr(lib(), f"oracle_sh_fwd_{mode}")(ctypes.byref(oc), n, int(degree), K, _p(means), _p(sh), float(offset),
+                                            _p(out))
+    return out
+
+
+def sh_bwd(cam, means, sh, degree: int, dL_dcolors, offset: float = 0.0, mode: str = "f64",
+           accumulate_into: Optional[Dict[str, np.ndarray]] = None) -> Dict[str, np.ndarray]:
+    dt = _dt(mode)
+    means, sh, g = _a(means, dt), _a(sh, dt), _a(dL_dcolors, dt)
+    n, K = means.shape[0], sh.shape[1]
+    out = accumulate_into or dict(dL_dsh=np.zeros_like(sh), dL_dmeans=np.zeros_like(means))
+    oc = camera(cam)
+    getattr(lib(), f"oracle_sh_bwd_{mode}")(ctypes.byref(oc), n, int(degree), K, _p(means), _p(sh), float(offset),
+                                            _p(g), _p(out["dL_dsh"]), _p(out["dL_dmeans"]))
+    return out

@@ -644,6 +644,122 @@ void preprocess_bwd(const oracle_camera* cam, int N, const Real* means, const Re
     }
 }
 
+// ---------------------------------------------------------------------------
+// Colour from real spherical harmonics ("Gaussian Splatting反向传播的CUDA实现",
+// section 4: the colour gradient reaches the SH coefficients through the
+// derivative of the SH basis, band-limited).  Reading: the orthonormal real SH
+// of degree <= 3 in Cartesian form on the unit view direction d = (x, y, z),
+// coefficients ordered k = l^2 + l + m; colour = max(0, sum_k Y_k(d) sh_k +
+// offset) per channel, d = normalise(mean - camera centre), camera centre
+// = -R^T t.  The clamp at 0 is the constraint; its derivative is 0 where it
+// is active.
+// ---------------------------------------------------------------------------
+template <typename Real>
+void sh_basis(const Real d[3], int degree, Real Y[16], Real dY[16][3]) {
+    const Real x = d[0], y = d[1], z = d[2];
+    const Real C0 = Real(0.28209479177387814), C1 = Real(0.4886025119029199);
+    const Real C2a = Real(1.0925484305920792), C2b = Real(0.31539156525252005), C2c = Real(0.5462742152960396);
+    const Real C3a = Real(0.5900435899266435), C3b = Real(2.890611442640554), C3c = Real(0.4570457994644658);
+    const Real C3d = Real(0.3731763325901154), C3e = Real(1.445305721320277);
+    for (int k = 0; k < 16; ++k) {
+        Y[k] = Real(0);
+        dY[k][0] = dY[k][1] = dY[k][2] = Real(0);
+    }
+    Y[0] = C0;
+    if (degree < 1) return;
+    Y[1] = C1 * y;  dY[1][1] = C1;
+    Y[2] = C1 * z;  dY[2][2] = C1;
+    Y[3] = C1 * x;  dY[3][0] = C1;
+    if (degree < 2) return;
+    Y[4] = C2a * x * y;               dY[4][0] = C2a * y;  dY[4][1] = C2a * x;
+    Y[5] = C2a * y * z;               dY[5][1] = C2a * z;  dY[5][2] = C2a * y;
+    Y[6] = C2b * (3 * z * z - 1);     dY[6][2] = C2b * 6 * z;
+    Y[7] = C2a * x * z;               dY[7][0] = C2a * z;  dY[7][2] = C2a * x;
+    Y[8] = C2c * (x * x - y * y);     dY[8][0] = C2c * 2 * x;  dY[8][1] = -C2c * 2 * y;
+    if (degree < 3) return;
+    Y[9] = C3a * y * (3 * x * x - y * y);
+    dY[9][0] = C3a * 6 * x * y;  dY[9][1] = C3a * (3 * x * x - 3 * y * y);
+    Y[10] = C3b * x * y * z;
+    dY[10][0] = C3b * y * z;  dY[10][1] = C3b * x * z;  dY[10][2] = C3b * x * y;
+    Y[11] = C3c * y * (5 * z * z - 1);
+    dY[11][1] = C3c * (5 * z * z - 1);  dY[11][2] = C3c * 10 * y * z;
+    Y[12] = C3d * z * (5 * z * z - 3);
+    dY[12][2] = C3d * (15 * z * z - 3);
+    Y[13] = C3c * x * (5 * z * z - 1);
+    dY[13][0] = C3c * (5 * z * z - 1);  dY[13][2] = C3c * 10 * x * z;
+    Y[14] = C3e * z * (x * x - y * y);
+    dY[14][0] = C3e * 2 * x * z;  dY[14][1] = -C3e * 2 * y * z;  dY[14][2] = C3e * (x * x - y * y);
+    Y[15] = C3a * x * (x * x - 3 * y * y);
+    dY[15][0] = C3a * (3 * x * x - 3 * y * y);  dY[15][1] = -C3a * 6 * x * y;
+}
+
+template <typename Real>
+void view_dir(const oracle_camera& cam, const Real* mu, Real v[3], Real d[3], Real& norm) {
+    for (int j = 0; j < 3; ++j) {
+        Real c = 0;
+        for (int i = 0; i < 3; ++i) c -= Real(cam.R[3 * i + j]) * Real(cam.t[i]);  // camera centre -R^T t
+        v[j] = mu[j] - c;
+    }
+    norm = std::sqrt(v[0] * v[0] + v[1] * v[1] + v[2] * v[2]);
+    for (int j = 0; j < 3; ++j) d[j] = v[j] / norm;
+}
+
+template <typename Real>
+void sh_fwd(const oracle_camera* cam, int N, int degree, int K, const Real* means, const Real* sh, Real offset,
+            Real* colors) {
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < N; ++i) {
+        Real v[3], d[3], nrm, Y[16], dY[16][3];
+        view_dir(*cam, means + 3 * i, v, d, nrm);
+        sh_basis(d, degree, Y, dY);
+        const int nk = (degree + 1) * (degree + 1);
+        for (int ch = 0; ch < 3; ++ch) {
+            Real acc = 0;
+            for (int k = 0; k < nk; ++k) acc += Y[k] * sh[((size_t)i * K + k) * 3 + ch];
+            colors[3 * i + ch] = std::max(acc + offset, Real(0));
+        }
+    }
+}
+
+template <typename Real>
+void sh_bwd(const oracle_camera* cam, int N, int degree, int K, const Real* means, const Real* sh, Real offset,
+            const Real* dL_dcolors, Real* dL_dsh, Real* dL_dmeans) {
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < N; ++i) {
+        Real v[3], d[3], nrm, Y[16], dY[16][3];
+        view_dir(*cam, means + 3 * i, v, d, nrm);
+        sh_basis(d, degree, Y, dY);
+        const int nk = (degree + 1) * (degree + 1);
+        Real g[3];
+        for (int ch = 0; ch < 3; ++ch) {
+            Real acc = 0;
+            for (int k = 0; k < nk; ++k) acc += Y[k] * sh[((size_t)i * K + k) * 3 + ch];
+            g[ch] = (acc + offset > Real(0)) ? dL_dcolors[3 * i + ch] : Real(0);  // clamp active: no gradient
+        }
+        Real dd[3] = {0, 0, 0};  // dL/d(direction), treating (x, y, z) as free
+        for (int k = 0; k < nk; ++k) {
+            Real s = 0;
+            for (int ch = 0; ch < 3; ++ch) {
+                dL_dsh[((size_t)i * K + k) * 3 + ch] += Y[k] * g[ch];
+                s += sh[((size_t)i * K + k) * 3 + ch] * g[ch];
+            }
+            for (int j = 0; j < 3; ++j) dd[j] += dY[k][j] * s;
+        }
+        // d = v / |v|: dL/dv = (I - d d^T) dL/dd / |v|, and v = mean - centre
+        const Real dot = d[0] * dd[0] + d[1] * dd[1] + d[2] * dd[2];
+        for (int j = 0; j < 3; ++j) dL_dmeans[3 * i + j] += (dd[j] - d[j] * dot) / nrm;
+    }
+}
+
+template <typename Real>
+void sh_basis_eval(int n, const Real* dirs, Real* out) {
+    for (int i = 0; i < n; ++i) {
+        Real Y[16], dY[16][3];
+        sh_basis(dirs + 3 * i, 3, Y, dY);
+        for (int k = 0; k < 16; ++k) out[16 * i + k] = Y[k];
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -709,5 +825,18 @@ void oracle_set_threads(int n) {
     }
 
 ORACLE_BOTH(DEF_PRE)
+
+#define DEF_SH(R, SUF)                                                                                        \
+    void oracle_sh_fwd_##SUF(const oracle_camera* cam, int N, int degree, int K, const R* means, const R* sh, \
+                             R offset, R* colors) {                                                          \
+        sh_fwd<R>(cam, N, degree, K, means, sh, offset, colors);                                             \
+    }                                                                                                        \
+    void oracle_sh_bwd_##SUF(const oracle_camera* cam, int N, int degree, int K, const R* means, const R* sh, \
+                             R offset, const R* dL_dcolors, R* dL_dsh, R* dL_dmeans) {                       \
+        sh_bwd<R>(cam, N, degree, K, means, sh, offset, dL_dcolors, dL_dsh, dL_dmeans);                      \
+    }                                                                                                        \
+    void oracle_sh_basis_##SUF(int n, const R* dirs, R* out) { sh_basis_eval<R>(n, dirs, out); }
+
+ORACLE_BOTH(DEF_SH)
 
 }  // extern "C"
