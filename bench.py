@@ -214,11 +214,24 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stages = ["preprocess_fwd", "bin_sort", "render_fwd", "render_bwd", "preprocess_bwd"]
+    sh_deg = args.sh_degree
+    if sh_deg is not None:
+        from differentiable_gaussian_splatting_preprocess_b200 import scenes as _scn
+        shd = torch.from_numpy(_scn.random_sh(sc.N, sh_deg, seed=1)).to(dev)
+        dsh = torch.zeros_like(shd)
+        colors = torch.empty((sc.N, 3), dtype=torch.float32, device=dev)
+        stages = ["sh_fwd"] + stages + ["sh_bwd"]
 
     def step(ev=None):
-        def mark(i):
+        marks = [0]
+
+        def mark(i=None):
             if ev is not None:
-                ev[i].record(stream)
+                ev[marks[0]].record(stream)
+            marks[0] += 1
+        if sh_deg is not None:
+            mark()
+            B.gs_sh_fwd(cam, sh_deg, means, shd, colors, offset=0.5)
         mark(0)
         pre = rz.preprocess(means, scales, quats, opacity)
         mark(1)
@@ -237,6 +250,9 @@ def run_ours(args):
                             rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"], grads["dL_dmeans"],
                             grads["dL_dscales"], grads["dL_dquats"], grads["dL_dopacity"], grads["dL_dcolors"])
         mark(5)
+        if sh_deg is not None:
+            B.gs_sh_bwd(cam, sh_deg, means, shd, grads["dL_dcolors"], dsh, grads["dL_dmeans"], offset=0.5)
+            mark()
 
     rz.backward(fr, means, scales, quats, colors, dL)  # allocate the 2D gradient buffers
     for _ in range(args.warmup):
@@ -256,7 +272,7 @@ def run_ours(args):
     evals_per_frame = n_evaluated + n_contrib
 
     sampler = ClockSampler(local)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -275,7 +291,7 @@ def run_ours(args):
     for ev in events:
         for i, s in enumerate(stages):
             stage_ms[s].append(ev[i].elapsed_time(ev[i + 1]))
-        step_ms.append(ev[0].elapsed_time(ev[5]))
+        step_ms.append(ev[0].elapsed_time(ev[len(stages)]))
     total_ms = sum(step_ms)
     if world > 1:
         tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
@@ -290,7 +306,7 @@ def run_ours(args):
     T = B.num_tiles(cam)
     tile_bits = max(0, (T - 1).bit_length())
     tpasses = (tile_bits + 7) // 8
-    launches = 1 + (1 + 4 * 3 + 3 + 1 + 3 * tpasses + 1) + 2 + 2 + 1
+    launches = 1 + (1 + 4 * 3 + 3 + 1 + 3 * tpasses + 1) + 2 + 2 + 1 + (2 if sh_deg is not None else 0)
 
     # roofline of the dominant kernel (render backward: FP32 ALU bound)
     peaks = _peaks()
@@ -368,7 +384,8 @@ def run_ours(args):
             metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
             ms_per_step=total_ms / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,
             dtype="f32", data="synthetic",
-            config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam.width}x{cam.height}, 16x16 tiles, fp32",
+            config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam.width}x{cam.height}, 16x16 tiles, fp32"
+                                 + (f", SH degree {sh_deg} colours" if sh_deg is not None else ""),
                         num_pairs=P, evals_per_frame=evals_per_frame, evaluated_fwd=n_evaluated,
                         contributor_prefix_bwd=n_contrib, blended=n_blended,
                         l2="flushed between steps (256 MiB write)",
@@ -396,6 +413,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sh-degree", type=int, default=None,
+                    help="colours from spherical harmonics of this degree (adds the SH stages to the step)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -31,7 +31,7 @@ TILE = 16
 # Every symbol include/gs.h declares.
 EXPORTED = ("gs_version", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
             "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd",
-            "gs_preprocess_fwd_noalloc", "gs_render_stats")
+            "gs_preprocess_fwd_noalloc", "gs_render_stats", "gs_sh_fwd", "gs_sh_bwd")
 
 
 class GsCamera(ctypes.Structure):
@@ -85,8 +85,12 @@ def lib() -> ctypes.CDLL:
         L.gs_render_stats.argtypes = [cam] + [P] * 6 + [P]
         L.gs_render_bwd.restype = I
         L.gs_render_bwd.argtypes = [cam, I] + [P] * 8 + [U] + [P] * 4 + [P]
+        L.gs_sh_fwd.restype = I
+        L.gs_sh_fwd.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P]
+        L.gs_sh_bwd.restype = I
+        L.gs_sh_bwd.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P, P, P]
         L.gs_preprocess_bwd.restype = I
-        L.gs_preprocess_bwd.argtypes = [cam, I] + [P] * 13 + [P]
+        L.gs_preprocess_bwd.argtypes = [cam, I] + [P] * 15 + [P]
         _lib = L
     return _lib
 
@@ -269,7 +273,8 @@ def gs_render_bwd(cam, ranges, ids, mean2d, conic_opacity, colors, final_T, n_co
 
 
 def gs_preprocess_bwd(cam, means, scales, quats, radius, conic_opacity, dL_dmean2d, dL_dconic_opacity,
-                      dL_dcolor2d, dL_dmeans, dL_dscales, dL_dquats, dL_dopacity, dL_dcolors, stream=None) -> None:
+                      dL_dcolor2d, dL_dmeans, dL_dscales, dL_dquats, dL_dopacity, dL_dcolors, grad2d_accum=None,
+                      vis_count=None, stream=None) -> None:
     N = means.shape[0]
     f32 = torch.float32
     _check(means, "means", f32, (N, 3))
@@ -285,14 +290,45 @@ def gs_preprocess_bwd(cam, means, scales, quats, radius, conic_opacity, dL_dmean
     _check(dL_dquats, "dL_dquats", f32, (N, 4))
     _check(dL_dopacity, "dL_dopacity", f32, (N,))
     _check(dL_dcolors, "dL_dcolors", f32, (N, 3))
+    _check(grad2d_accum, "grad2d_accum", f32, (N,), optional=True)
+    _check(vis_count, "vis_count", torch.uint32, (N,), optional=True)
     c = camera_struct(cam)
     _ok("gs_preprocess_bwd", lib().gs_preprocess_bwd(
         ctypes.byref(c), int(N), _ptr(means), _ptr(scales), _ptr(quats), _ptr(radius), _ptr(conic_opacity),
         _ptr(dL_dmean2d), _ptr(dL_dconic_opacity), _ptr(dL_dcolor2d), _ptr(dL_dmeans), _ptr(dL_dscales),
-        _ptr(dL_dquats), _ptr(dL_dopacity), _ptr(dL_dcolors), _stream(stream)))
+        _ptr(dL_dquats), _ptr(dL_dopacity), _ptr(dL_dcolors), _ptr(grad2d_accum), _ptr(vis_count),
+        _stream(stream)))
 
 
 NOALLOC_MAX_GAUSSIANS = 1 << 24
+SH_MAX_DEGREE = 3
+
+
+def gs_sh_fwd(cam, degree: int, means, sh, colors, offset: float = 0.0, stream=None) -> None:
+    N = means.shape[0]
+    _check(means, "means", torch.float32, (N, 3))
+    _check(sh, "sh", torch.float32)
+    if sh.dim() != 3 or sh.shape[0] != N or sh.shape[2] != 3:
+        raise ValueError("sh must have shape [N, K, 3]")
+    _check(colors, "colors", torch.float32, (N, 3))
+    c = camera_struct(cam)
+    _ok("gs_sh_fwd", lib().gs_sh_fwd(ctypes.byref(c), int(N), int(degree), int(sh.shape[1]), _ptr(means), _ptr(sh),
+                                     float(offset), _ptr(colors), _stream(stream)))
+
+
+def gs_sh_bwd(cam, degree: int, means, sh, dL_dcolors, dL_dsh, dL_dmeans, offset: float = 0.0, stream=None) -> None:
+    N = means.shape[0]
+    _check(means, "means", torch.float32, (N, 3))
+    _check(sh, "sh", torch.float32)
+    if sh.dim() != 3 or sh.shape[0] != N or sh.shape[2] != 3:
+        raise ValueError("sh must have shape [N, K, 3]")
+    _check(dL_dcolors, "dL_dcolors", torch.float32, (N, 3))
+    _check(dL_dsh, "dL_dsh", torch.float32, tuple(sh.shape))
+    _check(dL_dmeans, "dL_dmeans", torch.float32, (N, 3))
+    c = camera_struct(cam)
+    _ok("gs_sh_bwd", lib().gs_sh_bwd(ctypes.byref(c), int(N), int(degree), int(sh.shape[1]), _ptr(means), _ptr(sh),
+                                     float(offset), _ptr(dL_dcolors), _ptr(dL_dsh), _ptr(dL_dmeans),
+                                     _stream(stream)))
 
 
 def gs_preprocess_fwd_noalloc(cam, means, scales, quats, opacity, mean2d, depth, conic_opacity, radius, rect,

@@ -218,9 +218,16 @@ k_preprocess_bwd(gs_camera cam, int N, const float* __restrict__ means, const fl
                  const float4* __restrict__ conic_opacity, const float2* __restrict__ dL_dmean2d,
                  const float4* __restrict__ dL_dconic_opacity, const float* __restrict__ dL_dcolor2d,
                  float* __restrict__ dL_dmeans, float* __restrict__ dL_dscales, float4* __restrict__ dL_dquats,
-                 float* __restrict__ dL_dopacity, float* __restrict__ dL_dcolors) {
+                 float* __restrict__ dL_dopacity, float* __restrict__ dL_dcolors, float* __restrict__ grad2d_accum,
+                 unsigned* __restrict__ vis_count) {
     const int i = blockIdx.x * kPreBlock + threadIdx.x;
     if (i >= N || radius[i] == 0) return;
+    if (grad2d_accum) {
+        // densification statistics: |dL/dmean2d| of this view, and one more view
+        const float2 g2 = dL_dmean2d[i];
+        grad2d_accum[i] += sqrtf(g2.x * g2.x + g2.y * g2.y);
+        vis_count[i] += 1u;
+    }
     const float* W = cam.R;
     const float mx = means[3 * i], my = means[3 * i + 1], mz = means[3 * i + 2];
     const float tx = W[0] * mx + W[1] * my + W[2] * mz + cam.t[0];
@@ -374,8 +381,9 @@ extern "C" int gs_preprocess_bwd(const gs_camera* cam, int N, const float* means
                                  const float* quats, const int* radius, const float* conic_opacity,
                                  const float* dL_dmean2d, const float* dL_dconic_opacity, const float* dL_dcolor2d,
                                  float* dL_dmeans, float* dL_dscales, float* dL_dquats, float* dL_dopacity,
-                                 float* dL_dcolors, void* stream) {
+                                 float* dL_dcolors, float* grad2d_accum, unsigned* vis_count, void* stream) {
     if (!camera_ok(cam) || N < 0) return GS_ERR_INVALID_ARG;
+    if ((grad2d_accum == nullptr) != (vis_count == nullptr)) return GS_ERR_INVALID_ARG;
     if (N == 0) return GS_OK;
     if (!means || !scales || !quats || !radius || !conic_opacity || !dL_dmean2d || !dL_dconic_opacity ||
         !dL_dcolor2d || !dL_dmeans || !dL_dscales || !dL_dquats || !dL_dopacity || !dL_dcolors)
@@ -388,7 +396,7 @@ extern "C" int gs_preprocess_bwd(const gs_camera* cam, int N, const float* means
         *cam, N, means, scales, reinterpret_cast<const float4*>(quats), radius,
         reinterpret_cast<const float4*>(conic_opacity), reinterpret_cast<const float2*>(dL_dmean2d),
         reinterpret_cast<const float4*>(dL_dconic_opacity), dL_dcolor2d, dL_dmeans, dL_dscales,
-        reinterpret_cast<float4*>(dL_dquats), dL_dopacity, dL_dcolors);
+        reinterpret_cast<float4*>(dL_dquats), dL_dopacity, dL_dcolors, grad2d_accum, vis_count);
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

@@ -111,9 +111,12 @@ class Rasterizer:
                      n_contrib=n_contrib, contrib_mask=cmask, **pre)
 
     def backward(self, frame: Frame, means, scales, quats, colors, dL_dimage,
-                 grads: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
+                 grads: Optional[Dict[str, torch.Tensor]] = None, densify: Optional[Dict[str, torch.Tensor]] = None,
+                 stream=None) -> Dict[str, torch.Tensor]:
         """Render backward then preprocess backward.  3D gradients are
-        accumulated into ``grads`` (zeros are allocated when it is None)."""
+        accumulated into ``grads`` (zeros are allocated when it is None).
+        With ``densify`` = dict(grad2d_accum=[N] float32, vis_count=[N] uint32),
+        the densification statistics of this view are accumulated too."""
         N = frame.N
         g2 = dict(dL_dmean2d=self._buf("dL_dmean2d", (N, 2), torch.float32),
                   dL_dconic_opacity=self._buf("dL_dconic_opacity", (N, 4), torch.float32),
@@ -125,7 +128,9 @@ class Rasterizer:
             grads = zero_grads(N, self.device)
         B.gs_preprocess_bwd(self.cam, means, scales, quats, frame.radius, frame.conic_opacity, g2["dL_dmean2d"],
                             g2["dL_dconic_opacity"], g2["dL_dcolor"], grads["dL_dmeans"], grads["dL_dscales"],
-                            grads["dL_dquats"], grads["dL_dopacity"], grads["dL_dcolors"], stream)
+                            grads["dL_dquats"], grads["dL_dopacity"], grads["dL_dcolors"],
+                            None if densify is None else densify["grad2d_accum"],
+                            None if densify is None else densify["vis_count"], stream)
         grads.update(g2)
         return grads
 

@@ -257,12 +257,39 @@ GS_API int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges, co
  * Outputs are ACCUMULATED (+=) so that several cameras can sum into one set:
  *   dL_dmeans [N,3], dL_dscales [N,3], dL_dquats [N,4], dL_dopacity [N],
  *   dL_dcolors [N,3].  Culled Gaussians (radius 0) are left untouched.
+ * grad2d_accum [N] / vis_count [N] (optional, both or neither; may be NULL):
+ *   densification statistics ([TR] D.1: the position gradient of each
+ *   Gaussian accumulated over the views): for every Gaussian visible in this
+ *   view, grad2d_accum += |dL/dmean2d| (Euclidean norm, pixels) and
+ *   vis_count += 1.  Their ratio is the mean view-space gradient norm.
  */
 GS_API int gs_preprocess_bwd(const gs_camera* cam, int N, const float* means, const float* scales,
                       const float* quats, const int* radius, const float* conic_opacity,
                       const float* dL_dmean2d, const float* dL_dconic_opacity, const float* dL_dcolor2d,
                       float* dL_dmeans, float* dL_dscales, float* dL_dquats, float* dL_dopacity,
-                      float* dL_dcolors, void* stream);
+                      float* dL_dcolors, float* grad2d_accum, unsigned* vis_count, void* stream);
+
+/*
+ * gs_sh_fwd / gs_sh_bwd - colour from real spherical harmonics ([CB] 4: the
+ *   colour gradient reaches the SH coefficients through the derivative of
+ *   the SH basis, band-limited).  Orthonormal real SH of degree <= 3 in
+ *   Cartesian form on d = normalise(mean - camera centre), camera centre =
+ *   -R^T t; coefficients ordered k = l^2 + l + m (Y_00; Y_1-1 ~ y, Y_10 ~ z,
+ *   Y_11 ~ x; ...).  colour = max(0, sum_{k < (degree+1)^2} Y_k(d) sh[k] +
+ *   offset) per channel.
+ * sh [N, K, 3] with (degree + 1)^2 <= K <= 16 coefficients stored per
+ *   Gaussian (only the first (degree + 1)^2 are used); colors [N, 3]
+ *   (written).
+ * gs_sh_bwd ACCUMULATES (+=) into dL_dsh [N, K, 3] (first (degree+1)^2 rows)
+ *   and into dL_dmeans [N, 3] (the view-direction path; add the geometric
+ *   path with gs_preprocess_bwd).  Where the clamp is active the channel
+ *   passes no gradient.
+ */
+#define GS_SH_MAX_DEGREE 3
+GS_API int gs_sh_fwd(const gs_camera* cam, int N, int degree, int K, const float* means, const float* sh,
+                     float offset, float* colors, void* stream);
+GS_API int gs_sh_bwd(const gs_camera* cam, int N, int degree, int K, const float* means, const float* sh,
+                     float offset, const float* dL_dcolors, float* dL_dsh, float* dL_dmeans, void* stream);
 
 #ifdef __cplusplus
 }

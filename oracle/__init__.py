@@ -76,7 +76,7 @@ def lib():
             getattr(L, f"oracle_render_fwd_{suf}").restype = None
             getattr(L, f"oracle_render_bwd_{suf}").argtypes = [cam, I] + [P] * 10 + [I]
             getattr(L, f"oracle_render_bwd_{suf}").restype = None
-            getattr(L, f"oracle_preprocess_bwd_{suf}").argtypes = [cam, I] + [P] * 12
+            getattr(L, f"oracle_preprocess_bwd_{suf}").argtypes = [cam, I] + [P] * 14
             getattr(L, f"oracle_preprocess_bwd_{suf}").restype = None
         for suf, R in (("f32", ctypes.c_float), ("f64", ctypes.c_double)):
             getattr(L, f"oracle_sh_fwd_{suf}").argtypes = [cam, I, I, I, P, P, R, P]
@@ -213,8 +213,8 @@ def render_bwd(cam, N: int, ranges, ids, mean2d, conic_opacity, colors, dL_dimag
 
 
 def preprocess_bwd(cam, means, scales, quats, radius, dL_dmean2d, dL_dconic_opacity, dL_dcolor2d,
-                   mode: str = "f64", accumulate_into: Optional[Dict[str, np.ndarray]] = None
-                   ) -> Dict[str, np.ndarray]:
+                   mode: str = "f64", accumulate_into: Optional[Dict[str, np.ndarray]] = None,
+                   densify: bool = False) -> Dict[str, np.ndarray]:
     dt = _dt(mode)
     means, scales, quats = (_a(x, dt) for x in (means, scales, quats))
     radius = _a(radius, np.int32)
@@ -223,11 +223,14 @@ def preprocess_bwd(cam, means, scales, quats, radius, dL_dmean2d, dL_dconic_opac
     out = accumulate_into or dict(dL_dmeans=np.zeros((n, 3), dt), dL_dscales=np.zeros((n, 3), dt),
                                   dL_dquats=np.zeros((n, 4), dt), dL_dopacity=np.zeros(n, dt),
                                   dL_dcolors=np.zeros((n, 3), dt))
+    if densify and "grad2d_accum" not in out:
+        out["grad2d_accum"] = np.zeros(n, dt)
+        out["vis_count"] = np.zeros(n, np.uint32)
     oc = camera(cam)
     getattr(lib(), f"oracle_preprocess_bwd_{mode}")(
         ctypes.byref(oc), n, _p(means), _p(scales), _p(quats), _p(radius), _p(dm), _p(dc), _p(dcol),
         _p(out["dL_dmeans"]), _p(out["dL_dscales"]), _p(out["dL_dquats"]), _p(out["dL_dopacity"]),
-        _p(out["dL_dcolors"]))
+        _p(out["dL_dcolors"]), _p(out.get("grad2d_accum")), _p(out.get("vis_count")))
     return out
 
 

@@ -556,10 +556,18 @@ template <typename Real>
 void preprocess_bwd(const oracle_camera* cam, int N, const Real* means, const Real* scales, const Real* quats,
                     const int* radius, const Real* dL_dmean2d, const Real* dL_dconic_opacity,
                     const Real* dL_dcolor2d, Real* dL_dmeans, Real* dL_dscales, Real* dL_dquats,
-                    Real* dL_dopacity, Real* dL_dcolors) {
+                    Real* dL_dopacity, Real* dL_dcolors, Real* grad2d_accum, unsigned* vis_count) {
 #pragma omp parallel for schedule(static)
     for (int i = 0; i < N; ++i) {
         if (radius[i] == 0) continue;  // culled: exactly zero gradient
+        // Densification statistics (training page, section D.1: the position
+        // gradient accumulated over views): |dL/dmean2d| of this view, and the
+        // number of views in which the Gaussian is visible.
+        if (grad2d_accum) {
+            const Real gx = dL_dmean2d[2 * i], gy = dL_dmean2d[2 * i + 1];
+            grad2d_accum[i] += std::sqrt(gx * gx + gy * gy);
+            vis_count[i] += 1;
+        }
         Geom<Real> g;
         if (!geometry(*cam, means + 3 * i, scales + 3 * i, quats + 4 * i, g)) continue;
         const Real* s = scales + 3 * i;
@@ -819,9 +827,11 @@ void oracle_set_threads(int n) {
     void oracle_preprocess_bwd_##SUF(const oracle_camera* cam, int N, const R* means, const R* scales,       \
                                      const R* quats, const int* radius, const R* dL_dmean2d,                 \
                                      const R* dL_dconic_opacity, const R* dL_dcolor2d, R* dL_dmeans,         \
-                                     R* dL_dscales, R* dL_dquats, R* dL_dopacity, R* dL_dcolors) {           \
+                                     R* dL_dscales, R* dL_dquats, R* dL_dopacity, R* dL_dcolors,             \
+                                     R* grad2d_accum, unsigned* vis_count) {                                 \
         preprocess_bwd<R>(cam, N, means, scales, quats, radius, dL_dmean2d, dL_dconic_opacity, dL_dcolor2d,  \
-                          dL_dmeans, dL_dscales, dL_dquats, dL_dopacity, dL_dcolors);                        \
+                          dL_dmeans, dL_dscales, dL_dquats, dL_dopacity, dL_dcolors, grad2d_accum,           \
+                          vis_count);                                                                        \
     }
 
 ORACLE_BOTH(DEF_PRE)

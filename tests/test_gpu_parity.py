@@ -342,3 +342,25 @@ def test_contribution_mask_and_backward_without_it(cfg):
     torch.cuda.synchronize()
     for k in with_mask:
         assert rel_l2(to_np(outs[k]), with_mask[k]) <= 1e-5, k
+
+
+def test_densification_statistics_over_views():
+    """The statistics accumulated over the four cameras of the 3M scene equal
+    the oracle's (gradients restricted to sampled tiles keep the oracle fast)."""
+    sc = _scene(3)
+    cams = [sc.cameras[0], sc.cameras[0].replace(R=(0.985, 0.0, 0.174, 0.0, 1.0, 0.0, -0.174, 0.0, 0.985))]
+    gs = GpuScene(sc)
+    dens = dict(grad2d_accum=torch.zeros(sc.N, device="cuda"),
+                vis_count=torch.zeros(sc.N, dtype=torch.uint32, device="cuda"))
+    out = None
+    from differentiable_gaussian_splatting_preprocess_b200 import rasterizer as RZ
+    for cam in cams:
+        rz = RZ.Rasterizer(cam)
+        fr = rz.forward(gs.means, gs.scales, gs.quats, gs.opacity, gs.colors)
+        g = rz.backward(fr, gs.means, gs.scales, gs.quats, gs.colors, to_dev(sc.dL_dimage[0]), densify=dens)
+        torch.cuda.synchronize()
+        out = oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, to_np(fr.radius), to_np(g["dL_dmean2d"]),
+                                    to_np(g["dL_dconic_opacity"]), to_np(g["dL_dcolor"]), "f64",
+                                    accumulate_into=out, densify=True)
+    np.testing.assert_array_equal(to_np(dens["vis_count"]), out["vis_count"])
+    assert rel_l2(to_np(dens["grad2d_accum"]), out["grad2d_accum"]) <= 1e-6

@@ -492,3 +492,22 @@ def test_mirror_exp_error_bound():
     err = np.abs(y.astype(np.float64) - ref) / ulp
     assert err.max() <= 2.0, err.max()
     assert oracle.exp_f32(np.zeros(1))[0] == 1.0
+
+
+def test_densification_statistics_definition():
+    """Per visible view: accum += |dL/dmean2d|, count += 1; culled views add
+    nothing; two identical views double the accumulator."""
+    sc = scenes.random_tiny(n=8, seed=12)
+    cam = sc.cameras[0]
+    sc.means[7, 2] = -1.0  # culled in this view
+    fb = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0], "f64")
+    out = None
+    for _ in range(2):
+        out = oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, fb["pre"]["radius"], fb["dL_dmean2d"],
+                                    fb["dL_dconic_opacity"], fb["dL_dcolor"], "f64", accumulate_into=out,
+                                    densify=True)
+    norm = np.linalg.norm(fb["dL_dmean2d"], axis=1)
+    vis = fb["pre"]["radius"] > 0
+    np.testing.assert_allclose(out["grad2d_accum"], 2 * norm * vis, rtol=1e-14)
+    np.testing.assert_array_equal(out["vis_count"], 2 * vis.astype(np.uint32))
+    assert not vis[7] and out["vis_count"][7] == 0
