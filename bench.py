@@ -188,6 +188,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     from differentiable_gaussian_splatting_preprocess_b200 import binding as B
+    from differentiable_gaussian_splatting_preprocess_b200 import multiview as MV
     from differentiable_gaussian_splatting_preprocess_b200 import rasterizer as RZ
 
     world, rank, local = _dist()
@@ -201,129 +202,149 @@ def run_ours(args):
     B.lib()
 
     sc = _scene(args.config)
-    cam = sc.cameras[0]
+    cams = sc.cameras
+    # several views: split them over the ranks and sum the 3D gradients
+    # (camera-parallel); one view: every rank renders it (replicas)
+    multi = len(cams) > 1
+    mine = MV.assign_cameras(len(cams), world, rank) if multi else [0]
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
     means, scales, quats, opacity, colors = (t(x) for x in (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors))
-    dL = t(sc.dL_dimage[0])
-    rz = RZ.Rasterizer(cam, dev)
-    # size the pair buffers once (host read of P), then run in capacity mode
-    fr = rz.forward(means, scales, quats, opacity, colors)
-    P = fr.capacity
-    capacity = P
+    dLs = {i: t(sc.dL_dimage[i]) for i in mine}
+    rzs = {i: RZ.Rasterizer(cams[i], dev) for i in mine}
+    caps = {}
+    for i in mine:
+        # size the pair buffers once (host read of P), then run in capacity mode
+        fr = rzs[i].forward(means, scales, quats, opacity, colors)
+        caps[i] = fr.capacity
+        rzs[i].backward(fr, means, scales, quats, colors, dLs[i])  # allocates the 2D gradient buffers
     grads = RZ.zero_grads(sc.N, dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    stages = ["preprocess_fwd", "bin_sort", "render_fwd", "render_bwd", "preprocess_bwd"]
     sh_deg = args.sh_degree
     if sh_deg is not None:
         from differentiable_gaussian_splatting_preprocess_b200 import scenes as _scn
         shd = torch.from_numpy(_scn.random_sh(sc.N, sh_deg, seed=1)).to(dev)
         dsh = torch.zeros_like(shd)
         colors = torch.empty((sc.N, 3), dtype=torch.float32, device=dev)
-        stages = ["sh_fwd"] + stages + ["sh_bwd"]
+    exchange = multi and world > 1
 
-    def step(ev=None):
-        marks = [0]
+    def step(rec=None):
+        """One step: every view of this rank through a1-a8 (gradients summed),
+        then the gradient exchange when views are split over ranks.
+        ``rec`` collects (stage, start event, end event)."""
+        def timed(name, fn):
+            if rec is None:
+                fn()
+                return
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            rec.append((name, e0, e1))
 
-        def mark(i=None):
-            if ev is not None:
-                ev[marks[0]].record(stream)
-            marks[0] += 1
-        if sh_deg is not None:
-            mark()
-            B.gs_sh_fwd(cam, sh_deg, means, shd, colors, offset=0.5)
-        mark(0)
-        pre = rz.preprocess(means, scales, quats, opacity)
-        mark(1)
-        ws = rz.workspace(sc.N, capacity)
-        B.gs_bin_sort(cam, pre["depth"], pre["rect"], pre["tiles_touched"], pre["num_pairs"], capacity,
-                      rz._bufs["ids"], rz._bufs["ranges"], None, ws)
-        mark(2)
-        B.gs_render_fwd(cam, rz._bufs["ranges"], rz._bufs["ids"], pre["mean2d"], pre["conic_opacity"], colors,
-                        rz._bufs["image"], rz._bufs["final_T"], rz._bufs["n_contrib"], rz._bufs["contrib_mask"])
-        mark(3)
-        B.gs_render_bwd(cam, rz._bufs["ranges"], rz._bufs["ids"], pre["mean2d"], pre["conic_opacity"], colors,
-                        rz._bufs["final_T"], rz._bufs["n_contrib"], dL, rz._bufs["dL_dmean2d"],
-                        rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"], rz._bufs["contrib_mask"])
-        mark(4)
-        B.gs_preprocess_bwd(cam, means, scales, quats, pre["radius"], pre["conic_opacity"], rz._bufs["dL_dmean2d"],
-                            rz._bufs["dL_dconic_opacity"], rz._bufs["dL_dcolor"], grads["dL_dmeans"],
-                            grads["dL_dscales"], grads["dL_dquats"], grads["dL_dopacity"], grads["dL_dcolors"])
-        mark(5)
-        if sh_deg is not None:
-            B.gs_sh_bwd(cam, sh_deg, means, shd, grads["dL_dcolors"], dsh, grads["dL_dmeans"], offset=0.5)
-            mark()
+        for i in mine:
+            cam, rz, cap, dL = cams[i], rzs[i], caps[i], dLs[i]
+            b = rz._bufs
+            if sh_deg is not None:
+                timed("sh_fwd", lambda: B.gs_sh_fwd(cam, sh_deg, means, shd, colors, offset=0.5))
+            timed("preprocess_fwd", lambda: rz.preprocess(means, scales, quats, opacity))
+            timed("bin_sort", lambda: B.gs_bin_sort(cam, b["depth"], b["rect"], b["tiles_touched"], b["num_pairs"],
+                                                   cap, b["ids"], b["ranges"], None, rz.workspace(sc.N, cap)))
+            timed("render_fwd", lambda: B.gs_render_fwd(cam, b["ranges"], b["ids"], b["mean2d"], b["conic_opacity"],
+                                                       colors, b["image"], b["final_T"], b["n_contrib"],
+                                                       b["contrib_mask"]))
+            timed("render_bwd", lambda: B.gs_render_bwd(cam, b["ranges"], b["ids"], b["mean2d"], b["conic_opacity"],
+                                                       colors, b["final_T"], b["n_contrib"], dL, b["dL_dmean2d"],
+                                                       b["dL_dconic_opacity"], b["dL_dcolor"], b["contrib_mask"]))
+            timed("preprocess_bwd", lambda: B.gs_preprocess_bwd(
+                cam, means, scales, quats, b["radius"], b["conic_opacity"], b["dL_dmean2d"], b["dL_dconic_opacity"],
+                b["dL_dcolor"], grads["dL_dmeans"], grads["dL_dscales"], grads["dL_dquats"], grads["dL_dopacity"],
+                grads["dL_dcolors"]))
+            if sh_deg is not None:
+                timed("sh_bwd", lambda: B.gs_sh_bwd(cam, sh_deg, means, shd, grads["dL_dcolors"], dsh,
+                                                   grads["dL_dmeans"], offset=0.5))
+        if exchange:
+            timed("allreduce", lambda: MV.allreduce_grads(grads))
 
-    rz.backward(fr, means, scales, quats, colors, dL)  # allocate the 2D gradient buffers
     for _ in range(args.warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
-    st = rz.status()
-    if st != 0:
-        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
-    n_contrib = int(rz._bufs["n_contrib"].view(torch.int32).to(torch.int64).sum().item())
-    n_eval_t = torch.empty((cam.height, cam.width), dtype=torch.uint32, device=dev)
-    n_blend_t = torch.empty_like(n_eval_t)
-    pre0 = rz._bufs
-    B.gs_render_stats(cam, pre0["ranges"], pre0["ids"], pre0["mean2d"], pre0["conic_opacity"], n_eval_t, n_blend_t)
-    n_evaluated = int(n_eval_t.view(torch.int32).to(torch.int64).sum().item())
-    n_blended = int(n_blend_t.view(torch.int32).to(torch.int64).sum().item())
-    evals_per_frame = n_evaluated + n_contrib
+    for i in mine:
+        st = rzs[i].status()
+        if st != 0:
+            raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+    # work counts of this rank's views (outside the timed region)
+    n_contrib = n_evaluated = n_blended = P = 0
+    for i in mine:
+        b, cam = rzs[i]._bufs, cams[i]
+        ne = torch.empty((cam.height, cam.width), dtype=torch.uint32, device=dev)
+        nb = torch.empty_like(ne)
+        B.gs_render_stats(cam, b["ranges"], b["ids"], b["mean2d"], b["conic_opacity"], ne, nb)
+        n_contrib += int(b["n_contrib"].view(torch.int32).to(torch.int64).sum().item())
+        n_evaluated += int(ne.view(torch.int32).to(torch.int64).sum().item())
+        n_blended += int(nb.view(torch.int32).to(torch.int64).sum().item())
+        P += caps[i]
+    evals_per_step = n_evaluated + n_contrib
 
     sampler = ClockSampler(local)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    recs = [[] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
     time.sleep(0.3)
     for k in range(args.steps):
-        flush.zero_()  # L2 flush outside the timed interval
-        step(events[k])
+        flush.zero_()  # L2 flush outside the timed intervals
+        step(recs[k])
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     time.sleep(0.2)
     clocks = sampler.stop()
-    stage_ms = {s: [] for s in stages}
+    stage_ms = {}
     step_ms = []
-    for ev in events:
-        for i, s in enumerate(stages):
-            stage_ms[s].append(ev[i].elapsed_time(ev[i + 1]))
-        step_ms.append(ev[0].elapsed_time(ev[len(stages)]))
+    for rec in recs:
+        for name, e0, e1 in rec:
+            stage_ms.setdefault(name, []).append(e0.elapsed_time(e1))
+        step_ms.append(rec[0][1].elapsed_time(rec[-1][2]))
     total_ms = sum(step_ms)
+    evals_all = evals_per_step
     if world > 1:
         tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         total_ms = float(tt.item())
-    value = world * evals_per_frame * args.steps / (total_ms / 1e3)
-    st = rz.status()
-    if st != 0:
-        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+        ev_t = torch.tensor([float(evals_per_step)], device=dev, dtype=torch.float64)
+        dist.all_reduce(ev_t, op=dist.ReduceOp.SUM)
+        evals_all = float(ev_t.item())
+    value = evals_all * args.steps / (total_ms / 1e3)
+    for i in mine:
+        st = rzs[i].status()
+        if st != 0:
+            raise RuntimeError(f"device status {st}: {B.status_string(st)}")
 
     # launches of this library's kernels per step
-    T = B.num_tiles(cam)
-    tile_bits = max(0, (T - 1).bit_length())
-    tpasses = (tile_bits + 7) // 8
-    launches = 1 + (1 + 4 * 3 + 3 + 1 + 3 * tpasses + 1) + 2 + 2 + 1 + (2 if sh_deg is not None else 0)
+    tpasses = max(((B.num_tiles(cams[i]) - 1).bit_length() + 7) // 8 for i in mine)
+    per_view = 1 + (1 + 4 * 3 + 3 + 1 + 3 * tpasses + 1) + 2 + 2 + 1 + (2 if sh_deg is not None else 0)
+    launches = per_view * len(mine)
 
-    # roofline of the dominant kernel (render backward: FP32 ALU bound)
+    # roofline of the dominant kernel (render backward: FP32 issue bound)
     peaks = _peaks()
-    mean = {s: statistics.mean(v) for s, v in stage_ms.items()}
+    # per-step time of each stage, summed over this rank's views
+    mean = {s: statistics.mean(v) * len(v) / args.steps for s, v in stage_ms.items()}
     dominant = max(mean, key=mean.get)
     bwd_ops = n_blended * OPS_BWD_EVAL
     fwd_ops = n_blended * OPS_FWD_EVAL
     alu_peak = SMS * FP32_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12  # T lane-ops/s
     rb_ach = bwd_ops / (mean["render_bwd"] / 1e3) / 1e12
-    rec = RECORDED_TRAFFIC["k_render_bwd"]
-    traffic = rec["bytes"] if rec["sources_sha1"] == _render_sources_sha1() else None
+    rec_t = RECORDED_TRAFFIC["k_render_bwd"]
+    traffic = rec_t["bytes"] if (rec_t["sources_sha1"] == _render_sources_sha1() and len(mine) == 1) else None
     roofline = dict(kernel="k_render_bwd", bound="alu", achieved=rb_ach, peak=alu_peak, unit="Tops/s",
-                    frac=rb_ach / alu_peak, traffic=traffic, ops_per_launch=bwd_ops,
+                    frac=rb_ach / alu_peak, traffic=traffic, ops_per_launch=bwd_ops // len(mine),
                     ops_basis=f"{OPS_BWD_EVAL} FP32 ops x {n_blended} blended terms",
                     peak_src=f"148 SMs x 128 FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz (sm_max_mhz)")
     # HBM view of render fwd + bwd, as asked
-    pix = cam.width * cam.height
+    pix = sum(cams[i].width * cams[i].height for i in mine)
     fwd_bytes = P * BYTES_PAIR_READ + pix * BYTES_PIXEL
     bwd_bytes = P * (BYTES_PAIR_READ + BYTES_PAIR_ATOMIC) + pix * BYTES_PIXEL
     rfb_s = (mean["render_fwd"] + mean["render_bwd"]) / 1e3
@@ -333,13 +354,15 @@ def run_ours(args):
     fwd_alu = fwd_ops / (mean["render_fwd"] / 1e3) / 1e12
 
     # end to end through the public API: pinned host inputs -> device ->
-    # forward (host read of P) + backward -> 3D gradients back to the host
+    # forward (host read of P) + backward of every view of this rank, the
+    # gradient exchange, then the 3D gradients back to the host
     e2e = None
     if not args.no_e2e:
         host_in = [torch.from_numpy(np.ascontiguousarray(x)).pin_memory()
-                   for x in (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0])]
-        h2d = sum(x.numel() * x.element_size() for x in host_in)
-        rz2 = RZ.Rasterizer(cam, dev)
+                   for x in (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors)]
+        host_dl = [torch.from_numpy(np.ascontiguousarray(sc.dL_dimage[i])).pin_memory() for i in mine]
+        h2d = sum(x.numel() * x.element_size() for x in host_in + host_dl)
+        rz_e2e = {}
         host_out = None
         e2e_times = []
         for k in range(args.warmup + args.steps):
@@ -347,9 +370,12 @@ def run_ours(args):
             torch.cuda.synchronize(dev)
             t0 = time.perf_counter()
             d = [x.to(dev, non_blocking=True) for x in host_in]
-            f2 = rz2.forward(d[0], d[1], d[2], d[3], d[4])
-            g2 = rz2.backward(f2, d[0], d[1], d[2], d[4], d[5])
-            outs = [g2[k2] for k2 in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors")]
+            dls = [x.to(dev, non_blocking=True) for x in host_dl]
+            params = dict(means=d[0], scales=d[1], quats=d[2], opacity=d[3], colors=d[4])
+            g2 = MV.render_views([cams[i] for i in mine], params, dls, rasterizers=rz_e2e, camera_ids=mine)
+            if exchange:
+                MV.allreduce_grads(g2)
+            outs = [g2[k2] for k2 in MV.GRAD_KEYS]
             if host_out is None:
                 host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
             for ho, o in zip(host_out, outs):
@@ -363,7 +389,7 @@ def run_ours(args):
             tt = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             e2e_s = float(tt.item())
-        e2e = dict(value=world * evals_per_frame * args.steps / e2e_s, unit=UNIT, h2d_bytes_per_step=h2d,
+        e2e = dict(value=evals_all * args.steps / e2e_s, unit=UNIT, h2d_bytes_per_step=h2d,
                    d2h_bytes_per_step=d2h, ms_per_step=1e3 * e2e_s / args.steps)
 
     cpu = None
@@ -380,18 +406,20 @@ def run_ours(args):
                    sample=f"{reps} x ({c['sample']}); {tot_s:.1f} s in total")
 
     if rank == 0:
+        cam0 = cams[0]
+        par = (f"camera-parallel x{world}" if exchange else (f"replicas x{world}" if world > 1 else "1 GPU"))
         line = dict(
             metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
-            ms_per_step=total_ms / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,
-            dtype="f32", data="synthetic",
-            config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam.width}x{cam.height}, 16x16 tiles, fp32"
+            ms_per_step=total_ms / args.steps, higher_is_better=True, scaling="weak" if not exchange else "strong",
+            vs_baseline=None, dtype="f32", data="synthetic",
+            config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam0.width}x{cam0.height}, {len(cams)} view(s), "
+                                 f"16x16 tiles, fp32"
                                  + (f", SH degree {sh_deg} colours" if sh_deg is not None else ""),
-                        num_pairs=P, evals_per_frame=evals_per_frame, evaluated_fwd=n_evaluated,
-                        contributor_prefix_bwd=n_contrib, blended=n_blended,
-                        l2="flushed between steps (256 MiB write)",
-                        parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
-            fwd_ms_per_frame=mean["preprocess_fwd"] + mean["bin_sort"] + mean["render_fwd"],
-            bwd_ms_per_frame=mean["render_bwd"] + mean["preprocess_bwd"],
+                        views_per_rank=len(mine), num_pairs=P, evals_per_step=evals_per_step,
+                        evaluated_fwd=n_evaluated, contributor_prefix_bwd=n_contrib, blended=n_blended,
+                        l2="flushed between steps (256 MiB write)", parallelism=par),
+            fwd_ms_per_frame=(mean["preprocess_fwd"] + mean["bin_sort"] + mean["render_fwd"]) / len(mine),
+            bwd_ms_per_frame=(mean["render_bwd"] + mean["preprocess_bwd"]) / len(mine),
             stage_ms={s: round(v, 4) for s, v in mean.items()}, dominant_stage=dominant,
             roofline=roofline, render_fwd_alu=dict(achieved=fwd_alu, peak=alu_peak, unit="Tops/s",
                                                    frac=fwd_alu / alu_peak),

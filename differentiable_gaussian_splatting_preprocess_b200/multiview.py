@@ -1,0 +1,91 @@
+"""Several cameras of one scene: render each view forward and backward and sum
+the 3D gradients (the views of the 3M-Gaussian scene are rendered back to back
+with gradients accumulated).  Across processes the cameras are split between
+ranks and the per-rank sums are added with one all-reduce of a single flat
+buffer - the only exchange this path has (the Gaussians are replicated; each
+view is independent).  On GPUs the process group is NCCL over NVLink; the
+host logic is the same for any backend.
+"""
+from __future__ import annotations
+
+from typing import Callable, Dict, List, Optional, Sequence
+
+import torch
+import torch.distributed as dist
+
+from . import rasterizer as RZ
+
+GRAD_KEYS = ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors")
+
+
+def assign_cameras(n_cameras: int, world: int, rank: int) -> List[int]:
+    """Cameras of one rank: round-robin, so every camera belongs to exactly
+    one rank and the shares differ by at most one."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("bad rank / world size")
+    return [i for i in range(n_cameras) if i % world == rank]
+
+
+def render_views(cams: Sequence, params: Dict[str, torch.Tensor], dL_dimages: Sequence[torch.Tensor],
+                 grads: Optional[Dict[str, torch.Tensor]] = None,
+                 rasterizers: Optional[Dict[int, "RZ.Rasterizer"]] = None,
+                 densify: Optional[Dict[str, torch.Tensor]] = None, capacity: Optional[Sequence[int]] = None,
+                 camera_ids: Optional[Sequence[int]] = None) -> Dict[str, torch.Tensor]:
+    """Forward and backward of every camera in ``cams``; 3D gradients are
+    accumulated into ``grads`` (allocated when None).  ``rasterizers`` caches
+    one Rasterizer (and its buffers) per camera id across calls."""
+    means, scales, quats = params["means"], params["scales"], params["quats"]
+    opacity, colors = params["opacity"], params["colors"]
+    if grads is None:
+        grads = RZ.zero_grads(means.shape[0], means.device)
+    ids = list(range(len(cams))) if camera_ids is None else list(camera_ids)
+    for n, (cam, dl) in enumerate(zip(cams, dL_dimages)):
+        cid = ids[n]
+        rz = None if rasterizers is None else rasterizers.get(cid)
+        if rz is None:
+            rz = RZ.Rasterizer(cam, means.device)
+            if rasterizers is not None:
+                rasterizers[cid] = rz
+        cap = None if capacity is None else capacity[n]
+        fr = rz.forward(means, scales, quats, opacity, colors, capacity=cap)
+        rz.backward(fr, means, scales, quats, colors, dl, grads=grads, densify=densify)
+    return grads
+
+
+def flat_grads(grads: Dict[str, torch.Tensor], keys: Sequence[str] = GRAD_KEYS) -> torch.Tensor:
+    return torch.cat([grads[k].reshape(-1) for k in keys])
+
+
+def unflatten_into(flat: torch.Tensor, grads: Dict[str, torch.Tensor], keys: Sequence[str] = GRAD_KEYS) -> None:
+    off = 0
+    for k in keys:
+        n = grads[k].numel()
+        grads[k].copy_(flat[off:off + n].view_as(grads[k]))
+        off += n
+
+
+def allreduce_grads(grads: Dict[str, torch.Tensor], group=None, keys: Sequence[str] = GRAD_KEYS) -> None:
+    """Sum the gradient tensors over the ranks of ``group`` in place, with one
+    all-reduce of a single contiguous buffer (one launch, one NVLink
+    transfer schedule, whatever the number of tensors)."""
+    flat = flat_grads(grads, keys)
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    unflatten_into(flat, grads, keys)
+
+
+def render_views_distributed(cams: Sequence, params: Dict[str, torch.Tensor],
+                             dL_dimages: Sequence[torch.Tensor], group=None,
+                             render_fn: Callable = render_views, **kw) -> Dict[str, torch.Tensor]:
+    """Each rank renders its share of the cameras (assign_cameras), then the
+    3D gradients are summed over ranks: every rank ends with the gradient of
+    the sum of all views' losses."""
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    mine = assign_cameras(len(cams), world, rank)
+    grads = kw.pop("grads", None)
+    if grads is None:
+        grads = RZ.zero_grads(params["means"].shape[0], params["means"].device)
+    render_fn([cams[i] for i in mine], params, [dL_dimages[i] for i in mine], grads=grads, camera_ids=mine, **kw)
+    if world > 1:
+        allreduce_grads(grads, group)
+    return grads

@@ -364,3 +364,25 @@ def test_densification_statistics_over_views():
                                     accumulate_into=out, densify=True)
     np.testing.assert_array_equal(to_np(dens["vis_count"]), out["vis_count"])
     assert rel_l2(to_np(dens["grad2d_accum"]), out["grad2d_accum"]) <= 1e-6
+
+
+def test_render_views_sums_cameras():
+    """Several views rendered back to back with the 3D gradients summed equal
+    the sum of the oracle's per-view gradients."""
+    from differentiable_gaussian_splatting_preprocess_b200 import multiview as MV
+    sc = _scene(2)
+    base = sc.cameras[0]
+    cams = [base, base.replace(R=(0.985, 0.0, 0.174, 0.0, 1.0, 0.0, -0.174, 0.0, 0.985)),
+            base.replace(t=(0.2, -0.1, 0.0))]
+    gs = GpuScene(sc)
+    params = dict(means=gs.means, scales=gs.scales, quats=gs.quats, opacity=gs.opacity, colors=gs.colors)
+    dls = [to_dev(sc.dL_dimage[0])] * 3
+    grads = MV.render_views(cams, params, dls)
+    torch.cuda.synchronize()
+    ref = None
+    for cam in cams:
+        f = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0],
+                                    "f64")
+        ref = {k: f[k] for k in MV.GRAD_KEYS} if ref is None else {k: ref[k] + f[k] for k in MV.GRAD_KEYS}
+    for k in MV.GRAD_KEYS:
+        assert rel_l2(to_np(grads[k]), ref[k]) <= GRAD_REL_L2, k
