@@ -118,16 +118,14 @@ __global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const 
 template <int MAXB>
 struct RadixCfg {
     static constexpr int kRadix = 1 << MAXB;
-    static constexpr int kItems = MAXB >= 8 ? 4 : 8;
-    static constexpr int kTileKeys = kItems * kSortBlock;
+    static constexpr int kItems = 8;                        // keys per thread per tile
+    static constexpr int kTileKeys = kItems * kSortBlock;   // 2048
     static constexpr int kWarps = kSortBlock / 32;
-    static constexpr int kSlots = kItems * kWarps;  // (item, warp) groups per tile, in input order
-    // scatter shared memory: 16-bit per-(slot, digit) counts and tile-local
-    // offsets, 32-bit per-digit running bases / tile starts / tile bases,
-    // and the tile's keys and values regrouped by digit.
-    static constexpr size_t kScatterSmem = (size_t)2 * kSlots * kRadix * sizeof(unsigned short) +
-                                           (size_t)4 * kRadix * sizeof(unsigned) +
-                                           (size_t)2 * kTileKeys * sizeof(unsigned);
+    static constexpr int kWarpKeys = kItems * 32;           // each warp owns a contiguous block of the tile
+    // scatter shared memory: per-digit running bases / tile counts / tile
+    // starts / tile bases, per-(warp, digit) counts turned into offsets, and
+    // the tile's keys and values regrouped by digit
+    static constexpr size_t kScatterSmem = (size_t)(4 * kRadix + kWarps * kRadix + 2 * kTileKeys) * sizeof(unsigned);
 };
 
 template <int MAXB>
@@ -178,16 +176,25 @@ k_radix_hist(const unsigned* __restrict__ keys, const unsigned* __restrict__ n_p
     unsigned lo, hi;
     chunk_of<MAXB>(*n_ptr, lo, hi);
     const int warp = threadIdx.x >> 5;
+    // chunk boundaries are multiples of the tile (2048 keys), so every tile
+    // but the last is read with 16-byte loads, 4 keys per load
     for (unsigned base = lo; base < hi; base += C::kTileKeys) {
-        unsigned d[C::kItems];
+        if (base + C::kTileKeys <= hi) {
+            const uint4* k4 = reinterpret_cast<const uint4*>(keys + base);
+            uint4 v[C::kItems / 4];
 #pragma unroll
-        for (int j = 0; j < C::kItems; ++j) {
-            const unsigned i = base + j * kSortBlock + threadIdx.x;
-            d[j] = i < hi ? (keys[i] >> shift) & mask : kNoDigit;
+            for (int j = 0; j < C::kItems / 4; ++j) v[j] = k4[j * kSortBlock + threadIdx.x];
+#pragma unroll
+            for (int j = 0; j < C::kItems / 4; ++j) {
+                atomicAdd(&s_h[warp][(v[j].x >> shift) & mask], 1u);
+                atomicAdd(&s_h[warp][(v[j].y >> shift) & mask], 1u);
+                atomicAdd(&s_h[warp][(v[j].z >> shift) & mask], 1u);
+                atomicAdd(&s_h[warp][(v[j].w >> shift) & mask], 1u);
+            }
+        } else {
+            for (unsigned i = base + threadIdx.x; i < hi; i += kSortBlock)
+                atomicAdd(&s_h[warp][(keys[i] >> shift) & mask], 1u);
         }
-#pragma unroll
-        for (int j = 0; j < C::kItems; ++j)
-            if (d[j] != kNoDigit) atomicAdd(&s_h[warp][d[j]], 1u);
     }
     __syncthreads();
     const unsigned G = gridDim.x;
@@ -244,14 +251,15 @@ k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, i
         }
 }
 
-// Stable scatter.  Per tile of ITEMS x 256 keys:
-//   1. every warp ranks each of its item slots among its lanes (digit_peers)
-//      and records the group sizes per (slot, digit);
-//   2. one thread per digit turns those counts into tile-local offsets in
-//      input order (slot-major: item slot j, then warp), giving the tile's
-//      count per digit; the digit counts are scanned into tile-local starts;
-//   3. every key is placed in shared memory at its tile-local sorted
-//      position (keys regrouped by digit, input order kept within a digit);
+// Stable scatter.  Per tile of 2048 keys, each warp owning a contiguous block
+// of 256 of them (8 rows of 32):
+//   1. each warp ranks its keys row by row (digit_peers within the row, plus
+//      a running per-digit count of the warp's earlier rows), so ranks follow
+//      input order within the warp;
+//   2. one thread per digit turns the warps' counts into offsets (warp
+//      order), giving the tile's count per digit; one warp scans those into
+//      tile-local digit starts and advances the running global bases;
+//   3. every key is placed in shared memory at its tile-local sorted position;
 //   4. the regrouped tile is written out in order, so consecutive lanes write
 //      consecutive addresses of one digit's run (coalesced stores).
 template <int MAXB>
@@ -265,54 +273,56 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
     unsigned* s_tcnt = s_base + C::kRadix;                      // [radix] this tile's count per digit
     unsigned* s_tstart = s_tcnt + C::kRadix;                    // [radix] tile-local start per digit
     unsigned* s_tbase = s_tstart + C::kRadix;                   // [radix] global base for this tile
-    unsigned* s_keys = s_tbase + C::kRadix;                     // [tile] regrouped keys
+    unsigned* s_wcnt = s_tbase + C::kRadix;                     // [warps][radix] counts, then offsets
+    unsigned* s_keys = s_wcnt + C::kWarps * C::kRadix;          // [tile] regrouped keys
     unsigned* s_vals = s_keys + C::kTileKeys;                   // [tile] regrouped values
-    unsigned short* s_cnt = reinterpret_cast<unsigned short*>(s_vals + C::kTileKeys);  // [slots][radix]
-    unsigned short* s_off = s_cnt + C::kSlots * C::kRadix;                              // [slots][radix]
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
     const unsigned G = gridDim.x;
     for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) s_base[dd] = offsets[(size_t)dd * G + blockIdx.x];
-    for (int i = threadIdx.x; i < C::kSlots * C::kRadix; i += kSortBlock) s_cnt[i] = 0;
-    __syncthreads();
     unsigned lo, hi;
     chunk_of<MAXB>(*n_ptr, lo, hi);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned lt = lanemask_lt();
+    unsigned* wcnt = s_wcnt + warp * C::kRadix;
     for (unsigned base = lo; base < hi; base += C::kTileKeys) {
         const unsigned tile_n = min((unsigned)C::kTileKeys, hi - base);
+        for (int dd = lane; dd < radix; dd += 32) wcnt[dd] = 0;
+        __syncwarp();
         unsigned key[C::kItems], val[C::kItems], d[C::kItems], rank[C::kItems];
+        const unsigned wbase = base + warp * C::kWarpKeys;
 #pragma unroll
         for (int j = 0; j < C::kItems; ++j) {
-            const unsigned i = base + j * kSortBlock + threadIdx.x;
+            const unsigned i = wbase + j * 32 + lane;
             const bool valid = i < hi;
             key[j] = valid ? keys_in[i] : 0u;
             val[j] = valid ? vals_in[i] : 0u;
             d[j] = valid ? (key[j] >> shift) & mask : kNoDigit;
         }
-        // 1. ranks within each warp's slot
+        // 1. ranks within the warp, row after row
 #pragma unroll
         for (int j = 0; j < C::kItems; ++j) {
             const unsigned peers = digit_peers<MAXB>(d[j], bits);
-            rank[j] = __popc(peers & lt);
-            if (d[j] != kNoDigit && lane == __ffs(peers) - 1)
-                s_cnt[(j * C::kWarps + warp) * C::kRadix + d[j]] = (unsigned short)__popc(peers);
+            const bool valid = d[j] != kNoDigit;
+            const unsigned before = valid ? wcnt[d[j]] : 0u;
+            __syncwarp();
+            if (valid && lane == __ffs(peers) - 1) wcnt[d[j]] = before + __popc(peers);
+            __syncwarp();
+            rank[j] = before + __popc(peers & lt);
         }
         __syncthreads();
-        // 2. per digit: tile-local offsets in input order, and the tile count
+        // 2. per digit: warp offsets in warp order, and the tile count
         for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
             unsigned run = 0;
-#pragma unroll 8
-            for (int e = 0; e < C::kSlots; ++e) {
-                const unsigned c = s_cnt[e * C::kRadix + dd];
-                s_cnt[e * C::kRadix + dd] = 0;
-                s_off[e * C::kRadix + dd] = (unsigned short)run;
+#pragma unroll
+            for (int w = 0; w < C::kWarps; ++w) {
+                const unsigned c = s_wcnt[w * C::kRadix + dd];
+                s_wcnt[w * C::kRadix + dd] = run;
                 run += c;
             }
             s_tcnt[dd] = run;
         }
         __syncthreads();
-        // exclusive scan of the digit counts (one warp), bases for this tile
         if (warp == 0) {
             constexpr int per = (C::kRadix + 31) / 32;
             unsigned v[per], sum = 0;
@@ -345,7 +355,7 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
 #pragma unroll
         for (int j = 0; j < C::kItems; ++j) {
             if (d[j] != kNoDigit) {
-                const unsigned loc = s_tstart[d[j]] + s_off[(j * C::kWarps + warp) * C::kRadix + d[j]] + rank[j];
+                const unsigned loc = s_tstart[d[j]] + wcnt[d[j]] + rank[j];
                 s_keys[loc] = key[j];
                 s_vals[loc] = val[j];
             }
@@ -360,7 +370,7 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
             keys_out[pos] = k2;
             vals_out[pos] = s_vals[q];
         }
-        // the next tile's first barrier orders these reads before its writes
+        __syncthreads();  // the next tile reuses every shared array
     }
 }
 
@@ -447,83 +457,112 @@ k_scan_down(int N, const unsigned* __restrict__ order, const unsigned* __restric
     }
 }
 
-// Emit the (tile, Gaussian) pairs in depth-rank order.  A warp takes 32
-// consecutive ranks, whose pairs are contiguous in the output; each lane
-// writes every 32nd of those pairs, finding the Gaussian it belongs to by a
-// binary search over the warp's inclusive scan of pair counts (held in
-// registers, read with shuffles).  Stores are coalesced and the work per
-// lane is balanced however many tiles each Gaussian covers.
+// Emit the (tile, Gaussian) pairs in depth-rank order, balanced by pairs:
+// CTA c writes output positions [c * 2048, (c + 1) * 2048).  Visible
+// Gaussians come first in rank order and each has at least one pair, so
+// the ranks covering a segment are found by one binary search over the
+// exclusive pair offsets and number at most 2049; their offsets and ids are
+// staged in shared memory, and each thread finds the owner of each of its
+// output positions by a binary search there.  Row and column within the
+// Gaussian's tile rectangle come from a float quotient corrected by one step
+// (local < 2^24 and width <= 4096, so the float error is below one).
+constexpr int kEmitSeg = 2048;
+
+__device__ __forceinline__ unsigned upper_bound_global(const unsigned* __restrict__ a, unsigned n, unsigned x) {
+    // first index i in [0, n) with a[i] > x (n if none)
+    unsigned lo = 0, hi = n;
+    while (lo < hi) {
+        const unsigned mid = (lo + hi) >> 1;
+        if (a[mid] <= x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
 __global__ void __launch_bounds__(kSortBlock)
 k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
        const int4* __restrict__ rect, const unsigned* __restrict__ tiles_touched, const SortMisc* __restrict__ misc,
        unsigned* __restrict__ tkeys, unsigned* __restrict__ tvals) {
+    __shared__ unsigned s_off[kEmitSeg + 1];
+    __shared__ unsigned s_g[kEmitSeg + 1];
+    __shared__ unsigned s_r0, s_nr;
     const unsigned P = misc->p_eff;
     if (P == 0) return;  // nothing to emit, or over capacity
-    const int lane = threadIdx.x & 31;
-    const int warp_global = (blockIdx.x * kSortBlock + threadIdx.x) >> 5;
-    const int nwarps = (gridDim.x * kSortBlock) >> 5;
-    for (int r0 = warp_global * 32; r0 < N; r0 += nwarps * 32) {
-        const int r = r0 + lane;
-        unsigned g = 0, cnt = 0, off = 0;
-        int x0 = 0, y0 = 0, wdt = 1;
-        if (r < N) {
-            g = order[r];
-            cnt = tiles_touched[g];
-            off = pair_off[r];
-            if (cnt) {
-                const int4 rc = rect[g];
-                x0 = rc.x;
-                y0 = rc.y;
-                wdt = rc.z - rc.x;
-            }
+    for (unsigned p0 = blockIdx.x * kEmitSeg; p0 < P; p0 += gridDim.x * kEmitSeg) {
+        const unsigned p1 = min(P, p0 + kEmitSeg);
+        __syncthreads();  // the previous segment's readers are done
+        if (threadIdx.x == 0) {
+            // ranks r0 .. r1-1 cover [p0, p1): r0 = last rank with offset <= p0
+            const unsigned r0 = upper_bound_global(pair_off, (unsigned)N, p0) - 1;
+            const unsigned r1 = upper_bound_global(pair_off, (unsigned)N, p1 - 1);
+            s_r0 = r0;
+            s_nr = min(r1 - r0, (unsigned)kEmitSeg + 1);
         }
-        unsigned incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
+        __syncthreads();
+        const unsigned r0 = s_r0, nr = s_nr;
+        for (unsigned i = threadIdx.x; i < nr; i += kSortBlock) {
+            s_off[i] = pair_off[r0 + i];
+            s_g[i] = order[r0 + i];
         }
-        const unsigned total = __shfl_sync(0xffffffffu, incl, 31);
-        const unsigned off0 = __shfl_sync(0xffffffffu, off, 0);
-        const unsigned excl = incl - cnt;
-        // warp-uniform loop: every lane takes part in every shuffle
-        for (unsigned kb = 0; kb < total; kb += 32) {
-            const unsigned k = kb + lane;
-            // owner: the first lane whose inclusive count exceeds k
-            int sidx = 0;
-#pragma unroll
-            for (int b = 16; b >= 1; b >>= 1) {
-                const unsigned v = __shfl_sync(0xffffffffu, incl, sidx + b - 1);
-                if (v <= k) sidx += b;
+        __syncthreads();
+        for (unsigned p = p0 + threadIdx.x; p < p1; p += kSortBlock) {
+            // owner: last staged rank whose offset <= p
+            unsigned lo = 0, hi = nr;
+            while (hi - lo > 1) {
+                const unsigned mid = (lo + hi) >> 1;
+                if (s_off[mid] <= p) lo = mid; else hi = mid;
             }
-            sidx = min(sidx, 31);
-            const unsigned local = k - __shfl_sync(0xffffffffu, excl, sidx);
-            const unsigned gg = __shfl_sync(0xffffffffu, g, sidx);
-            const int ox = __shfl_sync(0xffffffffu, x0, sidx);
-            const int oy = __shfl_sync(0xffffffffu, y0, sidx);
-            const int ow = __shfl_sync(0xffffffffu, wdt, sidx);
-            const unsigned pos = off0 + k;
-            if (k < total && pos < P) {  // never write past P, even if the caller's counts disagree
-                tkeys[pos] = (unsigned)(oy + (int)(local / (unsigned)ow)) * (unsigned)TX +
-                             (unsigned)(ox + (int)(local % (unsigned)ow));
-                tvals[pos] = gg;
-            }
+            const unsigned g = s_g[lo];
+            const int4 rc = rect[g];
+            const unsigned w = (unsigned)(rc.z - rc.x);
+            const unsigned local = p - s_off[lo];
+            unsigned q = (unsigned)__fdividef((float)local, (float)w);
+            int r = (int)local - (int)(q * w);
+            if (r < 0) { --q; r += (int)w; }
+            else if (r >= (int)w) { ++q; r -= (int)w; }
+            tkeys[p] = (unsigned)(rc.y + (int)q) * (unsigned)TX + (unsigned)(rc.x + r);
+            tvals[p] = g;
         }
     }
 }
 
 // ranges[t] = [first, last + 1) of tile t in the sorted list, found by
-// comparing neighbours; optional 64-bit keys for callers that want them.
+// comparing neighbours; four keys per thread with 16-byte loads, neighbours
+// across lanes by shuffles.  Optional 64-bit keys for callers that want them.
 __global__ void k_ranges(const unsigned* __restrict__ tkeys, const unsigned* __restrict__ ids,
                          const float* __restrict__ depth, const SortMisc* __restrict__ misc, unsigned* __restrict__ ranges,
                          unsigned long long* __restrict__ keys) {
     const unsigned P = misc->p_eff;
+    const unsigned nq = (P + 3) / 4;  // quads, the last one partial
     const unsigned stride = gridDim.x * blockDim.x;
-    for (unsigned k = blockIdx.x * blockDim.x + threadIdx.x; k < P; k += stride) {
-        const unsigned t = tkeys[k];
-        if (k == 0 || tkeys[k - 1] != t) ranges[2 * t] = k;
-        if (k + 1 == P || tkeys[k + 1] != t) ranges[2 * t + 1] = k + 1;
-        if (keys) keys[k] = ((unsigned long long)t << 32) | __float_as_uint(depth[ids[k]]);
+    const int lane = threadIdx.x & 31;
+    // every lane of a warp iterates the same number of times (shuffles below)
+    for (unsigned qb = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); qb < nq; qb += stride) {
+        const unsigned qi = qb + lane;
+        const unsigned k0 = qi * 4;
+        unsigned t[4];
+        if (k0 + 3 < P) {
+            const uint4 v = reinterpret_cast<const uint4*>(tkeys)[qi];
+            t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) t[j] = k0 + j < P ? tkeys[k0 + j] : 0xFFFFFFFFu;
+        }
+        unsigned prev = __shfl_up_sync(0xffffffffu, t[3], 1);
+        unsigned next = __shfl_down_sync(0xffffffffu, t[0], 1);
+        if (lane == 0) prev = (k0 > 0 && k0 - 1 < P) ? tkeys[k0 - 1] : 0xFFFFFFFFu;
+        if (lane == 31) next = (k0 + 4 < P) ? tkeys[k0 + 4] : 0xFFFFFFFFu;
+        if (qi < nq) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const unsigned k = k0 + j;
+                if (k >= P) break;
+                const unsigned before = j == 0 ? prev : t[j - 1];
+                const unsigned after = (j == 3 || k + 1 == P) ? (k + 1 == P ? 0xFFFFFFFFu : next) : t[j + 1];
+                if (k == 0 || before != t[j]) ranges[2 * t[j]] = k;
+                if (k + 1 == P || after != t[j]) ranges[2 * t[j] + 1] = k + 1;
+                if (keys) keys[k] = ((unsigned long long)t[j] << 32) | __float_as_uint(depth[ids[k]]);
+            }
+        }
     }
 }
 
@@ -638,8 +677,10 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     const int tile_bits = ceil_log2((unsigned)T);
     const int tpasses = (tile_bits + 7) / 8;
     {
-        int blocks = (N + kSortBlock - 1) / kSortBlock;
-        if (blocks > 148 * 16) blocks = 148 * 16;
+        // one CTA per 2048 output pairs, up to a few waves (grid-stride beyond)
+        unsigned segs = (capacity + kEmitSeg - 1) / kEmitSeg;
+        int blocks = segs > 148u * 32u ? 148 * 32 : (int)segs;
+        if (blocks < 1) blocks = 1;
         unsigned* emit_vals = tpasses == 0 ? ids : w.tvals0;
         k_emit<<<blocks, kSortBlock, 0, st>>>(N, TX, order, w.pair_off, reinterpret_cast<const int4*>(rect),
                                               tiles_touched, w.misc, w.tkeys0, emit_vals);
@@ -653,8 +694,8 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
 
     // 4. tile ranges (and optional 64-bit keys)
     {
-        int blocks = (int)((capacity + 255u) / 256u);
-        if (blocks > 148 * 8) blocks = 148 * 8;
+        int blocks = (int)((capacity + 1023u) / 1024u);
+        if (blocks > 148 * 16) blocks = 148 * 16;
         if (blocks < 1) blocks = 1;
         k_ranges<<<blocks, 256, 0, st>>>(tkeys_sorted, ids, depth, w.misc, ranges, keys);
         GS_LAUNCH_CHECK();
