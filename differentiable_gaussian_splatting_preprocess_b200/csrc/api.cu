@@ -6,7 +6,7 @@
 #include "gs_internal.cuh"
 
 extern "C" size_t gs_preprocess_ws_bytes(int N);
-extern "C" size_t gs_bin_sort_ws_bytes(int N, unsigned capacity);
+extern "C" size_t gs_bin_sort_ws_bytes(int N, unsigned capacity, int width, int height);
 
 namespace {
 __global__ void k_clear_status(gs::WsHeader* h) { h->status = 0u; }
@@ -31,7 +31,7 @@ extern "C" size_t gs_workspace_bytes(int stage, int N, unsigned capacity, int wi
     if (N < 0 || width < 1 || height < 1) return 0;
     switch (stage) {
         case GS_STAGE_PREPROCESS_FWD: return gs_preprocess_ws_bytes(N);
-        case GS_STAGE_BIN_SORT: return gs_bin_sort_ws_bytes(N, capacity);
+        case GS_STAGE_BIN_SORT: return gs_bin_sort_ws_bytes(N, capacity, width, height);
         default: return 0;
     }
 }

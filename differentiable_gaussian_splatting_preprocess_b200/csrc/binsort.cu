@@ -33,11 +33,14 @@ constexpr int kRadixMax = 256;
 constexpr int kMaxPasses = 8;          // 4 depth passes + up to 3 tile passes (+1 spare)
 constexpr int kScanItems = 8;          // items per thread in the rank-order scan
 constexpr int kScanTile = kSortBlock * kScanItems;
+constexpr int kFusedMaxBits = 8;       // fused binning: TX and TY at most 256
 
 struct SortMisc {
     unsigned n_gauss;    // N
     unsigned p_eff;      // P if it fits the capacity, else 0
-    unsigned pad[62];
+    unsigned ps;         // super-tile pairs if P fits the capacity, else 0
+    unsigned nseg;       // segments of the super-tile lists
+    unsigned pad[60];
 };
 
 struct BinWs {
@@ -45,13 +48,39 @@ struct BinWs {
     SortMisc* misc;
     unsigned *dkeys0, *dvals0, *dkeys1, *dvals1;  // depth sort, N each
     unsigned* pair_off;                            // N + 1
+    unsigned* cnt_rank;                            // N: pairs of each rank (written by the scan's first kernel)
     unsigned* scan_part;                           // ceil(N / kScanTile) + 1
     unsigned *tkeys0, *tvals0, *tkeys1, *tvals1;   // pair sort, capacity each
     unsigned* hist;                                // kMaxPasses * kRadixMax * kSortMaxGrid
     unsigned* totals;                              // kMaxPasses * kRadixMax
+    // super-tile route only (empty otherwise)
+    unsigned* rc_rank;                             // N packed super-tile rectangles in rank order
+    unsigned *owner_lo, *owner_hi;                 // kSortMaxGrid each: ranks owning chunk ends
+    unsigned* cell_ranges;                         // 2 S: each super-tile's slice of the super list
+    unsigned* cell_seg0;                           // S + 1: first segment of each super-tile
+    unsigned *seg_cell, *seg_lo, *seg_hi;          // max_seg each
+    unsigned *seg_cnt, *seg_base;                  // max_seg * kCellTiles each
+    unsigned *tile_cnt, *tile_start;               // T each
+    unsigned short* seg_mask;                      // capacity: tile mask of each cell-list entry
+    unsigned max_seg;
+    int n_cells;                                   // S
 };
 
-size_t carve(void* base, int N, unsigned capacity, BinWs* w) {
+// Super-tiles (cells) of 4 x 4 tiles; a cell's Gaussian list is expanded to
+// its 16 tiles in segments of kSeg list entries.
+constexpr int kSuper = 4;
+constexpr int kCellTiles = kSuper * kSuper;
+constexpr int kSeg = 1024;
+static_assert(kCellTiles <= 32, "a cell's tile mask is one 32-bit word");
+
+// The super-tile route serves images of at most 256 x 256 cells (1024 tiles
+// a side); larger ones take the emit + radix-sort-by-tile-id route.
+inline bool super_binning(int TX, int TY) {
+    const int SX = (TX + kSuper - 1) / kSuper, SY = (TY + kSuper - 1) / kSuper;
+    return SX <= (1 << kFusedMaxBits) && SY <= (1 << kFusedMaxBits);
+}
+
+size_t carve(void* base, int N, unsigned capacity, int TX, int TY, BinWs* w) {
     size_t off = sizeof(WsHeader);
     char* b = reinterpret_cast<char*>(base);
     auto take = [&](size_t bytes) -> void* {
@@ -68,6 +97,7 @@ size_t carve(void* base, int N, unsigned capacity, BinWs* w) {
     t.dkeys1 = (unsigned*)take(n * 4);
     t.dvals1 = (unsigned*)take(n * 4);
     t.pair_off = (unsigned*)take((n + 1) * 4);
+    t.cnt_rank = (unsigned*)take(n * 4);
     t.scan_part = (unsigned*)take(((n + kScanTile - 1) / kScanTile + 1) * 4);
     t.tkeys0 = (unsigned*)take(cap * 4);
     t.tvals0 = (unsigned*)take(cap * 4);
@@ -75,9 +105,42 @@ size_t carve(void* base, int N, unsigned capacity, BinWs* w) {
     t.tvals1 = (unsigned*)take(cap * 4);
     t.hist = (unsigned*)take((size_t)kMaxPasses * kRadixMax * kSortMaxGrid * 4);
     t.totals = (unsigned*)take((size_t)kMaxPasses * kRadixMax * 4);
+    const bool sup = super_binning(TX, TY);
+    const size_t S = sup ? (size_t)((TX + kSuper - 1) / kSuper) * ((TY + kSuper - 1) / kSuper) : 0;
+    const size_t T = sup ? (size_t)TX * TY : 0;
+    t.max_seg = sup ? (unsigned)(cap / kSeg + S + 1) : 0u;
+    t.n_cells = (int)S;
+    const size_t ms = t.max_seg;
+    t.rc_rank = (unsigned*)take(sup ? n * 4 : 0);
+    t.owner_lo = (unsigned*)take((size_t)kSortMaxGrid * 4);
+    t.owner_hi = (unsigned*)take((size_t)kSortMaxGrid * 4);
+    t.cell_ranges = (unsigned*)take(2 * S * 4);
+    t.cell_seg0 = (unsigned*)take((S + 1) * 4);
+    t.seg_cell = (unsigned*)take(ms * 4);
+    t.seg_lo = (unsigned*)take(ms * 4);
+    t.seg_hi = (unsigned*)take(ms * 4);
+    t.seg_cnt = (unsigned*)take(ms * kCellTiles * 4);
+    t.seg_base = (unsigned*)take(ms * kCellTiles * 4);
+    t.tile_cnt = (unsigned*)take(T * 4);
+    t.tile_start = (unsigned*)take(T * 4);
+    t.seg_mask = (unsigned short*)take(sup ? cap * 2 : 0);
     if (w) *w = t;
     return off;
 }
+
+// A visible Gaussian's rectangle of super-tiles in 32 bits (x0, y0 < 256;
+// width and height in 1..256): x0 | (w - 1) << 8 | y0 << 16 | (h - 1) << 24.
+__device__ __forceinline__ int4 super_rect(int4 rc) {
+    return make_int4(rc.x / kSuper, rc.y / kSuper, (rc.z - 1) / kSuper + 1, (rc.w - 1) / kSuper + 1);
+}
+__device__ __forceinline__ unsigned pack_rect(int4 rc) {
+    return (unsigned)rc.x | ((unsigned)(rc.z - rc.x - 1) << 8) | ((unsigned)rc.y << 16) |
+           ((unsigned)(rc.w - rc.y - 1) << 24);
+}
+__device__ __forceinline__ int rect_x0(unsigned p) { return (int)(p & 255u); }
+__device__ __forceinline__ int rect_w(unsigned p) { return (int)((p >> 8) & 255u) + 1; }
+__device__ __forceinline__ int rect_y0(unsigned p) { return (int)((p >> 16) & 255u); }
+__device__ __forceinline__ int rect_h(unsigned p) { return (int)(p >> 24) + 1; }
 
 __device__ __forceinline__ unsigned lanemask_lt() {
     unsigned m;
@@ -94,6 +157,7 @@ __global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const 
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
     for (int i = tid; i < 2 * T; i += stride) ranges[i] = 0u;
     for (int i = tid; i < kMaxPasses * kRadixMax; i += stride) w.totals[i] = 0u;
+    for (int i = tid; i < 2 * w.n_cells; i += stride) w.cell_ranges[i] = 0u;
     for (int i = tid; i < N; i += stride) {
         w.dkeys0[i] = tiles_touched[i] > 0 ? __float_as_uint(depth[i]) : 0xFFFFFFFFu;
         w.dvals0[i] = (unsigned)i;
@@ -128,15 +192,21 @@ struct RadixCfg {
     static constexpr size_t kScatterSmem = (size_t)(4 * kRadix + kWarps * kRadix + 2 * kTileKeys) * sizeof(unsigned);
 };
 
+// Keys per CTA of a pass over n keys on G CTAs: ceil(n / G) rounded up to
+// whole 2048-key tiles (the same for every digit width).
+__host__ __device__ __forceinline__ unsigned chunk_size(unsigned n, unsigned G) {
+    constexpr unsigned tile = 2048;
+    const unsigned long long c = ((unsigned long long)n + G - 1) / G;
+    return (unsigned)((c + tile - 1) / tile * tile);
+}
+
 template <int MAXB>
 __device__ __forceinline__ void chunk_of(unsigned n, unsigned& lo, unsigned& hi) {
-    constexpr unsigned tile = RadixCfg<MAXB>::kTileKeys;
-    const unsigned G = gridDim.x;
-    unsigned chunk = (n + G - 1) / G;
-    chunk = (chunk + tile - 1) / tile * tile;
+    static_assert(RadixCfg<MAXB>::kTileKeys == 2048, "chunk_size assumes 2048-key tiles");
+    const unsigned chunk = chunk_size(n, gridDim.x);
     const unsigned long long l = (unsigned long long)blockIdx.x * chunk;
     lo = l < n ? (unsigned)l : n;
-    hi = min(n, lo + chunk);
+    hi = (unsigned)min((unsigned long long)n, (unsigned long long)lo + chunk);
 }
 
 constexpr unsigned kNoDigit = 0xFFFFFFFFu;
@@ -251,8 +321,9 @@ k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, i
         }
 }
 
-// Stable scatter.  Per tile of 2048 keys, each warp owning a contiguous block
-// of 256 of them (8 rows of 32):
+// Stable scatter of one tile of up to 2048 keys, each warp owning a
+// contiguous block of 256 of them (8 rows of 32), keys and digits already in
+// registers (row j of warp w = tile positions w*256 + j*32 + lane):
 //   1. each warp ranks its keys row by row (digit_peers within the row, plus
 //      a running per-digit count of the warp's earlier rows), so ranks follow
 //      input order within the warp;
@@ -262,6 +333,122 @@ k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, i
 //   3. every key is placed in shared memory at its tile-local sorted position;
 //   4. the regrouped tile is written out in order, so consecutive lanes write
 //      consecutive addresses of one digit's run (coalesced stores).
+// keys_out may be null (values only).  Ends with a block barrier.
+template <int MAXB>
+struct ScatterSmem {
+    using C = RadixCfg<MAXB>;
+    unsigned* base;   // [radix] running global base
+    unsigned* tcnt;   // [radix] this tile's count per digit
+    unsigned* tstart; // [radix] tile-local start per digit
+    unsigned* tbase;  // [radix] global base for this tile
+    unsigned* wcnt;   // [warps][radix] counts, then offsets
+    unsigned* keys;   // [tile (+ padding)] regrouped keys
+    unsigned* vals;   // [tile (+ padding)] regrouped values
+    __device__ ScatterSmem(unsigned char* raw, size_t tile_words) {
+        base = reinterpret_cast<unsigned*>(raw);
+        tcnt = base + C::kRadix;
+        tstart = tcnt + C::kRadix;
+        tbase = tstart + C::kRadix;
+        wcnt = tbase + C::kRadix;
+        keys = wcnt + C::kWarps * C::kRadix;
+        vals = keys + tile_words;
+    }
+    static constexpr size_t bytes(size_t tile_words) {
+        return (size_t)(4 * C::kRadix + C::kWarps * C::kRadix) * sizeof(unsigned) + 2 * tile_words * sizeof(unsigned);
+    }
+};
+
+template <int MAXB>
+__device__ __forceinline__ void scatter_tile(const ScatterSmem<MAXB>& sm, const unsigned (&key)[RadixCfg<MAXB>::kItems],
+                                             const unsigned (&val)[RadixCfg<MAXB>::kItems],
+                                             const unsigned (&d)[RadixCfg<MAXB>::kItems], unsigned tile_n, int shift,
+                                             int bits, unsigned* __restrict__ keys_out,
+                                             unsigned* __restrict__ vals_out) {
+    using C = RadixCfg<MAXB>;
+    const int radix = 1 << bits;
+    const unsigned mask = radix - 1;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt = lanemask_lt();
+    unsigned* wcnt = sm.wcnt + warp * C::kRadix;
+    unsigned rank[C::kItems];
+    for (int dd = lane; dd < radix; dd += 32) wcnt[dd] = 0;
+    __syncwarp();
+    // 1. ranks within the warp, row after row
+#pragma unroll
+    for (int j = 0; j < C::kItems; ++j) {
+        const unsigned peers = digit_peers<MAXB>(d[j], bits);
+        const bool valid = d[j] != kNoDigit;
+        const unsigned before = valid ? wcnt[d[j]] : 0u;
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) wcnt[d[j]] = before + __popc(peers);
+        __syncwarp();
+        rank[j] = before + __popc(peers & lt);
+    }
+    __syncthreads();
+    // 2. per digit: warp offsets in warp order, and the tile count
+    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
+        unsigned run = 0;
+#pragma unroll
+        for (int w = 0; w < C::kWarps; ++w) {
+            const unsigned c = sm.wcnt[w * C::kRadix + dd];
+            sm.wcnt[w * C::kRadix + dd] = run;
+            run += c;
+        }
+        sm.tcnt[dd] = run;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int per = (C::kRadix + 31) / 32;
+        unsigned v[per], sum = 0;
+#pragma unroll
+        for (int k = 0; k < per; ++k) {
+            const int dd = lane * per + k;
+            v[k] = dd < radix ? sm.tcnt[dd] : 0u;
+            sum += v[k];
+        }
+        unsigned incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        unsigned run = incl - sum;
+#pragma unroll
+        for (int k = 0; k < per; ++k) {
+            const int dd = lane * per + k;
+            if (dd < radix) {
+                sm.tstart[dd] = run;
+                sm.tbase[dd] = sm.base[dd];
+                sm.base[dd] += v[k];
+            }
+            run += v[k];
+        }
+    }
+    __syncthreads();
+    // 3. regroup the tile by digit in shared memory
+#pragma unroll
+    for (int j = 0; j < C::kItems; ++j) {
+        if (d[j] != kNoDigit) {
+            const unsigned loc = sm.tstart[d[j]] + wcnt[d[j]] + rank[j];
+            sm.keys[loc] = key[j];
+            sm.vals[loc] = val[j];
+        }
+    }
+    __syncthreads();
+    // 4. write the regrouped tile: consecutive q of one digit go to
+    //    consecutive output positions
+    for (unsigned q = threadIdx.x; q < tile_n; q += kSortBlock) {
+        const unsigned k2 = sm.keys[q];
+        const unsigned dq = (k2 >> shift) & mask;
+        const unsigned pos = sm.tbase[dq] + (q - sm.tstart[dq]);
+        if (keys_out) keys_out[pos] = k2;
+        vals_out[pos] = sm.vals[q];
+    }
+    __syncthreads();  // the next tile reuses every shared array
+}
+
+// Stable scatter pass over keys in global memory: each CTA walks its chunk
+// tile by tile.
 template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict__ vals_in,
@@ -269,27 +456,17 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
                 const unsigned* __restrict__ n_ptr, int shift, int bits, const unsigned* __restrict__ offsets) {
     using C = RadixCfg<MAXB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned* s_base = reinterpret_cast<unsigned*>(smem_raw);   // [radix] running global base
-    unsigned* s_tcnt = s_base + C::kRadix;                      // [radix] this tile's count per digit
-    unsigned* s_tstart = s_tcnt + C::kRadix;                    // [radix] tile-local start per digit
-    unsigned* s_tbase = s_tstart + C::kRadix;                   // [radix] global base for this tile
-    unsigned* s_wcnt = s_tbase + C::kRadix;                     // [warps][radix] counts, then offsets
-    unsigned* s_keys = s_wcnt + C::kWarps * C::kRadix;          // [tile] regrouped keys
-    unsigned* s_vals = s_keys + C::kTileKeys;                   // [tile] regrouped values
+    const ScatterSmem<MAXB> sm(smem_raw, C::kTileKeys);
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
     const unsigned G = gridDim.x;
-    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) s_base[dd] = offsets[(size_t)dd * G + blockIdx.x];
+    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) sm.base[dd] = offsets[(size_t)dd * G + blockIdx.x];
     unsigned lo, hi;
     chunk_of<MAXB>(*n_ptr, lo, hi);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned lt = lanemask_lt();
-    unsigned* wcnt = s_wcnt + warp * C::kRadix;
     for (unsigned base = lo; base < hi; base += C::kTileKeys) {
         const unsigned tile_n = min((unsigned)C::kTileKeys, hi - base);
-        for (int dd = lane; dd < radix; dd += 32) wcnt[dd] = 0;
-        __syncwarp();
-        unsigned key[C::kItems], val[C::kItems], d[C::kItems], rank[C::kItems];
+        unsigned key[C::kItems], val[C::kItems], d[C::kItems];
         const unsigned wbase = base + warp * C::kWarpKeys;
 #pragma unroll
         for (int j = 0; j < C::kItems; ++j) {
@@ -299,92 +476,35 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
             val[j] = valid ? vals_in[i] : 0u;
             d[j] = valid ? (key[j] >> shift) & mask : kNoDigit;
         }
-        // 1. ranks within the warp, row after row
-#pragma unroll
-        for (int j = 0; j < C::kItems; ++j) {
-            const unsigned peers = digit_peers<MAXB>(d[j], bits);
-            const bool valid = d[j] != kNoDigit;
-            const unsigned before = valid ? wcnt[d[j]] : 0u;
-            __syncwarp();
-            if (valid && lane == __ffs(peers) - 1) wcnt[d[j]] = before + __popc(peers);
-            __syncwarp();
-            rank[j] = before + __popc(peers & lt);
-        }
-        __syncthreads();
-        // 2. per digit: warp offsets in warp order, and the tile count
-        for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
-            unsigned run = 0;
-#pragma unroll
-            for (int w = 0; w < C::kWarps; ++w) {
-                const unsigned c = s_wcnt[w * C::kRadix + dd];
-                s_wcnt[w * C::kRadix + dd] = run;
-                run += c;
-            }
-            s_tcnt[dd] = run;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            constexpr int per = (C::kRadix + 31) / 32;
-            unsigned v[per], sum = 0;
-#pragma unroll
-            for (int k = 0; k < per; ++k) {
-                const int dd = lane * per + k;
-                v[k] = dd < radix ? s_tcnt[dd] : 0u;
-                sum += v[k];
-            }
-            unsigned incl = sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            unsigned run = incl - sum;
-#pragma unroll
-            for (int k = 0; k < per; ++k) {
-                const int dd = lane * per + k;
-                if (dd < radix) {
-                    s_tstart[dd] = run;
-                    s_tbase[dd] = s_base[dd];
-                    s_base[dd] += v[k];
-                }
-                run += v[k];
-            }
-        }
-        __syncthreads();
-        // 3. regroup the tile by digit in shared memory
-#pragma unroll
-        for (int j = 0; j < C::kItems; ++j) {
-            if (d[j] != kNoDigit) {
-                const unsigned loc = s_tstart[d[j]] + wcnt[d[j]] + rank[j];
-                s_keys[loc] = key[j];
-                s_vals[loc] = val[j];
-            }
-        }
-        __syncthreads();
-        // 4. write the regrouped tile: consecutive q of one digit go to
-        //    consecutive output positions
-        for (unsigned q = threadIdx.x; q < tile_n; q += kSortBlock) {
-            const unsigned k2 = s_keys[q];
-            const unsigned dq = (k2 >> shift) & mask;
-            const unsigned pos = s_tbase[dq] + (q - s_tstart[dq]);
-            keys_out[pos] = k2;
-            vals_out[pos] = s_vals[q];
-        }
-        __syncthreads();  // the next tile reuses every shared array
+        scatter_tile<MAXB>(sm, key, val, d, tile_n, shift, bits, keys_out, vals_out);
     }
 }
 
 // Exclusive scan, in depth-rank order, of the pair counts:
-// pair_off[r] = sum over ranks r' < r of tiles_touched[order[r']].
+// pair_off[r] = sum over ranks r' < r of cnt_rank[r'], where cnt_rank[r] is
+// the number of tiles of Gaussian order[r] or, with `rect` (super-tile
+// route), of its cells.  The first kernel gathers each rank's count once
+// (and, on the super-tile route, its packed cell rectangle).
 __global__ void __launch_bounds__(kSortBlock)
 k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ tiles_touched,
+                const int4* __restrict__ rect, unsigned* __restrict__ cnt_rank, unsigned* __restrict__ rc_rank,
                 unsigned* __restrict__ part) {
     const int base = blockIdx.x * kScanTile;
     unsigned s = 0;
 #pragma unroll
     for (int k = 0; k < kScanItems; ++k) {
         const int r = base + k * kSortBlock + threadIdx.x;
-        if (r < N) s += tiles_touched[order[r]];
+        if (r < N) {
+            const unsigned g = order[r];
+            unsigned v = tiles_touched[g];
+            if (rect && v) {
+                const int4 sr = super_rect(rect[g]);
+                v = (unsigned)((sr.z - sr.x) * (sr.w - sr.y));
+                rc_rank[r] = pack_rect(sr);
+            }
+            cnt_rank[r] = v;
+            s += v;
+        }
     }
     s = __reduce_add_sync(0xffffffffu, s);
     __shared__ unsigned s_w[kSortBlock / 32];
@@ -397,8 +517,10 @@ k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __res
     }
 }
 
-__global__ void __launch_bounds__(1024) k_scan_top(unsigned* __restrict__ part, int nb) {
-    // exclusive scan of nb partial sums by one CTA, each thread a contiguous run
+__global__ void __launch_bounds__(1024) k_scan_top(unsigned* __restrict__ part, int nb, SortMisc* __restrict__ misc) {
+    // exclusive scan of nb partial sums by one CTA, each thread a contiguous
+    // run; the total (of super-tile pairs, when that is what is scanned) goes
+    // to misc->ps, or 0 if the frame's pairs exceed the capacity
     __shared__ unsigned s_w[32];
     const int per = (nb + 1023) / 1024;
     const int c0 = threadIdx.x * per;
@@ -422,11 +544,17 @@ __global__ void __launch_bounds__(1024) k_scan_top(unsigned* __restrict__ part, 
             part[c0 + k] = run;
             run += c;
         }
+    if (threadIdx.x == 1023) misc->ps = misc->p_eff ? run : 0u;
 }
 
+// With `owner_lo` (super-tile route, G CTAs per pair pass), also records for
+// every chunk c of the pair stream the rank owning its first pair
+// (owner_lo[c]) and its last pair (owner_hi[c]): each rank checks the chunk
+// boundaries inside its own pair range, so no search is needed later.
 __global__ void __launch_bounds__(kSortBlock)
-k_scan_down(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ tiles_touched,
-            const unsigned* __restrict__ part, unsigned* __restrict__ pair_off) {
+k_scan_down(int N, const unsigned* __restrict__ cnt_rank, const unsigned* __restrict__ part,
+            unsigned* __restrict__ pair_off, const SortMisc* __restrict__ misc, unsigned G,
+            unsigned* __restrict__ owner_lo, unsigned* __restrict__ owner_hi) {
     // each thread owns kScanItems consecutive ranks
     const int base = blockIdx.x * kScanTile + threadIdx.x * kScanItems;
     unsigned v[kScanItems];
@@ -434,7 +562,7 @@ k_scan_down(int N, const unsigned* __restrict__ order, const unsigned* __restric
 #pragma unroll
     for (int k = 0; k < kScanItems; ++k) {
         const int r = base + k;
-        v[k] = r < N ? tiles_touched[order[r]] : 0u;
+        v[k] = r < N ? cnt_rank[r] : 0u;
         local += v[k];
     }
     __shared__ unsigned s_w[kSortBlock / 32];
@@ -449,10 +577,20 @@ k_scan_down(int N, const unsigned* __restrict__ order, const unsigned* __restric
     unsigned wbase = 0;
     for (int k = 0; k < warp; ++k) wbase += s_w[k];
     unsigned run = part[blockIdx.x] + wbase + incl - local;
+    const unsigned P = owner_lo ? misc->ps : 0u;
+    const unsigned long long chunk = P ? chunk_size(P, G) : 1ull;
 #pragma unroll
     for (int k = 0; k < kScanItems; ++k) {
         const int r = base + k;
         if (r < N) pair_off[r] = run;
+        if (P && v[k] && r < N) {
+            const unsigned long long off = run, e = off + v[k];
+            for (unsigned long long c = off / chunk; c * chunk < e && c < G; ++c) {
+                if (c * chunk >= off) owner_lo[c] = (unsigned)r;
+                const unsigned long long last = min((c + 1) * chunk, (unsigned long long)P) - 1;
+                if (last >= off && last < e) owner_hi[c] = (unsigned)r;
+            }
+        }
         run += v[k];
     }
 }
@@ -566,6 +704,481 @@ __global__ void k_ranges(const unsigned* __restrict__ tkeys, const unsigned* __r
     }
 }
 
+// ---------------------------------------------------------------------------
+// Super-tile binning (images of at most 256 x 256 cells of 4 x 4 tiles).
+// Most pairs come from Gaussians that cover many tiles, so instead
+// of sorting every (tile, Gaussian) pair, the Gaussians are first binned to
+// super-tiles (cells), which yields far fewer pairs, and each super-tile's
+// depth-ordered Gaussian list is then expanded to its 16 tiles directly into
+// the final per-tile lists:
+//   1. cell binning: the (cell, Gaussian) pairs of the rank-order stream are
+//      stably sorted by cell; the cell order cy * SX + cx equals the
+//      lexicographic (cy, cx) order, so this is a stable pass on cx followed
+//      by a stable pass on cy.  The first pass does not read a materialised
+//      pair list: it generates the pairs of its chunk of the stream on the
+//      fly (Gaussian by Gaussian, each cell rectangle row-major) and ranks
+//      them by cx; its histogram comes from the cell rectangles directly (a
+//      difference array over cx).  Intermediate key: cy << 16 | cx.
+//   2. each cell's list is cut into segments of kSeg entries; per segment and
+//      tile of the cell, the number of its Gaussians touching the tile
+//      (warp ballots over the 16-bit tile masks);
+//   3. prefix sums give every tile's range and every (segment, tile) base;
+//   4. each segment writes its Gaussians into the tiles' lists: for every
+//      tile bit, a ballot ranks the warp's Gaussians touching that tile, so
+//      consecutive lanes write consecutive positions.
+// Within a tile the order is the cell list's order, which is rank order, so
+// the result is the (tile, depth, id) order.
+constexpr int kGenWin = 9 * kSortBlock;   // staged ranks per 2048-pair tile (at most 2049 needed)
+constexpr int kPadTile = RadixCfg<8>::kTileKeys + RadixCfg<8>::kTileKeys / 32;
+
+// Padded shared-memory index: one spare word per 32, so that thread t's
+// consecutive slots 8t .. 8t+7 and a warp's row of 32 are both free of bank
+// conflicts.
+__device__ __forceinline__ unsigned pad_idx(unsigned q) { return q + (q >> 5); }
+
+// Per-CTA x histogram of the CTA's chunk of the cell-pair stream (the chunk that
+// k_gen_scatter will rank).  Gaussians entirely inside the chunk add their
+// height to tx in [x0, x0 + w) through a difference array; the (at most two)
+// Gaussians cut by the chunk's ends are counted pair by pair.
+template <int MAXB>
+__global__ void __launch_bounds__(kSortBlock)
+k_gen_hist(const unsigned* __restrict__ pair_off, const unsigned* __restrict__ rc_rank,
+           const unsigned* __restrict__ n_ptr, const unsigned* __restrict__ owner_lo,
+           const unsigned* __restrict__ owner_hi, unsigned* __restrict__ hist, unsigned* __restrict__ totals) {
+    using C = RadixCfg<MAXB>;
+    constexpr int kU = 4;  // ranks per thread in flight
+    __shared__ int s_d[C::kRadix + 1];
+    const unsigned P = *n_ptr;
+    for (int i = threadIdx.x; i <= C::kRadix; i += kSortBlock) s_d[i] = 0;
+    unsigned lo, hi;
+    chunk_of<MAXB>(P, lo, hi);
+    __syncthreads();
+    if (lo < hi) {
+        const unsigned ra = owner_lo[blockIdx.x], rb = owner_hi[blockIdx.x];
+        for (unsigned rbase = ra; rbase <= rb; rbase += kU * kSortBlock) {
+            unsigned off[kU], rc[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const unsigned r = rbase + u * kSortBlock + threadIdx.x;
+                const bool ok = r <= rb;
+                off[u] = ok ? pair_off[r] : 0xFFFFFFFFu;
+                rc[u] = ok ? rc_rank[r] : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                if (off[u] == 0xFFFFFFFFu) continue;
+                const int x0 = rect_x0(rc[u]), w = rect_w(rc[u]), h = rect_h(rc[u]);
+                const unsigned n = (unsigned)(w * h);
+                if (off[u] >= lo && off[u] + n <= hi) {
+                    atomicAdd(&s_d[x0], h);
+                    atomicAdd(&s_d[x0 + w], -h);
+                }
+            }
+        }
+        // the cut Gaussians, pair by pair, by the whole CTA
+        for (int e = 0; e < 2; ++e) {
+            const unsigned r = e == 0 ? ra : rb;
+            if (e == 1 && rb == ra) break;
+            const unsigned rc = rc_rank[r];
+            const unsigned off = pair_off[r];
+            const unsigned w = (unsigned)rect_w(rc);
+            const unsigned n = w * (unsigned)rect_h(rc);
+            if (off >= lo && off + n <= hi) continue;  // not cut: counted above
+            const unsigned a = max(off, lo) - off, b = min(off + n, hi) - off;
+            for (unsigned l = a + threadIdx.x; l < b; l += kSortBlock) {
+                const int tx = rect_x0(rc) + (int)(l % w);
+                atomicAdd(&s_d[tx], 1);
+                atomicAdd(&s_d[tx + 1], -1);
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        // inclusive prefix of the difference array: the count per digit
+        const int lane = threadIdx.x;
+        constexpr int per = C::kRadix / 32;
+        int v[per], sum = 0;
+#pragma unroll
+        for (int k = 0; k < per; ++k) {
+            v[k] = s_d[lane * per + k];
+            sum += v[k];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int run = incl - sum;
+        const unsigned G = gridDim.x;
+#pragma unroll
+        for (int k = 0; k < per; ++k) {
+            run += v[k];
+            const int dd = lane * per + k;
+            hist[(size_t)dd * G + blockIdx.x] = (unsigned)run;
+            if (run) atomicAdd(&totals[dd], (unsigned)run);
+        }
+    }
+}
+
+// First stable pass of the fused binning: per tile of 2048 consecutive pairs
+// of the rank-order stream, stage the ranks that own them (offsets, ids,
+// packed rectangles; three independent coalesced loads), generate the pairs
+// (thread t: tile slots 8t .. 8t+7, one binary search for the first slot,
+// then a walk), and hand them to scatter_tile ranked by tx.
+template <int MAXB>
+__global__ void __launch_bounds__(kSortBlock)
+k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
+              const unsigned* __restrict__ rc_rank, const unsigned* __restrict__ n_ptr,
+              const unsigned* __restrict__ owner_lo, int bits, const unsigned* __restrict__ offsets,
+              unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out) {
+    using C = RadixCfg<MAXB>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const ScatterSmem<MAXB> sm(smem_raw, kPadTile);
+    unsigned* s_off = sm.vals + kPadTile;  // [kGenWin] staged pair offsets
+    unsigned* s_g = s_off + kGenWin;      // [kGenWin] staged ids
+    unsigned* s_rc = s_g + kGenWin;       // [kGenWin] staged packed rectangles
+    __shared__ unsigned s_r0;
+    const int radix = 1 << bits;
+    const unsigned mask = radix - 1;
+    const unsigned G = gridDim.x;
+    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) sm.base[dd] = offsets[(size_t)dd * G + blockIdx.x];
+    const unsigned P = *n_ptr;
+    unsigned lo, hi;
+    chunk_of<MAXB>(P, lo, hi);
+    if (threadIdx.x == 0 && lo < hi) s_r0 = owner_lo[blockIdx.x];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (unsigned base = lo; base < hi; base += C::kTileKeys) {
+        const unsigned tile_n = min((unsigned)C::kTileKeys, hi - base);
+        const unsigned end = base + tile_n;
+        __syncthreads();  // s_r0 written; the previous tile is finished
+        const unsigned r0 = s_r0;
+        // stage the ranks with offsets below `end` (a prefix: offsets of
+        // visible ranks increase strictly, culled ranks sit at P)
+        unsigned nr = 0;
+        for (int round = 0; round * kSortBlock < kGenWin; ++round) {
+            const unsigned idx = round * kSortBlock + threadIdx.x;
+            const unsigned r = r0 + idx;
+            const bool inr = r < (unsigned)N;
+            const unsigned off = inr ? pair_off[r] : 0xFFFFFFFFu;
+            const unsigned g = inr ? order[r] : 0u;
+            const unsigned rc = inr ? rc_rank[r] : 0u;
+            const bool in = off < end;
+            if (in) {
+                s_off[idx] = off;
+                s_g[idx] = g;
+                s_rc[idx] = rc;
+            }
+            const int c = __syncthreads_count(in);
+            nr += (unsigned)c;
+            if (c < kSortBlock) break;
+        }
+        // owner of the next tile's first pair: the next rank if it starts there
+        if (threadIdx.x == 0) {
+            const unsigned nx = r0 + nr;
+            s_r0 = (nx < (unsigned)N && pair_off[nx] == end) ? nx : nx - 1;
+        }
+        // generate this thread's slots into the padded key/value arrays
+        const unsigned q0 = threadIdx.x * C::kItems;
+        if (q0 < tile_n) {
+            unsigned p = base + q0;
+            unsigned i = 0, top = nr;
+            while (top - i > 1) {
+                const unsigned mid = (i + top) >> 1;
+                if (s_off[mid] <= p) i = mid; else top = mid;
+            }
+            unsigned rc = s_rc[i], g = s_g[i];
+            int x0 = rect_x0(rc), x1 = x0 + rect_w(rc);
+            const unsigned w = (unsigned)(x1 - x0);
+            const unsigned local = p - s_off[i];
+            unsigned qq = (unsigned)__fdividef((float)local, (float)w);
+            int rr = (int)local - (int)(qq * w);
+            if (rr < 0) { --qq; rr += (int)w; }
+            else if (rr >= (int)w) { ++qq; rr -= (int)w; }
+            int tx = x0 + rr, ty = rect_y0(rc) + (int)qq;
+#pragma unroll
+            for (int j = 0; j < C::kItems; ++j) {
+                const unsigned q = q0 + j;
+                if (q < tile_n) {
+                    sm.keys[pad_idx(q)] = ((unsigned)ty << 16) | (unsigned)tx;
+                    sm.vals[pad_idx(q)] = g;
+                    ++p;
+                    if (i + 1 < nr && s_off[i + 1] == p) {
+                        ++i;
+                        rc = s_rc[i];
+                        g = s_g[i];
+                        x0 = rect_x0(rc);
+                        x1 = x0 + rect_w(rc);
+                        tx = x0;
+                        ty = rect_y0(rc);
+                    } else if (++tx == x1) {
+                        tx = x0;
+                        ++ty;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        unsigned key[C::kItems], val[C::kItems], d[C::kItems];
+        const unsigned wq = warp * C::kWarpKeys;
+#pragma unroll
+        for (int j = 0; j < C::kItems; ++j) {
+            const unsigned q = wq + j * 32 + lane;
+            const bool valid = q < tile_n;
+            key[j] = valid ? sm.keys[pad_idx(q)] : 0u;
+            val[j] = valid ? sm.vals[pad_idx(q)] : 0u;
+            d[j] = valid ? key[j] & mask : kNoDigit;
+        }
+        // scatter_tile's first barrier orders these reads before its regroup
+        scatter_tile<MAXB>(sm, key, val, d, tile_n, 0, bits, keys_out, vals_out);
+    }
+}
+
+template <int MAXB>
+constexpr size_t gen_scatter_smem() {
+    return ScatterSmem<MAXB>::bytes(kPadTile) + 3 * (size_t)kGenWin * sizeof(unsigned);
+}
+
+// Cell ranges of the cell-sorted list by comparing neighbours (keys
+// cy << 16 | cx); empty cells keep (0, 0).
+__global__ void k_cell_ranges(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ n_ptr, int SX,
+                              unsigned* __restrict__ cell_ranges) {
+    const unsigned n = *n_ptr;
+    for (unsigned k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
+        const unsigned key = ckeys[k];
+        const unsigned c = (key >> 16) * (unsigned)SX + (key & 0xFFFFu);
+        if (k == 0 || ckeys[k - 1] != key) cell_ranges[2 * c] = k;
+        if (k + 1 == n || ckeys[k + 1] != key) cell_ranges[2 * c + 1] = k + 1;
+    }
+}
+
+// Segments of the cell lists (one CTA): cell c gets ceil(len / kSeg)
+// segments, numbered in cell order; cell_seg0[c] is its first.
+__global__ void __launch_bounds__(1024)
+k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restrict__ cell_seg0,
+            unsigned* __restrict__ seg_cell, unsigned* __restrict__ seg_lo, unsigned* __restrict__ seg_hi,
+            SortMisc* __restrict__ misc) {
+    __shared__ unsigned s_w[32];
+    const int per = (S + 1023) / 1024;
+    const int c0 = threadIdx.x * per;
+    unsigned local = 0;
+    for (int k = 0; k < per; ++k) {
+        const int c = c0 + k;
+        if (c < S) local += (cell_ranges[2 * c + 1] - cell_ranges[2 * c] + kSeg - 1) / kSeg;
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_w[warp] = incl;
+    __syncthreads();
+    unsigned wbase = 0;
+    for (int k = 0; k < warp; ++k) wbase += s_w[k];
+    unsigned run = wbase + incl - local;
+    for (int k = 0; k < per; ++k) {
+        const int c = c0 + k;
+        if (c < S) {
+            cell_seg0[c] = run;
+            const unsigned a = cell_ranges[2 * c], b = cell_ranges[2 * c + 1];
+            for (unsigned lo = a; lo < b; lo += kSeg, ++run) {
+                seg_cell[run] = (unsigned)c;
+                seg_lo[run] = lo;
+                seg_hi[run] = min(b, lo + kSeg);
+            }
+        }
+    }
+    if (threadIdx.x == 1023) {
+        cell_seg0[S] = run;
+        misc->nseg = run;
+    }
+}
+
+// Mask of the tiles of cell (cx, cy) that tile rectangle rc covers; bit
+// ly * kSuper + lx is tile (kSuper cy + ly, kSuper cx + lx).
+__device__ __forceinline__ unsigned cell_mask(int4 rc, int cx, int cy) {
+    constexpr unsigned kRep = 0x1111u;  // one bit per row of 4
+    static_assert(kSuper == 4, "row replication constant assumes 4 x 4 cells");
+    const int lx0 = max(rc.x - kSuper * cx, 0), lx1 = min(rc.z - kSuper * cx, kSuper);
+    const int ly0 = max(rc.y - kSuper * cy, 0), ly1 = min(rc.w - kSuper * cy, kSuper);
+    if (lx1 <= lx0 || ly1 <= ly0) return 0u;
+    const unsigned row = (((1u << (lx1 - lx0)) - 1u) << lx0) * kRep;
+    const unsigned rows = ((1u << (kSuper * (ly1 - ly0))) - 1u) << (kSuper * ly0);
+    return row & rows;
+}
+
+// Per segment: count, per tile of its cell, the segment's Gaussians touching
+// it.  Warps count with one ballot per tile bit present in the warp.  Each
+// entry's tile mask is kept for k_seg_emit.
+__global__ void __launch_bounds__(kSortBlock)
+k_seg_count(int SX, const unsigned* __restrict__ clist, const int4* __restrict__ rect,
+            const unsigned* __restrict__ seg_cell, const unsigned* __restrict__ seg_lo,
+            const unsigned* __restrict__ seg_hi, const SortMisc* __restrict__ misc, unsigned* __restrict__ seg_cnt,
+            unsigned short* __restrict__ seg_mask) {
+    __shared__ unsigned s_c[kSortBlock / 32][kCellTiles];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned nseg = misc->nseg;
+    for (unsigned k = blockIdx.x; k < nseg; k += gridDim.x) {
+        if (lane < kCellTiles) s_c[warp][lane] = 0u;
+        __syncwarp();
+        const unsigned c = seg_cell[k], lo = seg_lo[k], hi = seg_hi[k];
+        const int cx = (int)(c % (unsigned)SX), cy = (int)(c / (unsigned)SX);
+        for (unsigned base = lo; base < hi; base += kSortBlock) {
+            const unsigned i = base + threadIdx.x;
+            const unsigned m = i < hi ? cell_mask(rect[clist[i]], cx, cy) : 0u;
+            if (i < hi) seg_mask[i] = (unsigned short)m;
+            for (unsigned u = __reduce_or_sync(0xffffffffu, m); u; u &= u - 1) {
+                const int b = __ffs(u) - 1;
+                const unsigned bal = __ballot_sync(0xffffffffu, (m >> b) & 1u);
+                if (lane == 0) s_c[warp][b] += __popc(bal);
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < kCellTiles) {
+            unsigned t = 0;
+#pragma unroll
+            for (int w = 0; w < kSortBlock / 32; ++w) t += s_c[w][threadIdx.x];
+            seg_cnt[(size_t)k * kCellTiles + threadIdx.x] = t;
+        }
+        __syncthreads();
+    }
+}
+
+// One thread per (cell, tile bit): exclusive prefix of the per-segment
+// counts over the cell's segments, and the tile's total.
+__global__ void __launch_bounds__(kCellTiles)
+k_cell_scan(int TX, int TY, int SX, const unsigned* __restrict__ cell_seg0, const unsigned* __restrict__ seg_cnt,
+            unsigned* __restrict__ seg_base, unsigned* __restrict__ tile_cnt) {
+    const unsigned c = blockIdx.x;
+    const int b = threadIdx.x;
+    const unsigned k0 = cell_seg0[c], k1 = cell_seg0[c + 1];
+    unsigned run = 0;
+    for (unsigned k = k0; k < k1; ++k) {
+        const unsigned v = seg_cnt[(size_t)k * kCellTiles + b];
+        seg_base[(size_t)k * kCellTiles + b] = run;
+        run += v;
+    }
+    const int tx = kSuper * (int)(c % (unsigned)SX) + b % kSuper, ty = kSuper * (int)(c / (unsigned)SX) + b / kSuper;
+    if (tx < TX && ty < TY) tile_cnt[ty * TX + tx] = run;
+}
+
+// Exclusive scan of the tile counts in tile order (one CTA, 4096 tiles per
+// round, four consecutive tiles per thread): tile starts and ranges; empty
+// tiles get (0, 0).
+__global__ void __launch_bounds__(1024)
+k_tile_scan(int T, const unsigned* __restrict__ tile_cnt, unsigned* __restrict__ tile_start,
+            unsigned* __restrict__ ranges) {
+    __shared__ unsigned s_w[32];
+    __shared__ unsigned s_carry;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) s_carry = 0u;
+    for (int t0 = 0; t0 < T; t0 += 4096) {
+        const int t = t0 + 4 * threadIdx.x;
+        unsigned v[4], local = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[j] = t + j < T ? tile_cnt[t + j] : 0u;
+            local += v[j];
+        }
+        unsigned incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        __syncthreads();  // s_w and s_carry of the previous round are consumed
+        if (lane == 31) s_w[warp] = incl;
+        __syncthreads();
+        unsigned wbase = 0;
+        for (int k = 0; k < warp; ++k) wbase += s_w[k];
+        unsigned run = s_carry + wbase + incl - local;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (t + j < T) {
+                tile_start[t + j] = run;
+                ranges[2 * (t + j)] = v[j] ? run : 0u;
+                ranges[2 * (t + j) + 1] = v[j] ? run + v[j] : 0u;
+            }
+            run += v[j];
+        }
+        __syncthreads();  // every thread has read s_carry
+        if (threadIdx.x == 1023) s_carry = run;
+    }
+}
+
+// Per segment: write its Gaussians into the lists of its cell's tiles.  Per
+// chunk of 256 list entries: each warp counts its Gaussians per tile bit
+// (ballots), one thread per bit turns the warps' counts into bases (warp
+// order after the running base), then each warp writes, per tile bit, its
+// Gaussians at base + ballot rank: consecutive lanes, consecutive addresses.
+// Optional 64-bit (tile << 32 | depth bits) keys.
+__global__ void __launch_bounds__(kSortBlock)
+k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const unsigned short* __restrict__ seg_mask,
+           const float* __restrict__ depth, const unsigned* __restrict__ seg_cell,
+           const unsigned* __restrict__ seg_lo, const unsigned* __restrict__ seg_hi,
+           const unsigned* __restrict__ seg_base, const unsigned* __restrict__ tile_start,
+           const SortMisc* __restrict__ misc, unsigned* __restrict__ ids, unsigned long long* __restrict__ keys) {
+    constexpr int kW = kSortBlock / 32;
+    __shared__ unsigned s_base[kCellTiles];
+    __shared__ unsigned s_wb[kW][kCellTiles];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt = lanemask_lt();
+    const unsigned nseg = misc->nseg;
+    for (unsigned k = blockIdx.x; k < nseg; k += gridDim.x) {
+        const unsigned c = seg_cell[k], lo = seg_lo[k], hi = seg_hi[k];
+        const int cx = (int)(c % (unsigned)SX), cy = (int)(c / (unsigned)SX);
+        if (threadIdx.x < kCellTiles) {
+            const int b = threadIdx.x;
+            const int tx = kSuper * cx + b % kSuper, ty = kSuper * cy + b / kSuper;
+            s_base[b] = (tx < TX && ty < TY) ? tile_start[ty * TX + tx] + seg_base[(size_t)k * kCellTiles + b] : 0u;
+        }
+        for (unsigned base = lo; base < hi; base += kSortBlock) {
+            const unsigned i = base + threadIdx.x;
+            const unsigned g = i < hi ? clist[i] : 0u;
+            const unsigned m = i < hi ? (unsigned)seg_mask[i] : 0u;
+            const unsigned un = __reduce_or_sync(0xffffffffu, m);
+            // this warp's count per tile bit
+            if (lane < kCellTiles) s_wb[warp][lane] = 0u;
+            __syncwarp();
+            for (unsigned u = un; u; u &= u - 1) {
+                const int b = __ffs(u) - 1;
+                const unsigned bal = __ballot_sync(0xffffffffu, (m >> b) & 1u);
+                if (lane == 0) s_wb[warp][b] = __popc(bal);
+            }
+            __syncthreads();
+            if (threadIdx.x < kCellTiles) {
+                const int b = threadIdx.x;
+                unsigned run = s_base[b];
+#pragma unroll
+                for (int w = 0; w < kW; ++w) {
+                    const unsigned cnt = s_wb[w][b];
+                    s_wb[w][b] = run;
+                    run += cnt;
+                }
+                s_base[b] = run;
+            }
+            __syncthreads();
+            const float dg = (keys && m) ? depth[g] : 0.0f;
+            for (unsigned u = un; u; u &= u - 1) {
+                const int b = __ffs(u) - 1;
+                const bool mine = (m >> b) & 1u;
+                const unsigned bal = __ballot_sync(0xffffffffu, mine);
+                if (mine) {
+                    const unsigned pos = s_wb[warp][b] + __popc(bal & lt);
+                    ids[pos] = g;
+                    if (keys) {
+                        const unsigned t = (unsigned)((kSuper * cy + b / kSuper) * TX + kSuper * cx + b % kSuper);
+                        keys[pos] = ((unsigned long long)t << 32) | __float_as_uint(dg);
+                    }
+                }
+            }
+        }
+        __syncthreads();  // s_base and s_wb are rebuilt for the next segment
+    }
+}
+
 int ceil_log2(unsigned x) {
     int b = 0;
     while ((1ull << b) < x) ++b;
@@ -628,9 +1241,9 @@ int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, un
 
 using namespace gs;
 
-extern "C" size_t gs_bin_sort_ws_bytes(int N, unsigned capacity) {
-    if (N < 0) return 0;
-    return carve(nullptr, N, capacity, nullptr);
+extern "C" size_t gs_bin_sort_ws_bytes(int N, unsigned capacity, int width, int height) {
+    if (N < 0 || width < 1 || height < 1) return 0;
+    return carve(nullptr, N, capacity, (width + kTile - 1) / kTile, (height + kTile - 1) / kTile, nullptr);
 }
 
 extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, const int* rect,
@@ -640,12 +1253,16 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     if (!camera_ok(cam) || N < 0 || !d_num_pairs || !ranges || !ws) return GS_ERR_INVALID_ARG;
     if (N > 0 && (!depth || !rect || !tiles_touched)) return GS_ERR_INVALID_ARG;
     if (capacity > 0 && !ids) return GS_ERR_INVALID_ARG;
-    if (!aligned(ws, 256) || ws_bytes < gs_bin_sort_ws_bytes(N, capacity)) return GS_ERR_INVALID_ARG;
+    if (!aligned(ws, 256) || ws_bytes < gs_bin_sort_ws_bytes(N, capacity, cam->width, cam->height))
+        return GS_ERR_INVALID_ARG;
     if (rect && !aligned(rect, 16)) return GS_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    BinWs w;
-    carve(ws, N, capacity, &w);
     const int TX = tiles_x(*cam), TY = tiles_y(*cam), T = TX * TY;
+    BinWs w;
+    carve(ws, N, capacity, TX, TY, &w);
+    const bool sup = w.n_cells > 0 && capacity > 0;  // super-tile route
+    const int SX = (TX + kSuper - 1) / kSuper, SY = (TY + kSuper - 1) / kSuper;
+    const int4* rect4 = reinterpret_cast<const int4*>(rect);
 
     {
         int work = N > 2 * T ? N : 2 * T;
@@ -665,13 +1282,66 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     const unsigned* order = (dpasses % 2 == 0) ? w.dvals0 : w.dvals1;
     GS_LAUNCH_CHECK();
 
-    // 2. pair offsets in rank order
+    // 2. pair offsets in rank order (of super-tile pairs on the super-tile route)
     const int nb = (N + kScanTile - 1) / kScanTile;
-    k_scan_partials<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, w.scan_part);
-    k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb);
-    k_scan_down<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, w.scan_part, w.pair_off);
+    const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
+    k_scan_partials<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
+                                               w.rc_rank, w.scan_part);
+    k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb, w.misc);
+    k_scan_down<<<nb, kSortBlock, 0, st>>>(N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
+                                           (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi);
     GS_LAUNCH_CHECK();
     if (capacity == 0) return GS_OK;
+
+    if (sup) {
+        // 3'. super-tile route: bin to cells (generate + stable pass on cx,
+        //     stable pass on cy), cell ranges, segments, per-tile counts,
+        //     tile ranges, expansion into the tile lists
+        const unsigned* ps = &w.misc->ps;
+        const int bx = ceil_log2((unsigned)SX), by = ceil_log2((unsigned)SY);
+        unsigned* h1 = w.hist + (size_t)4 * kRadixMax * kSortMaxGrid;
+        unsigned* t1 = w.totals + (size_t)4 * kRadixMax;
+        if (bx <= 7) {
+            k_gen_hist<7><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1);
+            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp);
+            cudaFuncSetAttribute(k_gen_scatter<7>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gen_scatter_smem<7>());
+            k_gen_scatter<7><<<Gp, kSortBlock, gen_scatter_smem<7>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
+                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0);
+        } else {
+            k_gen_hist<8><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1);
+            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp);
+            cudaFuncSetAttribute(k_gen_scatter<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gen_scatter_smem<8>());
+            k_gen_scatter<8><<<Gp, kSortBlock, gen_scatter_smem<8>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
+                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0);
+        }
+        GS_LAUNCH_CHECK();
+        unsigned* h2 = w.hist + (size_t)5 * kRadixMax * kSortMaxGrid;
+        unsigned* t2 = w.totals + (size_t)5 * kRadixMax;
+        if (by <= 7)
+            radix_pass<7>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+        else
+            radix_pass<8>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+        GS_LAUNCH_CHECK();
+        {
+            int blocks = (int)((capacity + 1023u) / 1024u);
+            if (blocks > 148 * 16) blocks = 148 * 16;
+            if (blocks < 1) blocks = 1;
+            k_cell_ranges<<<blocks, 256, 0, st>>>(w.tkeys1, ps, SX, w.cell_ranges);
+        }
+        const int S = SX * SY;
+        k_seg_table<<<1, 1024, 0, st>>>(S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc);
+        const int gseg = (int)(w.max_seg < 148u * 8u ? w.max_seg : 148u * 8u);
+        k_seg_count<<<gseg, kSortBlock, 0, st>>>(SX, w.tvals1, rect4, w.seg_cell, w.seg_lo, w.seg_hi, w.misc,
+                                                 w.seg_cnt, w.seg_mask);
+        k_cell_scan<<<S, kCellTiles, 0, st>>>(TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt);
+        k_tile_scan<<<1, 1024, 0, st>>>(T, w.tile_cnt, w.tile_start, ranges);
+        k_seg_emit<<<gseg, kSortBlock, 0, st>>>(TX, TY, SX, w.tvals1, w.seg_mask, depth, w.seg_cell, w.seg_lo,
+                                                w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys);
+        GS_LAUNCH_CHECK();
+        return GS_OK;
+    }
 
     // 3. emit pairs in rank order, then a stable sort by tile id
     const int tile_bits = ceil_log2((unsigned)T);
@@ -686,7 +1356,6 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
                                               tiles_touched, w.misc, w.tkeys0, emit_vals);
         GS_LAUNCH_CHECK();
     }
-    const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
     unsigned* tkeys_sorted = nullptr;
     radix_sort(st, Gp, &w.misc->p_eff, tile_bits, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, ids, &tkeys_sorted,
                w.hist, w.totals, 4);

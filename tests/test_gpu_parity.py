@@ -213,6 +213,23 @@ def test_ragged_and_tiny_images(W, H):
         assert rel_l2(to_np(r["grads"][k]), f[k]) <= GRAD_REL_L2, k
 
 
+@pytest.mark.parametrize("W,H,n,sigma_mult", [(4200, 24, 80, 3.0), (4096, 40, 80, 3.0), (40, 4096, 80, 3.0),
+                                              (800, 608, 2000, 1e3)])
+def test_binning_routes(W, H, n, sigma_mult):
+    """Both binning routes against the oracle's sort: more than 256 tile
+    columns (emit + sort by tile id), exactly 256 columns or rows (fused,
+    8-bit passes), and pairs of whole-image Gaussians cut by every chunk
+    boundary of the fused first pass."""
+    sc = _tiny(n=n, width=W, height=H, seed=W + 3 * H, z_range=(2.0, 6.0), sigma_mult=sigma_mult)
+    cam = sc.cameras[0].replace(fx=float(W), fy=float(H), cx=W / 2.0, cy=H / 2.0)
+    sc.cameras[0] = cam
+    gs = GpuScene(sc)
+    g = frame_np(run_gpu(gs, cam)["frame"])
+    pre = _check_preprocess(sc, cam, g)
+    assert g["num_pairs"] > 0
+    _check_bins(cam, g, pre)
+
+
 def test_no_thresholds_and_large_support():
     """alpha_min = T_min = 0 and a support radius covering the whole image."""
     sc = _tiny(n=24, width=64, height=48, seed=11, sigma_mult=1e3, alpha_min=0.0, T_min=0.0)

@@ -46,7 +46,9 @@ def _worker(rank, world, port, n_cams, N, out_q, fail_rank):
         grads["_seen"] = []
         MV.render_views_distributed(list(range(n_cams)), params, [None] * n_cams, render_fn=_fake_render,
                                     grads=grads)
-        out_q.put((rank, "ok", grads["_seen"], {k: grads[k].clone() for k in MV.GRAD_KEYS}))
+        # numpy copies: torch tensors would travel by file-descriptor sharing,
+        # which needs this process alive when the parent unpickles them
+        out_q.put((rank, "ok", grads["_seen"], {k: grads[k].numpy().copy() for k in MV.GRAD_KEYS}))
     except Exception as e:  # reported to the parent, never swallowed
         out_q.put((rank, "error", type(e).__name__, str(e)[:200]))
     finally:
@@ -99,7 +101,7 @@ def test_two_ranks_sum_every_camera_once(n_cams):
     total = float(sum(c + 1 for c in range(n_cams)))
     for r in res:
         for k, v in r[3].items():
-            assert torch.all(v == total), k
+            assert (v == total).all(), k
 
 
 def test_failed_rank_is_reported_not_hung():
