@@ -29,7 +29,7 @@ GS_STAGE_BIN_SORT = 1
 TILE = 16
 
 # Every symbol include/gs.h declares.
-EXPORTED = ("gs_version", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
+EXPORTED = ("gs_version", "gs_launch_count", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
             "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd",
             "gs_preprocess_fwd_noalloc", "gs_render_stats", "gs_sh_fwd", "gs_sh_bwd")
 
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         cam = ctypes.POINTER(GsCamera)
         L.gs_version.restype = I
         L.gs_version.argtypes = []
+        L.gs_launch_count.restype = ctypes.c_ulonglong
+        L.gs_launch_count.argtypes = []
         L.gs_status_string.restype = ctypes.c_char_p
         L.gs_status_string.argtypes = [I]
         L.gs_workspace_bytes.restype = S
@@ -101,6 +103,11 @@ def status_string(status: int) -> str:
 
 def version() -> int:
     return int(lib().gs_version())
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().gs_launch_count())
 
 
 def camera_struct(cam) -> GsCamera:

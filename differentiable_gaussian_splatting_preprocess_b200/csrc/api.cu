@@ -3,7 +3,16 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "gs_internal.cuh"
+
+namespace gs {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace gs
 
 extern "C" size_t gs_preprocess_ws_bytes(int N);
 extern "C" size_t gs_bin_sort_ws_bytes(int N, unsigned capacity, int width, int height);
@@ -13,6 +22,8 @@ __global__ void k_clear_status(gs::WsHeader* h) { h->status = 0u; }
 }  // namespace
 
 extern "C" int gs_version(void) { return (1 << 16) | 0; }
+
+extern "C" unsigned long long gs_launch_count(void) { return gs::g_launches.load(std::memory_order_relaxed); }
 
 extern "C" const char* gs_status_string(int status) {
     switch (status) {
@@ -54,7 +65,7 @@ extern "C" int gs_read_status(const void* ws, int* status, void* stream) {
 
 extern "C" int gs_clear_status(void* ws, void* stream) {
     if (!ws) return GS_ERR_INVALID_ARG;
-    k_clear_status<<<1, 1, 0, (cudaStream_t)stream>>>(reinterpret_cast<gs::WsHeader*>(ws));
+    k_clear_status<<<1, 1, 0, (cudaStream_t)stream>>>(reinterpret_cast<gs::WsHeader*>(ws)); gs::note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

@@ -1009,9 +1009,23 @@ __device__ __forceinline__ unsigned cell_mask(int4 rc, int cx, int cy) {
     return row & rows;
 }
 
+// Tile counts of a warp's masks, packed: bit b of a mask becomes byte b & 3
+// of word b >> 2 (a 4-bit slice spread to 4 bytes by one multiply, the
+// shifted copies disjoint), so one add per word counts 4 tiles and one
+// warp-wide add per word sums the warp (each byte stays below 256 as long as
+// no lane adds more than 7 masks).
+__device__ __forceinline__ unsigned spread4(unsigned x) { return (x * 0x00204081u) & 0x01010101u; }
+__device__ __forceinline__ void add_mask(unsigned (&acc)[kCellTiles / 4], unsigned m) {
+#pragma unroll
+    for (int j = 0; j < kCellTiles / 4; ++j) acc[j] += spread4((m >> (4 * j)) & 15u);
+}
+__device__ __forceinline__ unsigned packed_count(const unsigned (&acc)[kCellTiles / 4], int b) {
+    return (acc[b >> 2] >> (8 * (b & 3))) & 255u;
+}
+
 // Per segment: count, per tile of its cell, the segment's Gaussians touching
-// it.  Warps count with one ballot per tile bit present in the warp.  Each
-// entry's tile mask is kept for k_seg_emit.
+// it (packed byte counters, see add_mask).  Each entry's tile mask is kept
+// for k_seg_emit.
 __global__ void __launch_bounds__(kSortBlock)
 k_seg_count(int SX, const unsigned* __restrict__ clist, const int4* __restrict__ rect,
             const unsigned* __restrict__ seg_cell, const unsigned* __restrict__ seg_lo,
@@ -1021,20 +1035,19 @@ k_seg_count(int SX, const unsigned* __restrict__ clist, const int4* __restrict__
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned nseg = misc->nseg;
     for (unsigned k = blockIdx.x; k < nseg; k += gridDim.x) {
-        if (lane < kCellTiles) s_c[warp][lane] = 0u;
-        __syncwarp();
         const unsigned c = seg_cell[k], lo = seg_lo[k], hi = seg_hi[k];
         const int cx = (int)(c % (unsigned)SX), cy = (int)(c / (unsigned)SX);
+        static_assert(kSeg / kSortBlock <= 7, "packed byte counters hold at most 7 masks per lane");
+        unsigned acc[kCellTiles / 4] = {};
         for (unsigned base = lo; base < hi; base += kSortBlock) {
             const unsigned i = base + threadIdx.x;
             const unsigned m = i < hi ? cell_mask(rect[clist[i]], cx, cy) : 0u;
             if (i < hi) seg_mask[i] = (unsigned short)m;
-            for (unsigned u = __reduce_or_sync(0xffffffffu, m); u; u &= u - 1) {
-                const int b = __ffs(u) - 1;
-                const unsigned bal = __ballot_sync(0xffffffffu, (m >> b) & 1u);
-                if (lane == 0) s_c[warp][b] += __popc(bal);
-            }
+            add_mask(acc, m);
         }
+#pragma unroll
+        for (int j = 0; j < kCellTiles / 4; ++j) acc[j] = __reduce_add_sync(0xffffffffu, acc[j]);
+        if (lane < kCellTiles) s_c[warp][lane] = packed_count(acc, lane);
         __syncthreads();
         if (threadIdx.x < kCellTiles) {
             unsigned t = 0;
@@ -1110,7 +1123,7 @@ k_tile_scan(int T, const unsigned* __restrict__ tile_cnt, unsigned* __restrict__
 
 // Per segment: write its Gaussians into the lists of its cell's tiles.  Per
 // chunk of 256 list entries: each warp counts its Gaussians per tile bit
-// (ballots), one thread per bit turns the warps' counts into bases (warp
+// (packed byte counters), one thread per bit turns the warps' counts into bases (warp
 // order after the running base), then each warp writes, per tile bit, its
 // Gaussians at base + ballot rank: consecutive lanes, consecutive addresses.
 // Optional 64-bit (tile << 32 | depth bits) keys.
@@ -1139,14 +1152,12 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
             const unsigned g = i < hi ? clist[i] : 0u;
             const unsigned m = i < hi ? (unsigned)seg_mask[i] : 0u;
             const unsigned un = __reduce_or_sync(0xffffffffu, m);
-            // this warp's count per tile bit
-            if (lane < kCellTiles) s_wb[warp][lane] = 0u;
-            __syncwarp();
-            for (unsigned u = un; u; u &= u - 1) {
-                const int b = __ffs(u) - 1;
-                const unsigned bal = __ballot_sync(0xffffffffu, (m >> b) & 1u);
-                if (lane == 0) s_wb[warp][b] = __popc(bal);
-            }
+            // this warp's count per tile bit (packed byte counters)
+            unsigned acc[kCellTiles / 4] = {};
+            add_mask(acc, m);
+#pragma unroll
+            for (int j = 0; j < kCellTiles / 4; ++j) acc[j] = __reduce_add_sync(0xffffffffu, acc[j]);
+            if (lane < kCellTiles) s_wb[warp][lane] = packed_count(acc, lane);
             __syncthreads();
             if (threadIdx.x < kCellTiles) {
                 const int b = threadIdx.x;
@@ -1197,10 +1208,10 @@ template <int MAXB>
 void radix_pass(cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
                 const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals) {
     enable_scatter_smem<MAXB>();
-    k_radix_hist<MAXB><<<G, kSortBlock, 0, st>>>(ki, n_ptr, shift, bits, hist, totals);
-    k_radix_scan<<<1 << bits, kSortBlock, 0, st>>>(hist, totals, G);
+    k_radix_hist<MAXB><<<G, kSortBlock, 0, st>>>(ki, n_ptr, shift, bits, hist, totals); note_launch();
+    k_radix_scan<<<1 << bits, kSortBlock, 0, st>>>(hist, totals, G); note_launch();
     k_radix_scatter<MAXB><<<G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st>>>(ki, vi, ko, vo, n_ptr, shift, bits,
-                                                                                hist);
+                                                                                hist); note_launch();
 }
 
 // One stable LSD radix sort of (keys, vals) over bits [0, total_bits), with
@@ -1269,7 +1280,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = (work + 255) / 256;
         if (blocks < 1) blocks = 1;
         if (blocks > 148 * 8) blocks = 148 * 8;
-        k_bin_init<<<blocks, 256, 0, st>>>(N, T, depth, tiles_touched, d_num_pairs, capacity, w, ranges);
+        k_bin_init<<<blocks, 256, 0, st>>>(N, T, depth, tiles_touched, d_num_pairs, capacity, w, ranges); note_launch();
         GS_LAUNCH_CHECK();
     }
     if (N == 0) return GS_OK;
@@ -1286,10 +1297,10 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     const int nb = (N + kScanTile - 1) / kScanTile;
     const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
     k_scan_partials<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
-                                               w.rc_rank, w.scan_part);
-    k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb, w.misc);
+                                               w.rc_rank, w.scan_part); note_launch();
+    k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb, w.misc); note_launch();
     k_scan_down<<<nb, kSortBlock, 0, st>>>(N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
-                                           (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi);
+                                           (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi); note_launch();
     GS_LAUNCH_CHECK();
     if (capacity == 0) return GS_OK;
 
@@ -1302,19 +1313,19 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         unsigned* h1 = w.hist + (size_t)4 * kRadixMax * kSortMaxGrid;
         unsigned* t1 = w.totals + (size_t)4 * kRadixMax;
         if (bx <= 7) {
-            k_gen_hist<7><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1);
-            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp);
+            k_gen_hist<7><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
+            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
             cudaFuncSetAttribute(k_gen_scatter<7>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gen_scatter_smem<7>());
             k_gen_scatter<7><<<Gp, kSortBlock, gen_scatter_smem<7>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
-                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0);
+                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         } else {
-            k_gen_hist<8><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1);
-            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp);
+            k_gen_hist<8><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
+            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
             cudaFuncSetAttribute(k_gen_scatter<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gen_scatter_smem<8>());
             k_gen_scatter<8><<<Gp, kSortBlock, gen_scatter_smem<8>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
-                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0);
+                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         }
         GS_LAUNCH_CHECK();
         unsigned* h2 = w.hist + (size_t)5 * kRadixMax * kSortMaxGrid;
@@ -1328,17 +1339,17 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
             int blocks = (int)((capacity + 1023u) / 1024u);
             if (blocks > 148 * 16) blocks = 148 * 16;
             if (blocks < 1) blocks = 1;
-            k_cell_ranges<<<blocks, 256, 0, st>>>(w.tkeys1, ps, SX, w.cell_ranges);
+            k_cell_ranges<<<blocks, 256, 0, st>>>(w.tkeys1, ps, SX, w.cell_ranges); note_launch();
         }
         const int S = SX * SY;
-        k_seg_table<<<1, 1024, 0, st>>>(S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc);
+        k_seg_table<<<1, 1024, 0, st>>>(S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
         const int gseg = (int)(w.max_seg < 148u * 8u ? w.max_seg : 148u * 8u);
         k_seg_count<<<gseg, kSortBlock, 0, st>>>(SX, w.tvals1, rect4, w.seg_cell, w.seg_lo, w.seg_hi, w.misc,
-                                                 w.seg_cnt, w.seg_mask);
-        k_cell_scan<<<S, kCellTiles, 0, st>>>(TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt);
-        k_tile_scan<<<1, 1024, 0, st>>>(T, w.tile_cnt, w.tile_start, ranges);
+                                                 w.seg_cnt, w.seg_mask); note_launch();
+        k_cell_scan<<<S, kCellTiles, 0, st>>>(TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
+        k_tile_scan<<<1, 1024, 0, st>>>(T, w.tile_cnt, w.tile_start, ranges); note_launch();
         k_seg_emit<<<gseg, kSortBlock, 0, st>>>(TX, TY, SX, w.tvals1, w.seg_mask, depth, w.seg_cell, w.seg_lo,
-                                                w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys);
+                                                w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys); note_launch();
         GS_LAUNCH_CHECK();
         return GS_OK;
     }
@@ -1353,7 +1364,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         if (blocks < 1) blocks = 1;
         unsigned* emit_vals = tpasses == 0 ? ids : w.tvals0;
         k_emit<<<blocks, kSortBlock, 0, st>>>(N, TX, order, w.pair_off, reinterpret_cast<const int4*>(rect),
-                                              tiles_touched, w.misc, w.tkeys0, emit_vals);
+                                              tiles_touched, w.misc, w.tkeys0, emit_vals); note_launch();
         GS_LAUNCH_CHECK();
     }
     unsigned* tkeys_sorted = nullptr;
@@ -1366,7 +1377,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = (int)((capacity + 1023u) / 1024u);
         if (blocks > 148 * 16) blocks = 148 * 16;
         if (blocks < 1) blocks = 1;
-        k_ranges<<<blocks, 256, 0, st>>>(tkeys_sorted, ids, depth, w.misc, ranges, keys);
+        k_ranges<<<blocks, 256, 0, st>>>(tkeys_sorted, ids, depth, w.misc, ranges, keys); note_launch();
         GS_LAUNCH_CHECK();
     }
     return GS_OK;

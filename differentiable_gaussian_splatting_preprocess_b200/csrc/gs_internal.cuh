@@ -23,6 +23,10 @@ static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Host-side count of the kernels this library has launched (gs_launch_count);
+// called after every launch statement.
+void note_launch();
+
 inline int tiles_x(const gs_camera& c) { return (c.width + kTile - 1) / kTile; }
 inline int tiles_y(const gs_camera& c) { return (c.height + kTile - 1) / kTile; }
 

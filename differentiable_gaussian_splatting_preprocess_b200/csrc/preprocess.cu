@@ -372,7 +372,7 @@ extern "C" int gs_preprocess_fwd(const gs_camera* cam, int N, const float* means
     k_preprocess_fwd<<<blocks > 0 ? blocks : 1, kPreBlock, 0, (cudaStream_t)stream>>>(
         *cam, N, tiles_x(*cam), tiles_y(*cam), means, scales, reinterpret_cast<const float4*>(quats), opacity,
         reinterpret_cast<float2*>(mean2d), depth, reinterpret_cast<float4*>(conic_opacity), radius,
-        reinterpret_cast<int4*>(rect), tiles_touched, d_num_pairs, hdr, partials);
+        reinterpret_cast<int4*>(rect), tiles_touched, d_num_pairs, hdr, partials); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
@@ -396,7 +396,7 @@ extern "C" int gs_preprocess_bwd(const gs_camera* cam, int N, const float* means
         *cam, N, means, scales, reinterpret_cast<const float4*>(quats), radius,
         reinterpret_cast<const float4*>(conic_opacity), reinterpret_cast<const float2*>(dL_dmean2d),
         reinterpret_cast<const float4*>(dL_dconic_opacity), dL_dcolor2d, dL_dmeans, dL_dscales,
-        reinterpret_cast<float4*>(dL_dquats), dL_dopacity, dL_dcolors, grad2d_accum, vis_count);
+        reinterpret_cast<float4*>(dL_dquats), dL_dopacity, dL_dcolors, grad2d_accum, vis_count); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
@@ -479,7 +479,7 @@ extern "C" int gs_preprocess_fwd_noalloc(const gs_camera* cam, int N, const floa
     k_preprocess_fwd<<<blocks > 0 ? blocks : 1, kPreBlock, 0, st>>>(
         *cam, N, tiles_x(*cam), tiles_y(*cam), means, scales, reinterpret_cast<const float4*>(quats), opacity,
         reinterpret_cast<float2*>(mean2d), depth, reinterpret_cast<float4*>(conic_opacity), radius,
-        reinterpret_cast<int4*>(rect), tiles_touched, d_num_pairs, hdr, partials);
+        reinterpret_cast<int4*>(rect), tiles_touched, d_num_pairs, hdr, partials); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

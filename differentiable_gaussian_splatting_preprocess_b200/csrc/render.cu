@@ -452,13 +452,13 @@ extern "C" int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const
     if (contrib_mask) {
         int blocks = (int)((mask_words + 255u) / 256u);
         if (blocks > 148 * 8) blocks = 148 * 8;
-        k_zero<<<blocks, 256, 0, st>>>(reinterpret_cast<float*>(contrib_mask), mask_words, nullptr, 0, nullptr, 0);
+        k_zero<<<blocks, 256, 0, st>>>(reinterpret_cast<float*>(contrib_mask), mask_words, nullptr, 0, nullptr, 0); note_launch();
         GS_LAUNCH_CHECK();
     }
     k_render_fwd<<<T, kThreads, 0, st>>>(
         *cam, TX, reinterpret_cast<const uint2*>(ranges), ids, reinterpret_cast<const float2*>(mean2d),
         reinterpret_cast<const float4*>(conic_opacity), colors, image, final_T, n_contrib, contrib_mask,
-        contrib_mask ? mask_words : 0u);
+        contrib_mask ? mask_words : 0u); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
@@ -479,7 +479,7 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
         int blocks = (int)((work + 255) / 256);
         if (blocks > 148 * 8) blocks = 148 * 8;
         k_zero<<<blocks, 256, 0, st>>>(dL_dmean2d, (size_t)N * 2, dL_dconic_opacity, (size_t)N * 4, dL_dcolor,
-                                       (size_t)N * 3);
+                                       (size_t)N * 3); note_launch();
         GS_LAUNCH_CHECK();
     }
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
@@ -487,7 +487,7 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
                                        reinterpret_cast<const float2*>(mean2d),
                                        reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
                                        contrib_mask, contrib_mask ? mask_words : 0u, dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),
-                                       reinterpret_cast<float4*>(dL_dconic_opacity), dL_dcolor);
+                                       reinterpret_cast<float4*>(dL_dconic_opacity), dL_dcolor); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
@@ -500,7 +500,7 @@ extern "C" int gs_render_stats(const gs_camera* cam, const unsigned* ranges, con
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
     k_render_stats<<<T, kTilePixels, 0, (cudaStream_t)stream>>>(
         *cam, TX, reinterpret_cast<const uint2*>(ranges), ids, reinterpret_cast<const float2*>(mean2d),
-        reinterpret_cast<const float4*>(conic_opacity), n_evaluated, n_blended);
+        reinterpret_cast<const float4*>(conic_opacity), n_evaluated, n_blended); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

@@ -205,7 +205,7 @@ extern "C" int gs_sh_fwd(const gs_camera* cam, int N, int degree, int K, const f
     if (N == 0) return GS_OK;
     if (!means || !sh || !colors) return GS_ERR_INVALID_ARG;
     k_sh_fwd<<<(N + kShBlock - 1) / kShBlock, kShBlock, 0, (cudaStream_t)stream>>>(N, degree, K, camera_centre(*cam),
-                                                                                  offset, means, sh, colors);
+                                                                                  offset, means, sh, colors); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
@@ -216,7 +216,7 @@ extern "C" int gs_sh_bwd(const gs_camera* cam, int N, int degree, int K, const f
     if (N == 0) return GS_OK;
     if (!means || !sh || !dL_dcolors || !dL_dsh || !dL_dmeans) return GS_ERR_INVALID_ARG;
     k_sh_bwd<<<(N + kShBwdBlock - 1) / kShBwdBlock, kShBwdBlock, 0, (cudaStream_t)stream>>>(
-        N, degree, K, camera_centre(*cam), offset, means, sh, dL_dcolors, dL_dsh, dL_dmeans);
+        N, degree, K, camera_centre(*cam), offset, means, sh, dL_dcolors, dL_dsh, dL_dmeans); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

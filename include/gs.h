@@ -92,6 +92,12 @@ typedef struct gs_camera {
 /* Library version as (major << 16) | minor. */
 GS_API int gs_version(void);
 
+/* Number of kernels this library has launched in this process so far (all
+ * entry points, all streams, all threads).  Host-side count, taken when each
+ * launch is issued; a diagnostic for counting launches per frame.  Never
+ * fails. */
+GS_API unsigned long long gs_launch_count(void);
+
 /* Human-readable text for a status code or a combination of flags. */
 GS_API const char* gs_status_string(int status);
 

@@ -403,3 +403,23 @@ def test_render_views_sums_cameras():
         ref = {k: f[k] for k in MV.GRAD_KEYS} if ref is None else {k: ref[k] + f[k] for k in MV.GRAD_KEYS}
     for k in MV.GRAD_KEYS:
         assert rel_l2(to_np(grads[k]), ref[k]) <= GRAD_REL_L2, k
+
+
+def test_launch_count_is_fixed_per_frame():
+    """The library's launch counter: every frame of one configuration issues
+    the same number of kernels (no host-dependent fallbacks), and only the
+    library's own launches count."""
+    sc = _scene(2)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0], capacity=200_000)
+    deltas = []
+    for _ in range(2):
+        n0 = B.launch_count()
+        run_gpu(gs, cam, dL_dimage=sc.dL_dimage[0], capacity=200_000)
+        deltas.append(B.launch_count() - n0)
+    assert deltas[0] == deltas[1] > 10
+    n0 = B.launch_count()
+    torch.zeros(1000, device="cuda").add_(1.0)
+    torch.cuda.synchronize()
+    assert B.launch_count() == n0
