@@ -225,6 +225,8 @@ def run_ours(args):
         from differentiable_gaussian_splatting_preprocess_b200 import scenes as _scn
         shd = torch.from_numpy(_scn.random_sh(sc.N, sh_deg, seed=1)).to(dev)
         dsh = torch.zeros_like(shd)
+        if args.sh_f16:
+            shd = shd.half()  # binary16 storage, fp32 arithmetic (gs_sh_*_f16)
         colors = torch.empty((sc.N, 3), dtype=torch.float32, device=dev)
     exchange = multi and world > 1
 
@@ -411,7 +413,8 @@ def run_ours(args):
             vs_baseline=None, dtype="f32", data="synthetic",
             config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam0.width}x{cam0.height}, {len(cams)} view(s), "
                                  f"16x16 tiles, fp32"
-                                 + (f", SH degree {sh_deg} colours" if sh_deg is not None else ""),
+                                 + (f", SH degree {sh_deg} colours" if sh_deg is not None else "")
+                                 + (" (binary16 coefficient storage)" if sh_deg is not None and args.sh_f16 else ""),
                         views_per_rank=len(mine), num_pairs=P, evals_per_step=evals_per_step,
                         evaluated_fwd=n_evaluated, contributor_prefix_bwd=n_contrib, blended=n_blended,
                         l2="flushed between steps (256 MiB write)", parallelism=par),
@@ -440,6 +443,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--sh-degree", type=int, default=None,
                     help="colours from spherical harmonics of this degree (adds the SH stages to the step)")
+    ap.add_argument("--sh-f16", action="store_true",
+                    help="with --sh-degree: store the SH coefficients in binary16 (the mixed-precision variant)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -31,7 +31,8 @@ TILE = 16
 # Every symbol include/gs.h declares.
 EXPORTED = ("gs_version", "gs_launch_count", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
             "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd",
-            "gs_preprocess_fwd_noalloc", "gs_render_stats", "gs_sh_fwd", "gs_sh_bwd")
+            "gs_preprocess_fwd_noalloc", "gs_render_stats", "gs_sh_fwd", "gs_sh_bwd", "gs_sh_fwd_f16",
+            "gs_sh_bwd_f16")
 
 
 class GsCamera(ctypes.Structure):
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
         L.gs_sh_fwd.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P]
         L.gs_sh_bwd.restype = I
         L.gs_sh_bwd.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P, P, P]
+        L.gs_sh_fwd_f16.restype = I
+        L.gs_sh_fwd_f16.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P]
+        L.gs_sh_bwd_f16.restype = I
+        L.gs_sh_bwd_f16.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P, P, P]
         L.gs_preprocess_bwd.restype = I
         L.gs_preprocess_bwd.argtypes = [cam, I] + [P] * 15 + [P]
         _lib = L
@@ -311,31 +316,59 @@ NOALLOC_MAX_GAUSSIANS = 1 << 24
 SH_MAX_DEGREE = 3
 
 
+def _sh_entry(name: str, sh):
+    """The fp32 entry point, or its half-precision-storage twin for float16
+    coefficients."""
+    if sh.dtype == torch.float16:
+        return name + "_f16"
+    _check(sh, "sh", torch.float32)
+    return name
+
+
 def gs_sh_fwd(cam, degree: int, means, sh, colors, offset: float = 0.0, stream=None) -> None:
+    """SH colour; `sh` [N, K, 3] float32, or float16 (storage only: the
+    kernel computes in fp32)."""
     N = means.shape[0]
     _check(means, "means", torch.float32, (N, 3))
-    _check(sh, "sh", torch.float32)
+    name = _sh_entry("gs_sh_fwd", sh)
+    _check(sh, "sh", sh.dtype)
     if sh.dim() != 3 or sh.shape[0] != N or sh.shape[2] != 3:
         raise ValueError("sh must have shape [N, K, 3]")
     _check(colors, "colors", torch.float32, (N, 3))
     c = camera_struct(cam)
-    _ok("gs_sh_fwd", lib().gs_sh_fwd(ctypes.byref(c), int(N), int(degree), int(sh.shape[1]), _ptr(means), _ptr(sh),
-                                     float(offset), _ptr(colors), _stream(stream)))
+    _ok(name, getattr(lib(), name)(ctypes.byref(c), int(N), int(degree), int(sh.shape[1]), _ptr(means), _ptr(sh),
+                                   float(offset), _ptr(colors), _stream(stream)))
 
 
 def gs_sh_bwd(cam, degree: int, means, sh, dL_dcolors, dL_dsh, dL_dmeans, offset: float = 0.0, stream=None) -> None:
+    """SH backward; `sh` float32 or float16 (storage only); dL_dsh is float32
+    [N, K, 3] in both cases and is accumulated into."""
     N = means.shape[0]
     _check(means, "means", torch.float32, (N, 3))
-    _check(sh, "sh", torch.float32)
+    name = _sh_entry("gs_sh_bwd", sh)
+    _check(sh, "sh", sh.dtype)
     if sh.dim() != 3 or sh.shape[0] != N or sh.shape[2] != 3:
         raise ValueError("sh must have shape [N, K, 3]")
     _check(dL_dcolors, "dL_dcolors", torch.float32, (N, 3))
     _check(dL_dsh, "dL_dsh", torch.float32, tuple(sh.shape))
     _check(dL_dmeans, "dL_dmeans", torch.float32, (N, 3))
     c = camera_struct(cam)
-    _ok("gs_sh_bwd", lib().gs_sh_bwd(ctypes.byref(c), int(N), int(degree), int(sh.shape[1]), _ptr(means), _ptr(sh),
-                                     float(offset), _ptr(dL_dcolors), _ptr(dL_dsh), _ptr(dL_dmeans),
-                                     _stream(stream)))
+    _ok(name, getattr(lib(), name)(ctypes.byref(c), int(N), int(degree), int(sh.shape[1]), _ptr(means), _ptr(sh),
+                                   float(offset), _ptr(dL_dcolors), _ptr(dL_dsh), _ptr(dL_dmeans),
+                                   _stream(stream)))
+
+
+def gs_sh_fwd_f16(cam, degree: int, means, sh, colors, offset: float = 0.0, stream=None) -> None:
+    if sh.dtype != torch.float16:
+        raise TypeError("gs_sh_fwd_f16 takes float16 coefficients")
+    gs_sh_fwd(cam, degree, means, sh, colors, offset, stream)
+
+
+def gs_sh_bwd_f16(cam, degree: int, means, sh, dL_dcolors, dL_dsh, dL_dmeans, offset: float = 0.0,
+                  stream=None) -> None:
+    if sh.dtype != torch.float16:
+        raise TypeError("gs_sh_bwd_f16 takes float16 coefficients")
+    gs_sh_bwd(cam, degree, means, sh, dL_dcolors, dL_dsh, dL_dmeans, offset, stream)
 
 
 def gs_preprocess_fwd_noalloc(cam, means, scales, quats, opacity, mean2d, depth, conic_opacity, radius, rect,

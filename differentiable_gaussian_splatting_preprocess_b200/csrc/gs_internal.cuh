@@ -38,7 +38,7 @@ inline bool camera_ok(const gs_camera* c) {
     return true;
 }
 
-inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+__host__ __device__ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 #define GS_LAUNCH_CHECK()                                          \
     do {                                                           \

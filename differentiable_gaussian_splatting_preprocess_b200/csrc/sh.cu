@@ -8,7 +8,13 @@
 // ordered k = l^2 + l + m, colour = max(0, sum_k Y_k(d) sh_k + offset) per
 // channel; the clamp at 0 passes no gradient where it is active.
 // One thread per Gaussian; HBM-bound (16 x 3 coefficients per Gaussian).
+//
+// Mixed precision ([CB] sections 5 and 7 name half precision as a memory
+// optimisation): the *_f16 entry points read the coefficients stored as IEEE
+// binary16 (half the bytes of the largest per-Gaussian array) and compute in
+// fp32; colours, gradients and the accumulated dL/dsh stay fp32.
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "gs_internal.cuh"
@@ -81,27 +87,87 @@ constexpr int kShRow = kShMaxK * 3 + 1;  // padded row stride in shared memory, 
 // lanes reading "their" row at the same column hit 32 different banks.
 __device__ __forceinline__ int row_stride(int K) { return (K * 3) | 1; }
 
-__device__ __forceinline__ void warp_load_rows(float* dst, const float* __restrict__ src, int g0, int N, int K) {
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
+
+// The 32 rows of a warp are one contiguous block of rows * K * 3 elements
+// (16-byte aligned whenever the array base is, since g0 is a multiple of
+// 32).  It moves as 16-byte vectors: every lane issues all its loads before
+// its first shared-memory store, so the block costs one memory round trip.
+// Blocks that are not whole vectors (K = 1, a ragged last warp, an unaligned
+// base) move element by element.
+constexpr int kVecBytes = 16;
+
+template <typename T>
+__device__ __forceinline__ void warp_load_rows(float* dst, const T* __restrict__ src, int g0, int N, int K) {
+    constexpr int E = kVecBytes / sizeof(T);                       // elements per vector
+    constexpr int kMaxVec = (32 * kShMaxK * 3 + 32 * E - 1) / (32 * E);  // vectors per lane, at most
     const int lane = threadIdx.x & 31;
     const int rows = min(32, N - g0);
-    const int w = K * 3, rs = row_stride(K);
-    const float* s0 = src + (size_t)g0 * w;
-    for (int r = 0; r < rows; ++r)
-        for (int c = lane; c < w; c += 32) dst[r * rs + c] = s0[(size_t)r * w + c];
+    const int w = K * 3, rs = row_stride(K), total = rows * w;
+    const T* s0 = src + (size_t)g0 * w;
+    if (total % E == 0 && aligned(s0, kVecBytes)) {
+        const int nv = total / E;
+        uint4 v[kMaxVec];
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int idx = lane + 32 * j;
+            if (idx < nv) v[j] = reinterpret_cast<const uint4*>(s0)[idx];
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int idx = lane + 32 * j;
+            if (idx < nv) {
+                const T* e = reinterpret_cast<const T*>(&v[j]);
+                int r = (idx * E) / w, c = idx * E - r * w;
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    dst[r * rs + c] = to_f32(e[k]);
+                    if (++c == w) { c = 0; ++r; }
+                }
+            }
+        }
+    } else {
+        for (int idx = lane; idx < total; idx += 32) dst[(idx / w) * rs + idx % w] = to_f32(s0[idx]);
+    }
 }
 
 __device__ __forceinline__ void warp_store_rows(float* __restrict__ dst, const float* src, int g0, int N, int K) {
+    constexpr int kMaxVec = (32 * kShMaxK * 3 + 127) / 128;
     const int lane = threadIdx.x & 31;
     const int rows = min(32, N - g0);
-    const int w = K * 3, rs = row_stride(K);
+    const int w = K * 3, rs = row_stride(K), total = rows * w;
     float* d0 = dst + (size_t)g0 * w;
-    for (int r = 0; r < rows; ++r)
-        for (int c = lane; c < w; c += 32) d0[(size_t)r * w + c] = src[r * rs + c];
+    if (total % 4 == 0 && aligned(d0, kVecBytes)) {
+        const int nv = total / 4;
+        float4 v[kMaxVec];
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int idx = lane + 32 * j;
+            if (idx < nv) {
+                float* e = reinterpret_cast<float*>(&v[j]);
+                int r = (idx * 4) / w, c = idx * 4 - r * w;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    e[k] = src[r * rs + c];
+                    if (++c == w) { c = 0; ++r; }
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int idx = lane + 32 * j;
+            if (idx < nv) reinterpret_cast<float4*>(d0)[idx] = v[j];
+        }
+    } else {
+        for (int idx = lane; idx < total; idx += 32) d0[idx] = src[(idx / w) * rs + idx % w];
+    }
 }
 
+template <typename T>
 __global__ void __launch_bounds__(kShBlock)
 k_sh_fwd(int N, int degree, int K, float3 centre, float offset, const float* __restrict__ means,
-         const float* __restrict__ sh, float* __restrict__ colors) {
+         const T* __restrict__ sh, float* __restrict__ colors) {
     __shared__ float s_sh[kShWarps][32 * kShRow];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g0 = blockIdx.x * kShBlock + warp * 32;
@@ -129,9 +195,10 @@ k_sh_fwd(int N, int degree, int K, float3 centre, float offset, const float* __r
     colors[3 * i + 2] = fmaxf(bl + offset, 0.0f);
 }
 
+template <typename T>
 __global__ void __launch_bounds__(kShBwdBlock)
 k_sh_bwd(int N, int degree, int K, float3 centre, float offset, const float* __restrict__ means,
-         const float* __restrict__ sh, const float* __restrict__ dL_dcolors, float* __restrict__ dL_dsh,
+         const T* __restrict__ sh, const float* __restrict__ dL_dcolors, float* __restrict__ dL_dsh,
          float* __restrict__ dL_dmeans) {
     __shared__ float s_sh[kShBwdWarps][32 * kShRow];
     __shared__ float s_g[kShBwdWarps][32 * kShRow];
@@ -194,6 +261,30 @@ bool sh_args_ok(const gs_camera* cam, int N, int degree, int K) {
            K >= (degree + 1) * (degree + 1) && K <= kShMaxK;
 }
 
+template <typename T>
+int sh_fwd(const gs_camera* cam, int N, int degree, int K, const float* means, const T* sh, float offset,
+           float* colors, void* stream) {
+    if (!sh_args_ok(cam, N, degree, K)) return GS_ERR_INVALID_ARG;
+    if (N == 0) return GS_OK;
+    if (!means || !sh || !colors) return GS_ERR_INVALID_ARG;
+    k_sh_fwd<T><<<(N + kShBlock - 1) / kShBlock, kShBlock, 0, (cudaStream_t)stream>>>(
+        N, degree, K, camera_centre(*cam), offset, means, sh, colors); note_launch();
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+}
+
+template <typename T>
+int sh_bwd(const gs_camera* cam, int N, int degree, int K, const float* means, const T* sh, float offset,
+           const float* dL_dcolors, float* dL_dsh, float* dL_dmeans, void* stream) {
+    if (!sh_args_ok(cam, N, degree, K)) return GS_ERR_INVALID_ARG;
+    if (N == 0) return GS_OK;
+    if (!means || !sh || !dL_dcolors || !dL_dsh || !dL_dmeans) return GS_ERR_INVALID_ARG;
+    k_sh_bwd<T><<<(N + kShBwdBlock - 1) / kShBwdBlock, kShBwdBlock, 0, (cudaStream_t)stream>>>(
+        N, degree, K, camera_centre(*cam), offset, means, sh, dL_dcolors, dL_dsh, dL_dmeans); note_launch();
+    GS_LAUNCH_CHECK();
+    return GS_OK;
+}
+
 }  // namespace
 }  // namespace gs
 
@@ -201,22 +292,24 @@ using namespace gs;
 
 extern "C" int gs_sh_fwd(const gs_camera* cam, int N, int degree, int K, const float* means, const float* sh,
                          float offset, float* colors, void* stream) {
-    if (!sh_args_ok(cam, N, degree, K)) return GS_ERR_INVALID_ARG;
-    if (N == 0) return GS_OK;
-    if (!means || !sh || !colors) return GS_ERR_INVALID_ARG;
-    k_sh_fwd<<<(N + kShBlock - 1) / kShBlock, kShBlock, 0, (cudaStream_t)stream>>>(N, degree, K, camera_centre(*cam),
-                                                                                  offset, means, sh, colors); note_launch();
-    GS_LAUNCH_CHECK();
-    return GS_OK;
+    return sh_fwd<float>(cam, N, degree, K, means, sh, offset, colors, stream);
 }
 
 extern "C" int gs_sh_bwd(const gs_camera* cam, int N, int degree, int K, const float* means, const float* sh,
                          float offset, const float* dL_dcolors, float* dL_dsh, float* dL_dmeans, void* stream) {
-    if (!sh_args_ok(cam, N, degree, K)) return GS_ERR_INVALID_ARG;
-    if (N == 0) return GS_OK;
-    if (!means || !sh || !dL_dcolors || !dL_dsh || !dL_dmeans) return GS_ERR_INVALID_ARG;
-    k_sh_bwd<<<(N + kShBwdBlock - 1) / kShBwdBlock, kShBwdBlock, 0, (cudaStream_t)stream>>>(
-        N, degree, K, camera_centre(*cam), offset, means, sh, dL_dcolors, dL_dsh, dL_dmeans); note_launch();
-    GS_LAUNCH_CHECK();
-    return GS_OK;
+    return sh_bwd<float>(cam, N, degree, K, means, sh, offset, dL_dcolors, dL_dsh, dL_dmeans, stream);
+}
+
+extern "C" int gs_sh_fwd_f16(const gs_camera* cam, int N, int degree, int K, const float* means,
+                             const unsigned short* sh, float offset, float* colors, void* stream) {
+    if (sh && !aligned(sh, 2)) return GS_ERR_INVALID_ARG;
+    return sh_fwd<__half>(cam, N, degree, K, means, reinterpret_cast<const __half*>(sh), offset, colors, stream);
+}
+
+extern "C" int gs_sh_bwd_f16(const gs_camera* cam, int N, int degree, int K, const float* means,
+                             const unsigned short* sh, float offset, const float* dL_dcolors, float* dL_dsh,
+                             float* dL_dmeans, void* stream) {
+    if (sh && !aligned(sh, 2)) return GS_ERR_INVALID_ARG;
+    return sh_bwd<__half>(cam, N, degree, K, means, reinterpret_cast<const __half*>(sh), offset, dL_dcolors, dL_dsh,
+                          dL_dmeans, stream);
 }

@@ -297,6 +297,21 @@ GS_API int gs_sh_fwd(const gs_camera* cam, int N, int degree, int K, const float
 GS_API int gs_sh_bwd(const gs_camera* cam, int N, int degree, int K, const float* means, const float* sh,
                      float offset, const float* dL_dcolors, float* dL_dsh, float* dL_dmeans, void* stream);
 
+/*
+ * gs_sh_fwd_f16 / gs_sh_bwd_f16 - the same two operations with the
+ *   coefficients stored in half precision ([CB] 5 and 7 list half-precision
+ *   storage as a memory optimisation): sh [N, K, 3] holds IEEE binary16 bit
+ *   patterns (2-byte aligned), widened to fp32 on load; all arithmetic,
+ *   colors, dL_dcolors, the accumulated dL_dsh [N, K, 3] and dL_dmeans stay
+ *   fp32.  Results equal the fp32 entry points applied to the widened
+ *   coefficients.  Same ownership, accumulation and error behaviour as above.
+ */
+GS_API int gs_sh_fwd_f16(const gs_camera* cam, int N, int degree, int K, const float* means,
+                         const unsigned short* sh, float offset, float* colors, void* stream);
+GS_API int gs_sh_bwd_f16(const gs_camera* cam, int N, int degree, int K, const float* means,
+                         const unsigned short* sh, float offset, const float* dL_dcolors, float* dL_dsh,
+                         float* dL_dmeans, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -68,3 +68,42 @@ def test_render_with_sh_colours_end_to_end(cfg):
     assert rel_l2(to_np(dsh), ob["dL_dsh"]) <= GRAD_REL_L2
     for k in ("dL_dscales", "dL_dquats", "dL_dopacity"):
         assert rel_l2(to_np(g[k]), f[k]) <= GRAD_REL_L2, k
+
+
+@pytest.mark.parametrize("degree", [1, 3])
+def test_sh_half_precision_storage(degree):
+    """gs_sh_*_f16: coefficients stored as binary16, arithmetic in fp32.  The
+    bar is the fp32 one, against the oracle evaluated on the widened
+    coefficients (binary16 -> float64 is exact); the distance to the
+    full-precision colours is the storage rounding alone, at most
+    sum_k |Y_k| |sh_k| 2^-11 per channel."""
+    sc = scenes.preset(3)
+    cam = _rotated_cam(sc.cameras[0])
+    sh = scenes.random_sh(sc.N, degree, seed=11 + degree)
+    sh[:40, 0, :] = -5.0
+    sh16 = sh.astype(np.float16)
+    wide = sh16.astype(np.float64)
+    means = to_dev(sc.means)
+    shd16 = torch.from_numpy(sh16).cuda()
+    col = torch.empty((sc.N, 3), device="cuda")
+    B.gs_sh_fwd(cam, degree, means, shd16, col, offset=0.5)
+    g = np.random.default_rng(degree).normal(size=(sc.N, 3)).astype(np.float32)
+    dsh = torch.zeros(sh.shape, dtype=torch.float32, device="cuda")
+    dmu = torch.zeros_like(means)
+    B.gs_sh_bwd_f16(cam, degree, means, shd16, to_dev(g), dsh, dmu, offset=0.5)
+    torch.cuda.synchronize()
+    o64 = oracle.sh_fwd(cam, sc.means, wide, degree, 0.5, "f64")
+    np.testing.assert_allclose(to_np(col), o64, atol=1e-5)
+    assert not to_np(col)[:40].any()
+    ob = oracle.sh_bwd(cam, sc.means, wide, degree, g, 0.5, "f64")
+    assert rel_l2(to_np(dsh), ob["dL_dsh"]) <= 1e-5
+    assert rel_l2(to_np(dmu), ob["dL_dmeans"]) <= 1e-4
+    # storage rounding relative to the full-precision coefficients
+    full = oracle.sh_fwd(cam, sc.means, sh.astype(np.float64), degree, 0.5, "f64")
+    R = np.asarray(cam.R, np.float64).reshape(3, 3)
+    v = sc.means.astype(np.float64) + R.T @ np.asarray(cam.t, np.float64)  # mean - camera centre
+    Y = np.abs(oracle.sh_basis(v / np.linalg.norm(v, axis=1, keepdims=True)))[:, :(degree + 1) ** 2]
+    bound = np.einsum("nk,nkc->nc", Y, np.abs(sh[:, :(degree + 1) ** 2].astype(np.float64))) * 2.0 ** -11
+    assert np.all(np.abs(to_np(col) - full) <= bound + 1e-5)
+    with pytest.raises(TypeError):
+        B.gs_sh_fwd_f16(cam, degree, means, to_dev(sh), col)
