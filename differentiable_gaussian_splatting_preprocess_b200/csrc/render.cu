@@ -211,7 +211,11 @@ __device__ __forceinline__ float reduce8(float v[8], int lane) {
 
 constexpr int kGradStride = 9;  // floats per staged Gaussian in shared memory
 
-__global__ void __launch_bounds__(kThreads)
+// With the forward's contribution mask (kMask) the warps walk the recorded
+// positions and need no culling data: the staged boxes and thresholds are
+// dropped, which brings shared memory and registers down to ten CTAs per SM.
+template <bool kMask>
+__global__ void __launch_bounds__(kThreads, kMask ? 10 : 8)
 k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
              const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
              const float* __restrict__ colors, const float* __restrict__ final_T,
@@ -222,8 +226,8 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     __shared__ float2 s_xy[kBatch];
     __shared__ float4 s_co[kBatch];
     __shared__ float4 s_col[kBatch];
-    __shared__ float4 s_box[kBatch];
-    __shared__ float s_thr[kBatch];
+    __shared__ float4 s_box[kMask ? 1 : kBatch];
+    __shared__ float s_thr[kMask ? 1 : kBatch];
     __shared__ float s_grad[kBatch * kGradStride];
     __shared__ unsigned s_max[kWarps];
 
@@ -268,7 +272,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
         // the forward's contribution bits for this batch, loaded early so that
         // their latency overlaps the staging below
         unsigned mbits = 0;  // bit w: staged Gaussian w * 32 + lane blended a pixel of this warp
-        if (cmask) {
+        if (kMask) {
 #pragma unroll
             for (int w = 0; w < kWords; ++w) {
                 const int p = top - 1 - (w * 32 + lane);
@@ -291,8 +295,10 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 s_xy[r] = xy;
                 s_co[r] = co;
                 s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
-                s_box[r] = contrib_box(xy, co, amin);
-                s_thr[r] = contrib_threshold(co, amin);
+                if (!kMask) {
+                    s_box[r] = contrib_box(xy, co, amin);
+                    s_thr[r] = contrib_threshold(co, amin);
+                }
             }
         }
         __syncthreads();
@@ -301,7 +307,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
             const int jl = w * 32 + lane;
             const int p = top - 1 - jl;
             bool keep = jl < n && p < (int)wlast;
-            if (cmask) {
+            if (kMask) {
                 keep = keep && ((mbits >> w) & 1u);
             } else {
                 keep = keep && may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], q);
@@ -483,7 +489,8 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
         GS_LAUNCH_CHECK();
     }
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
-    k_render_bwd<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
+    auto kernel = contrib_mask ? k_render_bwd<true> : k_render_bwd<false>;
+    kernel<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
                                        reinterpret_cast<const float2*>(mean2d),
                                        reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
                                        contrib_mask, contrib_mask ? mask_words : 0u, dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),
