@@ -53,6 +53,16 @@ BYTES_PAIR_ATOMIC = 36
 BYTES_PIXEL = 20
 SMS = 148
 FP32_LANES_PER_SM = 128
+# Algorithmic bytes of gs_bin_sort on its cell (4x4-tile super-tile) route:
+# per Gaussian 156 B (key build 16, four depth-radix passes x 20, the
+# rank-order scans 40, the first cell pass's per-rank reads 20), per
+# (cell, Gaussian) pair 60 B (first pass write 8, second pass histogram +
+# scatter 20, cell ranges 4, segment counting 22 incl. the rectangle gather,
+# expansion reads 6), per (tile, Gaussian) pair the 4-byte id written.
+BIN_BYTES_GAUSSIAN = 156
+BIN_BYTES_CELL_PAIR = 60
+BIN_BYTES_PAIR = 4
+CELL = 4  # tiles per cell side
 
 
 def _peaks():
@@ -277,9 +287,13 @@ def run_ours(args):
         if st != 0:
             raise RuntimeError(f"device status {st}: {B.status_string(st)}")
     # work counts of this rank's views (outside the timed region)
-    n_contrib = n_evaluated = n_blended = P = 0
+    n_contrib = n_evaluated = n_blended = P = Ps = 0
     for i in mine:
         b, cam = rzs[i]._bufs, cams[i]
+        rc = b["rect"].to(torch.int64)
+        vis = b["tiles_touched"].view(torch.int32) > 0
+        cells = (((rc[:, 2] - 1) // CELL - rc[:, 0] // CELL + 1) * ((rc[:, 3] - 1) // CELL - rc[:, 1] // CELL + 1))
+        Ps += int(torch.where(vis, cells, torch.zeros_like(cells)).sum().item())
         ne = torch.empty((cam.height, cam.width), dtype=torch.uint32, device=dev)
         nb = torch.empty_like(ne)
         B.gs_render_stats(cam, b["ranges"], b["ids"], b["mean2d"], b["conic_opacity"], ne, nb)
@@ -351,6 +365,13 @@ def run_ours(args):
                       frac=(fwd_bytes + bwd_bytes) / rfb_s / 1e9 / peaks["hbm_gbs"],
                       bytes_per_frame=fwd_bytes + bwd_bytes, peak_src=peaks["src"])
     fwd_alu = fwd_ops / (mean["render_fwd"] / 1e3) / 1e12
+    # HBM view of the binning (the sort is the stage an HBM roofline fits)
+    bin_bytes = len(mine) * sc.N * BIN_BYTES_GAUSSIAN + Ps * BIN_BYTES_CELL_PAIR + P * BIN_BYTES_PAIR
+    bin_gbs = bin_bytes / (mean["bin_sort"] / 1e3) / 1e9
+    bin_hbm = dict(achieved_gbs=bin_gbs, peak_gbs=peaks["hbm_gbs"], frac=bin_gbs / peaks["hbm_gbs"],
+                   bytes_per_step=bin_bytes, cell_pairs=Ps, peak_src=peaks["src"],
+                   basis=f"{BIN_BYTES_GAUSSIAN} B/Gaussian + {BIN_BYTES_CELL_PAIR} B/cell pair + "
+                         f"{BIN_BYTES_PAIR} B/pair")
 
     # end to end through the public API: pinned host inputs -> device ->
     # forward (host read of P) + backward of every view of this rank, the
@@ -423,7 +444,7 @@ def run_ours(args):
             stage_ms={s: round(v, 4) for s, v in mean.items()}, dominant_stage=dominant,
             roofline=roofline, render_fwd_alu=dict(achieved=fwd_alu, peak=alu_peak, unit="Tops/s",
                                                    frac=fwd_alu / alu_peak),
-            render_hbm=render_hbm, cpu_baseline=cpu, e2e=e2e, gpu_launches=launches,
+            render_hbm=render_hbm, bin_sort_hbm=bin_hbm, cpu_baseline=cpu, e2e=e2e, gpu_launches=launches,
             clocks=clocks)
         print(json.dumps(line), flush=True)
     if world > 1:
