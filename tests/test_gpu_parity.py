@@ -213,13 +213,14 @@ def test_ragged_and_tiny_images(W, H):
         assert rel_l2(to_np(r["grads"][k]), f[k]) <= GRAD_REL_L2, k
 
 
-@pytest.mark.parametrize("W,H,n,sigma_mult", [(4200, 24, 80, 3.0), (4096, 40, 80, 3.0), (40, 4096, 80, 3.0),
+@pytest.mark.parametrize("W,H,n,sigma_mult", [(16400, 20, 80, 3.0), (8200, 40, 80, 3.0), (40, 8200, 80, 3.0),
                                               (800, 608, 2000, 1e3)])
 def test_binning_routes(W, H, n, sigma_mult):
-    """Both binning routes against the oracle's sort: more than 256 tile
-    columns (emit + sort by tile id), exactly 256 columns or rows (fused,
-    8-bit passes), and pairs of whole-image Gaussians cut by every chunk
-    boundary of the fused first pass."""
+    """Both binning routes against the oracle's sort: more than 1024 tile
+    columns (257 cells: emit + radix sort by tile id + boundary ranges),
+    129 cell columns or rows (cell passes with 8-bit digits), and cell pairs
+    of whole-image Gaussians cut by every chunk boundary of the generated
+    first pass."""
     sc = _tiny(n=n, width=W, height=H, seed=W + 3 * H, z_range=(2.0, 6.0), sigma_mult=sigma_mult)
     cam = sc.cameras[0].replace(fx=float(W), fy=float(H), cx=W / 2.0, cy=H / 2.0)
     sc.cameras[0] = cam
