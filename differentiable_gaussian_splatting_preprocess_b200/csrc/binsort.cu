@@ -940,15 +940,42 @@ constexpr size_t gen_scatter_smem() {
 }
 
 // Cell ranges of the cell-sorted list by comparing neighbours (keys
-// cy << 16 | cx); empty cells keep (0, 0).
+// cy << 16 | cx); empty cells keep (0, 0).  Four keys per thread with
+// 16-byte loads, neighbours across lanes by shuffles.
 __global__ void k_cell_ranges(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ n_ptr, int SX,
                               unsigned* __restrict__ cell_ranges) {
     const unsigned n = *n_ptr;
-    for (unsigned k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
-        const unsigned key = ckeys[k];
-        const unsigned c = (key >> 16) * (unsigned)SX + (key & 0xFFFFu);
-        if (k == 0 || ckeys[k - 1] != key) cell_ranges[2 * c] = k;
-        if (k + 1 == n || ckeys[k + 1] != key) cell_ranges[2 * c + 1] = k + 1;
+    const unsigned nq = (n + 3) / 4;
+    const unsigned stride = gridDim.x * blockDim.x;
+    const int lane = threadIdx.x & 31;
+    // every lane of a warp iterates the same number of times (shuffles below)
+    for (unsigned qb = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); qb < nq; qb += stride) {
+        const unsigned qi = qb + lane;
+        const unsigned k0 = qi * 4;
+        unsigned t[4];
+        if (k0 + 3 < n) {
+            const uint4 v = reinterpret_cast<const uint4*>(ckeys)[qi];
+            t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) t[j] = k0 + j < n ? ckeys[k0 + j] : 0xFFFFFFFFu;
+        }
+        unsigned prev = __shfl_up_sync(0xffffffffu, t[3], 1);
+        unsigned next = __shfl_down_sync(0xffffffffu, t[0], 1);
+        if (lane == 0) prev = (k0 > 0 && k0 - 1 < n) ? ckeys[k0 - 1] : 0xFFFFFFFFu;
+        if (lane == 31) next = (k0 + 4 < n) ? ckeys[k0 + 4] : 0xFFFFFFFFu;
+        if (qi < nq) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const unsigned k = k0 + j;
+                if (k >= n) break;
+                const unsigned before = j == 0 ? prev : t[j - 1];
+                const unsigned after = (j == 3 || k + 1 == n) ? (k + 1 == n ? 0xFFFFFFFFu : next) : t[j + 1];
+                const unsigned c = (t[j] >> 16) * (unsigned)SX + (t[j] & 0xFFFFu);
+                if (k == 0 || before != t[j]) cell_ranges[2 * c] = k;
+                if (k + 1 == n || after != t[j]) cell_ranges[2 * c + 1] = k + 1;
+            }
+        }
     }
 }
 
@@ -982,17 +1009,23 @@ k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restric
         const int c = c0 + k;
         if (c < S) {
             cell_seg0[c] = run;
-            const unsigned a = cell_ranges[2 * c], b = cell_ranges[2 * c + 1];
-            for (unsigned lo = a; lo < b; lo += kSeg, ++run) {
-                seg_cell[run] = (unsigned)c;
-                seg_lo[run] = lo;
-                seg_hi[run] = min(b, lo + kSeg);
-            }
+            run += (cell_ranges[2 * c + 1] - cell_ranges[2 * c] + kSeg - 1) / kSeg;
         }
     }
     if (threadIdx.x == 1023) {
         cell_seg0[S] = run;
         misc->nseg = run;
+    }
+    __syncthreads();
+    // one warp per cell writes the cell's segments, one lane per segment
+    for (int c = warp; c < S; c += 32) {
+        const unsigned a = cell_ranges[2 * c], b = cell_ranges[2 * c + 1], s0 = cell_seg0[c];
+        for (unsigned j = lane; a + j * kSeg < b; j += 32) {
+            const unsigned lo = a + j * kSeg;
+            seg_cell[s0 + j] = (unsigned)c;
+            seg_lo[s0 + j] = lo;
+            seg_hi[s0 + j] = min(b, lo + kSeg);
+        }
     }
 }
 
@@ -1172,8 +1205,11 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
             }
             __syncthreads();
             const float dg = (keys && m) ? depth[g] : 0.0f;
-            for (unsigned u = un; u; u &= u - 1) {
-                const int b = __ffs(u) - 1;
+            // tile bits in order, unrolled: no find-first-set / bit-reverse
+            // (XU) instructions; skipped bits cost one uniform branch
+#pragma unroll
+            for (int b = 0; b < kCellTiles; ++b) {
+                if (!((un >> b) & 1u)) continue;
                 const bool mine = (m >> b) & 1u;
                 const unsigned bal = __ballot_sync(0xffffffffu, mine);
                 if (mine) {
