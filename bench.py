@@ -373,37 +373,32 @@ def run_ours(args):
                    basis=f"{BIN_BYTES_GAUSSIAN} B/Gaussian + {BIN_BYTES_CELL_PAIR} B/cell pair + "
                          f"{BIN_BYTES_PAIR} B/pair")
 
-    # end to end through the public API: pinned host inputs -> device ->
-    # forward (host read of P) + backward of every view of this rank, the
+    # end to end through the public API: pinned host inputs -> device (on a
+    # side stream, overlapped with the kernels that do not read them yet) ->
+    # forward + backward of every view of this rank in capacity mode, the
     # gradient exchange, then the 3D gradients back to the host
     e2e = None
     if not args.no_e2e:
-        host_in = [torch.from_numpy(np.ascontiguousarray(x)).pin_memory()
-                   for x in (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors)]
+        host_params = {k: torch.from_numpy(np.ascontiguousarray(x)).pin_memory()
+                       for k, x in zip(("means", "scales", "quats", "opacity", "colors"),
+                                       (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors))}
         host_dl = [torch.from_numpy(np.ascontiguousarray(sc.dL_dimage[i])).pin_memory() for i in mine]
-        h2d = sum(x.numel() * x.element_size() for x in host_in + host_dl)
-        rz_e2e = {}
-        host_out = None
+        h2d = sum(x.numel() * x.element_size() for x in list(host_params.values()) + host_dl)
+        rz_e2e, e2e_state = {}, {}
+        host_out = {k: torch.empty(grads[k].shape, dtype=grads[k].dtype, pin_memory=True) for k in MV.GRAD_KEYS}
         e2e_times = []
         for k in range(args.warmup + args.steps):
             flush.zero_()
             torch.cuda.synchronize(dev)
             t0 = time.perf_counter()
-            d = [x.to(dev, non_blocking=True) for x in host_in]
-            dls = [x.to(dev, non_blocking=True) for x in host_dl]
-            params = dict(means=d[0], scales=d[1], quats=d[2], opacity=d[3], colors=d[4])
-            g2 = MV.render_views([cams[i] for i in mine], params, dls, rasterizers=rz_e2e, camera_ids=mine)
-            if exchange:
-                MV.allreduce_grads(g2)
-            outs = [g2[k2] for k2 in MV.GRAD_KEYS]
-            if host_out is None:
-                host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-            for ho, o in zip(host_out, outs):
-                ho.copy_(o, non_blocking=True)
+            MV.render_views_from_host([cams[i] for i in mine], host_params, host_dl, rz_e2e,
+                                      [caps[i] for i in mine], camera_ids=mine, state=e2e_state,
+                                      host_grads=host_out, reduce_fn=MV.allreduce_grads if exchange else None,
+                                      device=dev)
             torch.cuda.synchronize(dev)
             if k >= args.warmup:
                 e2e_times.append(time.perf_counter() - t0)
-        d2h = sum(o.numel() * o.element_size() for o in host_out)
+        d2h = sum(o.numel() * o.element_size() for o in host_out.values())
         e2e_s = sum(e2e_times)
         if world > 1:
             tt = torch.tensor([e2e_s], device=dev, dtype=torch.float64)

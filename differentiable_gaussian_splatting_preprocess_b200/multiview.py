@@ -52,6 +52,74 @@ def render_views(cams: Sequence, params: Dict[str, torch.Tensor], dL_dimages: Se
     return grads
 
 
+GEOMETRY_KEYS = ("means", "scales", "quats", "opacity")
+
+
+def render_views_from_host(cams: Sequence, host_params: Dict[str, torch.Tensor], host_dls: Sequence[torch.Tensor],
+                           rasterizers: Dict[int, "RZ.Rasterizer"], capacity: Sequence[int],
+                           camera_ids: Optional[Sequence[int]] = None, state: Optional[dict] = None,
+                           host_grads: Optional[Dict[str, torch.Tensor]] = None,
+                           reduce_fn: Optional[Callable[[Dict[str, torch.Tensor]], None]] = None,
+                           device=None) -> Dict[str, torch.Tensor]:
+    """One training step's rasterization from host (pinned) inputs to host
+    gradients, with the copies overlapped with the kernels.
+
+    The inputs move to reused device buffers on a side stream, in the order
+    the stages read them: the geometry (means, scales, quats, opacity) first
+    - the projection waits for it - then the colours, which the compositing
+    waits for while projection and binning run, then each view's dL/dimage,
+    which only its backward waits for.  Every view runs in capacity mode
+    (``capacity[n]`` pairs, no host round trip).  ``reduce_fn`` (e.g. the
+    cross-rank all-reduce) runs on the summed gradients before they are
+    copied to ``host_grads``.  ``state`` keeps the stream and buffers across
+    steps."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    st = state if state is not None else {}
+    cur = torch.cuda.current_stream(dev)
+    if "stream" not in st:
+        st["stream"] = torch.cuda.Stream(dev)
+        st["params"] = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_params.items()}
+        st["dls"] = [torch.empty(h.shape, dtype=h.dtype, device=dev) for h in host_dls]
+    cs, dp, dd = st["stream"], st["params"], st["dls"]
+    cs.wait_stream(cur)  # the previous step's readers of these buffers are done
+    with torch.cuda.stream(cs):
+        for k in GEOMETRY_KEYS:
+            dp[k].copy_(host_params[k], non_blocking=True)
+        e_geo = torch.cuda.Event()
+        e_geo.record(cs)
+        dp["colors"].copy_(host_params["colors"], non_blocking=True)
+        e_col = torch.cuda.Event()
+        e_col.record(cs)
+        e_dl = []
+        for d, h in zip(dd, host_dls):
+            d.copy_(h, non_blocking=True)
+            e = torch.cuda.Event()
+            e.record(cs)
+            e_dl.append(e)
+    cur.wait_event(e_geo)
+    grads = st.get("grads")
+    if grads is None:
+        grads = st["grads"] = RZ.zero_grads(dp["means"].shape[0], dev)
+    else:
+        for v in grads.values():
+            v.zero_()
+    ids = list(range(len(cams))) if camera_ids is None else list(camera_ids)
+    for n, cam in enumerate(cams):
+        rz = rasterizers.get(ids[n])
+        if rz is None:
+            rz = rasterizers[ids[n]] = RZ.Rasterizer(cam, dev)
+        fr = rz.forward(dp["means"], dp["scales"], dp["quats"], dp["opacity"], dp["colors"], capacity=capacity[n],
+                        colors_ready=e_col)
+        rz.backward(fr, dp["means"], dp["scales"], dp["quats"], dp["colors"], dd[n], grads=grads,
+                    dL_ready=e_dl[n])
+    if reduce_fn is not None:
+        reduce_fn(grads)
+    if host_grads is not None:
+        for k, h in host_grads.items():
+            h.copy_(grads[k], non_blocking=True)
+    return grads
+
+
 def flat_grads(grads: Dict[str, torch.Tensor], keys: Sequence[str] = GRAD_KEYS) -> torch.Tensor:
     return torch.cat([grads[k].reshape(-1) for k in keys])
 

@@ -82,13 +82,16 @@ class Rasterizer:
         return out
 
     def forward(self, means, scales, quats, opacity, colors, capacity: Optional[int] = None,
-                want_keys: bool = False, use_mask: bool = True, stream=None) -> Frame:
+                want_keys: bool = False, use_mask: bool = True, stream=None,
+                colors_ready: Optional[torch.cuda.Event] = None) -> Frame:
         """Preprocess, bin/sort and composite one frame.
 
         With ``capacity=None`` the pair count is read back to size the sort
         buffers (one device-to-host copy).  With a capacity the call makes no
         host round trip; if the frame needs more pairs, the status word of
         the workspace reports GS_ERR_CAPACITY and every tile range is empty.
+        ``colors_ready``: an event the compositing waits for (the colours may
+        still be arriving while the projection and the binning run).
         """
         N = means.shape[0]
         pre = self.preprocess(means, scales, quats, opacity, stream)
@@ -105,6 +108,8 @@ class Rasterizer:
         final_T = self._buf("final_T", (H, W), torch.float32)
         n_contrib = self._buf("n_contrib", (H, W), torch.uint32)
         cmask = self._buf("contrib_mask", (B.mask_words(max(capacity, 1)),), torch.uint32) if use_mask else None
+        if colors_ready is not None:
+            (stream or torch.cuda.current_stream(self.device)).wait_event(colors_ready)
         B.gs_render_fwd(self.cam, ranges, ids, pre["mean2d"], pre["conic_opacity"], colors, image, final_T,
                         n_contrib, cmask, stream)
         return Frame(N=N, capacity=capacity, ids=ids, ranges=ranges, keys=keys, image=image, final_T=final_T,
@@ -112,12 +117,16 @@ class Rasterizer:
 
     def backward(self, frame: Frame, means, scales, quats, colors, dL_dimage,
                  grads: Optional[Dict[str, torch.Tensor]] = None, densify: Optional[Dict[str, torch.Tensor]] = None,
-                 stream=None) -> Dict[str, torch.Tensor]:
+                 stream=None, dL_ready: Optional[torch.cuda.Event] = None) -> Dict[str, torch.Tensor]:
         """Render backward then preprocess backward.  3D gradients are
         accumulated into ``grads`` (zeros are allocated when it is None).
         With ``densify`` = dict(grad2d_accum=[N] float32, vis_count=[N] uint32),
-        the densification statistics of this view are accumulated too."""
+        the densification statistics of this view are accumulated too.
+        ``dL_ready``: an event the backward waits for before reading
+        ``dL_dimage``."""
         N = frame.N
+        if dL_ready is not None:
+            (stream or torch.cuda.current_stream(self.device)).wait_event(dL_ready)
         g2 = dict(dL_dmean2d=self._buf("dL_dmean2d", (N, 2), torch.float32),
                   dL_dconic_opacity=self._buf("dL_dconic_opacity", (N, 4), torch.float32),
                   dL_dcolor=self._buf("dL_dcolor", (N, 3), torch.float32))

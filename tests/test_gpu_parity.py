@@ -406,6 +406,32 @@ def test_render_views_sums_cameras():
         assert rel_l2(to_np(grads[k]), ref[k]) <= GRAD_REL_L2, k
 
 
+def test_render_views_from_host_overlapped_copies():
+    """The host-input step (copies on a side stream, compositing and backward
+    waiting on their inputs' events, capacity mode) gives the gradients of the
+    device-input path, twice in a row (buffers and stream reused)."""
+    from differentiable_gaussian_splatting_preprocess_b200 import multiview as MV
+    sc = _scene(2)
+    base = sc.cameras[0]
+    cams = [base, base.replace(R=(0.985, 0.0, 0.174, 0.0, 1.0, 0.0, -0.174, 0.0, 0.985))]
+    gs = GpuScene(sc)
+    params = dict(means=gs.means, scales=gs.scales, quats=gs.quats, opacity=gs.opacity, colors=gs.colors)
+    dl_np = [sc.dL_dimage[0], -0.5 * sc.dL_dimage[0]]
+    ref = MV.render_views(cams, params, [to_dev(d) for d in dl_np])
+    torch.cuda.synchronize()
+    host = {k: torch.from_numpy(np.ascontiguousarray(getattr(sc, k))).pin_memory()
+            for k in ("means", "scales", "quats", "opacity", "colors")}
+    host_dl = [torch.from_numpy(np.ascontiguousarray(d)).pin_memory() for d in dl_np]
+    out = {k: torch.empty(tuple(ref[k].shape), pin_memory=True) for k in MV.GRAD_KEYS}
+    rzs, state = {}, {}
+    for _ in range(2):
+        MV.render_views_from_host(cams, host, host_dl, rzs, [200_000, 200_000], state=state, host_grads=out)
+        torch.cuda.synchronize()
+        for k in MV.GRAD_KEYS:
+            assert rel_l2(out[k].numpy(), to_np(ref[k])) <= 1e-5, k
+    assert all(rz.status() == 0 for rz in rzs.values())
+
+
 def test_launch_count_is_fixed_per_frame():
     """The library's launch counter: every frame of one configuration issues
     the same number of kernels (no host-dependent fallbacks), and only the
