@@ -22,6 +22,10 @@
 
 #include <cuda_runtime.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "gs_internal.cuh"
 
 namespace gs {
@@ -1232,12 +1236,23 @@ int ceil_log2(unsigned x) {
     return b;
 }
 
-// The scatter needs more than the default 48 KiB of dynamic shared memory;
-// the attribute belongs to the current device, so it is set before each use.
+// Kernels that use more than the default 48 KiB of dynamic shared memory
+// must opt in once per device.  Done on first use and remembered, so later
+// calls (including calls recorded into a CUDA graph) issue no attribute call.
+template <typename Kernel>
+void opt_in_smem(Kernel kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.insert({dev, reinterpret_cast<const void*>(kernel)}).second)
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 template <int MAXB>
 void enable_scatter_smem() {
-    cudaFuncSetAttribute(k_radix_scatter<MAXB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)RadixCfg<MAXB>::kScatterSmem);
+    opt_in_smem(k_radix_scatter<MAXB>, RadixCfg<MAXB>::kScatterSmem);
 }
 
 template <int MAXB>
@@ -1351,15 +1366,13 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         if (bx <= 7) {
             k_gen_hist<7><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
             k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
-            cudaFuncSetAttribute(k_gen_scatter<7>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gen_scatter_smem<7>());
+            opt_in_smem(k_gen_scatter<7>, gen_scatter_smem<7>());
             k_gen_scatter<7><<<Gp, kSortBlock, gen_scatter_smem<7>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         } else {
             k_gen_hist<8><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
             k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
-            cudaFuncSetAttribute(k_gen_scatter<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gen_scatter_smem<8>());
+            opt_in_smem(k_gen_scatter<8>, gen_scatter_smem<8>());
             k_gen_scatter<8><<<Gp, kSortBlock, gen_scatter_smem<8>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         }
