@@ -209,6 +209,64 @@ __device__ __forceinline__ float reduce8(float v[8], int lane) {
     return v[0];
 }
 
+// One term of the reverse traversal for this thread's two pixels: undo the
+// term's transmittance step, accumulate the colour behind it, and produce the
+// pixel pair's share of the 9 gradient values (dL/du, dL/dv, dL/da, dL/db,
+// dL/dc, dL/dr, dL/dg, dL/dopacity; dL/db_colour in r9).  Returns false, with
+// nothing changed, when no pixel of the warp takes the term (a warp vote).
+// p is the term's position in the tile's list; last0/last1 the pixels'
+// contributor counts; terms the forward did not blend contribute nothing.
+__device__ __forceinline__ bool bwd_term(const PixelPair& q, float2 xy, float4 co, float4 c, int p, unsigned last0,
+                                         unsigned last1, float amax, float amin, float2 g0, float2 g1, float2 g2,
+                                         float2& T, float2& S0, float2& S1, float2& S2, float (&v)[8], float& r9) {
+    TermPair e;
+    eval_pair(q.px, q.py, xy, co, amax, amin, e);
+    const bool c0 = p < (int)last0 && e.ok0;
+    const bool c1 = p < (int)last1 && e.ok1;
+    if (!__any_sync(0xffffffffu, c0 || c1)) return false;
+    const float2 G = make_float2(c0 ? e.G.x : 0.0f, c1 ? e.G.y : 0.0f);
+    const float2 al = make_float2(c0 ? e.alpha.x : 0.0f, c1 ? e.alpha.y : 0.0f);
+    if (c0) T.x = __fdividef(T.x, 1.0f - al.x);
+    if (c1) T.y = __fdividef(T.y, 1.0f - al.y);
+    const float2 wgt = __fmul2_rn(al, T);
+    const float2 d0 = __fadd2_rn(make_float2(c.x, c.x), make_float2(-S0.x, -S0.y));
+    const float2 d1 = __fadd2_rn(make_float2(c.y, c.y), make_float2(-S1.x, -S1.y));
+    const float2 d2 = __fadd2_rn(make_float2(c.z, c.z), make_float2(-S2.x, -S2.y));
+    float2 dLda = __fmul2_rn(d0, g0);
+    dLda = __ffma2_rn(d1, g1, dLda);
+    dLda = __ffma2_rn(d2, g2, dLda);
+    dLda = __fmul2_rn(dLda, T);
+    // colour behind the next term towards the front: S <- alpha c + (1 - alpha) S
+    S0 = __ffma2_rn(al, d0, S0);
+    S1 = __ffma2_rn(al, d1, S1);
+    S2 = __ffma2_rn(al, d2, S2);
+    // exact derivative of min(alpha_max, opacity G): zero while capped
+    const float2 Gf = make_float2(e.at.x <= amax ? G.x : 0.0f, e.at.y <= amax ? G.y : 0.0f);
+    const float2 dsig = __fmul2_rn(Gf, dLda);                    // dL/dopacity
+    const float2 h = __fmul2_rn(dsig, make_float2(co.w, co.w));  // dL/dpower
+    const float2 hdx = __fmul2_rn(h, e.dx);
+    const float2 hdy = __fmul2_rn(h, make_float2(e.dy, e.dy));
+    float2 t2;
+    t2 = __ffma2_rn(make_float2(co.x, co.x), hdx, __fmul2_rn(make_float2(co.y, co.y), hdy));
+    v[0] = t2.x + t2.y;  // dL/du
+    t2 = __ffma2_rn(make_float2(co.y, co.y), hdx, __fmul2_rn(make_float2(co.z, co.z), hdy));
+    v[1] = t2.x + t2.y;  // dL/dv
+    t2 = __fmul2_rn(hdx, e.dx);
+    v[2] = -0.5f * (t2.x + t2.y);  // dL/da
+    t2 = __fmul2_rn(hdx, make_float2(e.dy, e.dy));
+    v[3] = -(t2.x + t2.y);  // dL/db
+    t2 = __fmul2_rn(hdy, make_float2(e.dy, e.dy));
+    v[4] = -0.5f * (t2.x + t2.y);  // dL/dc
+    t2 = __fmul2_rn(wgt, g0);
+    v[5] = t2.x + t2.y;  // dL/dcolor r
+    t2 = __fmul2_rn(wgt, g1);
+    v[6] = t2.x + t2.y;  // dL/dcolor g
+    v[7] = dsig.x + dsig.y;  // dL/dopacity
+    t2 = __fmul2_rn(wgt, g2);
+    r9 = t2.x + t2.y;  // dL/dcolor b
+    return true;
+}
+
 constexpr int kGradStride = 9;  // floats per staged Gaussian in shared memory
 
 // With the forward's contribution mask (kMask) the warps walk the recorded
@@ -317,56 +375,10 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 const int jj = w * 32 + __ffs(m) - 1;
                 m &= m - 1;
                 const int p = top - 1 - jj;
-                const float4 co = s_co[jj];
-                TermPair e;
-                eval_pair(q.px, q.py, s_xy[jj], co, amax, amin, e);
-                const bool c0 = p < (int)last0 && e.ok0;
-                const bool c1 = p < (int)last1 && e.ok1;
-                if (!__any_sync(0xffffffffu, c0 || c1)) continue;
-                // terms the forward did not blend contribute nothing
-                const float2 G = make_float2(c0 ? e.G.x : 0.0f, c1 ? e.G.y : 0.0f);
-                const float2 al = make_float2(c0 ? e.alpha.x : 0.0f, c1 ? e.alpha.y : 0.0f);
-                if (c0) T.x = __fdividef(T.x, 1.0f - al.x);
-                if (c1) T.y = __fdividef(T.y, 1.0f - al.y);
-                const float4 c = s_col[jj];
-                const float2 wgt = __fmul2_rn(al, T);
-                const float2 d0 = __fadd2_rn(make_float2(c.x, c.x), make_float2(-S0.x, -S0.y));
-                const float2 d1 = __fadd2_rn(make_float2(c.y, c.y), make_float2(-S1.x, -S1.y));
-                const float2 d2 = __fadd2_rn(make_float2(c.z, c.z), make_float2(-S2.x, -S2.y));
-                float2 dLda = __fmul2_rn(d0, g0);
-                dLda = __ffma2_rn(d1, g1, dLda);
-                dLda = __ffma2_rn(d2, g2, dLda);
-                dLda = __fmul2_rn(dLda, T);
-                // colour behind the next term towards the front: S <- alpha c + (1 - alpha) S
-                S0 = __ffma2_rn(al, d0, S0);
-                S1 = __ffma2_rn(al, d1, S1);
-                S2 = __ffma2_rn(al, d2, S2);
-                // exact derivative of min(alpha_max, opacity G): zero while capped
-                const float2 Gf = make_float2(e.at.x <= amax ? G.x : 0.0f, e.at.y <= amax ? G.y : 0.0f);
-                const float2 dsig = __fmul2_rn(Gf, dLda);                       // dL/dopacity
-                const float2 h = __fmul2_rn(dsig, make_float2(co.w, co.w));     // dL/dpower
-                const float2 hdx = __fmul2_rn(h, e.dx);
-                const float hdy_s = e.dy;
-                const float2 hdy = __fmul2_rn(h, make_float2(hdy_s, hdy_s));
-                float v[8];
-                float2 t2;
-                t2 = __ffma2_rn(make_float2(co.x, co.x), hdx, __fmul2_rn(make_float2(co.y, co.y), hdy));
-                v[0] = t2.x + t2.y;  // dL/du
-                t2 = __ffma2_rn(make_float2(co.y, co.y), hdx, __fmul2_rn(make_float2(co.z, co.z), hdy));
-                v[1] = t2.x + t2.y;  // dL/dv
-                t2 = __fmul2_rn(hdx, e.dx);
-                v[2] = -0.5f * (t2.x + t2.y);  // dL/da
-                t2 = __fmul2_rn(hdx, make_float2(e.dy, e.dy));
-                v[3] = -(t2.x + t2.y);  // dL/db
-                t2 = __fmul2_rn(hdy, make_float2(e.dy, e.dy));
-                v[4] = -0.5f * (t2.x + t2.y);  // dL/dc
-                t2 = __fmul2_rn(wgt, g0);
-                v[5] = t2.x + t2.y;  // dL/dcolor r
-                t2 = __fmul2_rn(wgt, g1);
-                v[6] = t2.x + t2.y;  // dL/dcolor g
-                v[7] = dsig.x + dsig.y;  // dL/dopacity
-                t2 = __fmul2_rn(wgt, g2);
-                float r9 = t2.x + t2.y;  // dL/dcolor b
+                float v[8], r9;
+                if (!bwd_term(q, s_xy[jj], s_co[jj], s_col[jj], p, last0, last1, amax, amin, g0, g1, g2, T, S0, S1, S2,
+                              v, r9))
+                    continue;
                 const float r8 = reduce8(v, lane);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
@@ -396,6 +408,103 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
             }
         }
         __syncthreads();
+    }
+}
+
+// Backward driven by the forward's contribution mask, one warp per 8x8
+// quadrant and no block barrier: each warp walks the mask words of its
+// quadrant from its last contributor towards the front; for each word the
+// lanes whose bit is set load that list entry into the warp's shared-memory
+// slots, and the warp then takes the set bits from the back.  After the
+// butterfly, the 9 gradient sums sit in 9 different lanes (value i in lane
+// 4i, the ninth in lane 1), which add them to the Gaussian's 2D gradients
+// with one atomic instruction.  A warp whose pixels are all finished leaves
+// at once instead of waiting at the other warps' batch barriers.
+__global__ void __launch_bounds__(kThreads, 9)
+k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
+                  const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
+                  const float* __restrict__ colors, const float* __restrict__ final_T,
+                  const unsigned* __restrict__ n_contrib, const unsigned* __restrict__ cmask, unsigned cmask_words,
+                  const float* __restrict__ dL_dimage, float* __restrict__ dL_dmean2d,
+                  float* __restrict__ dL_dconic_opacity, float* __restrict__ dL_dcolor) {
+    __shared__ unsigned s_id[kWarps][32];
+    __shared__ float2 s_xy[kWarps][32];
+    __shared__ float4 s_co[kWarps][32];
+    __shared__ float4 s_col[kWarps][32];
+    const PixelPair q = pixel_pair(cam, TX);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint2 rg = ranges[blockIdx.x];
+    const float amax = cam.alpha_max, amin = cam.alpha_min;
+    const size_t plane = (size_t)cam.width * cam.height;
+    const size_t pix = (size_t)q.y * cam.width + q.x0;
+
+    float2 T = make_float2(0.0f, 0.0f), g0 = T, g1 = T, g2 = T;
+    unsigned last0 = 0, last1 = 0;
+    if (q.in0) {
+        T.x = final_T[pix];
+        last0 = n_contrib[pix];
+        g0.x = dL_dimage[pix];
+        g1.x = dL_dimage[plane + pix];
+        g2.x = dL_dimage[2 * plane + pix];
+    }
+    if (q.in1) {
+        T.y = final_T[pix + 1];
+        last1 = n_contrib[pix + 1];
+        g0.y = dL_dimage[pix + 1];
+        g1.y = dL_dimage[plane + pix + 1];
+        g2.y = dL_dimage[2 * plane + pix + 1];
+    }
+    float2 S0 = make_float2(cam.bg[0], cam.bg[0]), S1 = make_float2(cam.bg[1], cam.bg[1]);
+    float2 S2 = make_float2(cam.bg[2], cam.bg[2]);
+    // furthest list position any pixel of this warp blended (a count), kept
+    // inside the tile's list
+    const unsigned wlast = min(__reduce_max_sync(0xffffffffu, max(last0, last1)), rg.y - rg.x);
+    if (wlast == 0) return;
+
+    // where this lane's flush goes: value i of the butterfly in lane 4i, the
+    // ninth (blue) in lane 1; each lane adds to one component of one array
+    float* gbase = nullptr;
+    unsigned gstride = 0;
+    if (lane == 0 || lane == 4) { gbase = dL_dmean2d + (lane >> 2); gstride = 2; }
+    else if (lane == 8 || lane == 12 || lane == 16) { gbase = dL_dconic_opacity + ((lane >> 2) - 2); gstride = 4; }
+    else if (lane == 28) { gbase = dL_dconic_opacity + 3; gstride = 4; }
+    else if (lane == 20 || lane == 24) { gbase = dL_dcolor + ((lane >> 2) - 5); gstride = 3; }
+    else if (lane == 1) { gbase = dL_dcolor + 2; gstride = 3; }
+
+    const unsigned k_hi = rg.x + wlast - 1;  // last list entry to visit (global index)
+    for (int wk = (int)(k_hi >> 5); wk >= (int)(rg.x >> 5); --wk) {
+        const unsigned kb = (unsigned)wk << 5;
+        const unsigned wi = (unsigned)wk * kWarps + warp;
+        unsigned bits = wi < cmask_words ? cmask[wi] : 0xFFFFFFFFu;
+        // entries of this word that belong to the tile's list up to k_hi
+        const unsigned lo = rg.x > kb ? rg.x - kb : 0u;
+        const unsigned hi = k_hi - kb;  // < 32 only in the first (highest) word
+        if (hi < 31u) bits &= (2u << hi) - 1u;
+        bits &= ~((1u << lo) - 1u);
+        if (!bits) continue;
+        if ((bits >> lane) & 1u) {
+            const unsigned j = ids[kb + lane];
+            s_id[warp][lane] = j;
+            s_xy[warp][lane] = mean2d[j];
+            s_co[warp][lane] = conic_opacity[j];
+            s_col[warp][lane] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+        }
+        __syncwarp();
+        while (bits) {
+            const int l = 31 - __clz(bits);
+            bits &= ~(1u << l);
+            const int p = (int)(kb + (unsigned)l - rg.x);
+            float v[8], r9;
+            if (!bwd_term(q, s_xy[warp][l], s_co[warp][l], s_col[warp][l], p, last0, last1, amax, amin, g0, g1, g2, T,
+                          S0, S1, S2, v, r9))
+                continue;
+            const float r8 = reduce8(v, lane);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
+            const float val = lane == 1 ? r9 : r8;
+            if (gbase && val != 0.0f) atomicAdd(gbase + (size_t)s_id[warp][l] * gstride, val);
+        }
+        __syncwarp();  // the next word reuses this warp's slots
     }
 }
 
@@ -489,7 +598,16 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
         GS_LAUNCH_CHECK();
     }
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
-    auto kernel = contrib_mask ? k_render_bwd<true> : k_render_bwd<false>;
+    if (contrib_mask) {
+        k_render_bwd_warp<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
+                                                  reinterpret_cast<const float2*>(mean2d),
+                                                  reinterpret_cast<const float4*>(conic_opacity), colors, final_T,
+                                                  n_contrib, contrib_mask, mask_words, dL_dimage, dL_dmean2d,
+                                                  dL_dconic_opacity, dL_dcolor); note_launch();
+        GS_LAUNCH_CHECK();
+        return GS_OK;
+    }
+    auto kernel = k_render_bwd<false>;
     kernel<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
                                        reinterpret_cast<const float2*>(mean2d),
                                        reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
