@@ -239,6 +239,22 @@ def run_ours(args):
             shd = shd.half()  # binary16 storage, fp32 arithmetic (gs_sh_*_f16)
         colors = torch.empty((sc.N, 3), dtype=torch.float32, device=dev)
     exchange = multi and world > 1
+    adam = None
+    if args.adam:
+        # the optimiser stage: raw parameters (log scales, logit opacity) whose
+        # activated values the step writes back into the rasterizer's inputs
+        adam = dict(cfg=B.GsAdamConfig(1.6e-4, 5e-3, 1e-3, 5e-2, 2.5e-3, 0.9, 0.999, 1e-15, 3000), step=[0],
+                    params=dict(means=means.clone(), log_scales=torch.log(scales), quats=quats.clone(),
+                                logit_opacity=torch.logit(opacity), colors=colors.clone()))
+        if sh_deg is not None:
+            raise SystemExit("--adam covers RGB colours (no --sh-degree)")
+        adam["m"] = torch.zeros((11 + 3) * sc.N, device=dev)
+        adam["v"] = torch.zeros_like(adam["m"])
+        # the optimiser updates its own copies and writes the activated
+        # values to scratch buffers, so the timed scene (and its pair count)
+        # stays that of the workload
+        adam["scales"] = torch.empty_like(scales)
+        adam["opacity"] = torch.empty_like(opacity)
 
     def step(rec=None):
         """One step: every view of this rank through a1-a8 (gradients summed),
@@ -277,6 +293,10 @@ def run_ours(args):
                                                    grads["dL_dmeans"], offset=0.5))
         if exchange:
             timed("allreduce", lambda: MV.allreduce_grads(grads))
+        if adam is not None:
+            adam["step"][0] += 1
+            timed("adam", lambda: B.gs_adam_step(adam["cfg"], adam["step"][0], adam["params"], grads, adam["m"],
+                                                 adam["v"], adam["scales"], adam["opacity"]))
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -307,7 +327,7 @@ def run_ours(args):
     # round trip, so every call is capturable) and replayed: one launch per
     # step instead of ~35 launches per view through the Python binding
     graph, graph_launches = None, 0
-    if not args.no_graph and not exchange:
+    if not args.no_graph and not exchange and adam is None:
         graph = torch.cuda.CUDAGraph()
         torch.cuda.synchronize(dev)
         n0 = B.launch_count()
@@ -492,6 +512,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--sh-degree", type=int, default=None,
                     help="colours from spherical harmonics of this degree (adds the SH stages to the step)")
+    ap.add_argument("--adam", action="store_true",
+                    help="add the fused optimiser step (gs_adam_step) to the step (eager timing only: the step "
+                         "number changes every step)")
     ap.add_argument("--sh-f16", action="store_true",
                     help="with --sh-degree: store the SH coefficients in binary16 (the mixed-precision variant)")
     args = ap.parse_args()

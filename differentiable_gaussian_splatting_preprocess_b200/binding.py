@@ -32,7 +32,7 @@ TILE = 16
 EXPORTED = ("gs_version", "gs_launch_count", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
             "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd",
             "gs_preprocess_fwd_noalloc", "gs_render_stats", "gs_sh_fwd", "gs_sh_bwd", "gs_sh_fwd_f16",
-            "gs_sh_bwd_f16")
+            "gs_sh_bwd_f16", "gs_adam_step")
 
 
 class GsCamera(ctypes.Structure):
@@ -45,6 +45,14 @@ class GsCamera(ctypes.Structure):
         ("alpha_min", ctypes.c_float), ("T_min", ctypes.c_float), ("sigma_mult", ctypes.c_float),
         ("bg", ctypes.c_float * 3),
     ]
+
+
+class GsAdamConfig(ctypes.Structure):
+    """gs_adam_config: per-group learning rates, Adam's betas and eps, and the
+    warm-up length of the position and scale rates."""
+    _fields_ = [("lr_means", ctypes.c_float), ("lr_scales", ctypes.c_float), ("lr_quats", ctypes.c_float),
+                ("lr_opacity", ctypes.c_float), ("lr_colors", ctypes.c_float), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("eps", ctypes.c_float), ("warmup_steps", ctypes.c_int)]
 
 
 class GsError(RuntimeError):
@@ -92,6 +100,10 @@ def lib() -> ctypes.CDLL:
         L.gs_sh_fwd.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P]
         L.gs_sh_bwd.restype = I
         L.gs_sh_bwd.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P, P, P]
+        L.gs_preprocess_fwd_noalloc.restype = I
+        L.gs_preprocess_fwd_noalloc.argtypes = [cam, I] + [P] * 11 + [P]
+        L.gs_adam_step.restype = I
+        L.gs_adam_step.argtypes = [ctypes.POINTER(GsAdamConfig), I, I, I] + [P] * 14 + [P]
         L.gs_sh_fwd_f16.restype = I
         L.gs_sh_fwd_f16.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P]
         L.gs_sh_bwd_f16.restype = I
@@ -376,11 +388,7 @@ def gs_preprocess_fwd_noalloc(cam, means, scales, quats, opacity, mean2d, depth,
     """gs_preprocess_fwd without a workspace, for callers that cannot
     allocate device memory: the scratch is a fixed array inside libgs.so
     (N up to NOALLOC_MAX_GAUSSIANS; calls on one device must not overlap)."""
-    L = lib()
-    fn = L.gs_preprocess_fwd_noalloc
-    if fn.argtypes is None:
-        fn.restype = ctypes.c_int
-        fn.argtypes = [ctypes.POINTER(GsCamera), ctypes.c_int] + [ctypes.c_void_p] * 11 + [ctypes.c_void_p]
+    fn = lib().gs_preprocess_fwd_noalloc
     N = means.shape[0]
     f32, i32, u32 = torch.float32, torch.int32, torch.uint32
     _check(means, "means", f32, (N, 3))
@@ -398,3 +406,32 @@ def gs_preprocess_fwd_noalloc(cam, means, scales, quats, opacity, mean2d, depth,
     _ok("gs_preprocess_fwd_noalloc", fn(
         ctypes.byref(c), int(N), _ptr(means), _ptr(scales), _ptr(quats), _ptr(opacity), _ptr(mean2d), _ptr(depth),
         _ptr(conic_opacity), _ptr(radius), _ptr(rect), _ptr(tiles_touched), _ptr(d_num_pairs), _stream(stream)))
+
+
+def gs_adam_step(cfg: GsAdamConfig, step: int, params: dict, grads: dict, m, v, scales=None, opacity=None,
+                 stream=None) -> None:
+    """Fused Adam step.  ``params``: means [N,3], log_scales [N,3], quats [N,4],
+    logit_opacity [N], colors [N,C] (float32, updated in place); ``grads``:
+    dL_dmeans, dL_dscales, dL_dquats, dL_dopacity, dL_dcolors as returned by
+    the rasterizer (w.r.t. activated scales and opacity); ``m``, ``v``: float32
+    [(11 + C) N] moments (zero before step 1); ``scales``, ``opacity``:
+    optional outputs of the new activated values."""
+    N = params["means"].shape[0]
+    colors = params["colors"]
+    C = colors.shape[1] if colors.dim() == 2 else int(colors[0].numel()) if N else 0
+    f32 = torch.float32
+    for k, shp in (("means", (N, 3)), ("log_scales", (N, 3)), ("quats", (N, 4)), ("logit_opacity", (N,))):
+        _check(params[k], k, f32, shp)
+    _check(colors, "colors", f32)
+    for k, shp in (("dL_dmeans", (N, 3)), ("dL_dscales", (N, 3)), ("dL_dquats", (N, 4)), ("dL_dopacity", (N,))):
+        _check(grads[k], k, f32, shp)
+    _check(grads["dL_dcolors"], "dL_dcolors", f32, tuple(colors.shape))
+    _check(m, "m", f32, ((11 + C) * N,))
+    _check(v, "v", f32, ((11 + C) * N,))
+    _check(scales, "scales", f32, (N, 3), optional=True)
+    _check(opacity, "opacity", f32, (N,), optional=True)
+    _ok("gs_adam_step", lib().gs_adam_step(
+        ctypes.byref(cfg), int(step), int(N), int(C), _ptr(params["means"]), _ptr(params["log_scales"]),
+        _ptr(params["quats"]), _ptr(params["logit_opacity"]), _ptr(colors), _ptr(grads["dL_dmeans"]),
+        _ptr(grads["dL_dscales"]), _ptr(grads["dL_dquats"]), _ptr(grads["dL_dopacity"]), _ptr(grads["dL_dcolors"]),
+        _ptr(m), _ptr(v), _ptr(scales), _ptr(opacity), _stream(stream)))

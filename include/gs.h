@@ -312,6 +312,38 @@ GS_API int gs_sh_bwd_f16(const gs_camera* cam, int N, int degree, int K, const f
                          const unsigned short* sh, float offset, const float* dL_dcolors, float* dL_dsh,
                          float* dL_dmeans, void* stream);
 
+/*
+ * gs_adam_step - fused optimiser step for the Gaussians' parameters
+ *   ([TR] C.2: Adam with one learning rate per parameter group and a linear
+ *   warm-up of the position and scale rates; Adam after Kingma and Ba).
+ *   Raw parameters: means [N,3], log_scales [N,3] (scales = exp), quats [N,4]
+ *   (16-byte aligned; renormalised to unit length after the update),
+ *   logit_opacity [N] (opacity = sigmoid), colors [N,C] (C = 3 for RGB,
+ *   3 * K for K spherical-harmonics coefficients; C = 0 skips the group).
+ *   Gradients are those the rasterizer returns, w.r.t. the ACTIVATED values
+ *   (dL_dscales w.r.t. exp(log_scales), dL_dopacity w.r.t. the opacity); they
+ *   are chained through exp / sigmoid here.  step counts from 1; the rate of
+ *   means and log_scales is multiplied by min(1, step / warmup_steps)
+ *   (warmup_steps = 0: no warm-up).
+ * m, v [(11 + C) N] each: first and second moments, group-major layout
+ *   [means 3N | log_scales 3N | quats 4N | opacity N | colors C N]; zero them
+ *   before step 1.  Parameters, m and v are updated in place.
+ * scales [N,3], opacity [N] (optional, NULL to skip): written with the new
+ *   activated values, ready for gs_preprocess_fwd.
+ * Errors: GS_ERR_INVALID_ARG for step < 1, negative sizes, betas outside
+ *   [0, 1), negative eps, missing pointers or unaligned quaternions.
+ */
+typedef struct {
+    float lr_means, lr_scales, lr_quats, lr_opacity, lr_colors;
+    float beta1, beta2, eps;
+    int warmup_steps;
+} gs_adam_config;
+
+GS_API int gs_adam_step(const gs_adam_config* cfg, int step, int N, int C, float* means, float* log_scales,
+                        float* quats, float* logit_opacity, float* colors, const float* dL_dmeans,
+                        const float* dL_dscales, const float* dL_dquats, const float* dL_dopacity,
+                        const float* dL_dcolors, float* m, float* v, float* scales, float* opacity, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

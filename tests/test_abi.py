@@ -34,6 +34,32 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, name), name
 
 
+def _prototypes():
+    """name -> number of parameters, from the GS_API declarations of include/*.h."""
+    protos = {}
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            for name, params in re.findall(r"GS_API\s+[\w\s\*]+?\b(gs_\w+)\s*\(([^)]*)\)", txt):
+                params = params.strip()
+                protos[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_signatures_match_header(lib):
+    """Every ctypes prototype of the binding has as many parameters as the C
+    declaration, so a call can never be marshalled against the wrong layout."""
+    protos = _prototypes()
+    assert set(protos) == set(B.EXPORTED)
+    for name, n in protos.items():
+        assert len(getattr(lib, name).argtypes) == n, name
+
+
+def test_adam_config_layout_matches_header():
+    # float lr x5, beta1, beta2, eps; int warmup_steps
+    assert ctypes.sizeof(B.GsAdamConfig) == 4 * 9
+
+
 def test_camera_struct_layout_matches_header():
     # int width, height, tile; float fx, fy, cx, cy, R[9], t[3], 6 scalars, bg[3]
     assert ctypes.sizeof(B.GsCamera) == 4 * (3 + 4 + 9 + 3 + 6 + 3)
