@@ -109,3 +109,19 @@ def test_failed_rank_is_reported_not_hung():
     assert res[1][1] == "error" and "injected" in res[1][3]
     # rank 0 reaches the all-reduce alone and gets an error from the timeout
     assert res[0][1] == "error"
+
+
+def test_split_image_bands_cover_the_frame():
+    from differentiable_gaussian_splatting_preprocess_b200 import scenes
+    cam = scenes.Camera(1920, 1080, 1600.0, 1600.0, 960.0, 540.0)
+    for parts in (1, 2, 3, 8, 68, 100):
+        bands = MV.split_image(cam, parts)
+        rows = MV.band_rows(cam, parts)
+        assert len(bands) == len(rows) <= min(parts, 68)
+        assert rows[0][0] == 0 and rows[-1][1] == 1080
+        for (a0, a1), (b0, b1) in zip(rows, rows[1:]):
+            assert a1 == b0 and a0 % 16 == 0
+        for bc, (y0, y1) in zip(bands, rows):
+            assert bc.height == y1 - y0 and bc.cy == cam.cy - y0 and bc.width == cam.width
+    with pytest.raises(ValueError):
+        MV.split_image(cam, 0)
