@@ -40,7 +40,7 @@ UNIT = "Gaussian·pixel evals/s"
 # count: any other term provably contributes nothing and may be skipped.
 OPS_FWD_EVAL = 24
 OPS_BWD_EVAL = 60
-# DRAM bytes per launch from the committed ncu capture of k_render_bwd
+# DRAM bytes per launch from the committed ncu capture of the render backward (k_render_bwd_warp)
 # (dram__bytes_read.sum + dram__bytes_write.sum) and the SHA-1 of the render
 # sources it was taken on; reported only while the sources are unchanged.
 RECORDED_TRAFFIC = {"k_render_bwd": dict(bytes=137050624, sources_sha1="98f976d872bb8d2f79ab231a2c5da36d56655d4b")}
@@ -401,7 +401,7 @@ def run_ours(args):
     rb_ach = bwd_ops / (mean["render_bwd"] / 1e3) / 1e12
     rec_t = RECORDED_TRAFFIC["k_render_bwd"]
     traffic = rec_t["bytes"] if (rec_t["sources_sha1"] == _render_sources_sha1() and len(mine) == 1) else None
-    roofline = dict(kernel="k_render_bwd", bound="alu", achieved=rb_ach, peak=alu_peak, unit="Tops/s",
+    roofline = dict(kernel="k_render_bwd_warp", bound="alu", achieved=rb_ach, peak=alu_peak, unit="Tops/s",
                     frac=rb_ach / alu_peak, traffic=traffic, ops_per_launch=bwd_ops // len(mine),
                     ops_basis=f"{OPS_BWD_EVAL} FP32 ops x {n_blended} blended terms",
                     peak_src=f"148 SMs x 128 FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz (sm_max_mhz)")
