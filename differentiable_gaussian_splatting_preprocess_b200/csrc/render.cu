@@ -11,9 +11,11 @@
 // list from the last contributor towards the front, recover T <- T / (1 - a),
 // and accumulate dL/dcolor = T a dL/dC and dL/da = T (c - C_behind) . dL/dC
 // (section 2's table), then through G to the conic and the 2D mean.
-// Per-Gaussian partial gradients are reduced across the warp and across the
-// CTA before any global atomic, so a (tile, Gaussian) pair costs at most one
-// float2, one float4 and three float atomics.
+// Per-Gaussian partial gradients are reduced across the warp before any
+// global atomic: with the forward's contribution mask, one 9-lane atomic
+// instruction per (quadrant, Gaussian); without it, the warps' sums are
+// added in shared memory first and a (tile, Gaussian) pair costs one float2,
+// one float4 and three float atomics.
 
 #include <cuda_runtime.h>
 
