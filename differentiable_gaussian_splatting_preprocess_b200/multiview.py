@@ -98,28 +98,48 @@ def render_views_from_host(cams: Sequence, host_params: Dict[str, torch.Tensor],
                            camera_ids: Optional[Sequence[int]] = None, state: Optional[dict] = None,
                            host_grads: Optional[Dict[str, torch.Tensor]] = None,
                            reduce_fn: Optional[Callable[[Dict[str, torch.Tensor]], None]] = None,
-                           device=None) -> Dict[str, torch.Tensor]:
+                           device=None, pipelined: bool = False) -> Dict[str, torch.Tensor]:
     """One training step's rasterization from host (pinned) inputs to host
     gradients, with the copies overlapped with the kernels.
 
-    The inputs move to reused device buffers on a side stream, in the order
-    the stages read them: the geometry (means, scales, quats, opacity) first
-    - the projection waits for it - then the colours, which the compositing
+    The inputs move to device buffers on a side stream, in the order the
+    stages read them: the geometry (means, scales, quats, opacity) first -
+    the projection waits for it - then the colours, which the compositing
     waits for while projection and binning run, then each view's dL/dimage,
     which only its backward waits for.  Every view runs in capacity mode
     (``capacity[n]`` pairs, no host round trip).  ``reduce_fn`` (e.g. the
     cross-rank all-reduce) runs on the summed gradients before they are
-    copied to ``host_grads``.  ``state`` keeps the stream and buffers across
-    steps."""
+    copied to ``host_grads``.  ``state`` keeps the streams and buffers across
+    steps.
+
+    Without ``pipelined`` the gradients are copied back on the compute stream
+    (the caller synchronises it before reading ``host_grads``).  With
+    ``pipelined`` the device buffers are double-buffered and the copy back
+    runs on a third stream: step k+1's inputs are copied while step k
+    computes and step k-1's gradients are copied back, and the call returns
+    without waiting; ``state["done"]`` is an event that completes when this
+    step's gradients are in ``host_grads``."""
     dev = torch.device("cuda") if device is None else torch.device(device)
     st = state if state is not None else {}
     cur = torch.cuda.current_stream(dev)
-    if "stream" not in st:
+    nslot = 2 if pipelined else 1
+    if "stream" not in st or st.get("nslot") != nslot:
+        st.clear()
+        st["nslot"] = nslot
         st["stream"] = torch.cuda.Stream(dev)
-        st["params"] = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_params.items()}
-        st["dls"] = [torch.empty(h.shape, dtype=h.dtype, device=dev) for h in host_dls]
-    cs, dp, dd = st["stream"], st["params"], st["dls"]
-    cs.wait_stream(cur)  # the previous step's readers of these buffers are done
+        st["d2h"] = torch.cuda.Stream(dev)
+        st["params"] = [{k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_params.items()}
+                        for _ in range(nslot)]
+        st["dls"] = [[torch.empty(h.shape, dtype=h.dtype, device=dev) for h in host_dls] for _ in range(nslot)]
+        st["grads"] = [RZ.zero_grads(host_params["means"].shape[0], dev) for _ in range(nslot)]
+        st["freed"] = [None] * nslot  # per slot: event after which its buffers may be overwritten
+        st["slot"] = -1
+    slot = st["slot"] = (st["slot"] + 1) % nslot
+    cs, dp, dd, grads = st["stream"], st["params"][slot], st["dls"][slot], st["grads"][slot]
+    if st["freed"][slot] is not None:
+        cs.wait_event(st["freed"][slot])  # the readers of this slot's inputs are done
+    else:
+        cs.wait_stream(cur)
     with torch.cuda.stream(cs):
         for k in GEOMETRY_KEYS:
             dp[k].copy_(host_params[k], non_blocking=True)
@@ -134,13 +154,12 @@ def render_views_from_host(cams: Sequence, host_params: Dict[str, torch.Tensor],
             e = torch.cuda.Event()
             e.record(cs)
             e_dl.append(e)
+    d2h_prev = st.get("d2h_done", [None] * nslot)[slot]
+    if d2h_prev is not None:
+        cur.wait_event(d2h_prev)  # this slot's gradients of two steps ago are back on the host
     cur.wait_event(e_geo)
-    grads = st.get("grads")
-    if grads is None:
-        grads = st["grads"] = RZ.zero_grads(dp["means"].shape[0], dev)
-    else:
-        for v in grads.values():
-            v.zero_()
+    for v in grads.values():
+        v.zero_()
     ids = list(range(len(cams))) if camera_ids is None else list(camera_ids)
     for n, cam in enumerate(cams):
         rz = rasterizers.get(ids[n])
@@ -152,9 +171,26 @@ def render_views_from_host(cams: Sequence, host_params: Dict[str, torch.Tensor],
                     dL_ready=e_dl[n])
     if reduce_fn is not None:
         reduce_fn(grads)
+    computed = torch.cuda.Event()
+    computed.record(cur)
+    st["freed"][slot] = computed
     if host_grads is not None:
-        for k, h in host_grads.items():
-            h.copy_(grads[k], non_blocking=True)
+        if pipelined:
+            ds = st["d2h"]
+            ds.wait_event(computed)
+            with torch.cuda.stream(ds):
+                for k, h in host_grads.items():
+                    h.copy_(grads[k], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(ds)
+            st.setdefault("d2h_done", [None] * nslot)[slot] = done
+            st["done"] = done
+        else:
+            for k, h in host_grads.items():
+                h.copy_(grads[k], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(cur)
+            st["done"] = done
     return grads
 
 

@@ -262,6 +262,35 @@ def test_capacity_overflow_is_reported_and_recoverable():
     assert rz.status() == 0 and int(to_np(fr.num_pairs)[0]) > 1000
 
 
+def test_pair_count_overflow_is_reported():
+    """A 65536 x 65536 image (4096 x 4096 tiles) with 300 Gaussians whose
+    support covers it: 300 * 2^24 pairs exceed 2^32 - 1.  The preprocess
+    reports GS_ERR_OVERFLOW, saturates the device pair count, and a binning
+    call then reports the capacity error and leaves every range empty."""
+    sc = _tiny(n=300, width=64, height=64, seed=9, sigma_mult=1e4)
+    cam = sc.cameras[0].replace(width=65536, height=65536, fx=65536.0, fy=65536.0, cx=32768.0, cy=32768.0)
+    gs = GpuScene(sc)
+    from differentiable_gaussian_splatting_preprocess_b200 import rasterizer as RZ
+    rz = RZ.Rasterizer(cam)
+    pre = rz.preprocess(gs.means, gs.scales, gs.quats, gs.opacity)
+    torch.cuda.synchronize()
+    tt = to_np(pre["tiles_touched"]).astype(np.int64)
+    o = oracle.preprocess(cam, sc.means, sc.scales, sc.quats, sc.opacity, "f32")
+    np.testing.assert_array_equal(tt, o["tiles_touched"])
+    assert tt.sum() > 0xFFFFFFFF and tt.max() == 4096 * 4096
+    assert rz.status() & B.GS_ERR_OVERFLOW
+    assert int(to_np(pre["num_pairs"]).view(np.uint32)[0]) == 0xFFFFFFFF
+    ids = torch.empty(1000, dtype=torch.uint32, device="cuda")
+    ranges = torch.full((B.num_tiles(cam), 2), 7, dtype=torch.uint32, device="cuda")
+    B.gs_bin_sort(cam, pre["depth"], pre["rect"], pre["tiles_touched"], pre["num_pairs"], 1000, ids, ranges, None,
+                  rz.workspace(sc.N, 1000))
+    torch.cuda.synchronize()
+    assert rz.status() & B.GS_ERR_CAPACITY
+    assert not to_np(ranges).any()
+    B.gs_clear_status(rz.ws)
+    assert rz.status() == 0
+
+
 def test_capacity_mode_matches_host_sized():
     sc = _scene(2)
     cam = sc.cameras[0]
@@ -430,6 +459,19 @@ def test_render_views_from_host_overlapped_copies():
         for k in MV.GRAD_KEYS:
             assert rel_l2(out[k].numpy(), to_np(ref[k])) <= 1e-5, k
     assert all(rz.status() == 0 for rz in rzs.values())
+    # pipelined: double-buffered inputs and gradients, copy-back on its own
+    # stream, no wait between steps; every step's gradients are the same
+    outs = []
+    pstate = {}
+    for _ in range(4):
+        o = {k: torch.empty(tuple(ref[k].shape), pin_memory=True) for k in MV.GRAD_KEYS}
+        MV.render_views_from_host(cams, host, host_dl, rzs, [200_000, 200_000], state=pstate, host_grads=o,
+                                  pipelined=True)
+        outs.append((o, pstate["done"]))
+    for o, done in outs:
+        done.synchronize()
+        for k in MV.GRAD_KEYS:
+            assert rel_l2(o[k].numpy(), to_np(ref[k])) <= 1e-5, k
 
 
 def test_cuda_graph_replay_matches_eager():
