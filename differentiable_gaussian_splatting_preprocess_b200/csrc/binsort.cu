@@ -7,16 +7,21 @@
 // reused by the backward.
 //
 // The order produced is that of a sort of 64-bit keys (tile << 32 |
-// float_bits(depth)) with ties broken by Gaussian id.  It is reached in two
-// sorts instead of one wide one:
+// float_bits(depth)) with ties broken by Gaussian id, reached without ever
+// sorting the (tile, Gaussian) pairs:
 //   1. the N Gaussians are sorted by depth bits (stable LSD radix sort, 8-bit
 //      digits, ids in increasing order initially, culled ones last), which
 //      gives every visible Gaussian its (depth, id) rank;
-//   2. the (tile, Gaussian) pairs are emitted in rank order and stably sorted
-//      by tile id alone (ceil(log2 T) bits, at most 8 per pass).
-// A stable sort by tile of a list already in (depth, id) order yields the
-// (tile, depth, id) order, so the result is the same as the 64-bit sort while
-// the pair-sized passes only move the tile bits.
+//   2. cell route (images of at most 1024 x 1024 tiles): the (cell,
+//      Gaussian) pairs of 4 x 4-tile cells are stably sorted by cell, and
+//      each cell's rank-ordered list is expanded into its 16 tiles' lists
+//      (see "Super-tile binning" below);
+//   3. wide-image route (otherwise): the (tile, Gaussian) pairs are emitted
+//      in rank order and stably sorted by tile id alone (ceil(log2 T) bits,
+//      at most 8 per pass), ranges found by comparing neighbours.
+// A stable sort by tile (or cell) of a list already in (depth, id) order
+// keeps that order within each tile, so both routes give the 64-bit sort's
+// result.
 //
 // Every kernel is a plain grid over its data; there are no inter-block waits.
 
