@@ -544,6 +544,38 @@ def test_image_space_split_equals_full_frame():
         assert rel_l2(to_np(grads[k]), to_np(full[k])) <= GRAD_REL_L2, k
 
 
+def test_autograd_binding_matches_direct_backward():
+    """rasterize() under torch.autograd: the image is the forward's, and
+    backpropagating sum(image * dL) gives the direct backward's gradients,
+    including through user-side activations (scales = exp, opacity = sigmoid)."""
+    from differentiable_gaussian_splatting_preprocess_b200 import autograd as AG
+    from differentiable_gaussian_splatting_preprocess_b200 import rasterizer as RZ
+    sc = _scene(2)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    dl = to_dev(sc.dL_dimage[0])
+    rz_ref = RZ.Rasterizer(cam)
+    fr = rz_ref.forward(gs.means, gs.scales, gs.quats, gs.opacity, gs.colors)
+    ref = rz_ref.backward(fr, gs.means, gs.scales, gs.quats, gs.colors, dl)
+    torch.cuda.synchronize()
+    log_s = torch.log(gs.scales).requires_grad_(True)
+    logit = torch.logit(gs.opacity).requires_grad_(True)
+    means = gs.means.clone().requires_grad_(True)
+    quats = gs.quats.clone().requires_grad_(True)
+    colors = gs.colors.clone().requires_grad_(True)
+    rz = RZ.Rasterizer(cam)
+    img = AG.rasterize(means, torch.exp(log_s), quats, torch.sigmoid(logit), colors, rz)
+    (img * dl).sum().backward()
+    torch.cuda.synchronize()
+    assert rel_l2(to_np(img.detach()), to_np(fr.image)) <= 1e-6
+    for t, k in ((means, "dL_dmeans"), (quats, "dL_dquats"), (colors, "dL_dcolors")):
+        assert rel_l2(to_np(t.grad), to_np(ref[k])) <= 1e-5, k
+    s = torch.exp(log_s).detach()
+    assert rel_l2(to_np(log_s.grad), to_np(ref["dL_dscales"] * s)) <= 1e-5
+    o = torch.sigmoid(logit).detach()
+    assert rel_l2(to_np(logit.grad), to_np(ref["dL_dopacity"] * o * (1 - o))) <= 1e-5
+
+
 def test_launch_count_is_fixed_per_frame():
     """The library's launch counter: every frame of one configuration issues
     the same number of kernels (no host-dependent fallbacks), and only the
