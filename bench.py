@@ -414,6 +414,12 @@ def run_ours(args):
                       frac=(fwd_bytes + bwd_bytes) / rfb_s / 1e9 / peaks["hbm_gbs"],
                       bytes_per_frame=fwd_bytes + bwd_bytes, peak_src=peaks["src"])
     fwd_alu = fwd_ops / (mean["render_fwd"] / 1e3) / 1e12
+    # the metric's "bwd HBM GB/s": the render backward alone, algorithmic
+    # bytes and, where the committed capture applies, measured DRAM bytes
+    rb_s = mean["render_bwd"] / 1e3
+    bwd_hbm = dict(achieved_gbs=bwd_bytes / rb_s / 1e9, peak_gbs=peaks["hbm_gbs"],
+                   frac=bwd_bytes / rb_s / 1e9 / peaks["hbm_gbs"], bytes_per_frame=bwd_bytes,
+                   dram_gbs=(traffic / (rb_s / len(mine)) / 1e9) if traffic else None, peak_src=peaks["src"])
     # HBM view of the binning (the sort is the stage an HBM roofline fits)
     bin_bytes = len(mine) * sc.N * BIN_BYTES_GAUSSIAN + Ps * BIN_BYTES_CELL_PAIR + P * BIN_BYTES_PAIR
     bin_gbs = bin_bytes / (mean["bin_sort"] / 1e3) / 1e9
@@ -497,7 +503,7 @@ def run_ours(args):
             stage_ms={s: round(v, 4) for s, v in mean.items()}, dominant_stage=dominant,
             roofline=roofline, render_fwd_alu=dict(achieved=fwd_alu, peak=alu_peak, unit="Tops/s",
                                                    frac=fwd_alu / alu_peak),
-            render_hbm=render_hbm, bin_sort_hbm=bin_hbm, cpu_baseline=cpu, e2e=e2e, gpu_launches=launches,
+            render_hbm=render_hbm, render_bwd_hbm=bwd_hbm, bin_sort_hbm=bin_hbm, cpu_baseline=cpu, e2e=e2e, gpu_launches=launches,
             clocks=clocks)
         print(json.dumps(line), flush=True)
     if world > 1:
