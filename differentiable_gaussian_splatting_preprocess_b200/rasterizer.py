@@ -152,3 +152,39 @@ def zero_grads(N: int, device) -> Dict[str, torch.Tensor]:
     return dict(dL_dmeans=torch.zeros((N, 3), **f), dL_dscales=torch.zeros((N, 3), **f),
                 dL_dquats=torch.zeros((N, 4), **f), dL_dopacity=torch.zeros((N,), **f),
                 dL_dcolors=torch.zeros((N, 3), **f))
+
+
+class GraphedStep:
+    """Forward + backward of one camera recorded once into a CUDA graph and
+    replayed: one launch per step instead of one per kernel.  The inputs are
+    the tensors given here, read in place at every replay (update them with
+    ``copy_`` between replays); the step runs in capacity mode, so the pair
+    count of every replayed frame must fit ``capacity`` (check ``status()``:
+    GS_ERR_CAPACITY otherwise).  ``grads`` (allocated when None) is zeroed and
+    refilled by every replay; ``frame`` holds the forward's outputs."""
+
+    def __init__(self, rz: Rasterizer, means, scales, quats, opacity, colors, dL_dimage, capacity: int,
+                 grads: Optional[Dict[str, torch.Tensor]] = None, use_mask: bool = True):
+        self.rz = rz
+        self.grads = zero_grads(means.shape[0], rz.device) if grads is None else grads
+        args = (means, scales, quats, opacity, colors)
+
+        def step():
+            for v in self.grads.values():
+                v.zero_()
+            fr = rz.forward(*args, capacity=capacity, use_mask=use_mask)
+            rz.backward(fr, means, scales, quats, colors, dL_dimage, grads=self.grads)
+            return fr
+
+        step()  # allocates every buffer and makes every one-time setup call outside the capture
+        torch.cuda.synchronize(rz.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.frame = step()
+
+    def replay(self) -> Dict[str, torch.Tensor]:
+        self.graph.replay()
+        return self.grads
+
+    def status(self) -> int:
+        return self.rz.status()

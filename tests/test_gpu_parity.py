@@ -511,6 +511,21 @@ def test_cuda_graph_replay_matches_eager():
     for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity"):
         assert rel_l2(to_np(grads[k]), ref[k]) <= 1e-5, k
     del g
+    # the same through the library's helper, with inputs updated in place
+    # between replays
+    gstep = RZ.GraphedStep(RZ.Rasterizer(cam), gs.means, gs.scales, gs.quats, gs.opacity, gs.colors, dl, cap)
+    for _ in range(2):
+        out = gstep.replay()
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(gstep.frame.image), ref["image"])
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity"):
+        assert rel_l2(to_np(out[k]), ref[k]) <= 1e-5, k
+    gs.colors.mul_(0.5)
+    gstep.replay()
+    torch.cuda.synchronize()
+    assert gstep.status() == 0
+    assert not np.array_equal(to_np(gstep.frame.image), ref["image"])
+    gs.colors.mul_(2.0)
 
 
 def test_image_space_split_equals_full_frame():
