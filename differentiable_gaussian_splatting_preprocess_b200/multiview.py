@@ -18,34 +18,12 @@ from . import rasterizer as RZ
 GRAD_KEYS = ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors")
 
 
-def split_image(cam, parts: int, tile: int = 16) -> List:
-    """Image-space split of one camera into ``parts`` horizontal bands of
-    whole tile rows (the last band takes the remainder; bands may be empty
-    when the image has fewer tile rows than parts, and are then omitted).
-
-    A band is the same camera with its principal point moved up by the
-    band's first pixel row: every pixel keeps its position relative to the
-    Gaussians, and tile rows coincide with the full frame's.  Because the
-    preprocess backward is linear in the 2D gradients, the 3D gradients of
-    the bands, summed, are those of the full frame: the band renders can run
-    on different ranks and meet in the same single all-reduce as the
-    camera-parallel split."""
+def band_rows(cam, parts: int, tile: int = 16) -> List[tuple]:
+    """Pixel row ranges [y0, y1) of ``parts`` horizontal bands of whole tile
+    rows (ceil(rows / parts) tile rows each, the last band the remainder;
+    empty bands, when the image has fewer tile rows than parts, are omitted)."""
     if parts < 1:
         raise ValueError("parts must be >= 1")
-    rows = (cam.height + tile - 1) // tile
-    per = (rows + parts - 1) // parts
-    bands = []
-    for b in range(parts):
-        r0, r1 = b * per, min(rows, (b + 1) * per)
-        if r0 >= r1:
-            continue
-        y0, y1 = r0 * tile, min(cam.height, r1 * tile)
-        bands.append(cam.replace(height=y1 - y0, cy=cam.cy - y0))
-    return bands
-
-
-def band_rows(cam, parts: int, tile: int = 16) -> List[tuple]:
-    """Pixel row ranges [y0, y1) of split_image's bands, in order."""
     rows = (cam.height + tile - 1) // tile
     per = (rows + parts - 1) // parts
     out = []
@@ -54,6 +32,19 @@ def band_rows(cam, parts: int, tile: int = 16) -> List[tuple]:
         if r0 < r1:
             out.append((r0 * tile, min(cam.height, r1 * tile)))
     return out
+
+
+def split_image(cam, parts: int, tile: int = 16) -> List:
+    """Image-space split of one camera into the bands of band_rows.
+
+    A band is the same camera with its principal point moved up by the
+    band's first pixel row: every pixel keeps its position relative to the
+    Gaussians, and tile rows coincide with the full frame's.  Because the
+    preprocess backward is linear in the 2D gradients, the 3D gradients of
+    the bands, summed, are those of the full frame: the band renders can run
+    on different ranks and meet in the same single all-reduce as the
+    camera-parallel split."""
+    return [cam.replace(height=y1 - y0, cy=cam.cy - y0) for y0, y1 in band_rows(cam, parts, tile)]
 
 
 def assign_cameras(n_cameras: int, world: int, rank: int) -> List[int]:
