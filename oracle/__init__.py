@@ -139,13 +139,16 @@ def preprocess(cam, means, scales, quats, opacity, mode: str = "f32") -> Dict[st
     return out
 
 
-def bin_pairs(cam, depth, rect, tiles_touched, mode: str = "f32") -> Dict[str, np.ndarray]:
+def bin_pairs(cam, depth, rect, tiles_touched, mode: str = "f32", want_keys: bool = True) -> Dict[str, np.ndarray]:
+    """Every (tile, Gaussian) pair in (tile, depth, id) order: ``ids`` [P],
+    ``ranges`` [T, 2] and, with ``want_keys``, the 64-bit (tile << 32 | depth
+    bits) keys."""
     dt = _dt(mode)
     depth = _a(depth, dt)
     rect = _a(rect, np.int32)
     tt = _a(tiles_touched, np.uint32)
     P = int(tt.astype(np.uint64).sum())
-    keys = np.zeros(P, np.uint64)
+    keys = np.zeros(P, np.uint64) if want_keys else None
     ids = np.zeros(P, np.uint32)
     ranges = np.zeros((cam.tiles_x * cam.tiles_y if hasattr(cam, "tiles_x") else
                        ((cam.width + cam.tile - 1) // cam.tile) * ((cam.height + cam.tile - 1) // cam.tile), 2),
@@ -234,11 +237,13 @@ def preprocess_bwd(cam, means, scales, quats, radius, dL_dmean2d, dL_dconic_opac
     return out
 
 
-def forward(cam, means, scales, quats, opacity, colors, mode: str = "f64") -> Dict[str, np.ndarray]:
-    """Preprocess, binning and compositing for one camera."""
+def forward(cam, means, scales, quats, opacity, colors, mode: str = "f64",
+            tiles: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray]:
+    """Preprocess, binning and compositing for one camera (compositing of
+    the listed ``tiles`` only, when given)."""
     pre = preprocess(cam, means, scales, quats, opacity, mode)
-    b = bin_pairs(cam, pre["depth"], pre["rect"], pre["tiles_touched"], mode)
-    r = render_fwd(cam, b["ranges"], b["ids"], pre["mean2d"], pre["conic_opacity"], colors, mode)
+    b = bin_pairs(cam, pre["depth"], pre["rect"], pre["tiles_touched"], mode, want_keys=False)
+    r = render_fwd(cam, b["ranges"], b["ids"], pre["mean2d"], pre["conic_opacity"], colors, mode, tiles=tiles)
     return dict(pre=pre, bins=b, **r)
 
 

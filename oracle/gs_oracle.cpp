@@ -46,7 +46,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <tuple>
+#include <utility>
 #include <vector>
 
 #ifdef _OPENMP
@@ -233,37 +233,51 @@ inline uint32_t float_bits(float f) {
 }
 
 // Binning: every (tile, Gaussian) pair, sorted lexicographically by
-// (tile, depth, id) with a plain comparison sort; ranges by scanning.
+// (tile, depth, id) (training page, section E.3: Gaussians are listed per
+// tile and each tile's list is sorted by depth).  The pairs are grouped by
+// tile (a count per tile, a prefix sum of the counts, then each Gaussian
+// written into the groups of the tiles its rectangle covers), and every
+// tile's group is sorted by (depth, id) with a plain comparison sort.  Tiles
+// are independent, so their sorts run in parallel; the result is the same
+// whatever the thread count.  ranges[t] = [first, last + 1) of tile t's
+// group; an empty tile gets (0, 0).
 template <typename Real>
 long long bin(const oracle_camera* cam, int N, const Real* depth, const int* rect, const unsigned* tiles_touched,
               unsigned long long* keys, unsigned* ids, unsigned* ranges) {
     const int TX = (cam->width + cam->tile - 1) / cam->tile;
     const int TY = (cam->height + cam->tile - 1) / cam->tile;
     const int T = TX * TY;
-    std::vector<std::tuple<uint32_t, Real, uint32_t>> pairs;
-    size_t P = 0;
-    for (int i = 0; i < N; ++i) P += tiles_touched[i];
-    pairs.reserve(P);
+    std::vector<size_t> count(T, 0), start(T + 1, 0);
     for (int i = 0; i < N; ++i) {
         if (tiles_touched[i] == 0) continue;
         const int* r = rect + 4 * i;
         for (int ty = r[1]; ty < r[3]; ++ty)
-            for (int tx = r[0]; tx < r[2]; ++tx)
-                pairs.emplace_back((uint32_t)(ty * TX + tx), depth[i], (uint32_t)i);
+            for (int tx = r[0]; tx < r[2]; ++tx) ++count[ty * TX + tx];
     }
-    std::sort(pairs.begin(), pairs.end());
-    for (int t = 0; t < T; ++t) ranges[2 * t] = ranges[2 * t + 1] = 0;
-    for (size_t k = 0; k < pairs.size(); ++k) {
-        const uint32_t tile = std::get<0>(pairs[k]);
-        if (ids) ids[k] = std::get<2>(pairs[k]);
-        if (keys) {
-            float df = (float)std::get<1>(pairs[k]);
-            keys[k] = ((unsigned long long)tile << 32) | float_bits(df);
+    for (int t = 0; t < T; ++t) start[t + 1] = start[t] + count[t];
+    const size_t P = start[T];
+    std::vector<std::pair<Real, uint32_t>> pairs(P);
+    std::vector<size_t> cursor(start.begin(), start.end() - 1);
+    for (int i = 0; i < N; ++i) {
+        if (tiles_touched[i] == 0) continue;
+        const int* r = rect + 4 * i;
+        for (int ty = r[1]; ty < r[3]; ++ty)
+            for (int tx = r[0]; tx < r[2]; ++tx) pairs[cursor[ty * TX + tx]++] = {depth[i], (uint32_t)i};
+    }
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int t = 0; t < T; ++t) {
+        std::sort(pairs.begin() + start[t], pairs.begin() + start[t + 1]);
+        ranges[2 * t] = count[t] ? (unsigned)start[t] : 0u;
+        ranges[2 * t + 1] = count[t] ? (unsigned)start[t + 1] : 0u;
+        for (size_t k = start[t]; k < start[t + 1]; ++k) {
+            if (ids) ids[k] = pairs[k].second;
+            if (keys) {
+                const float df = (float)pairs[k].first;
+                keys[k] = ((unsigned long long)t << 32) | float_bits(df);
+            }
         }
-        if (k == 0 || std::get<0>(pairs[k - 1]) != tile) ranges[2 * tile] = (unsigned)k;
-        if (k + 1 == pairs.size() || std::get<0>(pairs[k + 1]) != tile) ranges[2 * tile + 1] = (unsigned)(k + 1);
     }
-    return (long long)pairs.size();
+    return (long long)P;
 }
 
 // Brute-force list of one tile: every Gaussian whose rectangle contains the

@@ -106,17 +106,26 @@ def test_backward_parity(cfg):
     for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
         e = rel_l2(gr[k], o3[k])
         assert e <= 1e-4, (k, e)
-    # end to end: the float64 oracle's own forward and backward
-    if cfg <= 3:
-        f = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0],
-                                    "f64")
-        for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
-            e = rel_l2(gr[k], f[k])
-            assert e <= GRAD_REL_L2, (k, e)
-        # the float64 pipeline takes its alpha_min / T_min decisions in float64,
-        # so a few pixels may differ by one term; the rest agree to 1e-4
-        bad = (np.abs(g["image"] - f["image"]) > IMAGE_ATOL).any(0).mean()
-        assert bad <= 1.0 - N_CONTRIB_MATCH, bad
+    # end to end: the float64 oracle's own forward and backward (its own
+    # projection, binning and compositing decisions, rounded independently)
+    f = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0], "f64")
+    for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors"):
+        e = rel_l2(gr[k], f[k])
+        assert e <= GRAD_REL_L2, (k, e)
+    _check_against_f64(g, f)
+
+
+def _check_against_f64(g, f, mask=None):
+    """The acceptance bars against the float64 pipeline, which takes its
+    alpha_min / T_min decisions in float64: contributor counts equal on
+    >= 99.99% of pixels, and the image within 1e-4 on >= 99.99% of pixels (a
+    pixel whose decisions differ by one term may differ by more)."""
+    if mask is None:
+        mask = np.ones(g["n_contrib"].shape, bool)
+    match = (g["n_contrib"][mask] == f["n_contrib"][mask]).mean()
+    assert match >= N_CONTRIB_MATCH, f"n_contrib match vs float64 {match}"
+    bad = (np.abs(g["image"] - f["image"]) > IMAGE_ATOL).any(0)[mask].mean()
+    assert bad <= 1.0 - N_CONTRIB_MATCH, f"image pixels beyond {IMAGE_ATOL} vs float64: {bad}"
 
 
 def _sample_tiles(cam, n, seed):
@@ -125,12 +134,15 @@ def _sample_tiles(cam, n, seed):
 
 
 @pytest.mark.slow
-def test_config5_four_cameras_sampled():
+def test_config5_four_cameras():
     """3M Gaussians, four cameras rendered back to back with 3D gradients
-    accumulated: preprocess bit-exact per camera, sampled tile lists against
-    brute force, sampled tiles' compositing and gradients against the oracle
-    (the upstream gradient is restricted to the sampled tiles, so the oracle
-    only has to run those)."""
+    accumulated.  Per camera: preprocess bit-exact; every tile range and every
+    tile's sorted id list bit-exact against the oracle's binning; every tile
+    composited against the fp32 mirror (image, final T, contributor counts);
+    sampled tiles' image and contributor counts against the float64 pipeline;
+    sampled tiles' gradients against the float64 oracle (the upstream gradient
+    is restricted to the sampled tiles, so the oracle's backward only has to
+    run those)."""
     sc = _scene(5)
     gs = GpuScene(sc)
     grads = None
@@ -143,14 +155,23 @@ def test_config5_four_cameras_sampled():
             mask[ty * 16:(ty + 1) * 16, tx * 16:(tx + 1) * 16] = True
         dl = np.where(mask[None], sc.dL_dimage[ci], 0.0).astype(np.float32)
         r = run_gpu(gs, cam, dL_dimage=dl, want_keys=False, grads=grads)
+        assert r["rz"].status() == 0
         grads = {k: r["grads"][k] for k in ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors")}
         g = frame_np(r["frame"])
         pre = _check_preprocess(sc, cam, g)
-        for t in tiles[:6]:
+        b = oracle.bin_pairs(cam, pre["depth"], pre["rect"], pre["tiles_touched"], "f32", want_keys=False)
+        assert b["num_pairs"] == g["num_pairs"]
+        np.testing.assert_array_equal(g["ranges"], b["ranges"])
+        np.testing.assert_array_equal(g["ids"], b["ids"])
+        del b
+        for t in tiles[:3]:  # the per-tile brute force, independent of the oracle's grouping
             s, e = g["ranges"][t]
             np.testing.assert_array_equal(g["ids"][s:e], oracle.tile_list(cam, pre["depth"], pre["rect"],
                                                                           pre["tiles_touched"], int(t)))
-        _check_render_fwd(cam, sc, g, tiles=tiles)
+        _check_render_fwd(cam, sc, g)
+        f64 = oracle.forward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, "f64", tiles=tiles)
+        _check_against_f64(g, f64, mask)
+        del f64
         o2 = oracle.render_bwd(cam, sc.N, g["ranges"], g["ids"], g["mean2d"], g["conic_opacity"], sc.colors, dl,
                                "f64", tiles=tiles)
         gr = {k: to_np(r["grads"][k]) for k in ("dL_dmean2d", "dL_dconic_opacity", "dL_dcolor")}

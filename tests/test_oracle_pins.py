@@ -255,14 +255,16 @@ def test_golden_compositing(mode):
                             T_min=case["T_min"], bg=tuple(case["bg"]))
         gs = case["gaussians"]
         n = len(gs)
-        f = oracle.forward(cam, [x["mean"] for x in gs], _iso(n, 0.1), _ident_q(n), [x["opacity"] for x in gs],
-                           [x["color"] for x in gs], mode)
+        f = oracle.forward(cam, np.reshape([x["mean"] for x in gs], (n, 3)), _iso(n, 0.1), _ident_q(n),
+                           np.reshape([x["opacity"] for x in gs], (n,)), np.reshape([x["color"] for x in gs], (n, 3)),
+                           mode)
         exp = case["expected"]
         tol = max(case["tol"], 1e-7 if mode == "f32" else 1e-12)
         np.testing.assert_allclose(f["image"][:, py, px], exp["color"], atol=tol, err_msg=case["name"])
         assert f["final_T"][py, px] == pytest.approx(exp["final_T"], abs=tol), case["name"]
         assert f["n_contrib"][py, px] == exp["n_contrib"], case["name"]
         assert f["n_blended"][py, px] == exp["n_blended"], case["name"]
+        assert f["n_eval"][py, px] == exp["n_eval"], case["name"]
 
 
 def test_single_gaussian_closed_form():
@@ -290,11 +292,14 @@ def test_partition_of_unity(mode, tol):
     np.testing.assert_allclose(f["image"], 1.0, atol=tol)
 
 
-def test_brute_force_compositing_equals_tiled():
+@pytest.mark.parametrize("T_min", [1e-4, 0.5])
+def test_brute_force_compositing_equals_tiled(T_min):
     """With a support radius large enough that every rectangle covers the
     image, the tiled renderer equals compositing every Gaussian at every pixel
-    in (depth, id) order, with no tiles and no binning."""
-    sc = scenes.random_tiny(n=12, width=48, height=40, seed=7, sigma_mult=1e3)
+    in (depth, id) order, with no tiles and no binning; so do its work counts
+    (entries evaluated, the stopping one included; terms blended) and its
+    per-quadrant blend mask.  T_min = 0.5 makes pixels stop early."""
+    sc = scenes.random_tiny(n=12, width=48, height=40, seed=7, sigma_mult=1e3, T_min=T_min)
     cam = sc.cameras[0]
     f = oracle.forward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, "f64")
     pre = f["pre"]
@@ -302,10 +307,20 @@ def test_brute_force_compositing_equals_tiled():
     order = np.lexsort((np.arange(sc.N), pre["depth"]))
     H, W = cam.height, cam.width
     img = np.zeros((3, H, W))
+    n_eval = np.zeros((H, W), np.int64)
+    n_blend = np.zeros((H, W), np.int64)
+    # every tile's list is the whole depth order, so tile t holds list
+    # positions t*N .. t*N + N - 1; mask bit of position k in 8x8 quadrant q
+    # of its tile: word (k // 32) * 4 + q, bit k % 32
+    words = 4 * ((cam.num_tiles * sc.N + 31) // 32)
+    mask = np.zeros(words, np.uint32)
     for y in range(H):
         for x in range(W):
+            tile = (y // 16) * cam.tiles_x + x // 16
+            quad = ((y % 16) // 8) * 2 + (x % 16) // 8
             T, C, last = 1.0, np.zeros(3), 0
             for k, j in enumerate(order):
+                n_eval[y, x] += 1
                 d = np.array([x + 0.5, y + 0.5]) - pre["mean2d"][j]
                 a, b, c, o = pre["conic_opacity"][j]
                 power = -0.5 * (a * d[0] ** 2 + c * d[1] ** 2) - b * d[0] * d[1]
@@ -319,9 +334,23 @@ def test_brute_force_compositing_equals_tiled():
                 C += sc.colors[j] * al * T
                 T *= 1 - al
                 last = k + 1
+                n_blend[y, x] += 1
+                pos = tile * sc.N + k
+                mask[(pos // 32) * 4 + quad] |= np.uint32(1 << (pos % 32))
             img[:, y, x] = C + T * np.array(cam.bg)
             assert f["n_contrib"][y, x] == last
     np.testing.assert_allclose(f["image"], img, atol=1e-12)
+    # the work counts and the per-quadrant blend mask, from the same walk
+    np.testing.assert_array_equal(f["n_eval"], n_eval)
+    np.testing.assert_array_equal(f["n_blended"], n_blend)
+    assert (n_eval > n_blend).any()  # alpha_min skips occur
+    if T_min > 0.1:
+        assert (n_eval < sc.N).any()  # so do stops
+    b = f["bins"]
+    r = oracle.render_fwd(cam, b["ranges"], b["ids"], pre["mean2d"], pre["conic_opacity"], sc.colors, "f64",
+                          blend_mask=True)
+    np.testing.assert_array_equal(r["blend_mask"], mask)
+    assert mask.any()
 
 
 def test_translation_by_one_tile():
@@ -494,20 +523,34 @@ def test_mirror_exp_error_bound():
     assert oracle.exp_f32(np.zeros(1))[0] == 1.0
 
 
-def test_densification_statistics_definition():
-    """Per visible view: accum += |dL/dmean2d|, count += 1; culled views add
-    nothing; two identical views double the accumulator."""
-    sc = scenes.random_tiny(n=8, seed=12)
-    cam = sc.cameras[0]
-    sc.means[7, 2] = -1.0  # culled in this view
-    fb = oracle.forward_backward(cam, sc.means, sc.scales, sc.quats, sc.opacity, sc.colors, sc.dL_dimage[0], "f64")
+def test_densification_statistics_closed_form():
+    """The densification accumulator of one isotropic Gaussian on the optical
+    axis, seen by two identical views and by a third that culls it, equals
+    twice the norm of the hand-derived 2D mean gradient.  With one Gaussian,
+    alpha = sigma G (no cap, no thresholds), C = alpha c + (1 - alpha) bg, and
+    an upstream gradient of 1 on channel 0 of one pixel p0, the mean gradient
+    of the chain-rule page (dG/dmu = G Sigma^-1 (x - mu)) gives
+    dL/dmean2d = (c_0 - bg_0) sigma G(p0) (p0 - mu) / s2^2 with
+    s2^2 = (f s / z)^2 + eps."""
+    f, z, s, sig = 32.0, 3.0, 0.2, 0.8
+    cam = _cam(32, 32, f, sigma_mult=50.0, alpha_min=0.0, T_min=0.0, bg=(0.1, 0.2, 0.3))
+    col = [0.9, 0.4, 0.6]
+    x0, y0 = 19, 14
+    dl = np.zeros((3, 32, 32))
+    dl[0, y0, x0] = 1.0
+    means, scales, quats = np.array([[0.0, 0.0, z]]), np.array([[s, s, s]]), _ident_q(1)
+    s22 = (f * s / z) ** 2 + _f32(cam.eps2d)
+    d = np.array([x0 + 0.5 - 16.0, y0 + 0.5 - 16.0])
+    G = math.exp(-(d @ d) / (2.0 * s22))
+    expect = (col[0] - _f32(cam.bg[0])) * sig * G * d / s22
+    behind = cam.replace(t=(0.0, 0.0, -10.0))  # the Gaussian is behind this camera: culled
     out = None
-    for _ in range(2):
-        out = oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, fb["pre"]["radius"], fb["dL_dmean2d"],
+    for c in (cam, behind, cam):
+        fb = oracle.forward_backward(c, means, scales, quats, [sig], [col], dl, "f64")
+        if c is cam:
+            np.testing.assert_allclose(fb["dL_dmean2d"][0], expect, rtol=1e-10)
+        out = oracle.preprocess_bwd(c, means, scales, quats, fb["pre"]["radius"], fb["dL_dmean2d"],
                                     fb["dL_dconic_opacity"], fb["dL_dcolor"], "f64", accumulate_into=out,
                                     densify=True)
-    norm = np.linalg.norm(fb["dL_dmean2d"], axis=1)
-    vis = fb["pre"]["radius"] > 0
-    np.testing.assert_allclose(out["grad2d_accum"], 2 * norm * vis, rtol=1e-14)
-    np.testing.assert_array_equal(out["vis_count"], 2 * vis.astype(np.uint32))
-    assert not vis[7] and out["vis_count"][7] == 0
+    assert out["grad2d_accum"][0] == pytest.approx(2.0 * float(np.linalg.norm(expect)), rel=1e-10)
+    assert out["vis_count"][0] == 2
