@@ -143,28 +143,73 @@ def _scene(cfg: int):
     return scenes.preset(cfg)
 
 
-def cpu_oracle_sample(sc, tile_stride: int, max_seconds: float = 25.0):
-    """Time the oracle on a bounded sample of the workload: full preprocess
-    and binning, then compositing forward (fp32) and backward (fp64) on every
-    ``tile_stride``-th tile."""
+def cpu_tile_stride(cfg: int) -> int:
+    """Tile sample of the CPU oracle: every tile up to config 3, every 16th
+    tile of the 1080p configs (the same sample in both arms)."""
+    return 16 if cfg >= 4 else 1
+
+
+def cpu_oracle_sample(sc, tile_stride: int):
+    """Time the oracle on a bounded sample of the workload, forward and
+    backward separately: forward = full preprocess and binning, then
+    compositing (fp32 mirror) of every ``tile_stride``-th tile; backward =
+    compositing backward (float64) of the same tiles, then the full
+    preprocess backward.  Evaluations are counted like the GPU metric's:
+    per sampled pixel, entries evaluated in the forward plus the contributor
+    prefix walked by the backward."""
     import oracle
     cam = sc.cameras[0]
     t0 = time.perf_counter()
     pre = oracle.preprocess(cam, sc.means, sc.scales, sc.quats, sc.opacity, "f32")
-    b = oracle.bin_pairs(cam, pre["depth"], pre["rect"], pre["tiles_touched"], "f32")
+    b = oracle.bin_pairs(cam, pre["depth"], pre["rect"], pre["tiles_touched"], "f32", want_keys=False)
     tiles = np.arange(0, cam.num_tiles, tile_stride, dtype=np.int32)
     r = oracle.render_fwd(cam, b["ranges"], b["ids"], pre["mean2d"], pre["conic_opacity"], sc.colors, "f32",
                           tiles=tiles)
+    t1 = time.perf_counter()
     g = oracle.render_bwd(cam, sc.N, b["ranges"], b["ids"], pre["mean2d"], pre["conic_opacity"], sc.colors,
                           sc.dL_dimage[0], "f64", tiles=tiles)
     oracle.preprocess_bwd(cam, sc.means, sc.scales, sc.quats, pre["radius"], g["dL_dmean2d"],
                           g["dL_dconic_opacity"], g["dL_dcolor"], "f64")
-    dt = time.perf_counter() - t0
-    evals = int(r["n_eval"].astype(np.int64).sum()) + int(r["n_contrib"].astype(np.int64).sum())
-    return dict(value=evals / dt, unit=UNIT, cores=oracle.num_threads(), kind="oracle",
-                sample=(f"full preprocess + binning of the {sc.name} scene, compositing fwd (fp32) + bwd "
-                        f"(fp64) on every {tile_stride}th tile ({tiles.size} of {cam.num_tiles}), "
-                        f"{dt:.2f} s"), seconds=dt, evals=evals)
+    t2 = time.perf_counter()
+    ev_f = int(r["n_eval"].astype(np.int64).sum())
+    ev_b = int(r["n_contrib"].astype(np.int64).sum())
+    sample = (f"full preprocess + binning of the {sc.name} scene, compositing fwd (fp32) + bwd (fp64) on every "
+              f"{tile_stride}th tile ({tiles.size} of {cam.num_tiles})" if tile_stride > 1 else
+              f"the whole {sc.name} frame: preprocess, binning, compositing fwd (fp32) + bwd (fp64), "
+              f"preprocess bwd (fp64)")
+    return dict(evals=ev_f + ev_b, evals_fwd=ev_f, evals_bwd=ev_b, seconds=t2 - t0, fwd_s=t1 - t0, bwd_s=t2 - t1,
+                cores=oracle.num_threads(), sample=sample)
+
+
+def cpu_baseline(sc, cfg: int, min_seconds: float = 10.0, single_thread_cfgs=(1, 2, 3)):
+    """The oracle on the host cores: the bounded sample of ``cpu_oracle_sample``
+    repeated until about ``min_seconds`` of host work, forward and backward
+    reported separately; plus one-thread numbers for the small configs."""
+    import oracle
+    tot = dict(evals=0, evals_fwd=0, evals_bwd=0, seconds=0.0, fwd_s=0.0, bwd_s=0.0)
+    reps = 0
+    while tot["seconds"] < min_seconds and reps < 50:
+        c = cpu_oracle_sample(sc, cpu_tile_stride(cfg))
+        for k in tot:
+            tot[k] += c[k]
+        reps += 1
+    out = dict(value=tot["evals"] / tot["seconds"], unit=UNIT, cores=c["cores"], kind="oracle",
+               sample=f"{reps} x ({c['sample']}); {tot['seconds']:.1f} s in total",
+               fwd=dict(value=tot["evals_fwd"] / tot["fwd_s"], unit=UNIT, ms_per_sample=1e3 * tot["fwd_s"] / reps),
+               bwd=dict(value=tot["evals_bwd"] / tot["bwd_s"], unit=UNIT, ms_per_sample=1e3 * tot["bwd_s"] / reps))
+    n0 = oracle.num_threads()
+    st = {}
+    try:
+        oracle.set_threads(1)
+        for k in single_thread_cfgs:
+            c = cpu_oracle_sample(_scene(k), cpu_tile_stride(k))
+            st[f"config{k}"] = dict(value=c["evals"] / c["seconds"], fwd_evals_per_s=c["evals_fwd"] / c["fwd_s"],
+                                    bwd_evals_per_s=c["evals_bwd"] / c["bwd_s"], fwd_ms=1e3 * c["fwd_s"],
+                                    bwd_ms=1e3 * c["bwd_s"], unit=UNIT, cores=1, sample=c["sample"])
+    finally:
+        oracle.set_threads(n0)
+    out["single_thread"] = st
+    return out
 
 
 def run_reference(args):
@@ -172,23 +217,23 @@ def run_reference(args):
     if rank != 0:
         return 0
     sc = _scene(args.config)
-    stride = 16 if args.config >= 4 else 1
+    stride = cpu_tile_stride(args.config)
     import oracle
     for _ in range(args.warmup):
         cpu_oracle_sample(sc, stride * 4)
-    vals, secs = [], []
-    for _ in range(args.steps):
-        r = cpu_oracle_sample(sc, stride)
-        vals.append(r["evals"])
-        secs.append(r["seconds"])
-    value = sum(vals) / sum(secs)
+    recs = [cpu_oracle_sample(sc, stride) for _ in range(args.steps)]
+    secs = sum(r["seconds"] for r in recs)
+    value = sum(r["evals"] for r in recs) / secs
+    fwd = sum(r["evals_fwd"] for r in recs) / sum(r["fwd_s"] for r in recs)
+    bwd = sum(r["evals_bwd"] for r in recs) / sum(r["bwd_s"] for r in recs)
     line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=ws, steps=args.steps, warmup=args.warmup,
-                ms_per_step=1e3 * sum(secs) / len(secs), higher_is_better=True, scaling="weak", vs_baseline=None,
+                ms_per_step=1e3 * secs / len(recs), higher_is_better=True, scaling="weak", vs_baseline=None,
                 dtype="f32 fwd / f64 bwd", data="synthetic", impl="reference",
                 config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {sc.cameras[0].width}x{sc.cameras[0].height},"
                                      " 16x16 tiles (bounded tile sample per step)"),
                 cpu_baseline=dict(kind="oracle", cores=oracle.num_threads(), value=value, unit=UNIT,
-                                  sample=r["sample"]),
+                                  sample=recs[-1]["sample"], fwd=dict(value=fwd, unit=UNIT),
+                                  bwd=dict(value=bwd, unit=UNIT)),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
     return 0
@@ -212,14 +257,23 @@ def run_ours(args):
     B.lib()
 
     sc = _scene(args.config)
-    cams = sc.cameras
-    # several views: split them over the ranks and sum the 3D gradients
-    # (camera-parallel); one view: every rank renders it (replicas)
-    multi = len(cams) > 1
-    mine = MV.assign_cameras(len(cams), world, rank) if multi else [0]
+    # Work of this rank.  Several views, or --split image: the fixed
+    # workload is cut into (camera, band) units spread over the ranks
+    # (multiview.assign_work: whole cameras when the ranks divide them,
+    # tile-row bands otherwise) and the 3D gradients are summed with one
+    # all-reduce.  One view without --split: every rank renders the whole
+    # frame (replicas, no collective).
+    split = len(sc.cameras) > 1 or args.split == "image"
+    if split:
+        units = MV.assign_work(sc.cameras, world, rank)
+    else:
+        units = [MV.WorkUnit(0, 0, sc.cameras[0].height, True)]
+    cams = [MV.unit_view(sc.cameras, u) for u in units]
+    mine = list(range(len(units)))
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
     means, scales, quats, opacity, colors = (t(x) for x in (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors))
-    dLs = {i: t(sc.dL_dimage[i]) for i in mine}
+    dl_rows = [np.ascontiguousarray(sc.dL_dimage[u.camera][:, u.y0:u.y1]) for u in units]
+    dLs = {i: t(dl_rows[i]) for i in mine}
     rzs = {i: RZ.Rasterizer(cams[i], dev) for i in mine}
     caps = {}
     for i in mine:
@@ -238,7 +292,7 @@ def run_ours(args):
         if args.sh_f16:
             shd = shd.half()  # binary16 storage, fp32 arithmetic (gs_sh_*_f16)
         colors = torch.empty((sc.N, 3), dtype=torch.float32, device=dev)
-    exchange = multi and world > 1
+    exchange = split and world > 1
     adam = None
     if args.adam:
         # the optimiser stage: raw parameters (log scales, logit opacity) whose
@@ -308,6 +362,14 @@ def run_ours(args):
             raise RuntimeError(f"device status {st}: {B.status_string(st)}")
     # work counts of this rank's views (outside the timed region)
     n_contrib = n_evaluated = n_blended = P = Ps = 0
+    visited_fwd = visited_bwd = 0  # list entries a tile's walk reads: sum over tiles of the furthest pixel
+
+    def visited(counts, cam):
+        TX, TY = (cam.width + 15) // 16, (cam.height + 15) // 16
+        full = torch.zeros((TY * 16, TX * 16), dtype=torch.int64, device=dev)
+        full[:cam.height, :cam.width] = counts.view(torch.int32).to(torch.int64)
+        return int(full.view(TY, 16, TX, 16).amax(dim=(1, 3)).sum().item())
+
     for i in mine:
         b, cam = rzs[i]._bufs, cams[i]
         rc = b["rect"].to(torch.int64)
@@ -320,6 +382,8 @@ def run_ours(args):
         n_contrib += int(b["n_contrib"].view(torch.int32).to(torch.int64).sum().item())
         n_evaluated += int(ne.view(torch.int32).to(torch.int64).sum().item())
         n_blended += int(nb.view(torch.int32).to(torch.int64).sum().item())
+        visited_fwd += visited(ne, cam)
+        visited_bwd += visited(b["n_contrib"], cam)
         P += caps[i]
     evals_per_step = n_evaluated + n_contrib
 
@@ -392,37 +456,47 @@ def run_ours(args):
 
     # roofline of the dominant kernel (render backward: FP32 issue bound)
     peaks = _peaks()
-    # per-step time of each stage, summed over this rank's views
+    # per-step time of each stage, summed over this rank's views (a rank
+    # without a view has only the exchange; its stage times are 0)
     mean = {s: statistics.mean(v) * len(v) / args.steps for s, v in stage_ms.items()}
+    for s_ in ("preprocess_fwd", "bin_sort", "render_fwd", "render_bwd", "preprocess_bwd"):
+        mean.setdefault(s_, 0.0)
     dominant = max(mean, key=mean.get)
+    nv = max(len(mine), 1)
     bwd_ops = n_blended * OPS_BWD_EVAL
     fwd_ops = n_blended * OPS_FWD_EVAL
     alu_peak = SMS * FP32_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12  # T lane-ops/s
-    rb_ach = bwd_ops / (mean["render_bwd"] / 1e3) / 1e12
+    per_s = lambda x, ms: x / (ms / 1e3) if ms > 0 else 0.0
+    rb_ach = per_s(bwd_ops, mean["render_bwd"]) / 1e12
     rec_t = RECORDED_TRAFFIC["k_render_bwd"]
     traffic = rec_t["bytes"] if (rec_t["sources_sha1"] == _render_sources_sha1() and len(mine) == 1) else None
     roofline = dict(kernel="k_render_bwd_warp", bound="alu", achieved=rb_ach, peak=alu_peak, unit="Tops/s",
-                    frac=rb_ach / alu_peak, traffic=traffic, ops_per_launch=bwd_ops // len(mine),
+                    frac=rb_ach / alu_peak, traffic=traffic, ops_per_launch=bwd_ops // nv,
                     ops_basis=f"{OPS_BWD_EVAL} FP32 ops x {n_blended} blended terms",
                     peak_src=f"148 SMs x 128 FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz (sm_max_mhz)")
-    # HBM view of render fwd + bwd, as asked
+    # HBM view of render fwd + bwd, as asked, per VISITED pair: the list
+    # entries up to each tile's furthest evaluated (forward) or contributing
+    # (backward) position; entries beyond are never read
     pix = sum(cams[i].width * cams[i].height for i in mine)
-    fwd_bytes = P * BYTES_PAIR_READ + pix * BYTES_PIXEL
-    bwd_bytes = P * (BYTES_PAIR_READ + BYTES_PAIR_ATOMIC) + pix * BYTES_PIXEL
-    rfb_s = (mean["render_fwd"] + mean["render_bwd"]) / 1e3
+    fwd_bytes = visited_fwd * BYTES_PAIR_READ + pix * BYTES_PIXEL
+    bwd_bytes = visited_bwd * (BYTES_PAIR_READ + BYTES_PAIR_ATOMIC) + pix * BYTES_PIXEL
+    rfb_s = max((mean["render_fwd"] + mean["render_bwd"]) / 1e3, 1e-30)
     render_hbm = dict(achieved_gbs=(fwd_bytes + bwd_bytes) / rfb_s / 1e9, peak_gbs=peaks["hbm_gbs"],
                       frac=(fwd_bytes + bwd_bytes) / rfb_s / 1e9 / peaks["hbm_gbs"],
-                      bytes_per_frame=fwd_bytes + bwd_bytes, peak_src=peaks["src"])
-    fwd_alu = fwd_ops / (mean["render_fwd"] / 1e3) / 1e12
+                      bytes_per_frame=fwd_bytes + bwd_bytes, peak_src=peaks["src"],
+                      visited_pairs_fwd=visited_fwd, visited_pairs_bwd=visited_bwd,
+                      basis=f"{BYTES_PAIR_READ} B per visited pair read by each pass, {BYTES_PAIR_ATOMIC} B of "
+                            f"gradient atomics per pair visited by the backward, {BYTES_PIXEL} B per pixel per pass")
+    fwd_alu = per_s(fwd_ops, mean["render_fwd"]) / 1e12
     # the metric's "bwd HBM GB/s": the render backward alone, algorithmic
     # bytes and, where the committed capture applies, measured DRAM bytes
-    rb_s = mean["render_bwd"] / 1e3
+    rb_s = max(mean["render_bwd"] / 1e3, 1e-30)
     bwd_hbm = dict(achieved_gbs=bwd_bytes / rb_s / 1e9, peak_gbs=peaks["hbm_gbs"],
                    frac=bwd_bytes / rb_s / 1e9 / peaks["hbm_gbs"], bytes_per_frame=bwd_bytes,
                    dram_gbs=(traffic / (rb_s / len(mine)) / 1e9) if traffic else None, peak_src=peaks["src"])
     # HBM view of the binning (the sort is the stage an HBM roofline fits)
     bin_bytes = len(mine) * sc.N * BIN_BYTES_GAUSSIAN + Ps * BIN_BYTES_CELL_PAIR + P * BIN_BYTES_PAIR
-    bin_gbs = bin_bytes / (mean["bin_sort"] / 1e3) / 1e9
+    bin_gbs = per_s(bin_bytes, mean["bin_sort"]) / 1e9
     bin_hbm = dict(achieved_gbs=bin_gbs, peak_gbs=peaks["hbm_gbs"], frac=bin_gbs / peaks["hbm_gbs"],
                    bytes_per_step=bin_bytes, cell_pairs=Ps, peak_src=peaks["src"],
                    basis=f"{BIN_BYTES_GAUSSIAN} B/Gaussian + {BIN_BYTES_CELL_PAIR} B/cell pair + "
@@ -437,13 +511,13 @@ def run_ours(args):
         host_params = {k: torch.from_numpy(np.ascontiguousarray(x)).pin_memory()
                        for k, x in zip(("means", "scales", "quats", "opacity", "colors"),
                                        (sc.means, sc.scales, sc.quats, sc.opacity, sc.colors))}
-        host_dl = [torch.from_numpy(np.ascontiguousarray(sc.dL_dimage[i])).pin_memory() for i in mine]
+        host_dl = [torch.from_numpy(dl_rows[i]).pin_memory() for i in mine]
         h2d = sum(x.numel() * x.element_size() for x in list(host_params.values()) + host_dl)
         rz_e2e, e2e_state = {}, {}
         host_out = {k: torch.empty(grads[k].shape, dtype=grads[k].dtype, pin_memory=True) for k in MV.GRAD_KEYS}
         def e2e_step():
             MV.render_views_from_host([cams[i] for i in mine], host_params, host_dl, rz_e2e,
-                                      [caps[i] for i in mine], camera_ids=mine, state=e2e_state,
+                                      [caps[i] for i in mine], camera_ids=units, state=e2e_state,
                                       host_grads=host_out, reduce_fn=MV.allreduce_grads if exchange else None,
                                       device=dev, pipelined=True)
 
@@ -472,34 +546,30 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        # repeat the bounded sample until about 10 s of host work has been timed
-        stride = 4 if args.config >= 4 else 1
-        tot_s, tot_e, reps = 0.0, 0, 0
-        while tot_s < 10.0 and reps < 50:
-            c = cpu_oracle_sample(sc, tile_stride=stride)
-            tot_s += c["seconds"]
-            tot_e += c["evals"]
-            reps += 1
-        cpu = dict(value=tot_e / tot_s, unit=UNIT, cores=c["cores"], kind="oracle",
-                   sample=f"{reps} x ({c['sample']}); {tot_s:.1f} s in total")
+        cpu = cpu_baseline(sc, args.config)
 
     if rank == 0:
-        cam0 = cams[0]
-        par = (f"camera-parallel x{world}" if exchange else (f"replicas x{world}" if world > 1 else "1 GPU"))
+        cam0 = sc.cameras[0]
+        if exchange:
+            par = (f"image-space split x{world} (tile-row bands)" if len(sc.cameras) == 1 else
+                   f"camera-parallel x{world} ((camera, band) units)")
+        else:
+            par = f"replicas x{world}" if world > 1 else "1 GPU"
         line = dict(
             metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
             ms_per_step=total_ms / args.steps, ms_per_step_eager=eager_ms / args.steps,
             launch_mode="cuda graph replay" if graph is not None else "eager", higher_is_better=True, scaling="weak" if not exchange else "strong",
             vs_baseline=None, dtype="f32", data="synthetic",
-            config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam0.width}x{cam0.height}, {len(cams)} view(s), "
+            config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam0.width}x{cam0.height}, {len(sc.cameras)} view(s), "
                                  f"16x16 tiles, fp32"
                                  + (f", SH degree {sh_deg} colours" if sh_deg is not None else "")
                                  + (" (binary16 coefficient storage)" if sh_deg is not None and args.sh_f16 else ""),
-                        views_per_rank=len(mine), num_pairs=P, evals_per_step=evals_per_step,
+                        views_per_rank=len(mine), units_rank0=[(u.camera, u.y0, u.y1) for u in units],
+                        num_pairs=P, evals_per_step=evals_per_step,
                         evaluated_fwd=n_evaluated, contributor_prefix_bwd=n_contrib, blended=n_blended,
                         l2="flushed between steps (256 MiB write)", parallelism=par),
-            fwd_ms_per_frame=(mean["preprocess_fwd"] + mean["bin_sort"] + mean["render_fwd"]) / len(mine),
-            bwd_ms_per_frame=(mean["render_bwd"] + mean["preprocess_bwd"]) / len(mine),
+            fwd_ms_per_frame=(mean["preprocess_fwd"] + mean["bin_sort"] + mean["render_fwd"]) / nv,
+            bwd_ms_per_frame=(mean["render_bwd"] + mean["preprocess_bwd"]) / nv,
             stage_ms={s: round(v, 4) for s, v in mean.items()}, dominant_stage=dominant,
             roofline=roofline, render_fwd_alu=dict(achieved=fwd_alu, peak=alu_peak, unit="Tops/s",
                                                    frac=fwd_alu / alu_peak),
@@ -519,6 +589,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--split", choices=["replica", "image"], default="replica",
+                    help="one-view configs under torchrun: 'replica' (default) renders the whole frame on every "
+                         "rank; 'image' cuts the frame into tile-row bands, one per rank, and sums the 3D "
+                         "gradients with one all-reduce (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches only (default: the step is also captured in a CUDA graph and the "

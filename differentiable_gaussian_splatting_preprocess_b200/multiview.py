@@ -8,6 +8,8 @@ host logic is the same for any backend.
 """
 from __future__ import annotations
 
+import dataclasses
+import math
 from typing import Callable, Dict, List, Optional, Sequence
 
 import torch
@@ -18,33 +20,44 @@ from . import rasterizer as RZ
 GRAD_KEYS = ("dL_dmeans", "dL_dscales", "dL_dquats", "dL_dopacity", "dL_dcolors")
 
 
-def band_rows(cam, parts: int, tile: int = 16) -> List[tuple]:
-    """Pixel row ranges [y0, y1) of ``parts`` horizontal bands of whole tile
-    rows (ceil(rows / parts) tile rows each, the last band the remainder;
-    empty bands, when the image has fewer tile rows than parts, are omitted)."""
+def _band_bounds(tile_rows: int, parts: int) -> List[int]:
+    """parts + 1 tile-row boundaries: band k holds tile rows
+    [ceil(k rows / parts), ceil((k + 1) rows / parts)), so band sizes differ
+    by at most one tile row (when rows < parts, the last bands are empty)."""
     if parts < 1:
         raise ValueError("parts must be >= 1")
+    return [(k * tile_rows + parts - 1) // parts for k in range(parts + 1)]
+
+
+def band_rows(cam, parts: int, tile: int = 16) -> List[tuple]:
+    """Pixel row ranges [y0, y1) of ``parts`` horizontal bands of whole tile
+    rows, as equal as whole tile rows allow; empty bands (when the image has
+    fewer tile rows than parts) are omitted."""
     rows = (cam.height + tile - 1) // tile
-    per = (rows + parts - 1) // parts
-    out = []
-    for b in range(parts):
-        r0, r1 = b * per, min(rows, (b + 1) * per)
-        if r0 < r1:
-            out.append((r0 * tile, min(cam.height, r1 * tile)))
-    return out
+    b = _band_bounds(rows, parts)
+    return [(b[k] * tile, min(cam.height, b[k + 1] * tile)) for k in range(parts) if b[k] < b[k + 1]]
+
+
+def band_view(cam, y0: int, y1: int):
+    """The camera restricted to pixel rows [y0, y1): same camera with its
+    principal point moved up by y0, so every pixel keeps its position
+    relative to the Gaussians.  y0 must be a multiple of the tile size, so
+    that the band's tile rows coincide with the full frame's."""
+    return cam.replace(height=y1 - y0, cy=cam.cy - y0)
 
 
 def split_image(cam, parts: int, tile: int = 16) -> List:
     """Image-space split of one camera into the bands of band_rows.
 
-    A band is the same camera with its principal point moved up by the
-    band's first pixel row: every pixel keeps its position relative to the
-    Gaussians, and tile rows coincide with the full frame's.  Because the
-    preprocess backward is linear in the 2D gradients, the 3D gradients of
-    the bands, summed, are those of the full frame: the band renders can run
-    on different ranks and meet in the same single all-reduce as the
-    camera-parallel split."""
-    return [cam.replace(height=y1 - y0, cy=cam.cy - y0) for y0, y1 in band_rows(cam, parts, tile)]
+    The preprocess backward is linear in the 2D gradients, so the 3D
+    gradients of the bands, summed, equal those of the full frame up to fp32
+    rounding (each band projects the means with its own principal point, so
+    the pixel offsets round differently): the band renders can run on
+    different ranks and meet in the same single all-reduce as the
+    camera-parallel split.  The densification statistics are not linear in
+    the 2D gradients (a norm per view), so they must not be summed over
+    bands: compute them from whole views only."""
+    return [band_view(cam, y0, y1) for y0, y1 in band_rows(cam, parts, tile)]
 
 
 def assign_cameras(n_cameras: int, world: int, rank: int) -> List[int]:
@@ -53,6 +66,57 @@ def assign_cameras(n_cameras: int, world: int, rank: int) -> List[int]:
     if world < 1 or not 0 <= rank < world:
         raise ValueError("bad rank / world size")
     return [i for i in range(n_cameras) if i % world == rank]
+
+
+@dataclasses.dataclass(frozen=True)
+class WorkUnit:
+    """Rows [y0, y1) of camera ``camera``: one rank's share of a step."""
+    camera: int
+    y0: int
+    y1: int
+    whole: bool  # the unit is the camera's whole frame
+
+
+def assign_work(cams: Sequence, world: int, rank: int, tile: int = 16) -> List[WorkUnit]:
+    """The (camera, band) work units of one rank, for any number of ranks.
+
+    Each camera is cut into b = world / gcd(n_cameras, world) bands of whole
+    tile rows (_band_bounds), which makes n_cameras * b units, a multiple of
+    the number of ranks; rank r takes the contiguous run of U = n_cameras * b
+    / world units starting at r U, and neighbouring bands of one camera in
+    that run are merged into one taller band.  So every pixel row of every
+    camera belongs to exactly one rank, every rank gets the same number of
+    units, a rank splits a camera only where the ranks outnumber or do not
+    divide the cameras, and with world dividing n_cameras it is whole cameras
+    per rank.  Empty bands (fewer tile rows than bands) are dropped, so a
+    rank of a small image may get no unit: it then contributes zeros to the
+    gradient sum."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("bad rank / world size")
+    n = len(cams)
+    if n == 0:
+        return []
+    b = world // math.gcd(n, world)
+    per = n * b // world
+    first, last = rank * per, (rank + 1) * per  # unit u = camera u // b, band u % b
+    out = []
+    u = first
+    while u < last:
+        c, k0 = divmod(u, b)
+        k1 = min(b, k0 + (last - u))  # bands k0 .. k1 - 1 of camera c
+        rows = (cams[c].height + tile - 1) // tile
+        bd = _band_bounds(rows, b)
+        y0, y1 = bd[k0] * tile, min(cams[c].height, bd[k1] * tile)
+        if y0 < y1:
+            out.append(WorkUnit(c, y0, y1, y0 == 0 and y1 == cams[c].height))
+        u += k1 - k0
+    return out
+
+
+def unit_view(cams: Sequence, unit: WorkUnit):
+    """The camera a work unit renders (its band of the unit's camera)."""
+    cam = cams[unit.camera]
+    return cam if unit.whole else band_view(cam, unit.y0, unit.y1)
 
 
 def render_views(cams: Sequence, params: Dict[str, torch.Tensor], dL_dimages: Sequence[torch.Tensor],
@@ -209,16 +273,26 @@ def allreduce_grads(grads: Dict[str, torch.Tensor], group=None, keys: Sequence[s
 def render_views_distributed(cams: Sequence, params: Dict[str, torch.Tensor],
                              dL_dimages: Sequence[torch.Tensor], group=None,
                              render_fn: Callable = render_views, **kw) -> Dict[str, torch.Tensor]:
-    """Each rank renders its share of the cameras (assign_cameras), then the
-    3D gradients are summed over ranks: every rank ends with the gradient of
-    the sum of all views' losses."""
+    """Each rank renders its work units (assign_work: whole cameras, or bands
+    of cameras when the ranks outnumber or do not divide the cameras), then
+    the 3D gradients are summed over ranks: every rank ends with the gradient
+    of the sum of all views' losses.  A rank without a unit contributes
+    zeros.  ``render_fn`` receives the units' cameras, their rows of the
+    upstream gradients and ``camera_ids`` = the units (hashable keys for a
+    rasterizer cache)."""
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     rank = dist.get_rank(group) if dist.is_initialized() else 0
-    mine = assign_cameras(len(cams), world, rank)
+    units = assign_work(cams, world, rank)
+    if kw.get("densify") is not None and not all(u.whole for u in units):
+        raise ValueError("densification statistics are not additive over image bands")
     grads = kw.pop("grads", None)
     if grads is None:
         grads = RZ.zero_grads(params["means"].shape[0], params["means"].device)
-    render_fn([cams[i] for i in mine], params, [dL_dimages[i] for i in mine], grads=grads, camera_ids=mine, **kw)
+    if units:
+        views = [unit_view(cams, u) for u in units]
+        dls = [dL_dimages[u.camera] if (u.whole or dL_dimages[u.camera] is None)
+               else dL_dimages[u.camera][:, u.y0:u.y1].contiguous() for u in units]
+        render_fn(views, params, dls, grads=grads, camera_ids=units, **kw)
     if world > 1:
         allreduce_grads(grads, group)
     return grads

@@ -156,20 +156,36 @@ def zero_grads(N: int, device) -> Dict[str, torch.Tensor]:
 
 class GraphedStep:
     """Forward + backward of one camera recorded once into a CUDA graph and
-    replayed: one launch per step instead of one per kernel.  The inputs are
-    the tensors given here, read in place at every replay (update them with
-    ``copy_`` between replays); the step runs in capacity mode, so the pair
-    count of every replayed frame must fit ``capacity`` (check ``status()``:
-    GS_ERR_CAPACITY otherwise).  ``grads`` (allocated when None) is zeroed and
-    refilled by every replay; ``frame`` holds the forward's outputs."""
+    replayed: one launch per step instead of one per kernel.
 
-    def __init__(self, rz: Rasterizer, means, scales, quats, opacity, colors, dL_dimage, capacity: int,
+    The inputs are the tensors given here, read in place at every replay
+    (update them with ``copy_`` between replays); the step runs in capacity
+    mode, so the pair count of every replayed frame must fit ``capacity``.
+    ``grads`` (allocated when None) is zeroed and refilled by every replay;
+    ``frame`` holds the forward's outputs.
+
+    The graph records device addresses, so the step owns the buffers they
+    belong to: it builds its own Rasterizer (from ``cam``, or from the
+    camera of a Rasterizer passed instead), whose workspace, pair buffers,
+    frame and 2D gradient buffers live as long as the step and are used by
+    nothing else.  A Rasterizer passed in is not used and stays free for
+    eager calls.  Each replay begins by clearing the workspace's status
+    word, so ``status()`` reports the most recent replay (GS_ERR_CAPACITY
+    when its pair count did not fit)."""
+
+    def __init__(self, cam, means, scales, quats, opacity, colors, dL_dimage, capacity: int,
                  grads: Optional[Dict[str, torch.Tensor]] = None, use_mask: bool = True):
-        self.rz = rz
-        self.grads = zero_grads(means.shape[0], rz.device) if grads is None else grads
+        if isinstance(cam, Rasterizer):
+            cam, device = cam.cam, cam.device
+        else:
+            device = means.device
+        rz = self.rz = Rasterizer(cam, device)
+        self.grads = zero_grads(means.shape[0], device) if grads is None else grads
         args = (means, scales, quats, opacity, colors)
 
         def step():
+            if rz.ws is not None:
+                B.gs_clear_status(rz.ws)
             for v in self.grads.values():
                 v.zero_()
             fr = rz.forward(*args, capacity=capacity, use_mask=use_mask)
@@ -177,14 +193,18 @@ class GraphedStep:
             return fr
 
         step()  # allocates every buffer and makes every one-time setup call outside the capture
-        torch.cuda.synchronize(rz.device)
+        torch.cuda.synchronize(device)
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
             self.frame = step()
+        # the tensors whose addresses the graph holds
+        self.ws = rz.ws
+        self._held = (rz.ws, dict(rz._bufs), args, dL_dimage, self.grads)
 
     def replay(self) -> Dict[str, torch.Tensor]:
         self.graph.replay()
         return self.grads
 
     def status(self) -> int:
-        return self.rz.status()
+        """Status word of the workspace the graph uses (synchronises)."""
+        return B.gs_read_status(self.ws)

@@ -22,17 +22,31 @@ def _free_port():
     return port
 
 
+def _row_weight(c, y0, y1):
+    """Fake gradient of rows [y0, y1) of camera c: sum of (c + 1)(y + 1)."""
+    return float((c + 1) * ((y1 * (y1 + 1) - y0 * (y0 + 1)) // 2))
+
+
 def _fake_render(cams, params, dls, grads=None, camera_ids=None, **kw):
-    """Stands in for the per-camera kernels: camera c adds (c + 1) * ones to
-    every gradient and records that it ran."""
-    for cid in camera_ids:
+    """Stands in for the per-view kernels: the unit's rows of camera c add
+    _row_weight to every gradient, and the unit is recorded."""
+    for view, u in zip(cams, camera_ids):
+        assert view.height == u.y1 - u.y0 and view.cy == CAM_H / 2.0 - u.y0
         for k in MV.GRAD_KEYS:
-            grads[k] += float(cid + 1)
-        grads["_seen"].append(cid)
+            grads[k] += _row_weight(u.camera, u.y0, u.y1)
+        grads["_seen"].append((u.camera, u.y0, u.y1))
     return grads
 
 
-def _worker(rank, world, port, n_cams, N, out_q, fail_rank):
+CAM_H = 1080
+
+
+def _cams(n_cams, height=CAM_H):
+    from differentiable_gaussian_splatting_preprocess_b200 import scenes
+    return [scenes.Camera(1920, height, 1600.0, 1600.0, 960.0, CAM_H / 2.0) for _ in range(n_cams)]
+
+
+def _worker(rank, world, port, n_cams, N, out_q, fail_rank, height=CAM_H):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
@@ -44,7 +58,7 @@ def _worker(rank, world, port, n_cams, N, out_q, fail_rank):
                                                    ("dL_dquats", (N, 4)), ("dL_dopacity", (N,)),
                                                    ("dL_dcolors", (N, 3)))}
         grads["_seen"] = []
-        MV.render_views_distributed(list(range(n_cams)), params, [None] * n_cams, render_fn=_fake_render,
+        MV.render_views_distributed(_cams(n_cams, height), params, [None] * n_cams, render_fn=_fake_render,
                                     grads=grads)
         # numpy copies: torch tensors would travel by file-descriptor sharing,
         # which needs this process alive when the parent unpickles them
@@ -58,11 +72,12 @@ def _worker(rank, world, port, n_cams, N, out_q, fail_rank):
             pass
 
 
-def _run(world, n_cams, N, fail_rank=-1):
+def _run(world, n_cams, N, fail_rank=-1, height=CAM_H):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, n_cams, N, q, fail_rank)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, n_cams, N, q, fail_rank, height))
+             for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=120) for _ in range(world)]
@@ -92,16 +107,56 @@ def test_flat_roundtrip():
         assert torch.equal(g[k], h[k])
 
 
-@pytest.mark.parametrize("n_cams", [4, 3])
-def test_two_ranks_sum_every_camera_once(n_cams):
-    res = _run(2, n_cams, 7)
+@pytest.mark.parametrize("world,n_cams", [(2, 4), (2, 3), (3, 4), (8, 4), (3, 1)])
+def test_ranks_render_every_row_once_and_sum(world, n_cams):
+    """Every pixel row of every camera is rendered by exactly one rank (whole
+    cameras, or bands when the ranks outnumber or do not divide the
+    cameras), and after the all-reduce every rank holds the full sum."""
+    res = _run(world, n_cams, 7)
     assert all(r[1] == "ok" for r in res), res
-    seen = sorted(c for r in res for c in r[2])
-    assert seen == list(range(n_cams))
-    total = float(sum(c + 1 for c in range(n_cams)))
+    covered = {c: [] for c in range(n_cams)}
+    for r in res:
+        assert r[2], "every rank has work"
+        for c, y0, y1 in r[2]:
+            covered[c].append((y0, y1))
+    for c, spans in covered.items():
+        spans.sort()
+        assert spans[0][0] == 0 and spans[-1][1] == CAM_H
+        assert all(a[1] == b[0] for a, b in zip(spans, spans[1:])), spans
+        assert all(y0 % 16 == 0 for y0, _ in spans)
+    total = sum(_row_weight(c, 0, CAM_H) for c in range(n_cams))
     for r in res:
         for k, v in r[3].items():
             assert (v == total).all(), k
+
+
+def test_rank_without_work_contributes_zeros():
+    """One tile row and two ranks: the second rank gets no band, renders
+    nothing and still joins the all-reduce."""
+    res = _run(2, 1, 5, height=16)
+    assert all(r[1] == "ok" for r in res), res
+    assert res[0][2] == [(0, 0, 16)] and res[1][2] == []
+    for r in res:
+        for v in r[3].values():
+            assert (v == _row_weight(0, 0, 16)).all()
+
+
+def test_assign_work_partition():
+    """The unit assignment alone, for many world sizes: a partition of every
+    camera's rows into tile-aligned spans, equal unit counts per rank."""
+    for n_cams in (1, 2, 3, 4, 5):
+        cams = _cams(n_cams)
+        for world in range(1, 17):
+            spans = {c: [] for c in range(n_cams)}
+            for r in range(world):
+                for u in MV.assign_work(cams, world, r):
+                    spans[u.camera].append((u.y0, u.y1))
+                    assert u.whole == (u.y0 == 0 and u.y1 == CAM_H)
+            for c, sp in spans.items():
+                sp.sort()
+                assert sp[0][0] == 0 and sp[-1][1] == CAM_H and all(a[1] == b[0] for a, b in zip(sp, sp[1:]))
+    with pytest.raises(ValueError):
+        MV.assign_work(_cams(2), 2, 2)
 
 
 def test_failed_rank_is_reported_not_hung():
