@@ -66,6 +66,25 @@ __device__ __forceinline__ PixelPair pixel_pair(const gs_camera& cam, int TX) {
     return q;
 }
 
+// The pixel pair of this lane in quadrant `quad` (0..3: 8x8 quarters of the
+// tile, row-major) of tile `tile`.
+__device__ __forceinline__ PixelPair quad_pixel_pair(const gs_camera& cam, int TX, int tile, int quad, int lane) {
+    PixelPair q;
+    const int bx = (tile % TX) * kTile + (quad & 1) * 8;
+    const int by = (tile / TX) * kTile + (quad >> 1) * 8;
+    q.x0 = bx + 2 * (lane & 3);
+    q.y = by + (lane >> 2);
+    q.in0 = q.x0 < cam.width && q.y < cam.height;
+    q.in1 = q.x0 + 1 < cam.width && q.y < cam.height;
+    q.px = make_float2((float)q.x0 + 0.5f, (float)q.x0 + 1.5f);
+    q.py = (float)q.y + 0.5f;
+    q.sx0 = (float)bx + 0.5f;
+    q.sx1 = q.sx0 + 7.0f;
+    q.sy0 = (float)by + 0.5f;
+    q.sy1 = q.sy0 + 7.0f;
+    return q;
+}
+
 // Can the staged Gaussian reach alpha >= alpha_min in this warp's quadrant?
 __device__ __forceinline__ bool may_contribute(float4 box, float thr, float2 xy, float4 co, const PixelPair& q) {
     if (box_misses(box, q.sx0, q.sx1, q.sy0, q.sy1)) return false;
@@ -214,10 +233,15 @@ __device__ __forceinline__ float reduce8(float v[8], int lane) {
 // One term of the reverse traversal for this thread's two pixels: undo the
 // term's transmittance step, accumulate the colour behind it, and produce the
 // pixel pair's share of the 9 gradient values (dL/du, dL/dv, dL/da, dL/db,
-// dL/dc, dL/dr, dL/dg, dL/dopacity; dL/db_colour in r9).  Returns false, with
-// nothing changed, when no pixel of the warp takes the term (a warp vote).
-// p is the term's position in the tile's list; last0/last1 the pixels'
-// contributor counts; terms the forward did not blend contribute nothing.
+// dL/dc, dL/dr, dL/dg, dL/dopacity; dL/db_colour in r9).  p is the term's
+// position in the tile's list; last0/last1 the pixels' contributor counts;
+// terms the forward did not blend contribute nothing.  With kVote, returns
+// false, with nothing changed, when no pixel of the warp takes the term (a
+// warp vote; callers that only visit terms the forward blended in this warp
+// skip it).  With kFold, dL/da, dL/db and dL/dc are left without their
+// constant factors -1/2, -1 and -1/2 (exact powers of two, applied once after
+// the warp sum).
+template <bool kVote, bool kFold>
 __device__ __forceinline__ bool bwd_term(const PixelPair& q, float2 xy, float4 co, float4 c, int p, unsigned last0,
                                          unsigned last1, float amax, float amin, float2 g0, float2 g1, float2 g2,
                                          float2& T, float2& S0, float2& S1, float2& S2, float (&v)[8], float& r9) {
@@ -225,7 +249,7 @@ __device__ __forceinline__ bool bwd_term(const PixelPair& q, float2 xy, float4 c
     eval_pair(q.px, q.py, xy, co, amax, amin, e);
     const bool c0 = p < (int)last0 && e.ok0;
     const bool c1 = p < (int)last1 && e.ok1;
-    if (!__any_sync(0xffffffffu, c0 || c1)) return false;
+    if (kVote && !__any_sync(0xffffffffu, c0 || c1)) return false;
     const float2 G = make_float2(c0 ? e.G.x : 0.0f, c1 ? e.G.y : 0.0f);
     const float2 al = make_float2(c0 ? e.alpha.x : 0.0f, c1 ? e.alpha.y : 0.0f);
     if (c0) T.x = __fdividef(T.x, 1.0f - al.x);
@@ -254,11 +278,11 @@ __device__ __forceinline__ bool bwd_term(const PixelPair& q, float2 xy, float4 c
     t2 = __ffma2_rn(make_float2(co.y, co.y), hdx, __fmul2_rn(make_float2(co.z, co.z), hdy));
     v[1] = t2.x + t2.y;  // dL/dv
     t2 = __fmul2_rn(hdx, e.dx);
-    v[2] = -0.5f * (t2.x + t2.y);  // dL/da
+    v[2] = kFold ? t2.x + t2.y : -0.5f * (t2.x + t2.y);  // dL/da
     t2 = __fmul2_rn(hdx, make_float2(e.dy, e.dy));
-    v[3] = -(t2.x + t2.y);  // dL/db
+    v[3] = kFold ? t2.x + t2.y : -(t2.x + t2.y);  // dL/db
     t2 = __fmul2_rn(hdy, make_float2(e.dy, e.dy));
-    v[4] = -0.5f * (t2.x + t2.y);  // dL/dc
+    v[4] = kFold ? t2.x + t2.y : -0.5f * (t2.x + t2.y);  // dL/dc
     t2 = __fmul2_rn(wgt, g0);
     v[5] = t2.x + t2.y;  // dL/dcolor r
     t2 = __fmul2_rn(wgt, g1);
@@ -378,8 +402,8 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 m &= m - 1;
                 const int p = top - 1 - jj;
                 float v[8], r9;
-                if (!bwd_term(q, s_xy[jj], s_co[jj], s_col[jj], p, last0, last1, amax, amin, g0, g1, g2, T, S0, S1, S2,
-                              v, r9))
+                if (!bwd_term<true, false>(q, s_xy[jj], s_co[jj], s_col[jj], p, last0, last1, amax, amin, g0, g1, g2, T,
+                                           S0, S1, S2, v, r9))
                     continue;
                 const float r8 = reduce8(v, lane);
 #pragma unroll
@@ -413,29 +437,34 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     }
 }
 
-// Backward driven by the forward's contribution mask, one warp per 8x8
-// quadrant and no block barrier: each warp walks the mask words of its
-// quadrant from its last contributor towards the front; for each word the
-// lanes whose bit is set load that list entry into the warp's shared-memory
-// slots, and the warp then takes the set bits from the back.  After the
-// butterfly, the 9 gradient sums sit in 9 different lanes (value i in lane
-// 4i, the ninth in lane 1), which add them to the Gaussian's 2D gradients
-// with one atomic instruction.  A warp whose pixels are all finished leaves
-// at once instead of waiting at the other warps' batch barriers.
-__global__ void __launch_bounds__(kThreads, 9)
+// Backward driven by the forward's contribution mask: one CTA of one warp
+// per 8x8 quadrant (block b: tile b / 4, quadrant b % 4), so that a warp that
+// finishes frees its slot at once for the next quadrant.  The warp walks the
+// mask words of its quadrant from its last contributor towards the front;
+// for each word the lanes whose bit is set load that list entry into the
+// warp's shared-memory slots, and the warp then takes the set bits from the
+// back.  Every visited term was blended by some pixel of the quadrant, so no
+// vote is needed.  After the butterfly, the 9 gradient sums sit in 9
+// different lanes (value i in lane 4i, the ninth in lane 1), which scale
+// them by their constant factor and add them to the Gaussian's 2D gradients
+// with one atomic instruction.
+constexpr int kBwdWarpBlocksPerSM = 32;  // 64 registers per thread
+
+__global__ void __launch_bounds__(32, kBwdWarpBlocksPerSM)
 k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
                   const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
                   const float* __restrict__ colors, const float* __restrict__ final_T,
                   const unsigned* __restrict__ n_contrib, const unsigned* __restrict__ cmask, unsigned cmask_words,
                   const float* __restrict__ dL_dimage, float* __restrict__ dL_dmean2d,
                   float* __restrict__ dL_dconic_opacity, float* __restrict__ dL_dcolor) {
-    __shared__ unsigned s_id[kWarps][32];
-    __shared__ float2 s_xy[kWarps][32];
-    __shared__ float4 s_co[kWarps][32];
-    __shared__ float4 s_col[kWarps][32];
-    const PixelPair q = pixel_pair(cam, TX);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint2 rg = ranges[blockIdx.x];
+    __shared__ unsigned s_id[32];
+    __shared__ float2 s_xy[32];
+    __shared__ float4 s_co[32];
+    __shared__ float4 s_col[32];
+    const int lane = threadIdx.x;
+    const int tile = blockIdx.x >> 2, quad = blockIdx.x & 3;
+    const PixelPair q = quad_pixel_pair(cam, TX, tile, quad, lane);
+    const uint2 rg = ranges[tile];
     const float amax = cam.alpha_max, amin = cam.alpha_min;
     const size_t plane = (size_t)cam.width * cam.height;
     const size_t pix = (size_t)q.y * cam.width + q.x0;
@@ -464,11 +493,15 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
     if (wlast == 0) return;
 
     // where this lane's flush goes: value i of the butterfly in lane 4i, the
-    // ninth (blue) in lane 1; each lane adds to one component of one array
+    // ninth (blue) in lane 1; each lane adds to one component of one array,
+    // after the constant factor of its value (-1/2, -1, -1/2 for a, b, c)
     float* gbase = nullptr;
     unsigned gstride = 0;
+    float post = 1.0f;
     if (lane == 0 || lane == 4) { gbase = dL_dmean2d + (lane >> 2); gstride = 2; }
-    else if (lane == 8 || lane == 12 || lane == 16) { gbase = dL_dconic_opacity + ((lane >> 2) - 2); gstride = 4; }
+    else if (lane == 8 || lane == 12 || lane == 16) {
+        gbase = dL_dconic_opacity + ((lane >> 2) - 2); gstride = 4; post = lane == 12 ? -1.0f : -0.5f;
+    }
     else if (lane == 28) { gbase = dL_dconic_opacity + 3; gstride = 4; }
     else if (lane == 20 || lane == 24) { gbase = dL_dcolor + ((lane >> 2) - 5); gstride = 3; }
     else if (lane == 1) { gbase = dL_dcolor + 2; gstride = 3; }
@@ -476,7 +509,7 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
     const unsigned k_hi = rg.x + wlast - 1;  // last list entry to visit (global index)
     for (int wk = (int)(k_hi >> 5); wk >= (int)(rg.x >> 5); --wk) {
         const unsigned kb = (unsigned)wk << 5;
-        const unsigned wi = (unsigned)wk * kWarps + warp;
+        const unsigned wi = (unsigned)wk * kWarps + (unsigned)quad;
         unsigned bits = wi < cmask_words ? cmask[wi] : 0xFFFFFFFFu;
         // entries of this word that belong to the tile's list up to k_hi
         const unsigned lo = rg.x > kb ? rg.x - kb : 0u;
@@ -486,10 +519,10 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
         if (!bits) continue;
         if ((bits >> lane) & 1u) {
             const unsigned j = ids[kb + lane];
-            s_id[warp][lane] = j;
-            s_xy[warp][lane] = mean2d[j];
-            s_co[warp][lane] = conic_opacity[j];
-            s_col[warp][lane] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+            s_id[lane] = j;
+            s_xy[lane] = mean2d[j];
+            s_co[lane] = conic_opacity[j];
+            s_col[lane] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
         }
         __syncwarp();
         while (bits) {
@@ -497,14 +530,13 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
             bits &= ~(1u << l);
             const int p = (int)(kb + (unsigned)l - rg.x);
             float v[8], r9;
-            if (!bwd_term(q, s_xy[warp][l], s_co[warp][l], s_col[warp][l], p, last0, last1, amax, amin, g0, g1, g2, T,
-                          S0, S1, S2, v, r9))
-                continue;
+            bwd_term<false, true>(q, s_xy[l], s_co[l], s_col[l], p, last0, last1, amax, amin, g0, g1, g2, T, S0, S1,
+                                  S2, v, r9);
             const float r8 = reduce8(v, lane);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
-            const float val = lane == 1 ? r9 : r8;
-            if (gbase && val != 0.0f) atomicAdd(gbase + (size_t)s_id[warp][l] * gstride, val);
+            const float val = (lane == 1 ? r9 : r8) * post;
+            if (gbase && val != 0.0f) atomicAdd(gbase + (size_t)s_id[l] * gstride, val);
         }
         __syncwarp();  // the next word reuses this warp's slots
     }
@@ -601,7 +633,7 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
     }
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
     if (contrib_mask) {
-        k_render_bwd_warp<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
+        k_render_bwd_warp<<<4 * T, 32, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
                                                   reinterpret_cast<const float2*>(mean2d),
                                                   reinterpret_cast<const float4*>(conic_opacity), colors, final_T,
                                                   n_contrib, contrib_mask, mask_words, dL_dimage, dL_dmean2d,
