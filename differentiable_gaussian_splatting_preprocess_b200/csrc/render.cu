@@ -241,10 +241,13 @@ __device__ __forceinline__ float reduce8(float v[8], int lane) {
 // skip it).  With kFold, dL/da, dL/db and dL/dc are left without their
 // constant factors -1/2, -1 and -1/2 (exact powers of two, applied once after
 // the warp sum).
+// Sg = g . S, the upstream gradient dotted with the colour behind the term:
+// dL/dalpha = T (g . c - Sg), and S <- alpha c + (1 - alpha) S becomes
+// Sg <- Sg + alpha (g . c - Sg), one scalar per pixel instead of a colour.
 template <bool kVote, bool kFold>
 __device__ __forceinline__ bool bwd_term(const PixelPair& q, float2 xy, float4 co, float4 c, int p, unsigned last0,
                                          unsigned last1, float amax, float amin, float2 g0, float2 g1, float2 g2,
-                                         float2& T, float2& S0, float2& S1, float2& S2, float (&v)[8], float& r9) {
+                                         float2& T, float2& Sg, float (&v)[8], float& r9) {
     TermPair e;
     eval_pair(q.px, q.py, xy, co, amax, amin, e);
     const bool c0 = p < (int)last0 && e.ok0;
@@ -255,17 +258,13 @@ __device__ __forceinline__ bool bwd_term(const PixelPair& q, float2 xy, float4 c
     if (c0) T.x = __fdividef(T.x, 1.0f - al.x);
     if (c1) T.y = __fdividef(T.y, 1.0f - al.y);
     const float2 wgt = __fmul2_rn(al, T);
-    const float2 d0 = __fadd2_rn(make_float2(c.x, c.x), make_float2(-S0.x, -S0.y));
-    const float2 d1 = __fadd2_rn(make_float2(c.y, c.y), make_float2(-S1.x, -S1.y));
-    const float2 d2 = __fadd2_rn(make_float2(c.z, c.z), make_float2(-S2.x, -S2.y));
-    float2 dLda = __fmul2_rn(d0, g0);
-    dLda = __ffma2_rn(d1, g1, dLda);
-    dLda = __ffma2_rn(d2, g2, dLda);
-    dLda = __fmul2_rn(dLda, T);
-    // colour behind the next term towards the front: S <- alpha c + (1 - alpha) S
-    S0 = __ffma2_rn(al, d0, S0);
-    S1 = __ffma2_rn(al, d1, S1);
-    S2 = __ffma2_rn(al, d2, S2);
+    float2 gc = __fmul2_rn(make_float2(c.x, c.x), g0);  // g . c
+    gc = __ffma2_rn(make_float2(c.y, c.y), g1, gc);
+    gc = __ffma2_rn(make_float2(c.z, c.z), g2, gc);
+    const float2 diff = __fadd2_rn(gc, make_float2(-Sg.x, -Sg.y));
+    const float2 dLda = __fmul2_rn(diff, T);
+    // colour behind the next term towards the front, dotted with g
+    Sg = __ffma2_rn(al, diff, Sg);
     // exact derivative of min(alpha_max, opacity G): zero while capped
     const float2 Gf = make_float2(e.at.x <= amax ? G.x : 0.0f, e.at.y <= amax ? G.y : 0.0f);
     const float2 dsig = __fmul2_rn(Gf, dLda);                    // dL/dopacity
@@ -338,8 +337,10 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
         g1.y = dL_dimage[plane + pix + 1];
         g2.y = dL_dimage[2 * plane + pix + 1];
     }
-    float2 S0 = make_float2(cam.bg[0], cam.bg[0]), S1 = make_float2(cam.bg[1], cam.bg[1]);
-    float2 S2 = make_float2(cam.bg[2], cam.bg[2]);
+    // g . bg: the colour behind the last term is the background
+    float2 Sg = __fmul2_rn(make_float2(cam.bg[0], cam.bg[0]), g0);
+    Sg = __ffma2_rn(make_float2(cam.bg[1], cam.bg[1]), g1, Sg);
+    Sg = __ffma2_rn(make_float2(cam.bg[2], cam.bg[2]), g2, Sg);
 
     // furthest list position any pixel of the warp / of the tile blended
     const unsigned wlast = __reduce_max_sync(0xffffffffu, max(last0, last1));
@@ -403,7 +404,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 const int p = top - 1 - jj;
                 float v[8], r9;
                 if (!bwd_term<true, false>(q, s_xy[jj], s_co[jj], s_col[jj], p, last0, last1, amax, amin, g0, g1, g2, T,
-                                           S0, S1, S2, v, r9))
+                                           Sg, v, r9))
                     continue;
                 const float r8 = reduce8(v, lane);
 #pragma unroll
@@ -485,8 +486,10 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
         g1.y = dL_dimage[plane + pix + 1];
         g2.y = dL_dimage[2 * plane + pix + 1];
     }
-    float2 S0 = make_float2(cam.bg[0], cam.bg[0]), S1 = make_float2(cam.bg[1], cam.bg[1]);
-    float2 S2 = make_float2(cam.bg[2], cam.bg[2]);
+    // g . bg: the colour behind the last term is the background
+    float2 Sg = __fmul2_rn(make_float2(cam.bg[0], cam.bg[0]), g0);
+    Sg = __ffma2_rn(make_float2(cam.bg[1], cam.bg[1]), g1, Sg);
+    Sg = __ffma2_rn(make_float2(cam.bg[2], cam.bg[2]), g2, Sg);
     // furthest list position any pixel of this warp blended (a count), kept
     // inside the tile's list
     const unsigned wlast = min(__reduce_max_sync(0xffffffffu, max(last0, last1)), rg.y - rg.x);
@@ -530,8 +533,8 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
             bits &= ~(1u << l);
             const int p = (int)(kb + (unsigned)l - rg.x);
             float v[8], r9;
-            bwd_term<false, true>(q, s_xy[l], s_co[l], s_col[l], p, last0, last1, amax, amin, g0, g1, g2, T, S0, S1,
-                                  S2, v, r9);
+            bwd_term<false, true>(q, s_xy[l], s_co[l], s_col[l], p, last0, last1, amax, amin, g0, g1, g2, T, Sg, v,
+                                  r9);
             const float r8 = reduce8(v, lane);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
