@@ -126,18 +126,48 @@ __device__ __forceinline__ void eval_pair(float2 px, float py, float2 xy, float4
     e.ok1 = !(power.y > 0.0f) && !(e.alpha.y < alpha_min);
 }
 
-// Inflated threshold k on q = d^T A d: a pixel can reach alpha >= alpha_min
-// only where q <= k (see contrib_box).  +inf when no bound is available
-// (never culled), -1 when the Gaussian can never reach alpha_min.
-__device__ __forceinline__ float contrib_threshold(float4 co, float alpha_min) {
+// Culling parameters of one Gaussian, computed once per staged Gaussian:
+//  - thr: a pixel can reach alpha >= alpha_min only where q = d^T A d <= thr.
+//    The region is the ellipse q <= 2 ln(opacity / alpha_min); thr inflates
+//    that bound to cover the fp32 rounding of `power` in eval_pair, whose
+//    error grows with the conic's condition number (bounded by
+//    (a + c)^2 / det), and of exp.  +inf when no bound is available (never
+//    culled), -1 when the Gaussian can never reach alpha_min;
+//  - box: the axis-aligned box (pixel coordinates xmin, xmax, ymin, ymax) of
+//    that inflated ellipse, with extents sqrt(thr (A^-1)_xx) and
+//    sqrt(thr (A^-1)_yy); a warp whose pixels all lie outside may skip the
+//    Gaussian without changing any result.  A non-finite or undefined bound
+//    gives the infinite box (never skipped);
+//  - boc = b / c and boa = b / a, used by ellipse_misses.
+struct CullParams {
+    float4 box;
+    float thr, boc, boa;
+};
+
+__device__ __forceinline__ CullParams cull_params(float2 xy, float4 co, float alpha_min) {
     const float inf = __int_as_float(0x7f800000);
-    if (!(alpha_min > 0.0f)) return inf;
-    if (co.w < alpha_min) return -1.0f;
+    CullParams cp;
+    cp.box = make_float4(-inf, inf, -inf, inf);
+    cp.thr = inf;
+    cp.boc = co.y / co.z;
+    cp.boa = co.y / co.x;
+    if (!(alpha_min > 0.0f)) return cp;
+    if (co.w < alpha_min) {  // alpha <= opacity < alpha_min
+        cp.box = make_float4(inf, -inf, inf, -inf);
+        cp.thr = -1.0f;
+        return cp;
+    }
     const float det = co.x * co.z - co.y * co.y;
-    if (!(det > 0.0f)) return inf;
+    if (!(det > 0.0f)) return cp;
     const float tr = co.x + co.z;
-    const float k = 2.0f * logf(co.w / alpha_min) * (1.001f + 1e-6f * (tr * tr / det)) + 1e-5f;
-    return isfinite(k) ? k : inf;
+    const float ki = 2.0f * logf(co.w / alpha_min) * (1.001f + 1e-6f * (tr * tr / det)) + 1e-5f;
+    if (!isfinite(ki)) return cp;
+    cp.thr = ki;
+    const float ex = sqrtf(ki * co.z / det) + 0.01f;
+    const float ey = sqrtf(ki * co.x / det) + 0.01f;
+    const float4 b = make_float4(xy.x - ex, xy.x + ex, xy.y - ey, xy.y + ey);
+    if (isfinite(b.x) && isfinite(b.y) && isfinite(b.z) && isfinite(b.w)) cp.box = b;
+    return cp;
 }
 
 // True when q = a dx^2 + 2 b dx dy + c dy^2 exceeds `thr` at every point of
@@ -145,15 +175,14 @@ __device__ __forceinline__ float contrib_threshold(float4 co, float alpha_min) {
 // no pixel centre inside can reach alpha >= alpha_min.  The minimum of the
 // positive-definite q over the rectangle is 0 when the mean is inside, else
 // it lies on an edge, where q is a quadratic in one variable minimised in
-// closed form and clamped to the edge.  Any undefined value keeps the
-// Gaussian (the comparison is false).
-__device__ __forceinline__ bool ellipse_misses(float2 xy, float4 co, float thr, float x0, float x1, float y0,
-                                               float y1) {
+// closed form (boc = b / c, boa = b / a) and clamped to the edge.  Any
+// undefined value keeps the Gaussian (the comparison is false).
+__device__ __forceinline__ bool ellipse_misses(float2 xy, float4 co, float thr, float boc, float boa, float x0,
+                                               float x1, float y0, float y1) {
     if (xy.x >= x0 && xy.x <= x1 && xy.y >= y0 && xy.y <= y1) return false;
     const float a = co.x, b = co.y, c = co.z;
     if (!(a > 0.0f && c > 0.0f)) return false;
     const float ex0 = x0 - xy.x, ex1 = x1 - xy.x, ey0 = y0 - xy.y, ey1 = y1 - xy.y;
-    const float boc = b / c, boa = b / a;
     float best = __int_as_float(0x7f800000);
     // edges x = x0 and x = x1: minimise over dy in [ey0, ey1]; dy* = -b dx / c
 #pragma unroll
@@ -170,31 +199,6 @@ __device__ __forceinline__ bool ellipse_misses(float2 xy, float4 co, float thr, 
         best = fminf(best, a * dx * dx + 2.0f * b * dx * dy + c * dy * dy);
     }
     return best > thr;
-}
-
-// Axis-aligned box (pixel coordinates: xmin, xmax, ymin, ymax) outside of
-// which a Gaussian cannot reach alpha >= alpha_min, so a warp whose pixels
-// all lie outside may skip it without changing any result.  The region is
-// the ellipse d^T A d <= 2 ln(opacity / alpha_min); its extents are
-// sqrt(k (A^-1)_xx) and sqrt(k (A^-1)_yy).  k is inflated to cover the fp32
-// rounding of `power` in eval_term, whose error grows with the conic's
-// condition number (bounded by (a + c)^2 / det), and of exp.  A non-finite
-// or undefined bound gives the infinite box (never skipped).
-__device__ __forceinline__ float4 contrib_box(float2 xy, float4 co, float alpha_min) {
-    const float inf = __int_as_float(0x7f800000);
-    const float4 all = make_float4(-inf, inf, -inf, inf);
-    if (!(alpha_min > 0.0f)) return all;
-    if (co.w < alpha_min) return make_float4(inf, -inf, inf, -inf);  // alpha <= opacity < alpha_min
-    const float det = co.x * co.z - co.y * co.y;
-    if (!(det > 0.0f)) return all;
-    const float tr = co.x + co.z;
-    const float k = 2.0f * logf(co.w / alpha_min);
-    const float ki = k * (1.001f + 1e-6f * (tr * tr / det)) + 1e-5f;
-    const float ex = sqrtf(ki * co.z / det) + 0.01f;
-    const float ey = sqrtf(ki * co.x / det) + 0.01f;
-    const float4 b = make_float4(xy.x - ex, xy.x + ex, xy.y - ey, xy.y + ey);
-    if (!(isfinite(b.x) && isfinite(b.y) && isfinite(b.z) && isfinite(b.w))) return all;
-    return b;
 }
 
 // True when the box misses the rectangle of pixel centres [x0, x1] x [y0, y1].

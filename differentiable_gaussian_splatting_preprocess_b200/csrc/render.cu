@@ -26,7 +26,9 @@ namespace {
 
 // One CTA per 16x16 tile with 128 threads: each thread owns two horizontally
 // adjacent pixels, evaluated together with packed fp32x2 arithmetic; warp w
-// owns one 8x8 quadrant of the tile.  Gaussians are staged 256 at a time.
+// owns one 8x8 quadrant of the tile.  Gaussians are staged 128 at a time
+// (the forward; 256 in the backward without the mask), each with its culling
+// parameters computed once for the four warps.
 // Before a warp walks a batch it builds a ballot mask of the staged
 // Gaussians that can reach alpha >= alpha_min somewhere in its quadrant (a
 // box test, then an exact ellipse-versus-rectangle test, both inflated for
@@ -35,8 +37,10 @@ namespace {
 // are unchanged.
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 256;
+constexpr int kBatch = 256;       // staged Gaussians per batch (backward without the mask)
 constexpr int kWords = kBatch / 32;
+constexpr int kFwdBatch = 128;    // staged Gaussians per batch of the forward
+constexpr int kFwdWords = kFwdBatch / 32;
 static_assert(kThreads * 2 == kTilePixels, "two pixels per thread");
 
 struct PixelPair {
@@ -86,9 +90,17 @@ __device__ __forceinline__ PixelPair quad_pixel_pair(const gs_camera& cam, int T
 }
 
 // Can the staged Gaussian reach alpha >= alpha_min in this warp's quadrant?
-__device__ __forceinline__ bool may_contribute(float4 box, float thr, float2 xy, float4 co, const PixelPair& q) {
+// (box test, then the exact ellipse test; tr = (thr, b / c, b / a))
+__device__ __forceinline__ bool may_contribute(float4 box, float4 tr, float2 xy, float4 co, const PixelPair& q) {
     if (box_misses(box, q.sx0, q.sx1, q.sy0, q.sy1)) return false;
-    return !ellipse_misses(xy, co, thr, q.sx0, q.sx1, q.sy0, q.sy1);
+    return !ellipse_misses(xy, co, tr.x, tr.y, tr.z, q.sx0, q.sx1, q.sy0, q.sy1);
+}
+
+// Stage the culling parameters of one Gaussian (once per CTA and batch).
+__device__ __forceinline__ void stage_cull(float2 xy, float4 co, float alpha_min, float4& box, float4& tr) {
+    const CullParams cp = cull_params(xy, co, alpha_min);
+    box = cp.box;
+    tr = make_float4(cp.thr, cp.boc, cp.boa, 0.0f);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -96,11 +108,11 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
              const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
              const float* __restrict__ colors, float* __restrict__ image, float* __restrict__ final_T,
              unsigned* __restrict__ n_contrib, unsigned* __restrict__ cmask, unsigned cmask_words) {
-    __shared__ float2 s_xy[kBatch];
-    __shared__ float4 s_co[kBatch];
-    __shared__ float4 s_col[kBatch];
-    __shared__ float4 s_box[kBatch];
-    __shared__ float s_thr[kBatch];
+    __shared__ float2 s_xy[kFwdBatch];
+    __shared__ float4 s_co[kFwdBatch];
+    __shared__ float4 s_col[kFwdBatch];
+    __shared__ float4 s_box[kFwdBatch];
+    __shared__ float4 s_thr[kFwdBatch];  // threshold, b / c, b / a
     const PixelPair q = pixel_pair(cam, TX);
     const int lane = threadIdx.x & 31;
     const uint2 rg = ranges[blockIdx.x];
@@ -110,9 +122,9 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     float2 C0 = make_float2(0.0f, 0.0f), C1 = C0, C2 = C0;
     unsigned last0 = 0, last1 = 0;
     bool done0 = !q.in0, done1 = !q.in1;
-    for (unsigned b = rg.x; b < rg.y; b += kBatch) {
+    for (unsigned b = rg.x; b < rg.y; b += kFwdBatch) {
         if (__syncthreads_count(done0 && done1) == kThreads) break;
-        for (int r = threadIdx.x; r < kBatch; r += kThreads) {
+        for (int r = threadIdx.x; r < kFwdBatch; r += kThreads) {
             const unsigned k = b + r;
             if (k < rg.y) {
                 const unsigned j = ids[k];
@@ -121,12 +133,11 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 s_xy[r] = xy;
                 s_co[r] = co;
                 s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
-                s_box[r] = contrib_box(xy, co, amin);
-                s_thr[r] = contrib_threshold(co, amin);
+                stage_cull(xy, co, amin, s_box[r], s_thr[r]);
             }
         }
         __syncthreads();
-        const int n = min((unsigned)kBatch, rg.y - b);
+        const int n = min((unsigned)kFwdBatch, rg.y - b);
         bool warp_done = __all_sync(0xffffffffu, done0 && done1);
         // cull against the pixels of this warp that are still compositing
         PixelPair qa = q;
@@ -142,7 +153,7 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
             qa.sy0 = (float)aymin + 0.5f;
             qa.sy1 = (float)aymax + 0.5f;
         }
-        for (int w = 0; w < kWords && !warp_done; ++w) {
+        for (int w = 0; w < kFwdWords && !warp_done; ++w) {
             const int jl = w * 32 + lane;
             const bool keep = jl < n && may_contribute(s_box[jl], s_thr[jl], s_xy[jl], s_co[jl], qa);
             unsigned m = __ballot_sync(0xffffffffu, keep);
@@ -310,7 +321,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     __shared__ float4 s_co[kBatch];
     __shared__ float4 s_col[kBatch];
     __shared__ float4 s_box[kMask ? 1 : kBatch];
-    __shared__ float s_thr[kMask ? 1 : kBatch];
+    __shared__ float4 s_thr[kMask ? 1 : kBatch];  // threshold, b / c, b / a
     __shared__ float s_grad[kBatch * kGradStride];
     __shared__ unsigned s_max[kWarps];
 
@@ -380,10 +391,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 s_xy[r] = xy;
                 s_co[r] = co;
                 s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
-                if (!kMask) {
-                    s_box[r] = contrib_box(xy, co, amin);
-                    s_thr[r] = contrib_threshold(co, amin);
-                }
+                if (!kMask) stage_cull(xy, co, amin, s_box[r], s_thr[r]);
             }
         }
         __syncthreads();
