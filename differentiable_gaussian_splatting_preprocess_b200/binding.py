@@ -15,7 +15,11 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libgs.so")
+# GS_LIBRARY=debug loads libgs_debug.so (the index-checking build); any other
+# value is taken as a path to the library.
+_choice = os.environ.get("GS_LIBRARY", "")
+LIB_PATH = (os.path.join(_HERE, "libgs_debug.so") if _choice == "debug" else
+            (_choice or os.path.join(_HERE, "libgs.so")))
 
 GS_OK = 0
 GS_ERR_INVALID_ARG = 1
@@ -24,6 +28,7 @@ GS_ERR_TIMEOUT = 4
 GS_ERR_CUDA = 8
 GS_ERR_UNIMPLEMENTED = 16
 GS_ERR_OVERFLOW = 32
+GS_ERR_INDEX = 64
 GS_STAGE_PREPROCESS_FWD = 0
 GS_STAGE_BIN_SORT = 1
 TILE = 16
@@ -32,7 +37,7 @@ TILE = 16
 EXPORTED = ("gs_version", "gs_launch_count", "gs_status_string", "gs_workspace_bytes", "gs_read_status", "gs_clear_status",
             "gs_preprocess_fwd", "gs_bin_sort", "gs_render_fwd", "gs_render_bwd", "gs_preprocess_bwd",
             "gs_preprocess_fwd_noalloc", "gs_render_stats", "gs_sh_fwd", "gs_sh_bwd", "gs_sh_fwd_f16",
-            "gs_sh_bwd_f16", "gs_adam_step")
+            "gs_sh_bwd_f16", "gs_adam_step", "gs_debug_configure", "gs_debug_read")
 
 
 class GsCamera(ctypes.Structure):
@@ -110,6 +115,10 @@ def lib() -> ctypes.CDLL:
         L.gs_sh_bwd_f16.argtypes = [cam, I, I, I, P, P, ctypes.c_float, P, P, P, P]
         L.gs_preprocess_bwd.restype = I
         L.gs_preprocess_bwd.argtypes = [cam, I] + [P] * 15 + [P]
+        L.gs_debug_configure.restype = I
+        L.gs_debug_configure.argtypes = [U, U]
+        L.gs_debug_read.restype = I
+        L.gs_debug_read.argtypes = [ctypes.POINTER(I), I]
         _lib = L
     return _lib
 
@@ -173,6 +182,20 @@ def _ok(fn: str, status: int) -> None:
 
 def num_tiles(cam) -> int:
     return ((cam.width + TILE - 1) // TILE) * ((cam.height + TILE - 1) // TILE)
+
+
+def gs_debug_configure(n_gauss: int, capacity: int) -> None:
+    """Debug build only: the limits of its index checks (Gaussian ids below
+    n_gauss, list positions below capacity); clears the debug word."""
+    _ok("gs_debug_configure", lib().gs_debug_configure(int(n_gauss), int(capacity)))
+
+
+def gs_debug_read(clear: bool = False) -> int:
+    """Debug build only: the debug word (GS_ERR_INDEX once a check failed);
+    waits for the device."""
+    f = ctypes.c_int(0)
+    _ok("gs_debug_read", lib().gs_debug_read(ctypes.byref(f), 1 if clear else 0))
+    return int(f.value)
 
 
 def gs_workspace_bytes(stage: int, N: int, capacity: int, width: int, height: int) -> int:

@@ -4,6 +4,11 @@ Every translation unit under ``csrc/`` is compiled by nvcc for
 ``arch=compute_100a,code=sm_100a`` with line info, no fast-math, and the CUDA
 runtime linked statically, then linked into one shared object beside this
 file.  Objects go to ``_build/`` (git-ignored).
+
+``build(debug=True)`` builds ``libgs_debug.so`` from the same sources with
+GS_DEBUG defined (index checks before every gather by Gaussian id or list
+position; see gs_debug_configure in include/gs.h), as relocatable device code
+so that all translation units share one device-side debug word.
 """
 from __future__ import annotations
 
@@ -18,6 +23,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libgs.so")
+DEBUG_LIB = os.path.join(HERE, "libgs_debug.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -33,35 +39,40 @@ def _deps():
     return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(debug: bool = False) -> bool:
+    lib = DEBUG_LIB if debug else LIB
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OUT_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(debug):
+        return lib
+    out_dir = os.path.join(OUT_DIR, "debug") if debug else OUT_DIR
+    extra = ["-DGS_DEBUG", "-rdc=true"] if debug else []
+    os.makedirs(out_dir, exist_ok=True)
     objs = []
     for src in sources():
-        obj = os.path.join(OUT_DIR, os.path.basename(src) + ".o")
-        cmd = [NVCC, *ARCH, *CFLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(out_dir, os.path.basename(src) + ".o")
+        cmd = [NVCC, *ARCH, *CFLAGS, *extra, "-c", src, "-o", obj]
         if ptxas_info:
             cmd.insert(1, "-Xptxas=-v")
         if verbose:
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [NVCC, *ARCH, *extra, "-shared", "-cudart", "static", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, ptxas_info="--ptxas" in sys.argv))
+    dbg = "--debug" in sys.argv
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, ptxas_info="--ptxas" in sys.argv, debug=dbg))

@@ -34,6 +34,7 @@ extern "C" const char* gs_status_string(int status) {
         case GS_ERR_CUDA: return "CUDA launch or copy failed";
         case GS_ERR_UNIMPLEMENTED: return "not implemented";
         case GS_ERR_OVERFLOW: return "pair count does not fit in 32 bits";
+        case GS_ERR_INDEX: return "an index check of the debug build failed";
         default: return "several error flags are set";
     }
 }
@@ -62,6 +63,46 @@ extern "C" int gs_read_status(const void* ws, int* status, void* stream) {
     *status = (int)v;
     return GS_OK;
 }
+
+#ifdef GS_DEBUG
+namespace gs {
+__device__ DebugState g_debug = {0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u};
+}  // namespace gs
+
+extern "C" int gs_debug_configure(unsigned n_gauss, unsigned capacity) {
+    const gs::DebugState d = {n_gauss, capacity, 0u, 0u};
+    if (cudaMemcpyToSymbol(gs::g_debug, &d, sizeof d) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GS_ERR_CUDA;
+    }
+    return GS_OK;
+}
+
+extern "C" int gs_debug_read(int* flags, int clear) {
+    if (!flags) return GS_ERR_INVALID_ARG;
+    gs::DebugState d;
+    if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpyFromSymbol(&d, gs::g_debug, sizeof d) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GS_ERR_CUDA;
+    }
+    *flags = (int)d.flags;
+    if (clear) {
+        d.flags = 0u;
+        if (cudaMemcpyToSymbol(gs::g_debug, &d, sizeof d) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return GS_ERR_CUDA;
+        }
+    }
+    return GS_OK;
+}
+#else
+extern "C" int gs_debug_configure(unsigned, unsigned) { return GS_ERR_UNIMPLEMENTED; }
+
+extern "C" int gs_debug_read(int* flags, int) {
+    if (flags) *flags = 0;
+    return GS_ERR_UNIMPLEMENTED;
+}
+#endif
 
 extern "C" int gs_clear_status(void* ws, void* stream) {
     if (!ws) return GS_ERR_INVALID_ARG;

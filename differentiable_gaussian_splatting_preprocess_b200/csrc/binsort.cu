@@ -151,6 +151,13 @@ __device__ __forceinline__ int rect_w(unsigned p) { return (int)((p >> 8) & 255u
 __device__ __forceinline__ int rect_y0(unsigned p) { return (int)((p >> 16) & 255u); }
 __device__ __forceinline__ int rect_h(unsigned p) { return (int)(p >> 24) + 1; }
 
+// Debug build: after a failed index check inside the binning, later kernels
+// would see inconsistent inputs (a visible rank without pairs, an unwritten
+// pair), so the frame's usable pair count is set to 0: every later kernel of
+// the call then sees an empty frame (all ranges empty, no pair written), as
+// when the capacity is exceeded.
+__device__ __forceinline__ void abort_frame(SortMisc* misc) { atomicExch(&misc->p_eff, 0u); }
+
 __device__ __forceinline__ unsigned lanemask_lt() {
     unsigned m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -497,7 +504,7 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
 __global__ void __launch_bounds__(kSortBlock)
 k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ tiles_touched,
                 const int4* __restrict__ rect, unsigned* __restrict__ cnt_rank, unsigned* __restrict__ rc_rank,
-                unsigned* __restrict__ part) {
+                unsigned* __restrict__ part, SortMisc* __restrict__ misc) {
     const int base = blockIdx.x * kScanTile;
     unsigned s = 0;
 #pragma unroll
@@ -505,7 +512,9 @@ k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __res
         const int r = base + k * kSortBlock + threadIdx.x;
         if (r < N) {
             const unsigned g = order[r];
-            unsigned v = tiles_touched[g];
+            unsigned v = 0u;
+            if (id_ok(g)) v = tiles_touched[g];
+            else abort_frame(misc);
             if (rect && v) {
                 const int4 sr = super_rect(rect[g]);
                 v = (unsigned)((sr.z - sr.x) * (sr.w - sr.y));
@@ -627,7 +636,7 @@ __device__ __forceinline__ unsigned upper_bound_global(const unsigned* __restric
 
 __global__ void __launch_bounds__(kSortBlock)
 k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
-       const int4* __restrict__ rect, const unsigned* __restrict__ tiles_touched, const SortMisc* __restrict__ misc,
+       const int4* __restrict__ rect, const unsigned* __restrict__ tiles_touched, SortMisc* __restrict__ misc,
        unsigned* __restrict__ tkeys, unsigned* __restrict__ tvals) {
     __shared__ unsigned s_off[kEmitSeg + 1];
     __shared__ unsigned s_g[kEmitSeg + 1];
@@ -659,6 +668,10 @@ k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __rest
                 if (s_off[mid] <= p) lo = mid; else hi = mid;
             }
             const unsigned g = s_g[lo];
+            if (!id_ok(g) || !pos_ok(p)) {
+                abort_frame(misc);
+                continue;
+            }
             const int4 rc = rect[g];
             const unsigned w = (unsigned)(rc.z - rc.x);
             const unsigned local = p - s_off[lo];
@@ -707,7 +720,8 @@ __global__ void k_ranges(const unsigned* __restrict__ tkeys, const unsigned* __r
                 const unsigned after = (j == 3 || k + 1 == P) ? (k + 1 == P ? 0xFFFFFFFFu : next) : t[j + 1];
                 if (k == 0 || before != t[j]) ranges[2 * t[j]] = k;
                 if (k + 1 == P || after != t[j]) ranges[2 * t[j] + 1] = k + 1;
-                if (keys) keys[k] = ((unsigned long long)t[j] << 32) | __float_as_uint(depth[ids[k]]);
+                if (keys && pos_ok(k) && id_ok(ids[k]))
+                    keys[k] = ((unsigned long long)t[j] << 32) | __float_as_uint(depth[ids[k]]);
             }
         }
     }
@@ -1083,7 +1097,7 @@ k_seg_count(int SX, const unsigned* __restrict__ clist, const int4* __restrict__
         unsigned acc[kCellTiles / 4] = {};
         for (unsigned base = lo; base < hi; base += kSortBlock) {
             const unsigned i = base + threadIdx.x;
-            const unsigned m = i < hi ? cell_mask(rect[clist[i]], cx, cy) : 0u;
+            const unsigned m = (i < hi && id_ok(clist[i])) ? cell_mask(rect[clist[i]], cx, cy) : 0u;
             if (i < hi) seg_mask[i] = (unsigned short)m;
             add_mask(acc, m);
         }
@@ -1213,7 +1227,7 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
                 s_base[b] = run;
             }
             __syncthreads();
-            const float dg = (keys && m) ? depth[g] : 0.0f;
+            const float dg = (keys && m && id_ok(g)) ? depth[g] : 0.0f;
             // tile bits in order, unrolled: no find-first-set / bit-reverse
             // (XU) instructions; skipped bits cost one uniform branch
 #pragma unroll
@@ -1223,6 +1237,7 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
                 const unsigned bal = __ballot_sync(0xffffffffu, mine);
                 if (mine) {
                     const unsigned pos = s_wb[warp][b] + __popc(bal & lt);
+                    if (!pos_ok(pos)) continue;
                     ids[pos] = g;
                     if (keys) {
                         const unsigned t = (unsigned)((kSuper * cy + b / kSuper) * TX + kSuper * cx + b % kSuper);
@@ -1353,7 +1368,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     const int nb = (N + kScanTile - 1) / kScanTile;
     const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
     k_scan_partials<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
-                                               w.rc_rank, w.scan_part); note_launch();
+                                               w.rc_rank, w.scan_part, w.misc); note_launch();
     k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb, w.misc); note_launch();
     k_scan_down<<<nb, kSortBlock, 0, st>>>(N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
                                            (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi); note_launch();

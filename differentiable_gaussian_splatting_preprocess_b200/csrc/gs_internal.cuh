@@ -50,6 +50,32 @@ __host__ __device__ inline bool aligned(const void* p, size_t a) { return (reint
 
 __device__ __forceinline__ void raise_status(WsHeader* h, unsigned flag) { atomicOr(&h->status, flag); }
 
+// Index checks of the debug build (GS_DEBUG, compiled with relocatable
+// device code so that every translation unit shares g_debug).  Each returns
+// whether the index is inside its limit; a failed check ORs GS_ERR_INDEX
+// into the debug word, and the caller skips the access.  In the release
+// build they are constant true and cost nothing.
+#ifdef GS_DEBUG
+struct DebugState {
+    unsigned n_gauss;   // Gaussian ids must be below this
+    unsigned capacity;  // sorted-list positions must be below this
+    unsigned flags;     // GS_ERR_INDEX once a check failed
+    unsigned pad;
+};
+extern __device__ DebugState g_debug;
+__device__ __forceinline__ bool debug_check(bool ok) {
+    if (!ok) atomicOr(&g_debug.flags, (unsigned)GS_ERR_INDEX);
+    return ok;
+}
+__device__ __forceinline__ bool id_ok(unsigned j) { return debug_check(j < g_debug.n_gauss); }
+__device__ __forceinline__ bool pos_ok(unsigned k) { return debug_check(k < g_debug.capacity); }
+__device__ __forceinline__ bool end_ok(unsigned k) { return debug_check(k <= g_debug.capacity); }
+#else
+__device__ __forceinline__ constexpr bool id_ok(unsigned) { return true; }
+__device__ __forceinline__ constexpr bool pos_ok(unsigned) { return true; }
+__device__ __forceinline__ constexpr bool end_ok(unsigned) { return true; }
+#endif
+
 // exp(x) in fp32 as a fixed sequence of IEEE operations, so that any IEEE
 // machine with a correctly rounded fused multiply-add reproduces every bit
 // (the library's expf does not promise that, and a one-ulp difference can

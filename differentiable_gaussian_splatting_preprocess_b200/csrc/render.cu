@@ -96,6 +96,24 @@ __device__ __forceinline__ bool may_contribute(float4 box, float4 tr, float2 xy,
     return !ellipse_misses(xy, co, tr.x, tr.y, tr.z, q.sx0, q.sx1, q.sy0, q.sy1);
 }
 
+// A tile's range of the sorted list; in the debug build, an empty range if it
+// is not inside the list's capacity.
+__device__ __forceinline__ uint2 checked_range(uint2 rg) {
+    return (rg.x <= rg.y && end_ok(rg.y)) ? rg : make_uint2(0u, 0u);
+}
+
+// A staged entry that contributes nothing (zero opacity, never kept by the
+// cull), used by the debug build in place of an entry whose index failed its
+// check.
+__device__ __forceinline__ void stage_inert(float2& xy, float4& co, float4& col, float4& box, float4& thr) {
+    const float inf = __int_as_float(0x7f800000);
+    xy = make_float2(0.0f, 0.0f);
+    co = make_float4(1.0f, 0.0f, 1.0f, 0.0f);
+    col = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    box = make_float4(inf, -inf, inf, -inf);
+    thr = make_float4(-1.0f, 0.0f, 0.0f, 0.0f);
+}
+
 // Stage the culling parameters of one Gaussian (once per CTA and batch).
 __device__ __forceinline__ void stage_cull(float2 xy, float4 co, float alpha_min, float4& box, float4& tr) {
     const CullParams cp = cull_params(xy, co, alpha_min);
@@ -115,7 +133,7 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     __shared__ float4 s_thr[kFwdBatch];  // threshold, b / c, b / a
     const PixelPair q = pixel_pair(cam, TX);
     const int lane = threadIdx.x & 31;
-    const uint2 rg = ranges[blockIdx.x];
+    const uint2 rg = checked_range(ranges[blockIdx.x]);
     const float amax = cam.alpha_max, amin = cam.alpha_min, tmin = cam.T_min;
 
     float2 T = make_float2(1.0f, 1.0f);
@@ -127,13 +145,17 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
         for (int r = threadIdx.x; r < kFwdBatch; r += kThreads) {
             const unsigned k = b + r;
             if (k < rg.y) {
-                const unsigned j = ids[k];
-                const float2 xy = mean2d[j];
-                const float4 co = conic_opacity[j];
-                s_xy[r] = xy;
-                s_co[r] = co;
-                s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
-                stage_cull(xy, co, amin, s_box[r], s_thr[r]);
+                const unsigned j = pos_ok(k) ? ids[k] : 0xFFFFFFFFu;
+                if (id_ok(j)) {
+                    const float2 xy = mean2d[j];
+                    const float4 co = conic_opacity[j];
+                    s_xy[r] = xy;
+                    s_co[r] = co;
+                    s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+                    stage_cull(xy, co, amin, s_box[r], s_thr[r]);
+                } else {  // debug build, failed check: an inert entry (zero opacity)
+                    stage_inert(s_xy[r], s_co[r], s_col[r], s_box[r], s_thr[r]);
+                }
             }
         }
         __syncthreads();
@@ -327,7 +349,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
 
     const PixelPair q = pixel_pair(cam, TX);
     const int lane = threadIdx.x & 31;
-    const uint2 rg = ranges[blockIdx.x];
+    const uint2 rg = checked_range(ranges[blockIdx.x]);
     const float amax = cam.alpha_max, amin = cam.alpha_min;
     const size_t plane = (size_t)cam.width * cam.height;
     const size_t pix = (size_t)q.y * cam.width + q.x0;
@@ -384,14 +406,21 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
         for (int r = threadIdx.x; r < kBatch; r += kThreads) {
             const int pos = top - 1 - r;
             if (pos >= 0) {
-                const unsigned j = ids[rg.x + pos];
-                const float2 xy = mean2d[j];
-                const float4 co = conic_opacity[j];
-                s_id[r] = j;
-                s_xy[r] = xy;
-                s_co[r] = co;
-                s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
-                if (!kMask) stage_cull(xy, co, amin, s_box[r], s_thr[r]);
+                const unsigned j = pos_ok(rg.x + pos) ? ids[rg.x + pos] : 0xFFFFFFFFu;
+                if (id_ok(j)) {
+                    const float2 xy = mean2d[j];
+                    const float4 co = conic_opacity[j];
+                    s_id[r] = j;
+                    s_xy[r] = xy;
+                    s_co[r] = co;
+                    s_col[r] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+                    if (!kMask) stage_cull(xy, co, amin, s_box[r], s_thr[r]);
+                } else {  // debug build, failed check: an inert entry (zero opacity, id 0)
+                    s_id[r] = 0u;
+                    float4 box, thr;
+                    stage_inert(s_xy[r], s_co[r], s_col[r], box, thr);
+                    if (!kMask) { s_box[r] = box; s_thr[r] = thr; }
+                }
             }
         }
         __syncthreads();
@@ -473,7 +502,7 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
     const int lane = threadIdx.x;
     const int tile = blockIdx.x >> 2, quad = blockIdx.x & 3;
     const PixelPair q = quad_pixel_pair(cam, TX, tile, quad, lane);
-    const uint2 rg = ranges[tile];
+    const uint2 rg = checked_range(ranges[tile]);
     const float amax = cam.alpha_max, amin = cam.alpha_min;
     const size_t plane = (size_t)cam.width * cam.height;
     const size_t pix = (size_t)q.y * cam.width + q.x0;
@@ -529,11 +558,17 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
         bits &= ~((1u << lo) - 1u);
         if (!bits) continue;
         if ((bits >> lane) & 1u) {
-            const unsigned j = ids[kb + lane];
-            s_id[lane] = j;
-            s_xy[lane] = mean2d[j];
-            s_co[lane] = conic_opacity[j];
-            s_col[lane] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+            const unsigned j = pos_ok(kb + lane) ? ids[kb + lane] : 0xFFFFFFFFu;
+            if (id_ok(j)) {
+                s_id[lane] = j;
+                s_xy[lane] = mean2d[j];
+                s_co[lane] = conic_opacity[j];
+                s_col[lane] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+            } else {  // debug build, failed check: an inert entry (zero opacity, id 0)
+                s_id[lane] = 0u;
+                float4 box, thr;
+                stage_inert(s_xy[lane], s_co[lane], s_col[lane], box, thr);
+            }
         }
         __syncwarp();
         while (bits) {
@@ -566,13 +601,14 @@ k_render_stats(gs_camera cam, int TX, const uint2* __restrict__ ranges, const un
     const int x = (tile % TX) * kTile + (threadIdx.x & (kTile - 1));
     const int y = (tile / TX) * kTile + (threadIdx.x / kTile);
     if (x >= cam.width || y >= cam.height) return;
-    const uint2 rg = ranges[tile];
+    const uint2 rg = checked_range(ranges[tile]);
     const float2 px = make_float2((float)x + 0.5f, (float)x + 0.5f);
     const float py = (float)y + 0.5f;
     float T = 1.0f;
     unsigned ev = 0, bl = 0;
     for (unsigned k = rg.x; k < rg.y; ++k) {
-        const unsigned j = ids[k];
+        const unsigned j = pos_ok(k) ? ids[k] : 0xFFFFFFFFu;
+        if (!id_ok(j)) break;
         ++ev;
         TermPair e;
         eval_pair(px, py, mean2d[j], conic_opacity[j], cam.alpha_max, cam.alpha_min, e);

@@ -64,6 +64,7 @@ extern "C" {
 #define GS_ERR_CUDA 8          /* a CUDA launch or copy failed */
 #define GS_ERR_UNIMPLEMENTED 16
 #define GS_ERR_OVERFLOW 32     /* device: pair count does not fit in 32 bits */
+#define GS_ERR_INDEX 64        /* device, debug build only: an index check failed (the access was skipped) */
 
 /* Stages for gs_workspace_bytes(). */
 #define GS_STAGE_PREPROCESS_FWD 0
@@ -115,6 +116,26 @@ GS_API int gs_read_status(const void* ws, int* status, void* stream);
 
 /* Enqueue a reset of the status word of `ws` to GS_OK. */
 GS_API int gs_clear_status(void* ws, void* stream);
+
+/*
+ * Debug build (libgs_debug.so: the same sources compiled with GS_DEBUG; no
+ * counterpart on the pages, a tool for checking this library).  Before every
+ * gather by a Gaussian id or a sorted-list position, and before every write of
+ * a sorted-list entry, its kernels check the index against the limits set
+ * here (id < n_gauss, list position < capacity); a failed check skips the
+ * access and ORs GS_ERR_INDEX into a device-wide debug word instead of
+ * touching memory.  Tile indices come from the launch grid and the ranges;
+ * the ranges are checked against the capacity.
+ *
+ * gs_debug_configure - set the limits (and clear the debug word); blocks
+ *   until done.  Until it is first called every limit is unbounded.
+ * gs_debug_read - copy the debug word to *flags (host), after waiting for
+ *   all work on the device; with `clear` != 0 also reset it.
+ * In the release library (libgs.so) both return GS_ERR_UNIMPLEMENTED and
+ *   *flags is set to 0.
+ */
+GS_API int gs_debug_configure(unsigned n_gauss, unsigned capacity);
+GS_API int gs_debug_read(int* flags, int clear);
 
 /*
  * gs_preprocess_fwd - EWA projection of N 3D Gaussians ([TR] D.4, E.3; [CB] 4).

@@ -1,4 +1,4 @@
-"""CPU model of the cell-route binning's index arithmetic (no GPU).
+"""CPU model of the index arithmetic of the binning and render kernels (no GPU).
 
 The kernels in csrc/binsort.cu locate their work through derived indices:
 the ranks owning each chunk's first and last pair (recorded by the rank
@@ -9,6 +9,8 @@ restates those rules in Python and checks, on random rectangles, that they
 reproduce a direct construction: every generated pair, every chunk
 histogram, and the final per-tile lists (rank order) - and that no index
 leaves its buffer (staging window <= 2049 ranks, output positions < P).
+The render kernels' contribution-mask words (written per staged batch by the
+forward, walked back to front by the backward) are modelled the same way.
 """
 import random
 
@@ -193,3 +195,98 @@ def test_cell_route_index_model(TX, TY, N, seed, gmax):
     ref = [g for t in range(T) for g in order
            if rects[g][0] <= t % TX < rects[g][2] and rects[g][1] <= t // TX < rects[g][3]]
     assert ids == ref
+
+
+# --------------------------------------------------------------------------
+# Render kernels: contribution-mask words and the backward's walk
+# --------------------------------------------------------------------------
+
+FWD_BATCH = 128  # staged entries per forward batch
+QUADS = 4
+
+
+def _mask_model(ranges, blended, P):
+    """The forward's mask writes as render.cu indexes them: per tile, per
+    batch of FWD_BATCH entries starting at the tile's first position, per
+    word w of 32 staged entries (k0 = batch start + 32 w), quadrant q ORs its
+    32 blend bits shifted by o = k0 % 32 into word (k0 // 32) * 4 + q and, when
+    o > 0, the rest into the word four further on - each write only below the
+    mask's size 4 * ceil(P / 32)."""
+    words = QUADS * ((P + 31) // 32)
+    mask = np.zeros(words, np.uint64)
+    for t, (s, e) in enumerate(ranges):
+        for b in range(s, e, FWD_BATCH):
+            for w in range(FWD_BATCH // 32):
+                k0 = b + 32 * w
+                if k0 >= e:
+                    break
+                for q in range(QUADS):
+                    bw = 0
+                    for j in range(32):
+                        if k0 + j < e and (k0 + j, q) in blended:
+                            bw |= 1 << j
+                    if not bw:
+                        continue
+                    o = k0 & 31
+                    wi = (k0 >> 5) * QUADS + q
+                    assert wi < words
+                    mask[wi] |= (bw << o) & 0xFFFFFFFF
+                    if o and wi + QUADS < words:
+                        mask[wi + QUADS] |= bw >> (32 - o)
+                    elif o:
+                        assert (bw >> (32 - o)) == 0  # nothing lost at the end of the mask
+    return mask.astype(np.uint32)
+
+
+def _walk_model(mask, s, wlast, q):
+    """Positions the backward visits for quadrant q of a tile starting at s,
+    in visiting order, with their slot (lane) in the 32-entry staging."""
+    out = []
+    k_hi = s + wlast - 1
+    for wk in range(k_hi >> 5, (s >> 5) - 1, -1):
+        kb = wk << 5
+        wi = wk * QUADS + q
+        assert wi < len(mask)
+        bits = int(mask[wi])
+        lo = s - kb if s > kb else 0
+        hi = k_hi - kb
+        assert 0 <= lo <= 31
+        if hi < 31:
+            bits &= (2 << hi) - 1
+        bits &= ~((1 << lo) - 1) & 0xFFFFFFFF
+        while bits:
+            l = bits.bit_length() - 1
+            bits &= ~(1 << l)
+            assert 0 <= l < 32
+            out.append((kb + l, l))
+    return out
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_render_mask_words_and_backward_walk(seed):
+    """The forward's mask words equal the direct layout (bit k % 32 of word
+    (k // 32) * 4 + quadrant for every blended list position k), and the
+    backward visits exactly the blended positions up to the quadrant's last
+    contributor, back to front, each from its own staging slot k % 32."""
+    rng = np.random.default_rng(seed)
+    T = 37
+    lens = rng.integers(0, 300, T)
+    lens[rng.random(T) < 0.2] = 0
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    ranges = [(int(a), int(a + n)) for a, n in zip(starts, lens)]
+    P = int(lens.sum())
+    blended = {(k, q) for k in range(P) for q in range(QUADS) if rng.random() < 0.3}
+    mask = _mask_model(ranges, blended, P)
+    direct = np.zeros(QUADS * ((P + 31) // 32), np.uint32)
+    for k, q in blended:
+        direct[(k >> 5) * QUADS + q] |= np.uint32(1 << (k & 31))
+    np.testing.assert_array_equal(mask, direct)
+    for s, e in ranges:
+        for q in range(QUADS):
+            wlast = int(rng.integers(0, e - s + 1)) if e > s else 0
+            if wlast == 0:
+                continue
+            got = _walk_model(mask, s, wlast, q)
+            want = sorted((k for k in range(s, s + wlast) if (k, q) in blended), reverse=True)
+            assert [k for k, _ in got] == want
+            assert all(l == k % 32 for k, l in got)
