@@ -582,7 +582,8 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
             const float val = (lane == 1 ? r9 : r8) * post;
-            if (gbase && val != 0.0f) atomicAdd(gbase + (size_t)s_id[l] * gstride, val);
+            // (a zero sum is added too: testing for it costs more than the atomic)
+            if (gbase) atomicAdd(gbase + (size_t)s_id[l] * gstride, val);
         }
         __syncwarp();  // the next word reuses this warp's slots
     }
