@@ -391,6 +391,7 @@ def run_ours(args):
     # round trip, so every call is capturable) and replayed: one launch per
     # step instead of ~35 launches per view through the Python binding
     graph, graph_launches = None, 0
+    graph_spread = None
     if not args.no_graph and not exchange and adam is None:
         graph = torch.cuda.CUDAGraph()
         torch.cuda.synchronize(dev)
@@ -428,6 +429,8 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     if graph is not None:
         graph_ms = [a.elapsed_time(b) for a, b in ev]
+        srt = sorted(graph_ms)
+        graph_spread = dict(min=srt[0], median=srt[len(srt) // 2], max=srt[-1])
     if world > 1:
         dist.barrier()
     time.sleep(0.2)
@@ -558,7 +561,8 @@ def run_ours(args):
         line = dict(
             metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
             ms_per_step=total_ms / args.steps, ms_per_step_eager=eager_ms / args.steps,
-            launch_mode="cuda graph replay" if graph is not None else "eager", higher_is_better=True, scaling="weak" if not exchange else "strong",
+            launch_mode="cuda graph replay" if graph is not None else "eager", replay_ms=graph_spread,
+            higher_is_better=True, scaling="weak" if not exchange else "strong",
             vs_baseline=None, dtype="f32", data="synthetic",
             config=dict(workload=f"{sc.name}: {sc.N} Gaussians, {cam0.width}x{cam0.height}, {len(sc.cameras)} view(s), "
                                  f"16x16 tiles, fp32"
