@@ -256,9 +256,26 @@ def gs_bin_sort(cam, depth, rect, tiles_touched, d_num_pairs, capacity: int, ids
         _ptr(ids), _ptr(ranges), _ptr(keys), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def mask_words(capacity: int) -> int:
-    """Words of the contribution mask for `capacity` sorted pairs."""
-    return 4 * ((int(capacity) + 31) // 32)
+def order_words(n_tiles: int) -> int:
+    """Words of the dispatch-order block at the start of the contribution
+    mask (GS_ORDER_WORDS): per quadrant its blended-position count and the
+    backward's dispatch order, per tile the forward's dispatch order, and
+    the per-partition class counts of the quadrants."""
+    return 12 * int(n_tiles) + 256
+
+
+def mask_words(capacity: int, n_tiles: int) -> int:
+    """Words of the contribution mask (GS_MASK_WORDS) for `capacity` sorted
+    pairs on an image of `n_tiles` tiles: the dispatch-order block, then the
+    contribution bits."""
+    return order_words(n_tiles) + 4 * ((int(capacity) + 31) // 32)
+
+
+def _check_mask(cam, contrib_mask) -> None:
+    _check(contrib_mask, "contrib_mask", torch.uint32, optional=True)
+    if contrib_mask is not None and (contrib_mask.numel() < order_words(num_tiles(cam)) + 4
+                                     or contrib_mask.numel() % 4):
+        raise ValueError("contrib_mask needs a multiple of 4 words, at least mask_words(1, num_tiles(cam))")
 
 
 def gs_render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_T, n_contrib, contrib_mask=None,
@@ -273,7 +290,7 @@ def gs_render_fwd(cam, ranges, ids, mean2d, conic_opacity, colors, image, final_
     _check(image, "image", torch.float32, (3, H, W))
     _check(final_T, "final_T", torch.float32, (H, W))
     _check(n_contrib, "n_contrib", torch.uint32, (H, W))
-    _check(contrib_mask, "contrib_mask", torch.uint32, optional=True)
+    _check_mask(cam, contrib_mask)
     c = camera_struct(cam)
     _ok("gs_render_fwd", lib().gs_render_fwd(
         ctypes.byref(c), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(colors), _ptr(image),
@@ -311,7 +328,7 @@ def gs_render_bwd(cam, ranges, ids, mean2d, conic_opacity, colors, final_T, n_co
     _check(dL_dmean2d, "dL_dmean2d", torch.float32, (N, 2))
     _check(dL_dconic_opacity, "dL_dconic_opacity", torch.float32, (N, 4))
     _check(dL_dcolor, "dL_dcolor", torch.float32, (N, 3))
-    _check(contrib_mask, "contrib_mask", torch.uint32, optional=True)
+    _check_mask(cam, contrib_mask)
     c = camera_struct(cam)
     _ok("gs_render_bwd", lib().gs_render_bwd(
         ctypes.byref(c), int(N), _ptr(ranges), _ptr(ids), _ptr(mean2d), _ptr(conic_opacity), _ptr(colors),

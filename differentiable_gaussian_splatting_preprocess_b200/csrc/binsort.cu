@@ -27,10 +27,6 @@
 
 #include <cuda_runtime.h>
 
-#include <mutex>
-#include <set>
-#include <utility>
-
 #include "gs_internal.cuh"
 
 namespace gs {
@@ -1254,20 +1250,6 @@ int ceil_log2(unsigned x) {
     int b = 0;
     while ((1ull << b) < x) ++b;
     return b;
-}
-
-// Kernels that use more than the default 48 KiB of dynamic shared memory
-// must opt in once per device.  Done on first use and remembered, so later
-// calls (including calls recorded into a CUDA graph) issue no attribute call.
-template <typename Kernel>
-void opt_in_smem(Kernel kernel, size_t bytes) {
-    static std::mutex mu;
-    static std::set<std::pair<int, const void*>> done;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    std::lock_guard<std::mutex> lock(mu);
-    if (done.insert({dev, reinterpret_cast<const void*>(kernel)}).second)
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 template <int MAXB>

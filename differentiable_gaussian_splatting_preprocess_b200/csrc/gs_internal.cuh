@@ -4,6 +4,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "gs.h"
 
 namespace gs {
@@ -26,6 +30,20 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Host-side count of the kernels this library has launched (gs_launch_count);
 // called after every launch statement.
 void note_launch();
+
+// Kernels that use more than the default 48 KiB of dynamic shared memory
+// must opt in once per device.  Done on first use and remembered, so later
+// calls (including calls recorded into a CUDA graph) issue no attribute call.
+template <typename Kernel>
+void opt_in_smem(Kernel kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.insert({dev, reinterpret_cast<const void*>(kernel)}).second)
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
 
 inline int tiles_x(const gs_camera& c) { return (c.width + kTile - 1) / kTile; }
 inline int tiles_y(const gs_camera& c) { return (c.height + kTile - 1) / kTile; }

@@ -51,9 +51,8 @@ struct PixelPair {
     float sx0, sx1, sy0, sy1;  // pixel-centre rectangle of this warp's quadrant
 };
 
-__device__ __forceinline__ PixelPair pixel_pair(const gs_camera& cam, int TX) {
+__device__ __forceinline__ PixelPair pixel_pair(const gs_camera& cam, int TX, int tile) {
     PixelPair q;
-    const int tile = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bx = (tile % TX) * kTile + (warp & 1) * 8;
     const int by = (tile / TX) * kTile + (warp >> 1) * 8;
@@ -121,20 +120,37 @@ __device__ __forceinline__ void stage_cull(float2 xy, float4 co, float alpha_min
     tr = make_float4(cp.thr, cp.boc, cp.boa, 0.0f);
 }
 
+// Monotone 8-bit class of a work count, for the heaviest-first dispatch
+// order (see order_by_work): exact below 16, then 8 classes per octave (at
+// most 16 + 27 * 8 + 7 = 239).  Within a class the work differs by less than
+// 1/8.
+__device__ __forceinline__ unsigned order_code(unsigned w) {
+    if (w < 16u) return w;
+    const unsigned e = 31u - __clz(w);  // 4 .. 31
+    return 16u + (e - 4u) * 8u + ((w >> (e - 3u)) & 7u);
+}
+constexpr int kOrderCodes = 256;
+constexpr unsigned kPartUnits = 2048;  // quadrants per partition of the backward's order
+
 __global__ void __launch_bounds__(kThreads)
 k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsigned* __restrict__ ids,
              const float2* __restrict__ mean2d, const float4* __restrict__ conic_opacity,
              const float* __restrict__ colors, float* __restrict__ image, float* __restrict__ final_T,
-             unsigned* __restrict__ n_contrib, unsigned* __restrict__ cmask, unsigned cmask_words) {
+             unsigned* __restrict__ n_contrib, unsigned* __restrict__ cmask, unsigned cmask_words,
+             const unsigned* __restrict__ order, unsigned* __restrict__ quad_work,
+             unsigned* __restrict__ part_hist) {
     __shared__ float2 s_xy[kFwdBatch];
     __shared__ float4 s_co[kFwdBatch];
     __shared__ float4 s_col[kFwdBatch];
     __shared__ float4 s_box[kFwdBatch];
     __shared__ float4 s_thr[kFwdBatch];  // threshold, b / c, b / a
-    const PixelPair q = pixel_pair(cam, TX);
+    const unsigned tile = order ? order[blockIdx.x] : blockIdx.x;
+    if (tile >= gridDim.x) return;  // not a permutation of the tiles: nothing valid to do
+    const PixelPair q = pixel_pair(cam, TX, (int)tile);
     const int lane = threadIdx.x & 31;
-    const uint2 rg = checked_range(ranges[blockIdx.x]);
+    const uint2 rg = checked_range(ranges[tile]);
     const float amax = cam.alpha_max, amin = cam.alpha_min, tmin = cam.T_min;
+    unsigned n_blend_pos = 0;  // list positions blended into some pixel of this warp
 
     float2 T = make_float2(1.0f, 1.0f);
     float2 C0 = make_float2(0.0f, 0.0f), C1 = C0, C2 = C0;
@@ -206,6 +222,7 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                     break;
                 }
             }
+            n_blend_pos += __popc(blended_word);
             // record the word at global list positions b + w*32 .. b + w*32 + 31
             // (bit for position k: word (k >> 5) * 4 + warp, bit k & 31)
             if (cmask && blended_word && lane == 0) {
@@ -216,6 +233,13 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 if (o && wi + kWarps < cmask_words) atomicOr(&cmask[wi + kWarps], blended_word >> (32u - o));
             }
         }
+    }
+    // this quadrant's work for the backward's dispatch order: its count, and
+    // one more of its class in its partition's histogram
+    if (quad_work && lane == 0) {
+        const unsigned u = 4u * tile + (threadIdx.x >> 5);
+        quad_work[u] = n_blend_pos;
+        atomicAdd(&part_hist[(u / kPartUnits) * kOrderCodes + order_code(n_blend_pos)], 1u);
     }
     const size_t plane = (size_t)cam.width * cam.height;
     const size_t pix = (size_t)q.y * cam.width + q.x0;
@@ -347,7 +371,7 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     __shared__ float s_grad[kBatch * kGradStride];
     __shared__ unsigned s_max[kWarps];
 
-    const PixelPair q = pixel_pair(cam, TX);
+    const PixelPair q = pixel_pair(cam, TX, blockIdx.x);
     const int lane = threadIdx.x & 31;
     const uint2 rg = checked_range(ranges[blockIdx.x]);
     const float amax = cam.alpha_max, amin = cam.alpha_min;
@@ -476,7 +500,8 @@ k_render_bwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
 }
 
 // Backward driven by the forward's contribution mask: one CTA of one warp
-// per 8x8 quadrant (block b: tile b / 4, quadrant b % 4), so that a warp that
+// per 8x8 quadrant (block b takes unit order[b]: tile unit / 4, quadrant
+// unit % 4, the units dispatched most blended first), so that a warp that
 // finishes frees its slot at once for the next quadrant.  The warp walks the
 // mask words of its quadrant from its last contributor towards the front;
 // for each word the lanes whose bit is set load that list entry into the
@@ -494,13 +519,16 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
                   const float* __restrict__ colors, const float* __restrict__ final_T,
                   const unsigned* __restrict__ n_contrib, const unsigned* __restrict__ cmask, unsigned cmask_words,
                   const float* __restrict__ dL_dimage, float* __restrict__ dL_dmean2d,
-                  float* __restrict__ dL_dconic_opacity, float* __restrict__ dL_dcolor) {
+                  float* __restrict__ dL_dconic_opacity, float* __restrict__ dL_dcolor,
+                  const unsigned* __restrict__ order) {
     __shared__ unsigned s_id[32];
     __shared__ float2 s_xy[32];
     __shared__ float4 s_co[32];
     __shared__ float4 s_col[32];
     const int lane = threadIdx.x;
-    const int tile = blockIdx.x >> 2, quad = blockIdx.x & 3;
+    const unsigned unit = order[blockIdx.x];
+    if (unit >= gridDim.x) return;  // not a permutation of the quadrants: nothing valid to do
+    const int tile = (int)(unit >> 2), quad = (int)(unit & 3u);
     const PixelPair q = quad_pixel_pair(cam, TX, tile, quad, lane);
     const uint2 rg = checked_range(ranges[tile]);
     const float amax = cam.alpha_max, amin = cam.alpha_min;
@@ -589,6 +617,186 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
     }
 }
 
+// Dispatch order of the render CTAs, heaviest first.  The hardware starts
+// CTAs roughly in block-index order; a heavy tile that starts late (the
+// heavy tiles of a scene sit where its Gaussians crowd, anywhere in the
+// image) keeps its SM busy after the others have gone idle.  Dispatching in
+// decreasing order of work (longest processing time first) leaves the
+// light CTAs for the end.  The forward orders its tiles by list length (its
+// work before early termination is not known in advance); the backward
+// orders its quadrants by the number of list positions the forward blended
+// in them, which is the number of terms the quadrant's warp will visit.
+// The order changes which CTA runs when, never what a CTA computes.
+
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderWarps = kOrderThreads / 32;
+constexpr int kOrderCntStride = kOrderCodes + 1;  // per-warp row of class counters, padded
+constexpr int kOrderStage = 32768;                // items whose class and position stay in shared memory
+
+struct OrderSmem {
+    unsigned cnt[kOrderWarps * kOrderCntStride];  // (warp, class) at warp * 257 + class
+    unsigned wsum[kOrderWarps];
+    unsigned out[kOrderStage];                    // positions 0 .. kOrderStage-1 of the order
+    unsigned char code[kOrderStage];              // classes of items 0 .. kOrderStage-1
+};
+
+// Counting sort by one CTA of kOrderThreads threads: order[0 .. n) = the
+// items 0 .. n-1 in decreasing class (within a class in no particular order:
+// the order only decides which CTA starts when).
+//   0. the whole CTA loads the items' work counts (coalesced, many loads in
+//      flight) and keeps their classes in shared memory;
+//   1. warp w owns a contiguous run of 32-item rows and counts its items per
+//      class in its own row of counters (shared-memory atomics: lanes of one
+//      class serialise only within one instruction);
+//   2. an exclusive scan over the counters in (decreasing class, warp) order
+//      turns each into the first position of its (class, warp) group;
+//   3. each warp walks its rows again and takes positions with the same
+//      atomics; positions are gathered in shared memory and written out in
+//      order.
+// Items past kOrderStage (images of more than 8192 tiles) take the same
+// steps with their class recomputed from global memory and their position
+// stored directly.
+template <class Work>
+__device__ void order_by_work(unsigned n, Work work, unsigned* __restrict__ order, OrderSmem& sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kOrderWarps * kOrderCntStride; i += kOrderThreads) sm.cnt[i] = 0u;
+    const unsigned nc = min(n, (unsigned)kOrderStage);
+#pragma unroll 8
+    for (unsigned i = threadIdx.x; i < nc; i += kOrderThreads) sm.code[i] = (unsigned char)order_code(work(i));
+    __syncthreads();
+    const unsigned rows = (n + 31u) / 32u;
+    const unsigned per_warp = (rows + kOrderWarps - 1) / kOrderWarps;
+    const unsigned i0 = min(rows, (unsigned)warp * per_warp) * 32u + lane;
+    const unsigned i1 = min(n, min(rows, (unsigned)warp * per_warp + per_warp) * 32u);
+    unsigned* cnt = sm.cnt + warp * kOrderCntStride;
+    auto code_of = [&](unsigned i) { return i < nc ? (unsigned)sm.code[i] : order_code(work(i)); };
+    // 1. counts per (warp, class)
+#pragma unroll 4
+    for (unsigned i = i0; i < i1; i += 32u) atomicAdd(&cnt[code_of(i)], 1u);
+    __syncthreads();
+    // 2. exclusive scan; thread t takes flat entries 8t .. 8t+7, flat entry
+    // f = (255 - class) * 32 + warp
+    constexpr int per = kOrderCodes * kOrderWarps / kOrderThreads;
+    unsigned v[per], sum = 0;
+#pragma unroll
+    for (int k = 0; k < per; ++k) {
+        const unsigned f = threadIdx.x * per + k;
+        v[k] = sm.cnt[(f & 31u) * kOrderCntStride + (kOrderCodes - 1 - (f >> 5))];
+        sum += v[k];
+    }
+    unsigned incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) sm.wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned t = sm.wsum[lane];
+        unsigned ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += y;
+        }
+        sm.wsum[lane] = ti - t;
+    }
+    __syncthreads();
+    unsigned run = sm.wsum[warp] + incl - sum;
+#pragma unroll
+    for (int k = 0; k < per; ++k) {
+        const unsigned f = threadIdx.x * per + k;
+        sm.cnt[(f & 31u) * kOrderCntStride + (kOrderCodes - 1 - (f >> 5))] = run;
+        run += v[k];
+    }
+    __syncthreads();
+    // 3. positions
+#pragma unroll 4
+    for (unsigned i = i0; i < i1; i += 32u) {
+        const unsigned pos = atomicAdd(&cnt[code_of(i)], 1u);
+        if (pos < (unsigned)kOrderStage) sm.out[pos] = i;
+        else order[pos] = i;
+    }
+    __syncthreads();
+    for (unsigned p = threadIdx.x; p < nc; p += kOrderThreads) order[p] = sm.out[p];
+}
+
+__device__ __forceinline__ void zero_words(unsigned* __restrict__ a, size_t n, size_t first, size_t stride) {
+    for (size_t i = first; i < n; i += stride) a[i] = 0u;
+}
+
+// Before the forward: block 0 orders the tiles by list length into
+// tile_order[T]; the other blocks zero the backward's partition histograms
+// and the contribution bits (one range).  Launched with
+// sizeof(OrderSmem) bytes of dynamic shared memory (every block gets them;
+// one block uses them).
+__global__ void __launch_bounds__(kOrderThreads, 1)
+k_fwd_prep(int T, const uint2* __restrict__ ranges, unsigned* __restrict__ tile_order, unsigned* __restrict__ bits,
+           size_t n_bits) {
+    if (blockIdx.x == 0) {
+        extern __shared__ __align__(16) unsigned char order_smem[];
+        order_by_work((unsigned)T, [&](unsigned t) { const uint2 r = ranges[t]; return r.y - r.x; }, tile_order,
+                      *reinterpret_cast<OrderSmem*>(order_smem));
+        return;
+    }
+    zero_words(bits, n_bits, (size_t)(blockIdx.x - 1) * kOrderThreads + threadIdx.x,
+               (size_t)(gridDim.x - 1) * kOrderThreads);
+}
+
+// Before the backward: blocks 0 .. P-1 order the 4T quadrants by the
+// forward's blended-position counts into quad_order[4T] (decreasing class);
+// the other blocks zero the gradient outputs.  The forward counted every
+// partition's quadrants per class (part_hist[p][c], partition p = quadrants
+// p * kPartUnits ..), so block p knows where each class begins for its
+// quadrants - after every quadrant of a higher class, and after those of its
+// class in lower partitions - and places them with shared-memory atomics
+// (within a class in no particular order).
+__global__ void __launch_bounds__(kOrderThreads)
+k_bwd_prep(int T, int P, const unsigned* __restrict__ quad_work, const unsigned* __restrict__ part_hist,
+           unsigned* __restrict__ quad_order, float* __restrict__ a, size_t na, float* __restrict__ b, size_t nb,
+           float* __restrict__ c, size_t nc) {
+    if ((int)blockIdx.x < P) {
+        __shared__ unsigned s_cur[kOrderCodes];
+        __shared__ unsigned s_w[kOrderCodes / 32];
+        const int p = blockIdx.x, t = threadIdx.x, lane = t & 31;
+        unsigned tot = 0, before = 0;
+        if (t < kOrderCodes) {
+            const int cls = kOrderCodes - 1 - t;  // thread t: classes in decreasing order
+            for (int q = 0; q < P; ++q) {
+                const unsigned h = part_hist[q * kOrderCodes + cls];
+                tot += h;
+                before += q < p ? h : 0u;
+            }
+        }
+        // exclusive scan of the class totals in decreasing class order
+        unsigned incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (t < kOrderCodes && lane == 31) s_w[t >> 5] = incl;
+        __syncthreads();
+        if (t < kOrderCodes) {
+            unsigned above = incl - tot;
+            for (int w = 0; w < (t >> 5); ++w) above += s_w[w];
+            s_cur[kOrderCodes - 1 - t] = above + before;
+        }
+        __syncthreads();
+        const unsigned n = 4u * (unsigned)T;
+        const unsigned u1 = min(n, (unsigned)(p + 1) * kPartUnits);
+        for (unsigned u = (unsigned)p * kPartUnits + t; u < u1; u += kOrderThreads)
+            quad_order[atomicAdd(&s_cur[order_code(quad_work[u])], 1u)] = u;
+        return;
+    }
+    const size_t first = (size_t)(blockIdx.x - P) * kOrderThreads + threadIdx.x;
+    const size_t stride = (size_t)(gridDim.x - P) * kOrderThreads;
+    zero_words(reinterpret_cast<unsigned*>(a), na, first, stride);
+    zero_words(reinterpret_cast<unsigned*>(b), nb, first, stride);
+    zero_words(reinterpret_cast<unsigned*>(c), nc, first, stride);
+}
+
 // Work counts of the forward, per pixel: list entries evaluated before the
 // pixel stopped (the stopping entry included) and terms blended.  One thread
 // per pixel walking its tile's list in order with the same term evaluation as
@@ -632,6 +840,42 @@ __global__ void k_zero(float* __restrict__ a, size_t na, float* __restrict__ b, 
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nc; i += stride) c[i] = 0.0f;
 }
 
+// The contribution-mask buffer: the dispatch-order block, then the bits.
+struct MaskParts {
+    unsigned* quad_work = nullptr;    // [4T] blended positions per quadrant (forward output)
+    unsigned* quad_order = nullptr;   // [4T] backward dispatch order
+    unsigned* tile_order = nullptr;   // [T] forward dispatch order
+    unsigned* part_hist = nullptr;    // [P][256] quadrants per (partition, class) (forward output)
+    unsigned* bits = nullptr;         // contribution bits
+    unsigned bits_words = 0;
+    unsigned prep_words = 0;          // words from part_hist to the end: zeroed before the forward
+    int parts = 0;                    // P = ceil(4T / kPartUnits)
+};
+
+// Splits a caller's mask buffer; false if it is too small or not a multiple
+// of 4 words.
+bool mask_parts(unsigned* mask, unsigned mask_words, int T, MaskParts& m) {
+    if (!mask) return true;
+    const size_t order_words = 12 * (size_t)T + 256;  // GS_ORDER_WORDS
+    if (mask_words % kWarps != 0 || (size_t)mask_words < order_words + kWarps) return false;
+    m.parts = (int)((4 * (size_t)T + kPartUnits - 1) / kPartUnits);
+    m.quad_work = mask;
+    m.quad_order = mask + 4 * (size_t)T;
+    m.tile_order = mask + 8 * (size_t)T;
+    m.part_hist = mask + 9 * (size_t)T;  // P * 256 <= T / 2 + 256 words, inside the block
+    m.bits = mask + order_words;
+    m.bits_words = mask_words - (unsigned)order_words;
+    m.prep_words = mask_words - 9 * (unsigned)T;
+    return true;
+}
+
+// Blocks of a prep kernel: the ordering block plus enough to zero `words`
+// words, at most one block per SM in all (each holds sizeof(OrderSmem)).
+int prep_blocks(size_t words) {
+    const size_t z = (words + kOrderThreads - 1) / kOrderThreads;
+    return 1 + (int)(z < 147 ? z : 147);
+}
+
 }  // namespace
 }  // namespace gs
 
@@ -641,21 +885,22 @@ extern "C" int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const
                              const float* conic_opacity, const float* colors, float* image, float* final_T,
                              unsigned* n_contrib, unsigned* contrib_mask, unsigned mask_words, void* stream) {
     if (!camera_ok(cam) || !ranges || !image || !final_T || !n_contrib) return GS_ERR_INVALID_ARG;
-    if (contrib_mask && (mask_words == 0 || mask_words % kWarps != 0)) return GS_ERR_INVALID_ARG;
     if (!aligned(ranges, 8) || (conic_opacity && !aligned(conic_opacity, 16)) || (mean2d && !aligned(mean2d, 8)))
         return GS_ERR_INVALID_ARG;
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
+    MaskParts m;
+    if (!mask_parts(contrib_mask, mask_words, T, m)) return GS_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     if (contrib_mask) {
-        int blocks = (int)((mask_words + 255u) / 256u);
-        if (blocks > 148 * 8) blocks = 148 * 8;
-        k_zero<<<blocks, 256, 0, st>>>(reinterpret_cast<float*>(contrib_mask), mask_words, nullptr, 0, nullptr, 0); note_launch();
+        opt_in_smem(k_fwd_prep, sizeof(OrderSmem));
+        k_fwd_prep<<<prep_blocks(m.prep_words), kOrderThreads, sizeof(OrderSmem), st>>>(
+            T, reinterpret_cast<const uint2*>(ranges), m.tile_order, m.part_hist, m.prep_words); note_launch();
         GS_LAUNCH_CHECK();
     }
     k_render_fwd<<<T, kThreads, 0, st>>>(
         *cam, TX, reinterpret_cast<const uint2*>(ranges), ids, reinterpret_cast<const float2*>(mean2d),
-        reinterpret_cast<const float4*>(conic_opacity), colors, image, final_T, n_contrib, contrib_mask,
-        contrib_mask ? mask_words : 0u); note_launch();
+        reinterpret_cast<const float4*>(conic_opacity), colors, image, final_T, n_contrib, m.bits, m.bits_words,
+        m.tile_order, m.quad_work, m.part_hist); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
@@ -670,31 +915,39 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
     if (!aligned(ranges, 8) || (conic_opacity && !aligned(conic_opacity, 16)) || (mean2d && !aligned(mean2d, 8)) ||
         (dL_dmean2d && !aligned(dL_dmean2d, 8)) || (dL_dconic_opacity && !aligned(dL_dconic_opacity, 16)))
         return GS_ERR_INVALID_ARG;
-    cudaStream_t st = (cudaStream_t)stream;
-    if (N > 0) {
-        size_t work = (size_t)N * 4;
-        int blocks = (int)((work + 255) / 256);
-        if (blocks > 148 * 8) blocks = 148 * 8;
-        k_zero<<<blocks, 256, 0, st>>>(dL_dmean2d, (size_t)N * 2, dL_dconic_opacity, (size_t)N * 4, dL_dcolor,
-                                       (size_t)N * 3); note_launch();
-        GS_LAUNCH_CHECK();
-    }
     const int TX = tiles_x(*cam), T = TX * tiles_y(*cam);
+    // the buffer is only read here, except for the backward's own dispatch order
+    MaskParts m;
+    if (!mask_parts(const_cast<unsigned*>(contrib_mask), mask_words, T, m)) return GS_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t n = (size_t)N;
     if (contrib_mask) {
+        const size_t z = (n * 4 + kOrderThreads - 1) / kOrderThreads;
+        const int zb = (int)(z < 148 * 2 ? (z ? z : 1) : 148 * 2);
+        k_bwd_prep<<<m.parts + zb, kOrderThreads, 0, st>>>(T, m.parts, m.quad_work, m.part_hist, m.quad_order,
+                                                           dL_dmean2d, n * 2, dL_dconic_opacity, n * 4, dL_dcolor,
+                                                           n * 3); note_launch();
+        GS_LAUNCH_CHECK();
         k_render_bwd_warp<<<4 * T, 32, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
                                                   reinterpret_cast<const float2*>(mean2d),
                                                   reinterpret_cast<const float4*>(conic_opacity), colors, final_T,
-                                                  n_contrib, contrib_mask, mask_words, dL_dimage, dL_dmean2d,
-                                                  dL_dconic_opacity, dL_dcolor); note_launch();
+                                                  n_contrib, m.bits, m.bits_words, dL_dimage, dL_dmean2d,
+                                                  dL_dconic_opacity, dL_dcolor, m.quad_order); note_launch();
         GS_LAUNCH_CHECK();
         return GS_OK;
     }
+    if (N > 0) {
+        int blocks = (int)((n * 4 + 255) / 256);
+        if (blocks > 148 * 8) blocks = 148 * 8;
+        k_zero<<<blocks, 256, 0, st>>>(dL_dmean2d, n * 2, dL_dconic_opacity, n * 4, dL_dcolor, n * 3); note_launch();
+        GS_LAUNCH_CHECK();
+    }
     auto kernel = k_render_bwd<false>;
     kernel<<<T, kThreads, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
-                                       reinterpret_cast<const float2*>(mean2d),
-                                       reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
-                                       contrib_mask, contrib_mask ? mask_words : 0u, dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),
-                                       reinterpret_cast<float4*>(dL_dconic_opacity), dL_dcolor); note_launch();
+                                   reinterpret_cast<const float2*>(mean2d),
+                                   reinterpret_cast<const float4*>(conic_opacity), colors, final_T, n_contrib,
+                                   nullptr, 0u, dL_dimage, reinterpret_cast<float2*>(dL_dmean2d),
+                                   reinterpret_cast<float4*>(dL_dconic_opacity), dL_dcolor); note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

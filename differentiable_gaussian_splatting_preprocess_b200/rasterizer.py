@@ -107,7 +107,8 @@ class Rasterizer:
         image = self._buf("image", (3, H, W), torch.float32)
         final_T = self._buf("final_T", (H, W), torch.float32)
         n_contrib = self._buf("n_contrib", (H, W), torch.uint32)
-        cmask = self._buf("contrib_mask", (B.mask_words(max(capacity, 1)),), torch.uint32) if use_mask else None
+        cmask = (self._buf("contrib_mask", (B.mask_words(max(capacity, 1), B.num_tiles(self.cam)),), torch.uint32)
+                 if use_mask else None)
         if colors_ready is not None:
             (stream or torch.cuda.current_stream(self.device)).wait_event(colors_ready)
         B.gs_render_fwd(self.cam, ranges, ids, pre["mean2d"], pre["conic_opacity"], colors, image, final_T,

@@ -224,16 +224,33 @@ GS_API int gs_bin_sort(const gs_camera* cam, int N, const float* depth, const in
  * Outputs: image [3,H,W]; final_T [H,W]; n_contrib [H,W] uint32 = list
  *   position (within the tile) of the last blended term plus one.
  * colors [N,3] are indexed by the ids in `ids`.
- * contrib_mask (optional, may be NULL) receives, for every sorted position k
- *   and every 8x8 quadrant q of k's tile (row-major: top-left, top-right,
- *   bottom-left, bottom-right), bit (k & 31) of word (k >> 5) * 4 + q set when
- *   that Gaussian was blended into at least one pixel of the quadrant.  The
- *   call zeroes the first `mask_words` words, which must be a multiple of 4 and
- *   at least GS_MASK_WORDS(number of sorted pairs).  gs_render_bwd uses it to
- *   walk only the terms that contribute.
+ * contrib_mask (optional, may be NULL; mask_words words, a multiple of 4 and
+ *   at least GS_ORDER_WORDS(T) + 4) is the forward's record for gs_render_bwd,
+ *   in two parts:
+ *   - words [0, GS_ORDER_WORDS(T)): the dispatch-order block.  Words [0, 4T)
+ *     receive, per 8x8 quadrant q of tile t, the number of list positions
+ *     blended into at least one of its pixels (word 4t + q); words [4T, 8T)
+ *     receive the order in which gs_render_bwd dispatches those 4T quadrants
+ *     (most blended first); words [8T, 9T) the order in which this call
+ *     dispatched its tiles (longest list first); words from 9T on hold the
+ *     per-partition counts of quadrants by work class (256 words for each
+ *     2048 quadrants) that gs_render_bwd's ordering reads; the rest is
+ *     unused.  The orders change only the scheduling, never a result.
+ *   - words GS_ORDER_WORDS(T) onwards: the contribution bits.  For every
+ *     sorted position k and every 8x8 quadrant q of k's tile (row-major:
+ *     top-left, top-right, bottom-left, bottom-right), bit (k & 31) of word
+ *     GS_ORDER_WORDS(T) + (k >> 5) * 4 + q is set when that Gaussian was
+ *     blended into at least one pixel of the quadrant.  The call zeroes these
+ *     words; there should be at least GS_MASK_WORDS(P, T) - GS_ORDER_WORDS(T)
+ *     of them for P sorted pairs (positions beyond the buffer are not
+ *     recorded, and the backward then visits them all: correct, slower).
+ *   gs_render_bwd uses the bits to walk only the terms that contribute.
  */
-/* Words of the optional contribution mask for `capacity` sorted pairs. */
-#define GS_MASK_WORDS(capacity) (4u * (((unsigned)(capacity) + 31u) / 32u))
+/* Words of the dispatch-order block for an image of `n_tiles` tiles. */
+#define GS_ORDER_WORDS(n_tiles) (12u * (unsigned)(n_tiles) + 256u)
+/* Words of the optional contribution mask for `capacity` sorted pairs on an
+   image of `n_tiles` tiles. */
+#define GS_MASK_WORDS(capacity, n_tiles) (GS_ORDER_WORDS(n_tiles) + 4u * (((unsigned)(capacity) + 31u) / 32u))
 
 GS_API int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const unsigned* ids, const float* mean2d,
                   const float* conic_opacity, const float* colors, float* image, float* final_T,
@@ -261,7 +278,10 @@ GS_API int gs_render_stats(const gs_camera* cam, const unsigned* ranges, const u
  *   dL/d(u, v) = G dL/dG (a dx + b dy, b dx + c dy).
  * contrib_mask / mask_words: the forward's mask (see gs_render_fwd), or NULL
  *   to let the backward find the contributing terms itself (slower; same
- *   results up to the order of floating-point sums).
+ *   results up to the order of floating-point sums).  With the mask, the
+ *   call first writes its dispatch order (words [4T, 8T) of the block) from
+ *   the forward's per-quadrant counts, then dispatches one warp per quadrant
+ *   in that order.
  * Outputs (OVERWRITTEN; the call zeroes them first): dL_dmean2d [N,2];
  *   dL_dconic_opacity [N,4] = (dL/da, dL/db, dL/dc, dL/dopacity);
  *   dL_dcolor [N,3].  Summation order across pixels is unspecified

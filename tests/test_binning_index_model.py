@@ -290,3 +290,142 @@ def test_render_mask_words_and_backward_walk(seed):
             want = sorted((k for k in range(s, s + wlast) if (k, q) in blended), reverse=True)
             assert [k for k, _ in got] == want
             assert all(l == k % 32 for k, l in got)
+
+
+# ---------------------------------------------------------------------------
+# Dispatch order of the render CTAs (csrc/render.cu, order_by_work): one CTA
+# of 32 warps sorts n work counts into decreasing 8-bit classes, with the
+# classes and positions of the first 32768 items kept in shared memory.
+
+ORDER_THREADS = 1024
+ORDER_WARPS = 32
+ORDER_CODES = 256
+ORDER_STRIDE = ORDER_CODES + 1
+ORDER_CNT = ORDER_WARPS * ORDER_STRIDE
+ORDER_STAGE = 32768
+
+
+def _order_code(w):
+    if w < 16:
+        return w
+    e = w.bit_length() - 1
+    return 16 + (e - 4) * 8 + ((w >> (e - 3)) & 7)
+
+
+def _order_model(work):
+    """The kernel's phases warp by warp (lanes of one instruction in lane
+    order; the kernel's atomics may take any order, which moves items only
+    within their (class, warp) group); asserts that every shared-memory and
+    output index stays inside its buffer and that the scan's counter reads
+    of one warp instruction fall in distinct banks."""
+    n = len(work)
+    nc = min(n, ORDER_STAGE)
+    code = [_order_code(work[i]) for i in range(nc)]
+    cnt = [0] * ORDER_CNT
+    rows = (n + 31) // 32
+    per_warp = (rows + ORDER_WARPS - 1) // ORDER_WARPS
+
+    def items(w):
+        i0 = min(rows, w * per_warp) * 32
+        i1 = min(n, min(rows, w * per_warp + per_warp) * 32)
+        return range(i0, i1)
+
+    def code_of(i):
+        return code[i] if i < nc else _order_code(work[i])
+
+    for w in range(ORDER_WARPS):
+        for i in items(w):
+            x = w * ORDER_STRIDE + code_of(i)
+            assert 0 <= x < ORDER_CNT
+            cnt[x] += 1
+    per = ORDER_CODES * ORDER_WARPS // ORDER_THREADS
+
+    def flat_addr(f):
+        return (f & 31) * ORDER_STRIDE + (ORDER_CODES - 1 - (f >> 5))
+
+    for t0 in range(0, ORDER_THREADS, 32):
+        for k in range(per):
+            assert len({flat_addr((t0 + l) * per + k) % 32 for l in range(32)}) == 32
+    assert sorted(flat_addr(f) for f in range(ORDER_CODES * ORDER_WARPS)) == \
+        sorted(w * ORDER_STRIDE + c for w in range(ORDER_WARPS) for c in range(ORDER_CODES))
+    run = 0
+    for f in range(ORDER_CODES * ORDER_WARPS):
+        x = flat_addr(f)
+        cnt[x], run = run, run + cnt[x]
+    assert run == n
+    order = [None] * n
+    staged = [None] * ORDER_STAGE
+    for w in range(ORDER_WARPS):
+        for i in items(w):
+            x = w * ORDER_STRIDE + code_of(i)
+            pos = cnt[x]
+            cnt[x] += 1
+            assert 0 <= pos < n
+            if pos < ORDER_STAGE:
+                assert staged[pos] is None
+                staged[pos] = i
+            else:
+                assert order[pos] is None
+                order[pos] = i
+    for p in range(nc):
+        order[p] = staged[p]
+    return order
+
+
+def test_order_code_is_monotone_and_fits_a_byte():
+    prev = -1
+    for w in sorted(set(list(range(0, 5000)) + [2 ** k + d for k in range(12, 32) for d in (-1, 0, 1)] + [2 ** 32 - 1])):
+        c = _order_code(w)
+        assert prev <= c <= 239
+        prev = c
+    assert _order_code(15) == 15 and _order_code(16) == 16 and _order_code(2 ** 32 - 1) == 239
+
+
+@pytest.mark.parametrize("n", [1, 31, 33, 1023, 1025, 8160, 32640, 32769, 70001])
+def test_order_by_work_is_a_heaviest_first_permutation(n):
+    """The output is a permutation of 0 .. n-1 in decreasing work class, for
+    sizes that leave warps empty, end in a partial row or pass the
+    shared-memory staging."""
+    rng = np.random.default_rng(n)
+    work = [int(x) for x in rng.integers(0, 400, n)]
+    for i in rng.choice(n, size=min(n, 5), replace=False):
+        work[int(i)] = int(rng.integers(0, 2 ** 32))
+    order = _order_model(work)
+    assert sorted(order) == list(range(n))
+    codes = [_order_code(work[i]) for i in order]
+    assert all(a >= b for a, b in zip(codes, codes[1:]))
+
+
+PART_UNITS = 2048
+
+
+@pytest.mark.parametrize("T", [1, 16, 85, 103, 256, 2500, 8160])
+def test_backward_order_from_partition_histograms(T):
+    """The backward's order (csrc/render.cu, k_bwd_prep): the forward counts
+    the quadrants of every partition of 2048 per class; block p starts class
+    c after all quadrants of higher classes and after class c's quadrants in
+    partitions below p.  The result is a permutation of the 4T quadrants in
+    decreasing class, and the histograms fit the block between words 9T and
+    GS_ORDER_WORDS(T) = 12T + 256."""
+    rng = np.random.default_rng(T)
+    n = 4 * T
+    work = [int(x) for x in rng.integers(0, 600, n)]
+    P = (n + PART_UNITS - 1) // PART_UNITS
+    assert 9 * T + P * ORDER_CODES <= 12 * T + 256
+    hist = [[0] * ORDER_CODES for _ in range(P)]
+    for u in range(n):
+        hist[u // PART_UNITS][_order_code(work[u])] += 1
+    order = [None] * n
+    for p in range(P):
+        cur = [0] * ORDER_CODES
+        for c in range(ORDER_CODES):
+            above = sum(hist[q][c2] for q in range(P) for c2 in range(c + 1, ORDER_CODES))
+            cur[c] = above + sum(hist[q][c] for q in range(p))
+        for u in range(p * PART_UNITS, min(n, (p + 1) * PART_UNITS)):
+            c = _order_code(work[u])
+            pos = cur[c]
+            cur[c] += 1
+            assert 0 <= pos < n and order[pos] is None
+            order[pos] = u
+    codes = [_order_code(work[u]) for u in order]
+    assert all(a >= b for a, b in zip(codes, codes[1:]))

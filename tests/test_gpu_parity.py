@@ -406,10 +406,42 @@ def test_render_stats_match_oracle_counts(cfg):
     assert np.all(to_np(nb) <= g["n_contrib"])
 
 
+def _work_class(w: np.ndarray) -> np.ndarray:
+    """The render's 8-bit dispatch class: exact below 16, then 8 classes per octave."""
+    w = w.astype(np.int64)
+    e = np.floor(np.log2(np.maximum(w, 1))).astype(np.int64)
+    return np.where(w < 16, w, 16 + (e - 4) * 8 + ((w >> np.maximum(e - 3, 0)) & 7))
+
+
+def _check_dispatch_order(mask: np.ndarray, ranges: np.ndarray, blend_mask: np.ndarray) -> None:
+    """The dispatch-order block after a forward and a backward with the mask:
+    per quadrant the number of its blended positions (from the oracle's
+    contribution bits), the forward's tile order (a permutation of the tiles
+    in decreasing class of list length) and the backward's quadrant order (a
+    permutation of the quadrants in decreasing class of those counts)."""
+    T = ranges.shape[0]
+    rg = ranges.astype(np.int64)
+    L = rg[:, 1] - rg[:, 0]
+    k = np.concatenate([np.arange(a, b) for a, b in rg if b > a]) if L.sum() else np.zeros(0, np.int64)
+    tile_of = np.repeat(np.arange(T), L)
+    words = blend_mask.reshape(-1, 4)
+    want_work = np.zeros((T, 4), np.int64)
+    for q in range(4):
+        bit = (words[k >> 5, q] >> (k & 31).astype(np.uint32)) & 1
+        want_work[:, q] = np.bincount(tile_of, weights=bit, minlength=T).astype(np.int64)
+    quad_work = mask[:4 * T].astype(np.int64)
+    np.testing.assert_array_equal(quad_work, want_work.reshape(-1))
+    for order, work in ((mask[4 * T:8 * T].astype(np.int64), quad_work), (mask[8 * T:9 * T].astype(np.int64), L)):
+        np.testing.assert_array_equal(np.sort(order), np.arange(work.size))
+        assert np.all(np.diff(_work_class(work[order])) <= 0)
+
+
 @pytest.mark.parametrize("cfg", [2, 3, 4])
 def test_contribution_mask_and_backward_without_it(cfg):
     """The forward's per-quadrant contribution mask equals the oracle's bit for
-    bit, and the backward gives the same gradients with and without it."""
+    bit, the dispatch-order block holds the per-quadrant counts and the two
+    heaviest-first orders, and the backward gives the same gradients with and
+    without the mask."""
     sc = _scene(cfg)
     cam = sc.cameras[0]
     gs = GpuScene(sc)
@@ -420,7 +452,9 @@ def test_contribution_mask_and_backward_without_it(cfg):
     o = oracle.render_fwd(cam, g["ranges"], g["ids"], g["mean2d"], g["conic_opacity"], sc.colors, "f32",
                           blend_mask=True)
     words = 4 * ((P + 31) // 32)
-    np.testing.assert_array_equal(to_np(fr.contrib_mask)[:words], o["blend_mask"][:words])
+    ow = B.order_words(B.num_tiles(cam))
+    np.testing.assert_array_equal(to_np(fr.contrib_mask)[ow:ow + words], o["blend_mask"][:words])
+    _check_dispatch_order(to_np(fr.contrib_mask), g["ranges"], o["blend_mask"])
     with_mask = {k: to_np(r["grads"][k]).copy() for k in ("dL_dmean2d", "dL_dconic_opacity", "dL_dcolor")}
     outs = {k: torch.empty_like(r["grads"][k]) for k in with_mask}
     B.gs_render_bwd(cam, fr.ranges, fr.ids, fr.mean2d, fr.conic_opacity, gs.colors, fr.final_T, fr.n_contrib,
