@@ -998,52 +998,86 @@ __global__ void k_cell_ranges(const unsigned* __restrict__ ckeys, const unsigned
     }
 }
 
+// Exclusive scan of one value per thread across a CTA of 1024 threads;
+// returns this thread's exclusive prefix, and the total in *total.
+__device__ __forceinline__ unsigned block_exclusive_scan(unsigned x, unsigned* s_w, unsigned* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    __syncthreads();  // s_w of an earlier call is consumed
+    if (lane == 31) s_w[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned t = s_w[lane];
+        unsigned ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += y;
+        }
+        s_w[lane] = ti - t;
+        if (lane == 31) s_w[32] = ti;
+    }
+    __syncthreads();
+    *total = s_w[32];
+    return s_w[warp] + incl - x;
+}
+
 // Segments of the cell lists (one CTA): cell c gets ceil(len / kSeg)
-// segments, numbered in cell order; cell_seg0[c] is its first.
+// segments, numbered in cell order; cell_seg0[c] is its first.  The ranges
+// and first segments of up to kSegCache cells stay in shared memory for the
+// second phase (one warp per cell, one lane per segment: coalesced writes).
+constexpr int kSegCache = 2048;
+
 __global__ void __launch_bounds__(1024)
 k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restrict__ cell_seg0,
             unsigned* __restrict__ seg_cell, unsigned* __restrict__ seg_lo, unsigned* __restrict__ seg_hi,
             SortMisc* __restrict__ misc) {
-    __shared__ unsigned s_w[32];
+    __shared__ unsigned s_w[33];
+    __shared__ uint2 s_rg[kSegCache];
+    __shared__ unsigned s_s0[kSegCache];
+    const uint2* rg2 = reinterpret_cast<const uint2*>(cell_ranges);
     const int per = (S + 1023) / 1024;
     const int c0 = threadIdx.x * per;
     unsigned local = 0;
     for (int k = 0; k < per; ++k) {
         const int c = c0 + k;
-        if (c < S) local += (cell_ranges[2 * c + 1] - cell_ranges[2 * c] + kSeg - 1) / kSeg;
+        if (c < S) {
+            const uint2 r = rg2[c];
+            if (c < kSegCache) s_rg[c] = r;
+            local += (r.y - r.x + kSeg - 1) / kSeg;
+        }
     }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    if (lane == 31) s_w[warp] = incl;
-    __syncthreads();
-    unsigned wbase = 0;
-    for (int k = 0; k < warp; ++k) wbase += s_w[k];
-    unsigned run = wbase + incl - local;
+    unsigned total;
+    unsigned run = block_exclusive_scan(local, s_w, &total);
     for (int k = 0; k < per; ++k) {
         const int c = c0 + k;
         if (c < S) {
+            const uint2 r = c < kSegCache ? s_rg[c] : rg2[c];
             cell_seg0[c] = run;
-            run += (cell_ranges[2 * c + 1] - cell_ranges[2 * c] + kSeg - 1) / kSeg;
+            if (c < kSegCache) s_s0[c] = run;
+            run += (r.y - r.x + kSeg - 1) / kSeg;
         }
     }
-    if (threadIdx.x == 1023) {
-        cell_seg0[S] = run;
-        misc->nseg = run;
+    if (threadIdx.x == 0) {
+        cell_seg0[S] = total;
+        misc->nseg = total;
     }
     __syncthreads();
     // one warp per cell writes the cell's segments, one lane per segment
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int c = warp; c < S; c += 32) {
-        const unsigned a = cell_ranges[2 * c], b = cell_ranges[2 * c + 1], s0 = cell_seg0[c];
-        for (unsigned j = lane; a + j * kSeg < b; j += 32) {
-            const unsigned lo = a + j * kSeg;
+        const uint2 r = c < kSegCache ? s_rg[c] : rg2[c];
+        const unsigned s0 = c < kSegCache ? s_s0[c] : cell_seg0[c];
+        for (unsigned j = lane; r.x + j * kSeg < r.y; j += 32) {
+            const unsigned lo = r.x + j * kSeg;
             seg_cell[s0 + j] = (unsigned)c;
             seg_lo[s0 + j] = lo;
-            seg_hi[s0 + j] = min(b, lo + kSeg);
+            seg_hi[s0 + j] = min(r.y, lo + kSeg);
         }
     }
 }
@@ -1112,7 +1146,8 @@ k_seg_count(int SX, const unsigned* __restrict__ clist, const int4* __restrict__
 }
 
 // One thread per (cell, tile bit): exclusive prefix of the per-segment
-// counts over the cell's segments, and the tile's total.
+// counts over the cell's segments, and the tile's total.  Eight segments'
+// counts are loaded at a time, so their latencies overlap.
 __global__ void __launch_bounds__(kCellTiles)
 k_cell_scan(int TX, int TY, int SX, const unsigned* __restrict__ cell_seg0, const unsigned* __restrict__ seg_cnt,
             unsigned* __restrict__ seg_base, unsigned* __restrict__ tile_cnt) {
@@ -1120,7 +1155,18 @@ k_cell_scan(int TX, int TY, int SX, const unsigned* __restrict__ cell_seg0, cons
     const int b = threadIdx.x;
     const unsigned k0 = cell_seg0[c], k1 = cell_seg0[c + 1];
     unsigned run = 0;
-    for (unsigned k = k0; k < k1; ++k) {
+    unsigned k = k0;
+    for (; k + 8 <= k1; k += 8) {
+        unsigned v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = seg_cnt[(size_t)(k + j) * kCellTiles + b];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            seg_base[(size_t)(k + j) * kCellTiles + b] = run;
+            run += v[j];
+        }
+    }
+    for (; k < k1; ++k) {
         const unsigned v = seg_cnt[(size_t)k * kCellTiles + b];
         seg_base[(size_t)k * kCellTiles + b] = run;
         run += v;
@@ -1131,15 +1177,22 @@ k_cell_scan(int TX, int TY, int SX, const unsigned* __restrict__ cell_seg0, cons
 
 // Exclusive scan of the tile counts in tile order (one CTA, 4096 tiles per
 // round, four consecutive tiles per thread): tile starts and ranges; empty
-// tiles get (0, 0).
+// tiles get (0, 0).  Each round's results are gathered in shared memory
+// (padded: one spare word per 32) and written out with consecutive threads
+// on consecutive tiles.
+constexpr int kTileRound = 4096;
+
+__device__ __forceinline__ int pad32(int i) { return i + (i >> 5); }
+
 __global__ void __launch_bounds__(1024)
 k_tile_scan(int T, const unsigned* __restrict__ tile_cnt, unsigned* __restrict__ tile_start,
             unsigned* __restrict__ ranges) {
-    __shared__ unsigned s_w[32];
-    __shared__ unsigned s_carry;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) s_carry = 0u;
-    for (int t0 = 0; t0 < T; t0 += 4096) {
+    __shared__ unsigned s_w[33];
+    __shared__ unsigned s_start[kTileRound + kTileRound / 32];
+    __shared__ unsigned s_cnt[kTileRound + kTileRound / 32];
+    uint2* rg2 = reinterpret_cast<uint2*>(ranges);
+    unsigned carry = 0;
+    for (int t0 = 0; t0 < T; t0 += kTileRound) {
         const int t = t0 + 4 * threadIdx.x;
         unsigned v[4], local = 0;
 #pragma unroll
@@ -1147,29 +1200,23 @@ k_tile_scan(int T, const unsigned* __restrict__ tile_cnt, unsigned* __restrict__
             v[j] = t + j < T ? tile_cnt[t + j] : 0u;
             local += v[j];
         }
-        unsigned incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        __syncthreads();  // s_w and s_carry of the previous round are consumed
-        if (lane == 31) s_w[warp] = incl;
-        __syncthreads();
-        unsigned wbase = 0;
-        for (int k = 0; k < warp; ++k) wbase += s_w[k];
-        unsigned run = s_carry + wbase + incl - local;
+        unsigned total;
+        unsigned run = carry + block_exclusive_scan(local, s_w, &total);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            if (t + j < T) {
-                tile_start[t + j] = run;
-                ranges[2 * (t + j)] = v[j] ? run : 0u;
-                ranges[2 * (t + j) + 1] = v[j] ? run + v[j] : 0u;
-            }
+            s_start[pad32(4 * threadIdx.x + j)] = run;
+            s_cnt[pad32(4 * threadIdx.x + j)] = v[j];
             run += v[j];
         }
-        __syncthreads();  // every thread has read s_carry
-        if (threadIdx.x == 1023) s_carry = run;
+        __syncthreads();
+        const int nr = min(kTileRound, T - t0);
+        for (int i = threadIdx.x; i < nr; i += 1024) {
+            const unsigned st = s_start[pad32(i)], n = s_cnt[pad32(i)];
+            tile_start[t0 + i] = st;
+            rg2[t0 + i] = n ? make_uint2(st, st + n) : make_uint2(0u, 0u);
+        }
+        carry += total;
+        __syncthreads();  // s_start / s_cnt are rewritten next round
     }
 }
 
@@ -1320,6 +1367,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     if (!aligned(ws, 256) || ws_bytes < gs_bin_sort_ws_bytes(N, capacity, cam->width, cam->height))
         return GS_ERR_INVALID_ARG;
     if (rect && !aligned(rect, 16)) return GS_ERR_INVALID_ARG;
+    if (ranges && !aligned(ranges, 8)) return GS_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const int TX = tiles_x(*cam), TY = tiles_y(*cam), T = TX * TY;
     BinWs w;
