@@ -119,19 +119,46 @@ def unit_view(cams: Sequence, unit: WorkUnit):
     return cam if unit.whole else band_view(cam, unit.y0, unit.y1)
 
 
+_BIN_STREAMS: Dict[int, torch.cuda.Stream] = {}
+
+
+def binning_stream(device) -> torch.cuda.Stream:
+    """The high-priority stream that projects and bins the views ahead of
+    their compositing (one per device)."""
+    idx = torch.device(device).index
+    idx = torch.cuda.current_device() if idx is None else idx
+    if idx not in _BIN_STREAMS:
+        _BIN_STREAMS[idx] = torch.cuda.Stream(torch.device("cuda", idx), priority=-1)
+    return _BIN_STREAMS[idx]
+
+
 def render_views(cams: Sequence, params: Dict[str, torch.Tensor], dL_dimages: Sequence[torch.Tensor],
                  grads: Optional[Dict[str, torch.Tensor]] = None,
                  rasterizers: Optional[Dict[int, "RZ.Rasterizer"]] = None,
                  densify: Optional[Dict[str, torch.Tensor]] = None, capacity: Optional[Sequence[int]] = None,
-                 camera_ids: Optional[Sequence[int]] = None) -> Dict[str, torch.Tensor]:
+                 camera_ids: Optional[Sequence[int]] = None, overlap: bool = False) -> Dict[str, torch.Tensor]:
     """Forward and backward of every camera in ``cams``; 3D gradients are
     accumulated into ``grads`` (allocated when None).  ``rasterizers`` caches
-    one Rasterizer (and its buffers) per camera id across calls."""
+    one Rasterizer (and its buffers) per camera id across calls.
+
+    With ``overlap`` (capacity mode: ``capacity`` given) the views' projection
+    and binning run back to back on a high-priority side stream
+    (``binning_stream``) while the current stream composites, differentiates
+    and accumulates the views in order, each after its own binning: the
+    binning of view n + 1, bound by latency, fills the GPU beside the
+    compositing of view n.  The views must not share per-view buffers (one
+    Rasterizer per camera id), and the colours must not depend on the view."""
     means, scales, quats = params["means"], params["scales"], params["quats"]
     opacity, colors = params["opacity"], params["colors"]
     if grads is None:
         grads = RZ.zero_grads(means.shape[0], means.device)
     ids = list(range(len(cams))) if camera_ids is None else list(camera_ids)
+    if overlap and capacity is None:
+        raise ValueError("overlapped views run in capacity mode: pass capacity")
+    cur = torch.cuda.current_stream(means.device)
+    bs = binning_stream(means.device) if overlap else None
+    if bs is not None:
+        bs.wait_stream(cur)  # inputs written, earlier readers of the per-view buffers done
     for n, (cam, dl) in enumerate(zip(cams, dL_dimages)):
         cid = ids[n]
         rz = None if rasterizers is None else rasterizers.get(cid)
@@ -140,8 +167,11 @@ def render_views(cams: Sequence, params: Dict[str, torch.Tensor], dL_dimages: Se
             if rasterizers is not None:
                 rasterizers[cid] = rz
         cap = None if capacity is None else capacity[n]
-        fr = rz.forward(means, scales, quats, opacity, colors, capacity=cap)
+        fr = rz.forward(means, scales, quats, opacity, colors, capacity=cap, stream=bs,
+                        render_stream=cur if bs is not None else None)
         rz.backward(fr, means, scales, quats, colors, dl, grads=grads, densify=densify)
+    if bs is not None:
+        cur.wait_stream(bs)
     return grads
 
 

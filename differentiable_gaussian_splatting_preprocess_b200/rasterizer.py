@@ -83,7 +83,7 @@ class Rasterizer:
 
     def forward(self, means, scales, quats, opacity, colors, capacity: Optional[int] = None,
                 want_keys: bool = False, use_mask: bool = True, stream=None,
-                colors_ready: Optional[torch.cuda.Event] = None) -> Frame:
+                colors_ready: Optional[torch.cuda.Event] = None, render_stream=None) -> Frame:
         """Preprocess, bin/sort and composite one frame.
 
         With ``capacity=None`` the pair count is read back to size the sort
@@ -92,11 +92,15 @@ class Rasterizer:
         the workspace reports GS_ERR_CAPACITY and every tile range is empty.
         ``colors_ready``: an event the compositing waits for (the colours may
         still be arriving while the projection and the binning run).
+        ``render_stream``: run the compositing there instead of on
+        ``stream``, after the binning (an event joins the two), so that the
+        projection and binning of the next frame can go ahead on ``stream``.
         """
         N = means.shape[0]
         pre = self.preprocess(means, scales, quats, opacity, stream)
         if capacity is None:
-            capacity = int(pre["num_pairs"].to("cpu").view(torch.int32).item()) & 0xFFFFFFFF
+            with torch.cuda.stream(stream):  # the read waits for the projection
+                capacity = int(pre["num_pairs"].to("cpu").view(torch.int32).item()) & 0xFFFFFFFF
         ws = self.workspace(N, capacity)
         ids = self._buf("ids", (max(capacity, 1),), torch.uint32)
         ranges = self._buf("ranges", (B.num_tiles(self.cam), 2), torch.uint32)
@@ -109,6 +113,11 @@ class Rasterizer:
         n_contrib = self._buf("n_contrib", (H, W), torch.uint32)
         cmask = (self._buf("contrib_mask", (B.mask_words(max(capacity, 1), B.num_tiles(self.cam)),), torch.uint32)
                  if use_mask else None)
+        if render_stream is not None:
+            binned = torch.cuda.Event()
+            binned.record(stream or torch.cuda.current_stream(self.device))
+            render_stream.wait_event(binned)
+            stream = render_stream
         if colors_ready is not None:
             (stream or torch.cuda.current_stream(self.device)).wait_event(colors_ready)
         B.gs_render_fwd(self.cam, ranges, ids, pre["mean2d"], pre["conic_opacity"], colors, image, final_T,

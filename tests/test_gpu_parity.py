@@ -508,6 +508,47 @@ def test_render_views_sums_cameras():
         assert rel_l2(to_np(grads[k]), ref[k]) <= GRAD_REL_L2, k
 
 
+def test_render_views_overlapped_equals_sequential():
+    """Views whose projection and binning run ahead on the binning stream
+    give the gradients of the sequential path (same terms; only the order of
+    the floating-point atomics differs), eagerly twice in a row and replayed
+    from a CUDA graph."""
+    from differentiable_gaussian_splatting_preprocess_b200 import multiview as MV
+    sc = _scene(2)
+    base = sc.cameras[0]
+    cams = [base, base.replace(R=(0.985, 0.0, 0.174, 0.0, 1.0, 0.0, -0.174, 0.0, 0.985)),
+            base.replace(t=(0.2, -0.1, 0.0))]
+    gs = GpuScene(sc)
+    params = dict(means=gs.means, scales=gs.scales, quats=gs.quats, opacity=gs.opacity, colors=gs.colors)
+    dls = [to_dev(sc.dL_dimage[0])] * 3
+    rzs = {}
+    ref = {k: to_np(v).copy() for k, v in MV.render_views(cams, params, dls, rasterizers=rzs).items()
+           if k in MV.GRAD_KEYS}
+    torch.cuda.synchronize()
+    caps = [rzs[i]._bufs["ids"].numel() for i in range(len(cams))]
+    for _ in range(2):
+        got = MV.render_views(cams, params, dls, rasterizers=rzs, capacity=caps, overlap=True)
+        torch.cuda.synchronize()
+        for k in MV.GRAD_KEYS:
+            assert rel_l2(to_np(got[k]), ref[k]) <= 1e-5, k
+    grads = {k: torch.zeros_like(v) for k, v in got.items() if k in MV.GRAD_KEYS}
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up outside the capture, on a side stream
+        MV.render_views(cams, params, dls, grads=grads, rasterizers=rzs, capacity=caps, overlap=True)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for v in grads.values():
+            v.zero_()
+        MV.render_views(cams, params, dls, grads=grads, rasterizers=rzs, capacity=caps, overlap=True)
+    graph.replay()
+    torch.cuda.synchronize()
+    for k in MV.GRAD_KEYS:
+        assert rel_l2(to_np(grads[k]), ref[k]) <= 1e-5, k
+    assert all(rz.status() == 0 for rz in rzs.values())
+
+
 def test_render_views_from_host_overlapped_copies():
     """The host-input step (copies on a side stream, compositing and backward
     waiting on their inputs' events, capacity mode) gives the gradients of the
