@@ -43,7 +43,7 @@ OPS_BWD_EVAL = 60
 # DRAM bytes per launch from the committed ncu capture of the render backward (k_render_bwd_warp)
 # (dram__bytes_read.sum + dram__bytes_write.sum) and the SHA-1 of the render
 # sources it was taken on; reported only while the sources are unchanged.
-RECORDED_TRAFFIC = {"k_render_bwd": dict(bytes=138725632, sources_sha1="fa565619db6abdd936250267a6a1bbfa54ce6383")}
+RECORDED_TRAFFIC = {"k_render_bwd": dict(bytes=167509248, sources_sha1="8339ca8f1446b4ffd39383dcd2f97dbf7a61e451")}
 # Algorithmic bytes: per (tile, Gaussian) pair visited, id + mean2d +
 # conic/opacity + colour = 40 B read; the backward adds 36 B of gradient
 # atomics per pair; per pixel the forward writes 20 B (image, T, n_contrib)
