@@ -221,19 +221,36 @@ k_preprocess_bwd(gs_camera cam, int N, const float* __restrict__ means, const fl
                  float* __restrict__ dL_dopacity, float* __restrict__ dL_dcolors, float* __restrict__ grad2d_accum,
                  unsigned* __restrict__ vis_count) {
     const int i = blockIdx.x * kPreBlock + threadIdx.x;
-    if (i >= N || radius[i] == 0) return;
+    if (i >= N) return;
+    // Every load of this Gaussian - inputs and the accumulators read by the
+    // += below - is issued here, before the culling test, so that they are
+    // in flight together: one memory round trip instead of three (radius,
+    // then the inputs, then the accumulators).
+    const int rad = radius[i];
+    const float mx = means[3 * i], my = means[3 * i + 1], mz = means[3 * i + 2];
+    const float4 qv = quats[i];
+    const float s[3] = {scales[3 * i], scales[3 * i + 1], scales[3 * i + 2]};
+    const float4 co = conic_opacity[i];
+    const float4 gco = dL_dconic_opacity[i];
+    const float2 gm = dL_dmean2d[i];
+    const float gc0 = dL_dcolor2d[3 * i + 0], gc1 = dL_dcolor2d[3 * i + 1], gc2 = dL_dcolor2d[3 * i + 2];
+    const float am0 = dL_dmeans[3 * i + 0], am1 = dL_dmeans[3 * i + 1], am2 = dL_dmeans[3 * i + 2];
+    const float as0 = dL_dscales[3 * i + 0], as1 = dL_dscales[3 * i + 1], as2 = dL_dscales[3 * i + 2];
+    float4 dq = dL_dquats[i];
+    const float aop = dL_dopacity[i];
+    const float ac0 = dL_dcolors[3 * i + 0], ac1 = dL_dcolors[3 * i + 1], ac2 = dL_dcolors[3 * i + 2];
+    const float ga = grad2d_accum ? grad2d_accum[i] : 0.0f;
+    const unsigned vc = grad2d_accum ? vis_count[i] : 0u;
+    if (rad == 0) return;
     if (grad2d_accum) {
         // densification statistics: |dL/dmean2d| of this view, and one more view
-        const float2 g2 = dL_dmean2d[i];
-        grad2d_accum[i] += sqrtf(g2.x * g2.x + g2.y * g2.y);
-        vis_count[i] += 1u;
+        grad2d_accum[i] = ga + sqrtf(gm.x * gm.x + gm.y * gm.y);
+        vis_count[i] = vc + 1u;
     }
     const float* W = cam.R;
-    const float mx = means[3 * i], my = means[3 * i + 1], mz = means[3 * i + 2];
     const float tx = W[0] * mx + W[1] * my + W[2] * mz + cam.t[0];
     const float ty = W[3] * mx + W[4] * my + W[5] * mz + cam.t[1];
     const float tz = W[6] * mx + W[7] * my + W[8] * mz + cam.t[2];
-    const float4 qv = quats[i];
     const float qnorm = sqrtf(qv.x * qv.x + qv.y * qv.y + qv.z * qv.z + qv.w * qv.w);
     const float inv_n = 1.0f / qnorm;
     const float w = qv.x * inv_n, x = qv.y * inv_n, y = qv.z * inv_n, z = qv.w * inv_n;
@@ -247,7 +264,6 @@ k_preprocess_bwd(gs_camera cam, int N, const float* __restrict__ means, const fl
     R[2][0] = 2.f * (x * z - w * y);
     R[2][1] = 2.f * (y * z + w * x);
     R[2][2] = 1.f - 2.f * (x * x + y * y);
-    const float s[3] = {scales[3 * i], scales[3 * i + 1], scales[3 * i + 2]};
 
     const float iz = 1.0f / tz;
     const float iz2 = iz * iz;
@@ -267,8 +283,6 @@ k_preprocess_bwd(gs_camera cam, int N, const float* __restrict__ means, const fl
         for (int k = 0; k < 3; ++k) V[r][k] = (M[r][0] * R[0][k] + M[r][1] * R[1][k] + M[r][2] * R[2][k]) * s[k];
 
     // G2 = -A Gbar A
-    const float4 co = conic_opacity[i];
-    const float4 gco = dL_dconic_opacity[i];
     const float A00 = co.x, A01 = co.y, A11 = co.z;
     const float g00 = gco.x, g01 = 0.5f * gco.y, g11 = gco.z;
     const float P00 = A00 * g00 + A01 * g01, P01 = A00 * g01 + A01 * g11;
@@ -302,21 +316,21 @@ k_preprocess_bwd(gs_camera cam, int N, const float* __restrict__ means, const fl
     const float GJ11 = GM[1][0] * W[3] + GM[1][1] * W[4] + GM[1][2] * W[5];
     const float GJ12 = GM[1][0] * W[6] + GM[1][1] * W[7] + GM[1][2] * W[8];
 
-    const float2 gm = dL_dmean2d[i];
     const float iz3 = iz2 * iz;
     float dtx = cam.fx * iz * gm.x - cam.fx * iz2 * GJ02;
     float dty = cam.fy * iz * gm.y - cam.fy * iz2 * GJ12;
     float dtz = -cam.fx * tx * iz2 * gm.x - cam.fy * ty * iz2 * gm.y - cam.fx * iz2 * GJ00 +
                 2.f * cam.fx * tx * iz3 * GJ02 - cam.fy * iz2 * GJ11 + 2.f * cam.fy * ty * iz3 * GJ12;
-    dL_dmeans[3 * i + 0] += W[0] * dtx + W[3] * dty + W[6] * dtz;
-    dL_dmeans[3 * i + 1] += W[1] * dtx + W[4] * dty + W[7] * dtz;
-    dL_dmeans[3 * i + 2] += W[2] * dtx + W[5] * dty + W[8] * dtz;
+    dL_dmeans[3 * i + 0] = am0 + (W[0] * dtx + W[3] * dty + W[6] * dtz);
+    dL_dmeans[3 * i + 1] = am1 + (W[1] * dtx + W[4] * dty + W[7] * dtz);
+    dL_dmeans[3 * i + 2] = am2 + (W[2] * dtx + W[5] * dty + W[8] * dtz);
 
     // scales and rotation from dL/dL
     float GR[3][3];
+    const float as[3] = {as0, as1, as2};
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-        dL_dscales[3 * i + k] += GL[0][k] * R[0][k] + GL[1][k] * R[1][k] + GL[2][k] * R[2][k];
+        dL_dscales[3 * i + k] = as[k] + (GL[0][k] * R[0][k] + GL[1][k] * R[1][k] + GL[2][k] * R[2][k]);
 #pragma unroll
         for (int r = 0; r < 3; ++r) GR[r][k] = GL[r][k] * s[k];
     }
@@ -330,16 +344,15 @@ k_preprocess_bwd(gs_camera cam, int N, const float* __restrict__ means, const fl
                             y * GR[1][2] + x * GR[2][0] + y * GR[2][1]);
     // through q_hat = q / |q|
     const float dotp = w * dw + x * dx + y * dy + z * dz;
-    float4 dq = dL_dquats[i];
     dq.x += (dw - w * dotp) * inv_n;
     dq.y += (dx - x * dotp) * inv_n;
     dq.z += (dy - y * dotp) * inv_n;
     dq.w += (dz - z * dotp) * inv_n;
     dL_dquats[i] = dq;
-    dL_dopacity[i] += gco.w;
-    dL_dcolors[3 * i + 0] += dL_dcolor2d[3 * i + 0];
-    dL_dcolors[3 * i + 1] += dL_dcolor2d[3 * i + 1];
-    dL_dcolors[3 * i + 2] += dL_dcolor2d[3 * i + 2];
+    dL_dopacity[i] = aop + gco.w;
+    dL_dcolors[3 * i + 0] = ac0 + gc0;
+    dL_dcolors[3 * i + 1] = ac1 + gc1;
+    dL_dcolors[3 * i + 2] = ac2 + gc2;
 }
 
 }  // namespace
