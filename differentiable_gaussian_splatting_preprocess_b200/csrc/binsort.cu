@@ -1124,10 +1124,27 @@ k_seg_count(int SX, const unsigned* __restrict__ clist, const int4* __restrict__
         const unsigned c = seg_cell[k], lo = seg_lo[k], hi = seg_hi[k];
         const int cx = (int)(c % (unsigned)SX), cy = (int)(c / (unsigned)SX);
         static_assert(kSeg / kSortBlock <= 7, "packed byte counters hold at most 7 masks per lane");
+        // a segment holds at most kSeg entries: this thread's kJ entries are
+        // loaded first, then their rectangles, so that the loads of each
+        // step are in flight together
+        constexpr int kJ = kSeg / kSortBlock;
+        unsigned g[kJ];
+        int4 rc[kJ];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const unsigned i = lo + (unsigned)(j * kSortBlock) + threadIdx.x;
+            g[j] = i < hi ? clist[i] : 0xFFFFFFFFu;
+        }
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const bool ok = g[j] != 0xFFFFFFFFu && id_ok(g[j]);
+            rc[j] = ok ? rect[g[j]] : make_int4(0, 0, 0, 0);
+        }
         unsigned acc[kCellTiles / 4] = {};
-        for (unsigned base = lo; base < hi; base += kSortBlock) {
-            const unsigned i = base + threadIdx.x;
-            const unsigned m = (i < hi && id_ok(clist[i])) ? cell_mask(rect[clist[i]], cx, cy) : 0u;
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const unsigned i = lo + (unsigned)(j * kSortBlock) + threadIdx.x;
+            const unsigned m = g[j] != 0xFFFFFFFFu ? cell_mask(rc[j], cx, cy) : 0u;
             if (i < hi) seg_mask[i] = (unsigned short)m;
             add_mask(acc, m);
         }
@@ -1246,10 +1263,22 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
             const int tx = kSuper * cx + b % kSuper, ty = kSuper * cy + b / kSuper;
             s_base[b] = (tx < TX && ty < TY) ? tile_start[ty * TX + tx] + seg_base[(size_t)k * kCellTiles + b] : 0u;
         }
-        for (unsigned base = lo; base < hi; base += kSortBlock) {
-            const unsigned i = base + threadIdx.x;
-            const unsigned g = i < hi ? clist[i] : 0u;
-            const unsigned m = i < hi ? (unsigned)seg_mask[i] : 0u;
+        // a segment holds at most kSeg entries: this thread's entries and
+        // masks for the whole segment are loaded together, up front
+        constexpr int kJ = kSeg / kSortBlock;
+        unsigned gs[kJ], ms[kJ];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const unsigned i = lo + (unsigned)(j * kSortBlock) + threadIdx.x;
+            gs[j] = i < hi ? clist[i] : 0u;
+            ms[j] = i < hi ? (unsigned)seg_mask[i] : 0u;
+        }
+#pragma unroll
+        for (int jc = 0; jc < kJ; ++jc) {
+            const unsigned base = lo + (unsigned)(jc * kSortBlock);
+            if (base >= hi) break;  // block-uniform
+            const unsigned g = gs[jc];
+            const unsigned m = ms[jc];
             const unsigned un = __reduce_or_sync(0xffffffffu, m);
             // this warp's count per tile bit (packed byte counters)
             unsigned acc[kCellTiles / 4] = {};
