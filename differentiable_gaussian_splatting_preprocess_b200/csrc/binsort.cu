@@ -60,13 +60,13 @@ struct BinWs {
     unsigned* totals;                              // kMaxPasses * kRadixMax
     // super-tile route only (empty otherwise)
     unsigned* rc_rank;                             // N packed super-tile rectangles in rank order
+    unsigned char* sub_rank;                       // N: the tile rectangle's offsets in its edge cells (sub_offsets)
     unsigned *owner_lo, *owner_hi;                 // kSortMaxGrid each: ranks owning chunk ends
     unsigned* cell_ranges;                         // 2 S: each super-tile's slice of the super list
     unsigned* cell_seg0;                           // S + 1: first segment of each super-tile
     unsigned *seg_cell, *seg_lo, *seg_hi;          // max_seg each
     unsigned *seg_cnt, *seg_base;                  // max_seg * kCellTiles each
     unsigned *tile_cnt, *tile_start;               // T each
-    unsigned short* seg_mask;                      // capacity: tile mask of each cell-list entry
     unsigned max_seg;
     int n_cells;                                   // S
 };
@@ -117,6 +117,7 @@ size_t carve(void* base, int N, unsigned capacity, int TX, int TY, BinWs* w) {
     t.n_cells = (int)S;
     const size_t ms = t.max_seg;
     t.rc_rank = (unsigned*)take(sup ? n * 4 : 0);
+    t.sub_rank = (unsigned char*)take(sup ? n : 0);
     t.owner_lo = (unsigned*)take((size_t)kSortMaxGrid * 4);
     t.owner_hi = (unsigned*)take((size_t)kSortMaxGrid * 4);
     t.cell_ranges = (unsigned*)take(2 * S * 4);
@@ -128,7 +129,6 @@ size_t carve(void* base, int N, unsigned capacity, int TX, int TY, BinWs* w) {
     t.seg_base = (unsigned*)take(ms * kCellTiles * 4);
     t.tile_cnt = (unsigned*)take(T * 4);
     t.tile_start = (unsigned*)take(T * 4);
-    t.seg_mask = (unsigned short*)take(sup ? cap * 2 : 0);
     if (w) *w = t;
     return off;
 }
@@ -146,6 +146,38 @@ __device__ __forceinline__ int rect_x0(unsigned p) { return (int)(p & 255u); }
 __device__ __forceinline__ int rect_w(unsigned p) { return (int)((p >> 8) & 255u) + 1; }
 __device__ __forceinline__ int rect_y0(unsigned p) { return (int)((p >> 16) & 255u); }
 __device__ __forceinline__ int rect_h(unsigned p) { return (int)(p >> 24) + 1; }
+
+// Where a Gaussian's tile rectangle starts and ends inside the first and
+// last cells of its cell rectangle, in 8 bits: x0 mod 4 | (x1 - 1) mod 4 << 2
+// | y0 mod 4 << 4 | (y1 - 1) mod 4 << 6 (tile rectangle [x0, x1) x [y0, y1)).
+__device__ __forceinline__ unsigned sub_offsets(int4 rc) {
+    static_assert(kSuper == 4, "two bits per offset assume 4 x 4 cells");
+    return (unsigned)(rc.x & 3) | (unsigned)((rc.z - 1) & 3) << 2 | (unsigned)(rc.y & 3) << 4 |
+           (unsigned)((rc.w - 1) & 3) << 6;
+}
+
+// Cell-pair keys: cell x in bits 0-7 and cell y in bits 16-23 (the radix
+// digits), the 16-bit mask of the cell's tiles that the Gaussian covers in
+// bits 8-15 (mask bits 0-7) and 24-31 (mask bits 8-15); bit ly * 4 + lx of
+// the mask is tile (4 cy + ly, 4 cx + lx).
+constexpr unsigned kCellBits = 0x00FF00FFu;
+__device__ __forceinline__ unsigned key_mask(unsigned key) { return ((key >> 8) & 0xFFu) | ((key >> 24) << 8); }
+
+// The key of the pair (cell (cx, cy), Gaussian) from the Gaussian's packed
+// cell rectangle rc and sub_offsets byte sb: the tiles covered span lx0..lx1
+// in x (the rectangle's offsets in its first / last cell column, else 0 / 3)
+// and ly0..ly1 in y.
+__device__ __forceinline__ unsigned cell_pair_key(unsigned rc, unsigned sb, int cx, int cy) {
+    const int cx0 = rect_x0(rc), cy0 = rect_y0(rc);
+    const unsigned lx0 = cx == cx0 ? (sb & 3u) : 0u;
+    const unsigned lx1 = cx == cx0 + rect_w(rc) - 1 ? ((sb >> 2) & 3u) : 3u;
+    const unsigned ly0 = cy == cy0 ? ((sb >> 4) & 3u) : 0u;
+    const unsigned ly1 = cy == cy0 + rect_h(rc) - 1 ? (sb >> 6) : 3u;
+    const unsigned row = ((2u << lx1) - (1u << lx0)) * 0x1111u;  // tiles lx0..lx1 of every row
+    const unsigned rows = (2u << (4u * ly1 + 3u)) - (1u << (4u * ly0));  // rows ly0..ly1
+    const unsigned m = row & rows;
+    return (unsigned)cx | (m & 0xFFu) << 8 | (unsigned)cy << 16 | (m >> 8) << 24;
+}
 
 // Debug build: after a failed index check inside the binning, later kernels
 // would see inconsistent inputs (a visible rank without pairs, an unwritten
@@ -500,6 +532,7 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
 __global__ void __launch_bounds__(kSortBlock)
 k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ tiles_touched,
                 const int4* __restrict__ rect, unsigned* __restrict__ cnt_rank, unsigned* __restrict__ rc_rank,
+                unsigned char* __restrict__ sub_rank,
                 unsigned* __restrict__ part, SortMisc* __restrict__ misc) {
     const int base = blockIdx.x * kScanTile;
     unsigned s = 0;
@@ -512,9 +545,11 @@ k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __res
             if (id_ok(g)) v = tiles_touched[g];
             else abort_frame(misc);
             if (rect && v) {
-                const int4 sr = super_rect(rect[g]);
+                const int4 tr = rect[g];
+                const int4 sr = super_rect(tr);
                 v = (unsigned)((sr.z - sr.x) * (sr.w - sr.y));
                 rc_rank[r] = pack_rect(sr);
+                sub_rank[r] = (unsigned char)sub_offsets(tr);
             }
             cnt_rank[r] = v;
             s += v;
@@ -737,7 +772,9 @@ __global__ void k_ranges(const unsigned* __restrict__ tkeys, const unsigned* __r
 //      pair list: it generates the pairs of its chunk of the stream on the
 //      fly (Gaussian by Gaussian, each cell rectangle row-major) and ranks
 //      them by cx; its histogram comes from the cell rectangles directly (a
-//      difference array over cx).  Intermediate key: cy << 16 | cx.
+//      difference array over cx).  Intermediate key: cx | cy << 16, with
+//      the pair's 16-bit tile mask in the other bits (cell_pair_key), so
+//      that later steps never look the Gaussian's rectangle up again.
 //   2. each cell's list is cut into segments of kSeg entries; per segment and
 //      tile of the cell, the number of its Gaussians touching the tile
 //      (warp ballots over the 16-bit tile masks);
@@ -848,15 +885,16 @@ k_gen_hist(const unsigned* __restrict__ pair_off, const unsigned* __restrict__ r
 template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
-              const unsigned* __restrict__ rc_rank, const unsigned* __restrict__ n_ptr,
-              const unsigned* __restrict__ owner_lo, int bits, const unsigned* __restrict__ offsets,
-              unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out) {
+              const unsigned* __restrict__ rc_rank, const unsigned char* __restrict__ sub_rank,
+              const unsigned* __restrict__ n_ptr, const unsigned* __restrict__ owner_lo, int bits,
+              const unsigned* __restrict__ offsets, unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out) {
     using C = RadixCfg<MAXB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const ScatterSmem<MAXB> sm(smem_raw, kPadTile);
     unsigned* s_off = sm.vals + kPadTile;  // [kGenWin] staged pair offsets
     unsigned* s_g = s_off + kGenWin;      // [kGenWin] staged ids
     unsigned* s_rc = s_g + kGenWin;       // [kGenWin] staged packed rectangles
+    unsigned char* s_sb = reinterpret_cast<unsigned char*>(s_rc + kGenWin);  // [kGenWin] staged sub_offsets
     __shared__ unsigned s_r0;
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
@@ -882,11 +920,13 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
             const unsigned off = inr ? pair_off[r] : 0xFFFFFFFFu;
             const unsigned g = inr ? order[r] : 0u;
             const unsigned rc = inr ? rc_rank[r] : 0u;
+            const unsigned sb = inr ? sub_rank[r] : 0u;
             const bool in = off < end;
             if (in) {
                 s_off[idx] = off;
                 s_g[idx] = g;
                 s_rc[idx] = rc;
+                s_sb[idx] = (unsigned char)sb;
             }
             const int c = __syncthreads_count(in);
             nr += (unsigned)c;
@@ -906,7 +946,7 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
                 const unsigned mid = (i + top) >> 1;
                 if (s_off[mid] <= p) i = mid; else top = mid;
             }
-            unsigned rc = s_rc[i], g = s_g[i];
+            unsigned rc = s_rc[i], g = s_g[i], sb = s_sb[i];
             int x0 = rect_x0(rc), x1 = x0 + rect_w(rc);
             const unsigned w = (unsigned)(x1 - x0);
             const unsigned local = p - s_off[i];
@@ -919,13 +959,14 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
             for (int j = 0; j < C::kItems; ++j) {
                 const unsigned q = q0 + j;
                 if (q < tile_n) {
-                    sm.keys[pad_idx(q)] = ((unsigned)ty << 16) | (unsigned)tx;
+                    sm.keys[pad_idx(q)] = cell_pair_key(rc, sb, tx, ty);
                     sm.vals[pad_idx(q)] = g;
                     ++p;
                     if (i + 1 < nr && s_off[i + 1] == p) {
                         ++i;
                         rc = s_rc[i];
                         g = s_g[i];
+                        sb = s_sb[i];
                         x0 = rect_x0(rc);
                         x1 = x0 + rect_w(rc);
                         tx = x0;
@@ -955,11 +996,11 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
 
 template <int MAXB>
 constexpr size_t gen_scatter_smem() {
-    return ScatterSmem<MAXB>::bytes(kPadTile) + 3 * (size_t)kGenWin * sizeof(unsigned);
+    return ScatterSmem<MAXB>::bytes(kPadTile) + 3 * (size_t)kGenWin * sizeof(unsigned) + (size_t)kGenWin;
 }
 
-// Cell ranges of the cell-sorted list by comparing neighbours (keys
-// cy << 16 | cx); empty cells keep (0, 0).  Four keys per thread with
+// Cell ranges of the cell-sorted list by comparing neighbours' cells (the
+// kCellBits of the keys); empty cells keep (0, 0).  Four keys per thread with
 // 16-byte loads, neighbours across lanes by shuffles.
 __global__ void k_cell_ranges(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ n_ptr, int SX,
                               unsigned* __restrict__ cell_ranges) {
@@ -988,11 +1029,13 @@ __global__ void k_cell_ranges(const unsigned* __restrict__ ckeys, const unsigned
             for (int j = 0; j < 4; ++j) {
                 const unsigned k = k0 + j;
                 if (k >= n) break;
-                const unsigned before = j == 0 ? prev : t[j - 1];
-                const unsigned after = (j == 3 || k + 1 == n) ? (k + 1 == n ? 0xFFFFFFFFu : next) : t[j + 1];
-                const unsigned c = (t[j] >> 16) * (unsigned)SX + (t[j] & 0xFFFFu);
-                if (k == 0 || before != t[j]) cell_ranges[2 * c] = k;
-                if (k + 1 == n || after != t[j]) cell_ranges[2 * c + 1] = k + 1;
+                const unsigned cell = t[j] & kCellBits;
+                const unsigned before = (j == 0 ? prev : t[j - 1]) & kCellBits;
+                const unsigned after =
+                    ((j == 3 || k + 1 == n) ? (k + 1 == n ? 0xFFFFFFFFu : next) : t[j + 1]) & kCellBits;
+                const unsigned c = (cell >> 16) * (unsigned)SX + (cell & 0xFFu);
+                if (k == 0 || before != cell) cell_ranges[2 * c] = k;
+                if (k + 1 == n || after != cell) cell_ranges[2 * c + 1] = k + 1;
             }
         }
     }
@@ -1082,19 +1125,6 @@ k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restric
     }
 }
 
-// Mask of the tiles of cell (cx, cy) that tile rectangle rc covers; bit
-// ly * kSuper + lx is tile (kSuper cy + ly, kSuper cx + lx).
-__device__ __forceinline__ unsigned cell_mask(int4 rc, int cx, int cy) {
-    constexpr unsigned kRep = 0x1111u;  // one bit per row of 4
-    static_assert(kSuper == 4, "row replication constant assumes 4 x 4 cells");
-    const int lx0 = max(rc.x - kSuper * cx, 0), lx1 = min(rc.z - kSuper * cx, kSuper);
-    const int ly0 = max(rc.y - kSuper * cy, 0), ly1 = min(rc.w - kSuper * cy, kSuper);
-    if (lx1 <= lx0 || ly1 <= ly0) return 0u;
-    const unsigned row = (((1u << (lx1 - lx0)) - 1u) << lx0) * kRep;
-    const unsigned rows = ((1u << (kSuper * (ly1 - ly0))) - 1u) << (kSuper * ly0);
-    return row & rows;
-}
-
 // Tile counts of a warp's masks, packed: bit b of a mask becomes byte b & 3
 // of word b >> 2 (a 4-bit slice spread to 4 bytes by one multiply, the
 // shifted copies disjoint), so one add per word counts 4 tiles and one
@@ -1110,44 +1140,29 @@ __device__ __forceinline__ unsigned packed_count(const unsigned (&acc)[kCellTile
 }
 
 // Per segment: count, per tile of its cell, the segment's Gaussians touching
-// it (packed byte counters, see add_mask).  Each entry's tile mask is kept
-// for k_seg_emit.
+// it (packed byte counters, see add_mask), from the tile masks the cell-pair
+// keys carry.
 __global__ void __launch_bounds__(kSortBlock)
-k_seg_count(int SX, const unsigned* __restrict__ clist, const int4* __restrict__ rect,
-            const unsigned* __restrict__ seg_cell, const unsigned* __restrict__ seg_lo,
-            const unsigned* __restrict__ seg_hi, const SortMisc* __restrict__ misc, unsigned* __restrict__ seg_cnt,
-            unsigned short* __restrict__ seg_mask) {
+k_seg_count(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ seg_lo,
+            const unsigned* __restrict__ seg_hi, const SortMisc* __restrict__ misc, unsigned* __restrict__ seg_cnt) {
     __shared__ unsigned s_c[kSortBlock / 32][kCellTiles];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned nseg = misc->nseg;
     for (unsigned k = blockIdx.x; k < nseg; k += gridDim.x) {
-        const unsigned c = seg_cell[k], lo = seg_lo[k], hi = seg_hi[k];
-        const int cx = (int)(c % (unsigned)SX), cy = (int)(c / (unsigned)SX);
+        const unsigned lo = seg_lo[k], hi = seg_hi[k];
         static_assert(kSeg / kSortBlock <= 7, "packed byte counters hold at most 7 masks per lane");
-        // a segment holds at most kSeg entries: this thread's kJ entries are
-        // loaded first, then their rectangles, so that the loads of each
-        // step are in flight together
+        // a segment holds at most kSeg entries: this thread's kJ keys are
+        // loaded together
         constexpr int kJ = kSeg / kSortBlock;
-        unsigned g[kJ];
-        int4 rc[kJ];
-#pragma unroll
-        for (int j = 0; j < kJ; ++j) {
-            const unsigned i = lo + (unsigned)(j * kSortBlock) + threadIdx.x;
-            g[j] = i < hi ? clist[i] : 0xFFFFFFFFu;
-        }
-#pragma unroll
-        for (int j = 0; j < kJ; ++j) {
-            const bool ok = g[j] != 0xFFFFFFFFu && id_ok(g[j]);
-            rc[j] = ok ? rect[g[j]] : make_int4(0, 0, 0, 0);
-        }
         unsigned acc[kCellTiles / 4] = {};
+        unsigned key[kJ];
 #pragma unroll
         for (int j = 0; j < kJ; ++j) {
             const unsigned i = lo + (unsigned)(j * kSortBlock) + threadIdx.x;
-            const unsigned m = g[j] != 0xFFFFFFFFu ? cell_mask(rc[j], cx, cy) : 0u;
-            if (i < hi) seg_mask[i] = (unsigned short)m;
-            add_mask(acc, m);
+            key[j] = i < hi ? ckeys[i] : 0u;  // a key of 0 carries no tile
         }
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) add_mask(acc, key_mask(key[j]));
 #pragma unroll
         for (int j = 0; j < kCellTiles / 4; ++j) acc[j] = __reduce_add_sync(0xffffffffu, acc[j]);
         if (lane < kCellTiles) s_c[warp][lane] = packed_count(acc, lane);
@@ -1244,7 +1259,7 @@ k_tile_scan(int T, const unsigned* __restrict__ tile_cnt, unsigned* __restrict__
 // Gaussians at base + ballot rank: consecutive lanes, consecutive addresses.
 // Optional 64-bit (tile << 32 | depth bits) keys.
 __global__ void __launch_bounds__(kSortBlock)
-k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const unsigned short* __restrict__ seg_mask,
+k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const unsigned* __restrict__ ckeys,
            const float* __restrict__ depth, const unsigned* __restrict__ seg_cell,
            const unsigned* __restrict__ seg_lo, const unsigned* __restrict__ seg_hi,
            const unsigned* __restrict__ seg_base, const unsigned* __restrict__ tile_start,
@@ -1271,7 +1286,7 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
         for (int j = 0; j < kJ; ++j) {
             const unsigned i = lo + (unsigned)(j * kSortBlock) + threadIdx.x;
             gs[j] = i < hi ? clist[i] : 0u;
-            ms[j] = i < hi ? (unsigned)seg_mask[i] : 0u;
+            ms[j] = i < hi ? key_mask(ckeys[i]) : 0u;
         }
 #pragma unroll
         for (int jc = 0; jc < kJ; ++jc) {
@@ -1427,7 +1442,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     const int nb = (N + kScanTile - 1) / kScanTile;
     const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
     k_scan_partials<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
-                                               w.rc_rank, w.scan_part, w.misc); note_launch();
+                                               w.rc_rank, w.sub_rank, w.scan_part, w.misc); note_launch();
     k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb, w.misc); note_launch();
     k_scan_down<<<nb, kSortBlock, 0, st>>>(N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
                                            (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi); note_launch();
@@ -1446,13 +1461,15 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
             k_gen_hist<7><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
             k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
             opt_in_smem(k_gen_scatter<7>, gen_scatter_smem<7>());
-            k_gen_scatter<7><<<Gp, kSortBlock, gen_scatter_smem<7>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
+            k_gen_scatter<7><<<Gp, kSortBlock, gen_scatter_smem<7>(), st>>>(N, order, w.pair_off, w.rc_rank,
+                                                                           w.sub_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         } else {
             k_gen_hist<8><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
             k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
             opt_in_smem(k_gen_scatter<8>, gen_scatter_smem<8>());
-            k_gen_scatter<8><<<Gp, kSortBlock, gen_scatter_smem<8>(), st>>>(N, order, w.pair_off, w.rc_rank, ps,
+            k_gen_scatter<8><<<Gp, kSortBlock, gen_scatter_smem<8>(), st>>>(N, order, w.pair_off, w.rc_rank,
+                                                                           w.sub_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         }
         GS_LAUNCH_CHECK();
@@ -1472,11 +1489,10 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         const int S = SX * SY;
         k_seg_table<<<1, 1024, 0, st>>>(S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
         const int gseg = (int)(w.max_seg < 148u * 8u ? w.max_seg : 148u * 8u);
-        k_seg_count<<<gseg, kSortBlock, 0, st>>>(SX, w.tvals1, rect4, w.seg_cell, w.seg_lo, w.seg_hi, w.misc,
-                                                 w.seg_cnt, w.seg_mask); note_launch();
+        k_seg_count<<<gseg, kSortBlock, 0, st>>>(w.tkeys1, w.seg_lo, w.seg_hi, w.misc, w.seg_cnt); note_launch();
         k_cell_scan<<<S, kCellTiles, 0, st>>>(TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
         k_tile_scan<<<1, 1024, 0, st>>>(T, w.tile_cnt, w.tile_start, ranges); note_launch();
-        k_seg_emit<<<gseg, kSortBlock, 0, st>>>(TX, TY, SX, w.tvals1, w.seg_mask, depth, w.seg_cell, w.seg_lo,
+        k_seg_emit<<<gseg, kSortBlock, 0, st>>>(TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell, w.seg_lo,
                                                 w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys); note_launch();
         GS_LAUNCH_CHECK();
         return GS_OK;

@@ -3,7 +3,8 @@
 The kernels in csrc/binsort.cu locate their work through derived indices:
 the ranks owning each chunk's first and last pair (recorded by the rank
 scan), the window of ranks a 2048-pair tile stages, the walk that generates
-the pairs of a tile, the tile mask of a Gaussian inside a 4x4-tile cell, the
+the pairs of a tile, the tile mask of a Gaussian inside a 4x4-tile cell (as the
+cell-pair key carries it, from the cell rectangle and 8 bits of offsets), the
 segments of a cell list and the (segment, tile) output bases.  This test
 restates those rules in Python and checks, on random rectangles, that they
 reproduce a direct construction: every generated pair, every chunk
@@ -65,6 +66,33 @@ def _owners(off, cnt, P, G):
     return chunk, lo_own, hi_own
 
 
+def _sub_offsets(r):
+    """The 8-bit offsets of a tile rectangle inside its first and last cells
+    (csrc/binsort.cu, sub_offsets)."""
+    x0, y0, x1, y1 = r
+    return (x0 & 3) | ((x1 - 1) & 3) << 2 | (y0 & 3) << 4 | ((y1 - 1) & 3) << 6
+
+
+def _cell_pair_key(crect, sb, cx, cy):
+    """The cell-pair key with the pair's tile mask in bits 8-15 and 24-31
+    (csrc/binsort.cu, cell_pair_key), from the cell rectangle and the
+    sub-offsets only."""
+    cx0, cy0, cx1, cy1 = crect
+    lx0 = sb & 3 if cx == cx0 else 0
+    lx1 = (sb >> 2) & 3 if cx == cx1 - 1 else 3
+    ly0 = (sb >> 4) & 3 if cy == cy0 else 0
+    ly1 = sb >> 6 if cy == cy1 - 1 else 3
+    row = ((2 << lx1) - (1 << lx0)) * 0x1111
+    rows = (2 << (4 * ly1 + 3)) - (1 << (4 * ly0))
+    m = row & rows
+    assert 0 <= cx < 256 and 0 <= cy < 256 and 0 < m < (1 << 16)
+    return cx | (m & 0xFF) << 8 | cy << 16 | (m >> 8) << 24
+
+
+def _key_mask(key):
+    return ((key >> 8) & 0xFF) | ((key >> 24) << 8)
+
+
 def _cell_mask(rc, cx, cy):
     x0, y0, x1, y1 = rc
     lx0, lx1 = max(x0 - CELL * cx, 0), min(x1 - CELL * cx, CELL)
@@ -122,6 +150,10 @@ def test_cell_route_index_model(TX, TY, N, seed, gmax):
                     if base + q0 + j >= end:
                         break
                     generated.append((cy, cx, g))
+                    # the key carries the cell (the radix digits) and the pair's tile mask
+                    key = _cell_pair_key(crect[g], _sub_offsets(rects[g]), cx, cy)
+                    assert key & 0x00FF00FF == cy << 16 | cx
+                    assert _key_mask(key) == _cell_mask(rects[g], cx, cy)
                     p += 1
                     if i + 1 < len(win) and off[win[i + 1]] == p:
                         i += 1
