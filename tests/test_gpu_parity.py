@@ -253,13 +253,14 @@ def test_ragged_and_tiny_images(W, H):
 
 
 @pytest.mark.parametrize("W,H,n,sigma_mult", [(16400, 20, 80, 3.0), (8200, 40, 80, 3.0), (40, 8200, 80, 3.0),
-                                              (800, 608, 2000, 1e3)])
+                                              (800, 608, 2000, 1e3), (2000, 1200, 300, 3.0), (2000, 2100, 200, 3.0),
+                                              (8200, 600, 80, 3.0)])
 def test_binning_routes(W, H, n, sigma_mult):
     """Both binning routes against the oracle's sort: more than 1024 tile
     columns (257 cells: emit + radix sort by tile id + boundary ranges),
-    129 cell columns or rows (cell passes with 8-bit digits), and cell pairs
-    of whole-image Gaussians cut by every chunk boundary of the generated
-    first pass."""
+    129 cell columns or rows (cell passes with 8-bit digits), cell pairs of
+    whole-image Gaussians cut by every chunk boundary of the generated first
+    pass, and larger cell grids (32 x 19, 32 x 33, 129 x 10 cells)."""
     sc = _tiny(n=n, width=W, height=H, seed=W + 3 * H, z_range=(2.0, 6.0), sigma_mult=sigma_mult)
     cam = sc.cameras[0].replace(fx=float(W), fy=float(H), cx=W / 2.0, cy=H / 2.0)
     sc.cameras[0] = cam
