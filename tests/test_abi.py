@@ -93,3 +93,30 @@ def test_host_argument_checks_need_no_device(lib):
     assert rc == B.GS_ERR_INVALID_ARG
     rc = lib.gs_bin_sort(ctypes.byref(cam), -1, None, None, None, None, 0, None, None, None, None, 0, None)
     assert rc == B.GS_ERR_INVALID_ARG
+
+
+def test_mask_and_range_buffer_checks_need_no_device(lib):
+    """The contribution mask must hold the dispatch-order block plus at least
+    one group of bits and be a multiple of 4 words; tile ranges must be
+    8-byte aligned.  Both are rejected before anything is enqueued (host
+    arrays stand in for device buffers: nothing is dereferenced)."""
+    import numpy as np
+    cam = B.GsCamera()
+    cam.width, cam.height, cam.tile = 64, 48, 16
+    T = 4 * 3
+    buf = np.zeros(1 << 16, np.uint64)  # 8-byte aligned host storage
+    p = lambda off: ctypes.c_void_p(buf.ctypes.data + off)
+    need = B.order_words(T) + 4
+    assert need == 12 * T + 256 + 4
+    for words in (need - 4, need + 2, 0):
+        rc = lib.gs_render_fwd(ctypes.byref(cam), p(0), p(0), p(0), p(0), p(0), p(0), p(0), p(0), p(0), words, None)
+        assert rc == B.GS_ERR_INVALID_ARG, words
+        rc = lib.gs_render_bwd(ctypes.byref(cam), 0, p(0), p(0), p(0), p(0), p(0), p(0), p(0), p(0), words, p(0),
+                               None, None, None, None)
+        assert rc == B.GS_ERR_INVALID_ARG, words
+    assert B.mask_words(100, T) == B.order_words(T) + 4 * 4
+    ws_bytes = B.gs_workspace_bytes(B.GS_STAGE_BIN_SORT, 0, 0, cam.width, cam.height)
+    ws = np.zeros(ws_bytes + 512, np.uint8)
+    ws_p = ctypes.c_void_p((ws.ctypes.data + 255) // 256 * 256)
+    rc = lib.gs_bin_sort(ctypes.byref(cam), 0, None, None, None, p(0), 0, None, p(4), None, ws_p, ws_bytes, None)
+    assert rc == B.GS_ERR_INVALID_ARG
