@@ -197,6 +197,7 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 __global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const unsigned* __restrict__ tiles_touched,
                            const unsigned* __restrict__ d_num_pairs, unsigned capacity, BinWs w,
                            unsigned* __restrict__ ranges) {
+    pdl_enter();
     const int stride = gridDim.x * blockDim.x;
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
     for (int i = tid; i < 2 * T; i += stride) ranges[i] = 0u;
@@ -281,6 +282,7 @@ template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_radix_hist(const unsigned* __restrict__ keys, const unsigned* __restrict__ n_ptr, int shift, int bits,
              unsigned* __restrict__ hist, unsigned* __restrict__ totals) {
+    pdl_enter();
     using C = RadixCfg<MAXB>;
     __shared__ unsigned s_h[C::kWarps][C::kRadix];
     const int radix = 1 << bits;
@@ -325,6 +327,7 @@ k_radix_hist(const unsigned* __restrict__ keys, const unsigned* __restrict__ n_p
 // prefix over CTAs of hist[d][.], in place.
 __global__ void __launch_bounds__(kSortBlock)
 k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, int G) {
+    pdl_enter();
     const int d = blockIdx.x;
     __shared__ unsigned s_w[kSortBlock / 32];
     __shared__ unsigned s_base;
@@ -498,6 +501,7 @@ __global__ void __launch_bounds__(kSortBlock)
 k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict__ vals_in,
                 unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out,
                 const unsigned* __restrict__ n_ptr, int shift, int bits, const unsigned* __restrict__ offsets) {
+    pdl_enter();
     using C = RadixCfg<MAXB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const ScatterSmem<MAXB> sm(smem_raw, C::kTileKeys);
@@ -534,6 +538,7 @@ k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __res
                 const int4* __restrict__ rect, unsigned* __restrict__ cnt_rank, unsigned* __restrict__ rc_rank,
                 unsigned char* __restrict__ sub_rank,
                 unsigned* __restrict__ part, SortMisc* __restrict__ misc) {
+    pdl_enter();
     const int base = blockIdx.x * kScanTile;
     unsigned s = 0;
 #pragma unroll
@@ -567,6 +572,7 @@ k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __res
 }
 
 __global__ void __launch_bounds__(1024) k_scan_top(unsigned* __restrict__ part, int nb, SortMisc* __restrict__ misc) {
+    pdl_enter();
     // exclusive scan of nb partial sums by one CTA, each thread a contiguous
     // run; the total (of super-tile pairs, when that is what is scanned) goes
     // to misc->ps, or 0 if the frame's pairs exceed the capacity
@@ -604,6 +610,7 @@ __global__ void __launch_bounds__(kSortBlock)
 k_scan_down(int N, const unsigned* __restrict__ cnt_rank, const unsigned* __restrict__ part,
             unsigned* __restrict__ pair_off, const SortMisc* __restrict__ misc, unsigned G,
             unsigned* __restrict__ owner_lo, unsigned* __restrict__ owner_hi) {
+    pdl_enter();
     // each thread owns kScanItems consecutive ranks
     const int base = blockIdx.x * kScanTile + threadIdx.x * kScanItems;
     unsigned v[kScanItems];
@@ -669,6 +676,7 @@ __global__ void __launch_bounds__(kSortBlock)
 k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
        const int4* __restrict__ rect, const unsigned* __restrict__ tiles_touched, SortMisc* __restrict__ misc,
        unsigned* __restrict__ tkeys, unsigned* __restrict__ tvals) {
+    pdl_enter();
     __shared__ unsigned s_off[kEmitSeg + 1];
     __shared__ unsigned s_g[kEmitSeg + 1];
     __shared__ unsigned s_r0, s_nr;
@@ -722,6 +730,7 @@ k_emit(int N, int TX, const unsigned* __restrict__ order, const unsigned* __rest
 __global__ void k_ranges(const unsigned* __restrict__ tkeys, const unsigned* __restrict__ ids,
                          const float* __restrict__ depth, const SortMisc* __restrict__ misc, unsigned* __restrict__ ranges,
                          unsigned long long* __restrict__ keys) {
+    pdl_enter();
     const unsigned P = misc->p_eff;
     const unsigned nq = (P + 3) / 4;  // quads, the last one partial
     const unsigned stride = gridDim.x * blockDim.x;
@@ -801,6 +810,7 @@ __global__ void __launch_bounds__(kSortBlock)
 k_gen_hist(const unsigned* __restrict__ pair_off, const unsigned* __restrict__ rc_rank,
            const unsigned* __restrict__ n_ptr, const unsigned* __restrict__ owner_lo,
            const unsigned* __restrict__ owner_hi, unsigned* __restrict__ hist, unsigned* __restrict__ totals) {
+    pdl_enter();
     using C = RadixCfg<MAXB>;
     constexpr int kU = 4;  // ranks per thread in flight
     __shared__ int s_d[C::kRadix + 1];
@@ -888,6 +898,7 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
               const unsigned* __restrict__ rc_rank, const unsigned char* __restrict__ sub_rank,
               const unsigned* __restrict__ n_ptr, const unsigned* __restrict__ owner_lo, int bits,
               const unsigned* __restrict__ offsets, unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out) {
+    pdl_enter();
     using C = RadixCfg<MAXB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const ScatterSmem<MAXB> sm(smem_raw, kPadTile);
@@ -1004,6 +1015,7 @@ constexpr size_t gen_scatter_smem() {
 // 16-byte loads, neighbours across lanes by shuffles.
 __global__ void k_cell_ranges(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ n_ptr, int SX,
                               unsigned* __restrict__ cell_ranges) {
+    pdl_enter();
     const unsigned n = *n_ptr;
     const unsigned nq = (n + 3) / 4;
     const unsigned stride = gridDim.x * blockDim.x;
@@ -1080,6 +1092,7 @@ __global__ void __launch_bounds__(1024)
 k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restrict__ cell_seg0,
             unsigned* __restrict__ seg_cell, unsigned* __restrict__ seg_lo, unsigned* __restrict__ seg_hi,
             SortMisc* __restrict__ misc) {
+    pdl_enter();
     __shared__ unsigned s_w[33];
     __shared__ uint2 s_rg[kSegCache];
     __shared__ unsigned s_s0[kSegCache];
@@ -1145,6 +1158,7 @@ __device__ __forceinline__ unsigned packed_count(const unsigned (&acc)[kCellTile
 __global__ void __launch_bounds__(kSortBlock)
 k_seg_count(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ seg_lo,
             const unsigned* __restrict__ seg_hi, const SortMisc* __restrict__ misc, unsigned* __restrict__ seg_cnt) {
+    pdl_enter();
     __shared__ unsigned s_c[kSortBlock / 32][kCellTiles];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned nseg = misc->nseg;
@@ -1183,6 +1197,7 @@ k_seg_count(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ seg
 __global__ void __launch_bounds__(kCellTiles)
 k_cell_scan(int TX, int TY, int SX, const unsigned* __restrict__ cell_seg0, const unsigned* __restrict__ seg_cnt,
             unsigned* __restrict__ seg_base, unsigned* __restrict__ tile_cnt) {
+    pdl_enter();
     const unsigned c = blockIdx.x;
     const int b = threadIdx.x;
     const unsigned k0 = cell_seg0[c], k1 = cell_seg0[c + 1];
@@ -1219,6 +1234,7 @@ __device__ __forceinline__ int pad32(int i) { return i + (i >> 5); }
 __global__ void __launch_bounds__(1024)
 k_tile_scan(int T, const unsigned* __restrict__ tile_cnt, unsigned* __restrict__ tile_start,
             unsigned* __restrict__ ranges) {
+    pdl_enter();
     __shared__ unsigned s_w[33];
     __shared__ unsigned s_start[kTileRound + kTileRound / 32];
     __shared__ unsigned s_cnt[kTileRound + kTileRound / 32];
@@ -1264,6 +1280,7 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
            const unsigned* __restrict__ seg_lo, const unsigned* __restrict__ seg_hi,
            const unsigned* __restrict__ seg_base, const unsigned* __restrict__ tile_start,
            const SortMisc* __restrict__ misc, unsigned* __restrict__ ids, unsigned long long* __restrict__ keys) {
+    pdl_enter();
     constexpr int kW = kSortBlock / 32;
     __shared__ unsigned s_base[kCellTiles];
     __shared__ unsigned s_wb[kW][kCellTiles];
@@ -1349,19 +1366,19 @@ void enable_scatter_smem() {
 }
 
 template <int MAXB>
-void radix_pass(cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
+void radix_pass(bool pdl, cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
                 const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals) {
     enable_scatter_smem<MAXB>();
-    k_radix_hist<MAXB><<<G, kSortBlock, 0, st>>>(ki, n_ptr, shift, bits, hist, totals); note_launch();
-    k_radix_scan<<<1 << bits, kSortBlock, 0, st>>>(hist, totals, G); note_launch();
-    k_radix_scatter<MAXB><<<G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st>>>(ki, vi, ko, vo, n_ptr, shift, bits,
+    launch_pdl(pdl, k_radix_hist<MAXB>, G, kSortBlock, 0, st, ki, n_ptr, shift, bits, hist, totals); note_launch();
+    launch_pdl(pdl, k_radix_scan, 1 << bits, kSortBlock, 0, st, hist, totals, G); note_launch();
+    launch_pdl(pdl, k_radix_scatter<MAXB>, G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st, ki, vi, ko, vo, n_ptr, shift, bits,
                                                                                 hist); note_launch();
 }
 
 // One stable LSD radix sort of (keys, vals) over bits [0, total_bits), with
 // at most 8 bits per pass.  The final pass writes to (final_keys, final_vals)
 // when they are given.  Returns the number of passes.
-int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, unsigned* k0, unsigned* v0,
+int radix_sort(bool pdl, cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, unsigned* k0, unsigned* v0,
                unsigned* k1, unsigned* v1, unsigned* final_vals, unsigned** out_keys, unsigned* hist,
                unsigned* totals, int pass_base) {
     const int passes = (total_bits + 7) / 8;
@@ -1377,9 +1394,9 @@ int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, un
         unsigned* h = hist + (size_t)(pass_base + p) * kRadixMax * kSortMaxGrid;
         unsigned* tot = totals + (size_t)(pass_base + p) * kRadixMax;
         if (bits <= 7)
-            radix_pass<7>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
+            radix_pass<7>(pdl, st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
         else
-            radix_pass<8>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
+            radix_pass<8>(pdl, st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
         unsigned* tk = ki;
         ki = ko;
         ko = tk;
@@ -1413,6 +1430,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     if (rect && !aligned(rect, 16)) return GS_ERR_INVALID_ARG;
     if (ranges && !aligned(ranges, 8)) return GS_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
+    const bool pdl = pdl_allowed(st);  // programmatic dependent launch outside graph capture
     const int TX = tiles_x(*cam), TY = tiles_y(*cam), T = TX * TY;
     BinWs w;
     carve(ws, N, capacity, TX, TY, &w);
@@ -1425,7 +1443,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = (work + 255) / 256;
         if (blocks < 1) blocks = 1;
         if (blocks > 148 * 8) blocks = 148 * 8;
-        k_bin_init<<<blocks, 256, 0, st>>>(N, T, depth, tiles_touched, d_num_pairs, capacity, w, ranges); note_launch();
+        launch_pdl(pdl, k_bin_init, blocks, 256, 0, st, N, T, depth, tiles_touched, d_num_pairs, capacity, w, ranges); note_launch();
         GS_LAUNCH_CHECK();
     }
     if (N == 0) return GS_OK;
@@ -1433,7 +1451,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     // 1. depth ranks of the Gaussians (32-bit keys, culled ones last)
     const int Gd = (N + 2047) / 2048 < kSortMaxGrid ? (N + 2047) / 2048 : kSortMaxGrid;
     unsigned* dkeys_sorted = nullptr;
-    const int dpasses = radix_sort(st, Gd, &w.misc->n_gauss, 32, w.dkeys0, w.dvals0, w.dkeys1, w.dvals1, nullptr,
+    const int dpasses = radix_sort(pdl, st, Gd, &w.misc->n_gauss, 32, w.dkeys0, w.dvals0, w.dkeys1, w.dvals1, nullptr,
                                    &dkeys_sorted, w.hist, w.totals, 0);
     const unsigned* order = (dpasses % 2 == 0) ? w.dvals0 : w.dvals1;
     GS_LAUNCH_CHECK();
@@ -1441,10 +1459,10 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     // 2. pair offsets in rank order (of super-tile pairs on the super-tile route)
     const int nb = (N + kScanTile - 1) / kScanTile;
     const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
-    k_scan_partials<<<nb, kSortBlock, 0, st>>>(N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
+    launch_pdl(pdl, k_scan_partials, nb, kSortBlock, 0, st, N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
                                                w.rc_rank, w.sub_rank, w.scan_part, w.misc); note_launch();
-    k_scan_top<<<1, 1024, 0, st>>>(w.scan_part, nb, w.misc); note_launch();
-    k_scan_down<<<nb, kSortBlock, 0, st>>>(N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
+    launch_pdl(pdl, k_scan_top, 1, 1024, 0, st, w.scan_part, nb, w.misc); note_launch();
+    launch_pdl(pdl, k_scan_down, nb, kSortBlock, 0, st, N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
                                            (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi); note_launch();
     GS_LAUNCH_CHECK();
     if (capacity == 0) return GS_OK;
@@ -1458,17 +1476,17 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         unsigned* h1 = w.hist + (size_t)4 * kRadixMax * kSortMaxGrid;
         unsigned* t1 = w.totals + (size_t)4 * kRadixMax;
         if (bx <= 7) {
-            k_gen_hist<7><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
-            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
+            launch_pdl(pdl, k_gen_hist<7>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
+            launch_pdl(pdl, k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
             opt_in_smem(k_gen_scatter<7>, gen_scatter_smem<7>());
-            k_gen_scatter<7><<<Gp, kSortBlock, gen_scatter_smem<7>(), st>>>(N, order, w.pair_off, w.rc_rank,
+            launch_pdl(pdl, k_gen_scatter<7>, Gp, kSortBlock, gen_scatter_smem<7>(), st, N, order, w.pair_off, w.rc_rank,
                                                                            w.sub_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         } else {
-            k_gen_hist<8><<<Gp, kSortBlock, 0, st>>>(w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
-            k_radix_scan<<<1 << bx, kSortBlock, 0, st>>>(h1, t1, Gp); note_launch();
+            launch_pdl(pdl, k_gen_hist<8>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
+            launch_pdl(pdl, k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
             opt_in_smem(k_gen_scatter<8>, gen_scatter_smem<8>());
-            k_gen_scatter<8><<<Gp, kSortBlock, gen_scatter_smem<8>(), st>>>(N, order, w.pair_off, w.rc_rank,
+            launch_pdl(pdl, k_gen_scatter<8>, Gp, kSortBlock, gen_scatter_smem<8>(), st, N, order, w.pair_off, w.rc_rank,
                                                                            w.sub_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         }
@@ -1476,23 +1494,23 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         unsigned* h2 = w.hist + (size_t)5 * kRadixMax * kSortMaxGrid;
         unsigned* t2 = w.totals + (size_t)5 * kRadixMax;
         if (by <= 7)
-            radix_pass<7>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+            radix_pass<7>(pdl, st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
         else
-            radix_pass<8>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+            radix_pass<8>(pdl, st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
         GS_LAUNCH_CHECK();
         {
             int blocks = (int)((capacity + 1023u) / 1024u);
             if (blocks > 148 * 16) blocks = 148 * 16;
             if (blocks < 1) blocks = 1;
-            k_cell_ranges<<<blocks, 256, 0, st>>>(w.tkeys1, ps, SX, w.cell_ranges); note_launch();
+            launch_pdl(pdl, k_cell_ranges, blocks, 256, 0, st, w.tkeys1, ps, SX, w.cell_ranges); note_launch();
         }
         const int S = SX * SY;
-        k_seg_table<<<1, 1024, 0, st>>>(S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
+        launch_pdl(pdl, k_seg_table, 1, 1024, 0, st, S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
         const int gseg = (int)(w.max_seg < 148u * 8u ? w.max_seg : 148u * 8u);
-        k_seg_count<<<gseg, kSortBlock, 0, st>>>(w.tkeys1, w.seg_lo, w.seg_hi, w.misc, w.seg_cnt); note_launch();
-        k_cell_scan<<<S, kCellTiles, 0, st>>>(TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
-        k_tile_scan<<<1, 1024, 0, st>>>(T, w.tile_cnt, w.tile_start, ranges); note_launch();
-        k_seg_emit<<<gseg, kSortBlock, 0, st>>>(TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell, w.seg_lo,
+        launch_pdl(pdl, k_seg_count, gseg, kSortBlock, 0, st, w.tkeys1, w.seg_lo, w.seg_hi, w.misc, w.seg_cnt); note_launch();
+        launch_pdl(pdl, k_cell_scan, S, kCellTiles, 0, st, TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
+        launch_pdl(pdl, k_tile_scan, 1, 1024, 0, st, T, w.tile_cnt, w.tile_start, ranges); note_launch();
+        launch_pdl(pdl, k_seg_emit, gseg, kSortBlock, 0, st, TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell, w.seg_lo,
                                                 w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys); note_launch();
         GS_LAUNCH_CHECK();
         return GS_OK;
@@ -1507,12 +1525,12 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = segs > 148u * 32u ? 148 * 32 : (int)segs;
         if (blocks < 1) blocks = 1;
         unsigned* emit_vals = tpasses == 0 ? ids : w.tvals0;
-        k_emit<<<blocks, kSortBlock, 0, st>>>(N, TX, order, w.pair_off, reinterpret_cast<const int4*>(rect),
+        launch_pdl(pdl, k_emit, blocks, kSortBlock, 0, st, N, TX, order, w.pair_off, reinterpret_cast<const int4*>(rect),
                                               tiles_touched, w.misc, w.tkeys0, emit_vals); note_launch();
         GS_LAUNCH_CHECK();
     }
     unsigned* tkeys_sorted = nullptr;
-    radix_sort(st, Gp, &w.misc->p_eff, tile_bits, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, ids, &tkeys_sorted,
+    radix_sort(pdl, st, Gp, &w.misc->p_eff, tile_bits, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, ids, &tkeys_sorted,
                w.hist, w.totals, 4);
     GS_LAUNCH_CHECK();
 
@@ -1521,7 +1539,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = (int)((capacity + 1023u) / 1024u);
         if (blocks > 148 * 16) blocks = 148 * 16;
         if (blocks < 1) blocks = 1;
-        k_ranges<<<blocks, 256, 0, st>>>(tkeys_sorted, ids, depth, w.misc, ranges, keys); note_launch();
+        launch_pdl(pdl, k_ranges, blocks, 256, 0, st, tkeys_sorted, ids, depth, w.misc, ranges, keys); note_launch();
         GS_LAUNCH_CHECK();
     }
     return GS_OK;
