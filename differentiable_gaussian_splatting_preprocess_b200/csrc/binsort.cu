@@ -28,6 +28,7 @@
 #include <cuda_runtime.h>
 
 #include "gs_internal.cuh"
+#include "pdl.cuh"
 
 namespace gs {
 namespace {
@@ -1366,19 +1367,19 @@ void enable_scatter_smem() {
 }
 
 template <int MAXB>
-void radix_pass(bool pdl, cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
+void radix_pass(cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
                 const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals) {
     enable_scatter_smem<MAXB>();
-    launch_pdl(pdl, k_radix_hist<MAXB>, G, kSortBlock, 0, st, ki, n_ptr, shift, bits, hist, totals); note_launch();
-    launch_pdl(pdl, k_radix_scan, 1 << bits, kSortBlock, 0, st, hist, totals, G); note_launch();
-    launch_pdl(pdl, k_radix_scatter<MAXB>, G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st, ki, vi, ko, vo, n_ptr, shift, bits,
+    launch_pdl(k_radix_hist<MAXB>, G, kSortBlock, 0, st, ki, n_ptr, shift, bits, hist, totals); note_launch();
+    launch_pdl(k_radix_scan, 1 << bits, kSortBlock, 0, st, hist, totals, G); note_launch();
+    launch_pdl(k_radix_scatter<MAXB>, G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st, ki, vi, ko, vo, n_ptr, shift, bits,
                                                                                 hist); note_launch();
 }
 
 // One stable LSD radix sort of (keys, vals) over bits [0, total_bits), with
 // at most 8 bits per pass.  The final pass writes to (final_keys, final_vals)
 // when they are given.  Returns the number of passes.
-int radix_sort(bool pdl, cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, unsigned* k0, unsigned* v0,
+int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, unsigned* k0, unsigned* v0,
                unsigned* k1, unsigned* v1, unsigned* final_vals, unsigned** out_keys, unsigned* hist,
                unsigned* totals, int pass_base) {
     const int passes = (total_bits + 7) / 8;
@@ -1394,9 +1395,9 @@ int radix_sort(bool pdl, cudaStream_t st, int G, const unsigned* n_ptr, int tota
         unsigned* h = hist + (size_t)(pass_base + p) * kRadixMax * kSortMaxGrid;
         unsigned* tot = totals + (size_t)(pass_base + p) * kRadixMax;
         if (bits <= 7)
-            radix_pass<7>(pdl, st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
+            radix_pass<7>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
         else
-            radix_pass<8>(pdl, st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
+            radix_pass<8>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
         unsigned* tk = ki;
         ki = ko;
         ko = tk;
@@ -1430,7 +1431,6 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     if (rect && !aligned(rect, 16)) return GS_ERR_INVALID_ARG;
     if (ranges && !aligned(ranges, 8)) return GS_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    const bool pdl = pdl_allowed(st);  // programmatic dependent launch outside graph capture
     const int TX = tiles_x(*cam), TY = tiles_y(*cam), T = TX * TY;
     BinWs w;
     carve(ws, N, capacity, TX, TY, &w);
@@ -1443,7 +1443,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = (work + 255) / 256;
         if (blocks < 1) blocks = 1;
         if (blocks > 148 * 8) blocks = 148 * 8;
-        launch_pdl(pdl, k_bin_init, blocks, 256, 0, st, N, T, depth, tiles_touched, d_num_pairs, capacity, w, ranges); note_launch();
+        launch_pdl(k_bin_init, blocks, 256, 0, st, N, T, depth, tiles_touched, d_num_pairs, capacity, w, ranges); note_launch();
         GS_LAUNCH_CHECK();
     }
     if (N == 0) return GS_OK;
@@ -1451,7 +1451,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     // 1. depth ranks of the Gaussians (32-bit keys, culled ones last)
     const int Gd = (N + 2047) / 2048 < kSortMaxGrid ? (N + 2047) / 2048 : kSortMaxGrid;
     unsigned* dkeys_sorted = nullptr;
-    const int dpasses = radix_sort(pdl, st, Gd, &w.misc->n_gauss, 32, w.dkeys0, w.dvals0, w.dkeys1, w.dvals1, nullptr,
+    const int dpasses = radix_sort(st, Gd, &w.misc->n_gauss, 32, w.dkeys0, w.dvals0, w.dkeys1, w.dvals1, nullptr,
                                    &dkeys_sorted, w.hist, w.totals, 0);
     const unsigned* order = (dpasses % 2 == 0) ? w.dvals0 : w.dvals1;
     GS_LAUNCH_CHECK();
@@ -1459,10 +1459,10 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     // 2. pair offsets in rank order (of super-tile pairs on the super-tile route)
     const int nb = (N + kScanTile - 1) / kScanTile;
     const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
-    launch_pdl(pdl, k_scan_partials, nb, kSortBlock, 0, st, N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
+    launch_pdl(k_scan_partials, nb, kSortBlock, 0, st, N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
                                                w.rc_rank, w.sub_rank, w.scan_part, w.misc); note_launch();
-    launch_pdl(pdl, k_scan_top, 1, 1024, 0, st, w.scan_part, nb, w.misc); note_launch();
-    launch_pdl(pdl, k_scan_down, nb, kSortBlock, 0, st, N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
+    launch_pdl(k_scan_top, 1, 1024, 0, st, w.scan_part, nb, w.misc); note_launch();
+    launch_pdl(k_scan_down, nb, kSortBlock, 0, st, N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
                                            (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi); note_launch();
     GS_LAUNCH_CHECK();
     if (capacity == 0) return GS_OK;
@@ -1476,17 +1476,17 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         unsigned* h1 = w.hist + (size_t)4 * kRadixMax * kSortMaxGrid;
         unsigned* t1 = w.totals + (size_t)4 * kRadixMax;
         if (bx <= 7) {
-            launch_pdl(pdl, k_gen_hist<7>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
-            launch_pdl(pdl, k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
+            launch_pdl(k_gen_hist<7>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
+            launch_pdl(k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
             opt_in_smem(k_gen_scatter<7>, gen_scatter_smem<7>());
-            launch_pdl(pdl, k_gen_scatter<7>, Gp, kSortBlock, gen_scatter_smem<7>(), st, N, order, w.pair_off, w.rc_rank,
+            launch_pdl(k_gen_scatter<7>, Gp, kSortBlock, gen_scatter_smem<7>(), st, N, order, w.pair_off, w.rc_rank,
                                                                            w.sub_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         } else {
-            launch_pdl(pdl, k_gen_hist<8>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
-            launch_pdl(pdl, k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
+            launch_pdl(k_gen_hist<8>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
+            launch_pdl(k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
             opt_in_smem(k_gen_scatter<8>, gen_scatter_smem<8>());
-            launch_pdl(pdl, k_gen_scatter<8>, Gp, kSortBlock, gen_scatter_smem<8>(), st, N, order, w.pair_off, w.rc_rank,
+            launch_pdl(k_gen_scatter<8>, Gp, kSortBlock, gen_scatter_smem<8>(), st, N, order, w.pair_off, w.rc_rank,
                                                                            w.sub_rank, ps,
                                                                            w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
         }
@@ -1494,23 +1494,23 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         unsigned* h2 = w.hist + (size_t)5 * kRadixMax * kSortMaxGrid;
         unsigned* t2 = w.totals + (size_t)5 * kRadixMax;
         if (by <= 7)
-            radix_pass<7>(pdl, st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+            radix_pass<7>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
         else
-            radix_pass<8>(pdl, st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+            radix_pass<8>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
         GS_LAUNCH_CHECK();
         {
             int blocks = (int)((capacity + 1023u) / 1024u);
             if (blocks > 148 * 16) blocks = 148 * 16;
             if (blocks < 1) blocks = 1;
-            launch_pdl(pdl, k_cell_ranges, blocks, 256, 0, st, w.tkeys1, ps, SX, w.cell_ranges); note_launch();
+            launch_pdl(k_cell_ranges, blocks, 256, 0, st, w.tkeys1, ps, SX, w.cell_ranges); note_launch();
         }
         const int S = SX * SY;
-        launch_pdl(pdl, k_seg_table, 1, 1024, 0, st, S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
+        launch_pdl(k_seg_table, 1, 1024, 0, st, S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
         const int gseg = (int)(w.max_seg < 148u * 8u ? w.max_seg : 148u * 8u);
-        launch_pdl(pdl, k_seg_count, gseg, kSortBlock, 0, st, w.tkeys1, w.seg_lo, w.seg_hi, w.misc, w.seg_cnt); note_launch();
-        launch_pdl(pdl, k_cell_scan, S, kCellTiles, 0, st, TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
-        launch_pdl(pdl, k_tile_scan, 1, 1024, 0, st, T, w.tile_cnt, w.tile_start, ranges); note_launch();
-        launch_pdl(pdl, k_seg_emit, gseg, kSortBlock, 0, st, TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell, w.seg_lo,
+        launch_pdl(k_seg_count, gseg, kSortBlock, 0, st, w.tkeys1, w.seg_lo, w.seg_hi, w.misc, w.seg_cnt); note_launch();
+        launch_pdl(k_cell_scan, S, kCellTiles, 0, st, TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
+        launch_pdl(k_tile_scan, 1, 1024, 0, st, T, w.tile_cnt, w.tile_start, ranges); note_launch();
+        launch_pdl(k_seg_emit, gseg, kSortBlock, 0, st, TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell, w.seg_lo,
                                                 w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys); note_launch();
         GS_LAUNCH_CHECK();
         return GS_OK;
@@ -1525,12 +1525,12 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = segs > 148u * 32u ? 148 * 32 : (int)segs;
         if (blocks < 1) blocks = 1;
         unsigned* emit_vals = tpasses == 0 ? ids : w.tvals0;
-        launch_pdl(pdl, k_emit, blocks, kSortBlock, 0, st, N, TX, order, w.pair_off, reinterpret_cast<const int4*>(rect),
+        launch_pdl(k_emit, blocks, kSortBlock, 0, st, N, TX, order, w.pair_off, reinterpret_cast<const int4*>(rect),
                                               tiles_touched, w.misc, w.tkeys0, emit_vals); note_launch();
         GS_LAUNCH_CHECK();
     }
     unsigned* tkeys_sorted = nullptr;
-    radix_sort(pdl, st, Gp, &w.misc->p_eff, tile_bits, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, ids, &tkeys_sorted,
+    radix_sort(st, Gp, &w.misc->p_eff, tile_bits, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, ids, &tkeys_sorted,
                w.hist, w.totals, 4);
     GS_LAUNCH_CHECK();
 
@@ -1539,7 +1539,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         int blocks = (int)((capacity + 1023u) / 1024u);
         if (blocks > 148 * 16) blocks = 148 * 16;
         if (blocks < 1) blocks = 1;
-        launch_pdl(pdl, k_ranges, blocks, 256, 0, st, tkeys_sorted, ids, depth, w.misc, ranges, keys); note_launch();
+        launch_pdl(k_ranges, blocks, 256, 0, st, tkeys_sorted, ids, depth, w.misc, ranges, keys); note_launch();
         GS_LAUNCH_CHECK();
     }
     return GS_OK;

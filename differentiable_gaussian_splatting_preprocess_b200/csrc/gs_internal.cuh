@@ -31,49 +31,6 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // called after every launch statement.
 void note_launch();
 
-// Programmatic dependent launch (sm_90 and later): a kernel launched with
-// launch_pdl(true, ...) may be scheduled while the kernel before it in the stream is
-// still running; its threads first wait (griddepcontrol.wait: until that
-// kernel has completed and its memory operations are visible), then allow
-// the next kernel to be scheduled in turn.  Only the launch latency and the
-// ramp-up overlap the previous kernel's tail; no kernel reads anything
-// before its predecessor is complete.  The wait is the hardware's; without
-// the launch attribute both instructions do nothing.
-__device__ __forceinline__ void pdl_enter() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// Whether launches on `st` should use programmatic dependent launch: only
-// when the stream is not being captured into a CUDA graph (measured: eager
-// chains of short kernels gain, graph replays lose - a graph already
-// launches its kernels back to back, and blocks launched early wait on SMs
-// that other work could use).
-inline bool pdl_allowed(cudaStream_t st) {
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
-        cudaGetLastError();  // clear the query's error; launch plainly
-        return false;
-    }
-    return cs == cudaStreamCaptureStatusNone;
-}
-
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                              cudaStream_t st, Args&&... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
-}
-
 // Kernels that use more than the default 48 KiB of dynamic shared memory
 // must opt in once per device.  Done on first use and remembered, so later
 // calls (including calls recorded into a CUDA graph) issue no attribute call.
