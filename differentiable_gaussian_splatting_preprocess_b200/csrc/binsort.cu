@@ -204,9 +204,24 @@ __global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const 
     for (int i = tid; i < 2 * T; i += stride) ranges[i] = 0u;
     for (int i = tid; i < kMaxPasses * kRadixMax; i += stride) w.totals[i] = 0u;
     for (int i = tid; i < 2 * w.n_cells; i += stride) w.cell_ranges[i] = 0u;
-    for (int i = tid; i < N; i += stride) {
-        w.dkeys0[i] = tiles_touched[i] > 0 ? __float_as_uint(depth[i]) : 0xFFFFFFFFu;
-        w.dvals0[i] = (unsigned)i;
+    // four items per thread and round, their loads issued together
+    constexpr int kU = 4;
+    for (long long i0 = tid; i0 < N; i0 += (long long)kU * stride) {
+        unsigned tt[kU], dk[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const long long i = i0 + (long long)u * stride;
+            tt[u] = i < N ? tiles_touched[i] : 0u;
+            dk[u] = i < N ? __float_as_uint(depth[i]) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const long long i = i0 + (long long)u * stride;
+            if (i < N) {
+                w.dkeys0[i] = tt[u] > 0 ? dk[u] : 0xFFFFFFFFu;
+                w.dvals0[i] = (unsigned)i;
+            }
+        }
     }
     if (tid == 0) {
         const unsigned P = *d_num_pairs;
@@ -541,24 +556,37 @@ k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __res
                 unsigned* __restrict__ part, SortMisc* __restrict__ misc) {
     pdl_enter();
     const int base = blockIdx.x * kScanTile;
+    // the gathers are issued in two rounds of independent loads (all ids,
+    // then every count and rectangle), not as one dependent chain per rank
+    unsigned g[kScanItems];
+#pragma unroll
+    for (int k = 0; k < kScanItems; ++k) {
+        const int r = base + k * kSortBlock + threadIdx.x;
+        g[k] = r < N ? order[r] : 0xFFFFFFFFu;
+    }
+    unsigned v[kScanItems];
+    int4 tr[kScanItems];
+#pragma unroll
+    for (int k = 0; k < kScanItems; ++k) {
+        const bool ok = g[k] < (unsigned)N && id_ok(g[k]);
+        v[k] = ok ? tiles_touched[g[k]] : 0u;
+        if (rect) tr[k] = ok ? rect[g[k]] : make_int4(0, 0, 0, 0);
+    }
     unsigned s = 0;
 #pragma unroll
     for (int k = 0; k < kScanItems; ++k) {
         const int r = base + k * kSortBlock + threadIdx.x;
         if (r < N) {
-            const unsigned g = order[r];
-            unsigned v = 0u;
-            if (id_ok(g)) v = tiles_touched[g];
-            else abort_frame(misc);
-            if (rect && v) {
-                const int4 tr = rect[g];
-                const int4 sr = super_rect(tr);
-                v = (unsigned)((sr.z - sr.x) * (sr.w - sr.y));
+            if (!id_ok(g[k])) abort_frame(misc);
+            unsigned c = v[k];
+            if (rect && c) {
+                const int4 sr = super_rect(tr[k]);
+                c = (unsigned)((sr.z - sr.x) * (sr.w - sr.y));
                 rc_rank[r] = pack_rect(sr);
-                sub_rank[r] = (unsigned char)sub_offsets(tr);
+                sub_rank[r] = (unsigned char)sub_offsets(tr[k]);
             }
-            cnt_rank[r] = v;
-            s += v;
+            cnt_rank[r] = c;
+            s += c;
         }
     }
     s = __reduce_add_sync(0xffffffffu, s);
