@@ -1220,35 +1220,41 @@ k_seg_count(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ seg
     }
 }
 
-// One thread per (cell, tile bit): exclusive prefix of the per-segment
-// counts over the cell's segments, and the tile's total.  Eight segments'
-// counts are loaded at a time, so their latencies overlap.
-__global__ void __launch_bounds__(kCellTiles)
+// One CTA per cell: exclusive prefix of the per-segment counts over the
+// cell's segments, per tile bit, and the tile's total.  The cell's segments
+// are cut into kCellScanGroups contiguous runs; thread (run g, tile bit b)
+// sums run g's counts of bit b, the runs' sums are scanned in shared memory,
+// and each thread then writes its run's bases.  All loads of a pass are
+// independent, so a cell with many segments costs two rounds of latency.
+constexpr int kCellScanGroups = 16;
+
+__global__ void __launch_bounds__(kCellTiles * kCellScanGroups)
 k_cell_scan(int TX, int TY, int SX, const unsigned* __restrict__ cell_seg0, const unsigned* __restrict__ seg_cnt,
             unsigned* __restrict__ seg_base, unsigned* __restrict__ tile_cnt) {
     pdl_enter();
+    __shared__ unsigned s_sum[kCellScanGroups][kCellTiles];
     const unsigned c = blockIdx.x;
-    const int b = threadIdx.x;
+    const int b = threadIdx.x % kCellTiles, grp = threadIdx.x / kCellTiles;
     const unsigned k0 = cell_seg0[c], k1 = cell_seg0[c + 1];
+    const unsigned n = k1 - k0;
+    const unsigned per = (n + kCellScanGroups - 1) / kCellScanGroups;
+    const unsigned ka = k0 + min(n, (unsigned)grp * per), kb = k0 + min(n, (unsigned)(grp + 1) * per);
+    unsigned sum = 0;
+    for (unsigned k = ka; k < kb; ++k) sum += seg_cnt[(size_t)k * kCellTiles + b];
+    s_sum[grp][b] = sum;
+    __syncthreads();
     unsigned run = 0;
-    unsigned k = k0;
-    for (; k + 8 <= k1; k += 8) {
-        unsigned v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = seg_cnt[(size_t)(k + j) * kCellTiles + b];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            seg_base[(size_t)(k + j) * kCellTiles + b] = run;
-            run += v[j];
-        }
-    }
-    for (; k < k1; ++k) {
+    for (int g2 = 0; g2 < grp; ++g2) run += s_sum[g2][b];
+    for (unsigned k = ka; k < kb; ++k) {
         const unsigned v = seg_cnt[(size_t)k * kCellTiles + b];
         seg_base[(size_t)k * kCellTiles + b] = run;
         run += v;
     }
-    const int tx = kSuper * (int)(c % (unsigned)SX) + b % kSuper, ty = kSuper * (int)(c / (unsigned)SX) + b / kSuper;
-    if (tx < TX && ty < TY) tile_cnt[ty * TX + tx] = run;
+    if (grp == kCellScanGroups - 1) {  // run is now the cell's total for bit b
+        const int tx = kSuper * (int)(c % (unsigned)SX) + b % kSuper;
+        const int ty = kSuper * (int)(c / (unsigned)SX) + b / kSuper;
+        if (tx < TX && ty < TY) tile_cnt[ty * TX + tx] = run;
+    }
 }
 
 // Exclusive scan of the tile counts in tile order (one CTA, 4096 tiles per
@@ -1303,6 +1309,7 @@ k_tile_scan(int T, const unsigned* __restrict__ tile_cnt, unsigned* __restrict__
 // order after the running base), then each warp writes, per tile bit, its
 // Gaussians at base + ballot rank: consecutive lanes, consecutive addresses.
 // Optional 64-bit (tile << 32 | depth bits) keys.
+template <bool kKeys>
 __global__ void __launch_bounds__(kSortBlock)
 k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const unsigned* __restrict__ ckeys,
            const float* __restrict__ depth, const unsigned* __restrict__ seg_cell,
@@ -1312,7 +1319,7 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
     pdl_enter();
     constexpr int kW = kSortBlock / 32;
     __shared__ unsigned s_base[kCellTiles];
-    __shared__ unsigned s_wb[kW][kCellTiles];
+    __shared__ __align__(16) unsigned s_wb[kW][kCellTiles];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned lt = lanemask_lt();
     const unsigned nseg = misc->nseg;
@@ -1340,7 +1347,6 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
             if (base >= hi) break;  // block-uniform
             const unsigned g = gs[jc];
             const unsigned m = ms[jc];
-            const unsigned un = __reduce_or_sync(0xffffffffu, m);
             // this warp's count per tile bit (packed byte counters)
             unsigned acc[kCellTiles / 4] = {};
             add_mask(acc, m);
@@ -1360,21 +1366,30 @@ k_seg_emit(int TX, int TY, int SX, const unsigned* __restrict__ clist, const uns
                 s_base[b] = run;
             }
             __syncthreads();
-            const float dg = (keys && m && id_ok(g)) ? depth[g] : 0.0f;
+            const float dg = (kKeys && m && id_ok(g)) ? depth[g] : 0.0f;
             // tile bits in order, unrolled: no find-first-set / bit-reverse
-            // (XU) instructions; skipped bits cost one uniform branch
+            // (XU) instructions, and no test of the warp's union of masks
+            // (a row of 32 list entries almost always touches all 16 tiles);
+            // the warp's bases come four at a time
 #pragma unroll
-            for (int b = 0; b < kCellTiles; ++b) {
-                if (!((un >> b) & 1u)) continue;
-                const bool mine = (m >> b) & 1u;
-                const unsigned bal = __ballot_sync(0xffffffffu, mine);
-                if (mine) {
-                    const unsigned pos = s_wb[warp][b] + __popc(bal & lt);
-                    if (!pos_ok(pos)) continue;
-                    ids[pos] = g;
-                    if (keys) {
-                        const unsigned t = (unsigned)((kSuper * cy + b / kSuper) * TX + kSuper * cx + b % kSuper);
-                        keys[pos] = ((unsigned long long)t << 32) | __float_as_uint(dg);
+            for (int q = 0; q < kCellTiles / 4; ++q) {
+                const uint4 b4 = *reinterpret_cast<const uint4*>(&s_wb[warp][4 * q]);
+                const unsigned wb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int b = 4 * q + i;
+                    const bool mine = (m >> b) & 1u;
+                    const unsigned bal = __ballot_sync(0xffffffffu, mine);
+                    if (mine) {
+                        const unsigned pos = wb[i] + __popc(bal & lt);
+                        if (pos_ok(pos)) {
+                            ids[pos] = g;
+                            if (kKeys) {
+                                const unsigned t =
+                                    (unsigned)((kSuper * cy + b / kSuper) * TX + kSuper * cx + b % kSuper);
+                                keys[pos] = ((unsigned long long)t << 32) | __float_as_uint(dg);
+                            }
+                        }
                     }
                 }
             }
@@ -1536,10 +1551,15 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         launch_pdl(k_seg_table, 1, 1024, 0, st, S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
         const int gseg = (int)(w.max_seg < 148u * 8u ? w.max_seg : 148u * 8u);
         launch_pdl(k_seg_count, gseg, kSortBlock, 0, st, w.tkeys1, w.seg_lo, w.seg_hi, w.misc, w.seg_cnt); note_launch();
-        launch_pdl(k_cell_scan, S, kCellTiles, 0, st, TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
+        launch_pdl(k_cell_scan, S, kCellTiles * kCellScanGroups, 0, st, TX, TY, SX, w.cell_seg0, w.seg_cnt, w.seg_base, w.tile_cnt); note_launch();
         launch_pdl(k_tile_scan, 1, 1024, 0, st, T, w.tile_cnt, w.tile_start, ranges); note_launch();
-        launch_pdl(k_seg_emit, gseg, kSortBlock, 0, st, TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell, w.seg_lo,
-                                                w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys); note_launch();
+        if (keys)
+            launch_pdl(k_seg_emit<true>, gseg, kSortBlock, 0, st, TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell,
+                       w.seg_lo, w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys);
+        else
+            launch_pdl(k_seg_emit<false>, gseg, kSortBlock, 0, st, TX, TY, SX, w.tvals1, w.tkeys1, depth, w.seg_cell,
+                       w.seg_lo, w.seg_hi, w.seg_base, w.tile_start, w.misc, ids, keys);
+        note_launch();
         GS_LAUNCH_CHECK();
         return GS_OK;
     }
