@@ -36,6 +36,8 @@ namespace {
 constexpr int kSortBlock = 256;
 constexpr int kSortMaxGrid = 148 * 4;  // CTAs per radix pass: a multiple of the SM count
 constexpr int kRadixMax = 256;
+constexpr int kScanGroup = 32;         // chunks per group of the per-group digit totals
+constexpr int kMaxGroups = (kSortMaxGrid + kScanGroup - 1) / kScanGroup;
 constexpr int kMaxPasses = 8;          // 4 depth passes + up to 3 tile passes (+1 spare)
 constexpr int kScanItems = 8;          // items per thread in the rank-order scan
 constexpr int kScanTile = kSortBlock * kScanItems;
@@ -57,8 +59,9 @@ struct BinWs {
     unsigned* cnt_rank;                            // N: pairs of each rank (written by the scan's first kernel)
     unsigned* scan_part;                           // ceil(N / kScanTile) + 1
     unsigned *tkeys0, *tvals0, *tkeys1, *tvals1;   // pair sort, capacity each
-    unsigned* hist;                                // kMaxPasses * kRadixMax * kSortMaxGrid
+    unsigned* hist;                                // kMaxPasses * kSortMaxGrid * kRadixMax (chunk-major)
     unsigned* totals;                              // kMaxPasses * kRadixMax
+    unsigned* gtot;                                // kMaxPasses * kMaxGroups * kRadixMax (group-major)
     // super-tile route only (empty otherwise)
     unsigned* rc_rank;                             // N packed super-tile rectangles in rank order
     unsigned char* sub_rank;                       // N: the tile rectangle's offsets in its edge cells (sub_offsets)
@@ -111,6 +114,7 @@ size_t carve(void* base, int N, unsigned capacity, int TX, int TY, BinWs* w) {
     t.tvals1 = (unsigned*)take(cap * 4);
     t.hist = (unsigned*)take((size_t)kMaxPasses * kRadixMax * kSortMaxGrid * 4);
     t.totals = (unsigned*)take((size_t)kMaxPasses * kRadixMax * 4);
+    t.gtot = (unsigned*)take((size_t)kMaxPasses * kMaxGroups * kRadixMax * 4);
     const bool sup = super_binning(TX, TY);
     const size_t S = sup ? (size_t)((TX + kSuper - 1) / kSuper) * ((TY + kSuper - 1) / kSuper) : 0;
     const size_t T = sup ? (size_t)TX * TY : 0;
@@ -203,6 +207,7 @@ __global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const 
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
     for (int i = tid; i < 2 * T; i += stride) ranges[i] = 0u;
     for (int i = tid; i < kMaxPasses * kRadixMax; i += stride) w.totals[i] = 0u;
+    for (int i = tid; i < kMaxPasses * kMaxGroups * kRadixMax; i += stride) w.gtot[i] = 0u;
     for (int i = tid; i < 2 * w.n_cells; i += stride) w.cell_ranges[i] = 0u;
     // four items per thread and round, their loads issued together
     constexpr int kU = 4;
@@ -291,13 +296,15 @@ __device__ __forceinline__ unsigned digit_peers(unsigned d, int bits) {
     return m;
 }
 
-// Per-CTA digit histogram of its chunk, stored digit-major (hist[d * G + cta]);
-// digit totals accumulate into totals[d].  Each warp counts into its own
-// shared-memory histogram.
+// Per-CTA digit histogram of its chunk, stored chunk-major
+// (hist[cta * kRadixMax + d]); digit totals accumulate into totals[d] and the
+// totals of each group of kScanGroup consecutive chunks into
+// gtot[group * kRadixMax + d] (see chunk_bases).  Each warp counts into its
+// own shared-memory histogram.
 template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_radix_hist(const unsigned* __restrict__ keys, const unsigned* __restrict__ n_ptr, int shift, int bits,
-             unsigned* __restrict__ hist, unsigned* __restrict__ totals) {
+             unsigned* __restrict__ hist, unsigned* __restrict__ totals, unsigned* __restrict__ gtot) {
     pdl_enter();
     using C = RadixCfg<MAXB>;
     __shared__ unsigned s_h[C::kWarps][C::kRadix];
@@ -329,59 +336,60 @@ k_radix_hist(const unsigned* __restrict__ keys, const unsigned* __restrict__ n_p
         }
     }
     __syncthreads();
-    const unsigned G = gridDim.x;
     for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) {
         unsigned c = 0;
 #pragma unroll
         for (int w = 0; w < C::kWarps; ++w) c += s_h[w][dd];
-        hist[(size_t)dd * G + blockIdx.x] = c;
-        if (c) atomicAdd(&totals[dd], c);
+        hist[(size_t)blockIdx.x * kRadixMax + dd] = c;
+        if (c) {
+            atomicAdd(&totals[dd], c);
+            atomicAdd(&gtot[(blockIdx.x / kScanGroup) * kRadixMax + dd], c);
+        }
     }
 }
 
-// One CTA per digit d: offsets[d][c] = (sum of totals below d) + exclusive
-// prefix over CTAs of hist[d][.], in place.
-__global__ void __launch_bounds__(kSortBlock)
-k_radix_scan(unsigned* __restrict__ hist, const unsigned* __restrict__ totals, int G) {
-    pdl_enter();
-    const int d = blockIdx.x;
-    __shared__ unsigned s_w[kSortBlock / 32];
-    __shared__ unsigned s_base;
-    unsigned b = 0;
-    for (int e = threadIdx.x; e < d; e += kSortBlock) b += totals[e];
-    b = __reduce_add_sync(0xffffffffu, b);
-    if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = b;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned s2 = 0;
-        for (int k = 0; k < kSortBlock / 32; ++k) s2 += s_w[k];
-        s_base = s2;
+// Global output base of each digit for this CTA's chunk (thread d < radix
+// writes base[d]): the totals of the smaller digits, plus digit d's counts in
+// the chunks before this one - whole groups of kScanGroup chunks from the
+// group totals, the rest of this chunk's group from the chunk counts.  At
+// most kMaxGroups - 1 + kScanGroup - 1 independent loads per thread, each a
+// coalesced row over the digits; no separate scan pass over the histograms.
+// Ends with a block barrier.
+__device__ __forceinline__ void chunk_bases(const unsigned* __restrict__ hist, const unsigned* __restrict__ totals,
+                                            const unsigned* __restrict__ gtot, int radix, unsigned* __restrict__ base) {
+    static_assert(kSortBlock == kRadixMax, "one thread per digit");
+    __shared__ unsigned s_w[kSortBlock / 32 + 1];
+    const int d = threadIdx.x;
+    const unsigned c = blockIdx.x, g = c / kScanGroup;
+    const bool in = d < radix;
+    const unsigned t = in ? totals[d] : 0u;
+    unsigned pre = 0;
+    if (in) {
+#pragma unroll
+        for (int k = 0; k < kMaxGroups - 1; ++k)
+            if ((unsigned)k < g) pre += gtot[k * kRadixMax + d];
+#pragma unroll
+        for (int k = 0; k < kScanGroup - 1; ++k) {
+            const unsigned cc = g * kScanGroup + (unsigned)k;
+            if (cc < c) pre += hist[(size_t)cc * kRadixMax + d];
+        }
     }
-    __syncthreads();
-    const int per = (G + kSortBlock - 1) / kSortBlock;
-    unsigned* row = hist + (size_t)d * G;
-    const int c0 = threadIdx.x * per;
-    unsigned local = 0;
-    for (int k = 0; k < per; ++k)
-        if (c0 + k < G) local += row[c0 + k];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned incl = local;
+    // exclusive prefix of the digit totals over the block
+    const int lane = d & 31, warp = d >> 5;
+    unsigned incl = t;
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
     }
-    __syncthreads();
     if (lane == 31) s_w[warp] = incl;
     __syncthreads();
     unsigned wbase = 0;
-    for (int k = 0; k < warp; ++k) wbase += s_w[k];
-    unsigned run = s_base + wbase + incl - local;
-    for (int k = 0; k < per; ++k)
-        if (c0 + k < G) {
-            const unsigned c = row[c0 + k];
-            row[c0 + k] = run;
-            run += c;
-        }
+#pragma unroll
+    for (int k = 0; k < kSortBlock / 32; ++k)
+        if (k < warp) wbase += s_w[k];
+    if (in) base[d] = wbase + incl - t + pre;
+    __syncthreads();
 }
 
 // Stable scatter of one tile of up to 2048 keys, each warp owning a
@@ -516,15 +524,15 @@ template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict__ vals_in,
                 unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out,
-                const unsigned* __restrict__ n_ptr, int shift, int bits, const unsigned* __restrict__ offsets) {
+                const unsigned* __restrict__ n_ptr, int shift, int bits, const unsigned* __restrict__ hist,
+                const unsigned* __restrict__ totals, const unsigned* __restrict__ gtot) {
     pdl_enter();
     using C = RadixCfg<MAXB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const ScatterSmem<MAXB> sm(smem_raw, C::kTileKeys);
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
-    const unsigned G = gridDim.x;
-    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) sm.base[dd] = offsets[(size_t)dd * G + blockIdx.x];
+    chunk_bases(hist, totals, gtot, radix, sm.base);
     unsigned lo, hi;
     chunk_of<MAXB>(*n_ptr, lo, hi);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -838,7 +846,8 @@ template <int MAXB>
 __global__ void __launch_bounds__(kSortBlock)
 k_gen_hist(const unsigned* __restrict__ pair_off, const unsigned* __restrict__ rc_rank,
            const unsigned* __restrict__ n_ptr, const unsigned* __restrict__ owner_lo,
-           const unsigned* __restrict__ owner_hi, unsigned* __restrict__ hist, unsigned* __restrict__ totals) {
+           const unsigned* __restrict__ owner_hi, unsigned* __restrict__ hist, unsigned* __restrict__ totals,
+           unsigned* __restrict__ gtot) {
     pdl_enter();
     using C = RadixCfg<MAXB>;
     constexpr int kU = 4;  // ranks per thread in flight
@@ -905,13 +914,15 @@ k_gen_hist(const unsigned* __restrict__ pair_off, const unsigned* __restrict__ r
             if (lane >= o) incl += y;
         }
         int run = incl - sum;
-        const unsigned G = gridDim.x;
 #pragma unroll
         for (int k = 0; k < per; ++k) {
             run += v[k];
             const int dd = lane * per + k;
-            hist[(size_t)dd * G + blockIdx.x] = (unsigned)run;
-            if (run) atomicAdd(&totals[dd], (unsigned)run);
+            hist[(size_t)blockIdx.x * kRadixMax + dd] = (unsigned)run;
+            if (run) {
+                atomicAdd(&totals[dd], (unsigned)run);
+                atomicAdd(&gtot[(blockIdx.x / kScanGroup) * kRadixMax + dd], (unsigned)run);
+            }
         }
     }
 }
@@ -922,11 +933,12 @@ k_gen_hist(const unsigned* __restrict__ pair_off, const unsigned* __restrict__ r
 // (thread t: tile slots 8t .. 8t+7, one binary search for the first slot,
 // then a walk), and hand them to scatter_tile ranked by tx.
 template <int MAXB>
-__global__ void __launch_bounds__(kSortBlock)
+__global__ void __launch_bounds__(kSortBlock, 4)
 k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restrict__ pair_off,
               const unsigned* __restrict__ rc_rank, const unsigned char* __restrict__ sub_rank,
               const unsigned* __restrict__ n_ptr, const unsigned* __restrict__ owner_lo, int bits,
-              const unsigned* __restrict__ offsets, unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out) {
+              const unsigned* __restrict__ hist, const unsigned* __restrict__ totals,
+              const unsigned* __restrict__ gtot, unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out) {
     pdl_enter();
     using C = RadixCfg<MAXB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -938,8 +950,7 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
     __shared__ unsigned s_r0;
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
-    const unsigned G = gridDim.x;
-    for (int dd = threadIdx.x; dd < radix; dd += kSortBlock) sm.base[dd] = offsets[(size_t)dd * G + blockIdx.x];
+    chunk_bases(hist, totals, gtot, radix, sm.base);
     const unsigned P = *n_ptr;
     unsigned lo, hi;
     chunk_of<MAXB>(P, lo, hi);
@@ -1411,12 +1422,12 @@ void enable_scatter_smem() {
 
 template <int MAXB>
 void radix_pass(cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
-                const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals) {
+                const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals, unsigned* gtot) {
     enable_scatter_smem<MAXB>();
-    launch_pdl(k_radix_hist<MAXB>, G, kSortBlock, 0, st, ki, n_ptr, shift, bits, hist, totals); note_launch();
-    launch_pdl(k_radix_scan, 1 << bits, kSortBlock, 0, st, hist, totals, G); note_launch();
+    launch_pdl(k_radix_hist<MAXB>, G, kSortBlock, 0, st, ki, n_ptr, shift, bits, hist, totals, gtot); note_launch();
     launch_pdl(k_radix_scatter<MAXB>, G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st, ki, vi, ko, vo, n_ptr, shift, bits,
-                                                                                hist); note_launch();
+               hist, totals, gtot);
+    note_launch();
 }
 
 // One stable LSD radix sort of (keys, vals) over bits [0, total_bits), with
@@ -1424,7 +1435,7 @@ void radix_pass(cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bi
 // when they are given.  Returns the number of passes.
 int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, unsigned* k0, unsigned* v0,
                unsigned* k1, unsigned* v1, unsigned* final_vals, unsigned** out_keys, unsigned* hist,
-               unsigned* totals, int pass_base) {
+               unsigned* totals, unsigned* gtot, int pass_base) {
     const int passes = (total_bits + 7) / 8;
     if (passes == 0) {
         *out_keys = k0;
@@ -1437,10 +1448,11 @@ int radix_sort(cudaStream_t st, int G, const unsigned* n_ptr, int total_bits, un
         unsigned* vdst = (last && final_vals) ? final_vals : vo;
         unsigned* h = hist + (size_t)(pass_base + p) * kRadixMax * kSortMaxGrid;
         unsigned* tot = totals + (size_t)(pass_base + p) * kRadixMax;
+        unsigned* gt = gtot + (size_t)(pass_base + p) * kMaxGroups * kRadixMax;
         if (bits <= 7)
-            radix_pass<7>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
+            radix_pass<7>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot, gt);
         else
-            radix_pass<8>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot);
+            radix_pass<8>(st, G, n_ptr, p * bits, bits, ki, vi, ko, vdst, h, tot, gt);
         unsigned* tk = ki;
         ki = ko;
         ko = tk;
@@ -1495,7 +1507,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     const int Gd = (N + 2047) / 2048 < kSortMaxGrid ? (N + 2047) / 2048 : kSortMaxGrid;
     unsigned* dkeys_sorted = nullptr;
     const int dpasses = radix_sort(st, Gd, &w.misc->n_gauss, 32, w.dkeys0, w.dvals0, w.dkeys1, w.dvals1, nullptr,
-                                   &dkeys_sorted, w.hist, w.totals, 0);
+                                   &dkeys_sorted, w.hist, w.totals, w.gtot, 0);
     const unsigned* order = (dpasses % 2 == 0) ? w.dvals0 : w.dvals1;
     GS_LAUNCH_CHECK();
 
@@ -1518,28 +1530,32 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         const int bx = ceil_log2((unsigned)SX), by = ceil_log2((unsigned)SY);
         unsigned* h1 = w.hist + (size_t)4 * kRadixMax * kSortMaxGrid;
         unsigned* t1 = w.totals + (size_t)4 * kRadixMax;
+        unsigned* g1 = w.gtot + (size_t)4 * kMaxGroups * kRadixMax;
         if (bx <= 7) {
-            launch_pdl(k_gen_hist<7>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
-            launch_pdl(k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
+            launch_pdl(k_gen_hist<7>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1,
+                       g1);
+            note_launch();
             opt_in_smem(k_gen_scatter<7>, gen_scatter_smem<7>());
             launch_pdl(k_gen_scatter<7>, Gp, kSortBlock, gen_scatter_smem<7>(), st, N, order, w.pair_off, w.rc_rank,
-                                                                           w.sub_rank, ps,
-                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
+                       w.sub_rank, ps, w.owner_lo, bx, h1, t1, g1, w.tkeys0, w.tvals0);
+            note_launch();
         } else {
-            launch_pdl(k_gen_hist<8>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1); note_launch();
-            launch_pdl(k_radix_scan, 1 << bx, kSortBlock, 0, st, h1, t1, Gp); note_launch();
+            launch_pdl(k_gen_hist<8>, Gp, kSortBlock, 0, st, w.pair_off, w.rc_rank, ps, w.owner_lo, w.owner_hi, h1, t1,
+                       g1);
+            note_launch();
             opt_in_smem(k_gen_scatter<8>, gen_scatter_smem<8>());
             launch_pdl(k_gen_scatter<8>, Gp, kSortBlock, gen_scatter_smem<8>(), st, N, order, w.pair_off, w.rc_rank,
-                                                                           w.sub_rank, ps,
-                                                                           w.owner_lo, bx, h1, w.tkeys0, w.tvals0); note_launch();
+                       w.sub_rank, ps, w.owner_lo, bx, h1, t1, g1, w.tkeys0, w.tvals0);
+            note_launch();
         }
         GS_LAUNCH_CHECK();
         unsigned* h2 = w.hist + (size_t)5 * kRadixMax * kSortMaxGrid;
         unsigned* t2 = w.totals + (size_t)5 * kRadixMax;
+        unsigned* g2 = w.gtot + (size_t)5 * kMaxGroups * kRadixMax;
         if (by <= 7)
-            radix_pass<7>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+            radix_pass<7>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2, g2);
         else
-            radix_pass<8>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2);
+            radix_pass<8>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2, g2);
         GS_LAUNCH_CHECK();
         {
             int blocks = (int)((capacity + 1023u) / 1024u);
@@ -1579,7 +1595,7 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     }
     unsigned* tkeys_sorted = nullptr;
     radix_sort(st, Gp, &w.misc->p_eff, tile_bits, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, ids, &tkeys_sorted,
-               w.hist, w.totals, 4);
+               w.hist, w.totals, w.gtot, 4);
     GS_LAUNCH_CHECK();
 
     // 4. tile ranges (and optional 64-bit keys)

@@ -461,3 +461,49 @@ def test_backward_order_from_partition_histograms(T):
             order[pos] = u
     codes = [_order_code(work[u]) for u in order]
     assert all(a >= b for a, b in zip(codes, codes[1:]))
+
+
+# --- radix pass bases: each scatter CTA derives its own digit bases ---------
+SORT_MAX_GRID = 148 * 4
+SCAN_GROUP = 32
+MAX_GROUPS = (SORT_MAX_GRID + SCAN_GROUP - 1) // SCAN_GROUP
+
+
+def _chunk_bases_model(hist, totals, gtot, c):
+    """chunk_bases as the kernel computes it for CTA c: the digit totals'
+    exclusive prefix, the group totals of the whole groups before c's group
+    (loop over MAX_GROUPS - 1 slots) and the chunk counts of c's group before
+    c (loop over SCAN_GROUP - 1 slots)."""
+    radix = hist.shape[1]
+    g = c // SCAN_GROUP
+    base = np.zeros(radix, dtype=np.int64)
+    for d in range(radix):
+        pre = 0
+        for k in range(MAX_GROUPS - 1):
+            if k < g:
+                pre += int(gtot[k, d])
+        for k in range(SCAN_GROUP - 1):
+            cc = g * SCAN_GROUP + k
+            if cc < c:
+                pre += int(hist[cc, d])
+        base[d] = int(totals[:d].sum()) + pre
+    return base
+
+
+@pytest.mark.parametrize("G", [1, 2, 31, 32, 33, 64, 65, 300, SORT_MAX_GRID])
+@pytest.mark.parametrize("radix", [128, 256])
+def test_chunk_bases_equal_a_scan_over_chunks(G, radix):
+    rng = np.random.default_rng(G * 7 + radix)
+    hist = rng.integers(0, 50, size=(G, radix)) * (rng.random((G, radix)) < 0.6)
+    totals = hist.sum(axis=0)
+    gtot = np.zeros((MAX_GROUPS, radix), dtype=np.int64)
+    for c in range(G):  # what the histogram kernels accumulate
+        gtot[c // SCAN_GROUP] += hist[c]
+    # reference: the stable pass's offsets, an exclusive scan in (digit, chunk) order
+    flat = hist.T.reshape(-1)
+    excl = np.concatenate([[0], np.cumsum(flat)[:-1]]).reshape(radix, G)
+    cs = sorted({0, G - 1, G // 2, min(G - 1, SCAN_GROUP), min(G - 1, SCAN_GROUP - 1)}
+                | set(int(x) for x in rng.integers(0, G, size=min(G, 12))))
+    for c in cs:
+        assert np.array_equal(_chunk_bases_model(hist, totals, gtot, c), excl[:, c]), (G, radix, c)
+    assert (G - 1) // SCAN_GROUP <= MAX_GROUPS - 1  # every group before the last fits the loop
