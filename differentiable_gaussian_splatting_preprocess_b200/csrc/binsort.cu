@@ -411,7 +411,7 @@ struct ScatterSmem {
     unsigned* base;   // [radix] running global base
     unsigned* tcnt;   // [radix] this tile's count per digit
     unsigned* tstart; // [radix] tile-local start per digit
-    unsigned* tbase;  // [radix] global base for this tile
+    unsigned* tdelta; // [radix] global base for this tile minus the tile-local start (mod 2^32)
     unsigned* wcnt;   // [warps][radix] counts, then offsets
     unsigned* keys;   // [tile (+ padding)] regrouped keys
     unsigned* vals;   // [tile (+ padding)] regrouped values
@@ -419,8 +419,8 @@ struct ScatterSmem {
         base = reinterpret_cast<unsigned*>(raw);
         tcnt = base + C::kRadix;
         tstart = tcnt + C::kRadix;
-        tbase = tstart + C::kRadix;
-        wcnt = tbase + C::kRadix;
+        tdelta = tstart + C::kRadix;
+        wcnt = tdelta + C::kRadix;
         keys = wcnt + C::kWarps * C::kRadix;
         vals = keys + tile_words;
     }
@@ -489,7 +489,7 @@ __device__ __forceinline__ void scatter_tile(const ScatterSmem<MAXB>& sm, const 
             const int dd = lane * per + k;
             if (dd < radix) {
                 sm.tstart[dd] = run;
-                sm.tbase[dd] = sm.base[dd];
+                sm.tdelta[dd] = sm.base[dd] - run;
                 sm.base[dd] += v[k];
             }
             run += v[k];
@@ -511,7 +511,7 @@ __device__ __forceinline__ void scatter_tile(const ScatterSmem<MAXB>& sm, const 
     for (unsigned q = threadIdx.x; q < tile_n; q += kSortBlock) {
         const unsigned k2 = sm.keys[q];
         const unsigned dq = (k2 >> shift) & mask;
-        const unsigned pos = sm.tbase[dq] + (q - sm.tstart[dq]);
+        const unsigned pos = q + sm.tdelta[dq];
         if (keys_out) keys_out[pos] = k2;
         vals_out[pos] = sm.vals[q];
     }
@@ -608,46 +608,38 @@ k_scan_partials(int N, const unsigned* __restrict__ order, const unsigned* __res
     }
 }
 
-__global__ void __launch_bounds__(1024) k_scan_top(unsigned* __restrict__ part, int nb, SortMisc* __restrict__ misc) {
-    pdl_enter();
-    // exclusive scan of nb partial sums by one CTA, each thread a contiguous
-    // run; the total (of super-tile pairs, when that is what is scanned) goes
-    // to misc->ps, or 0 if the frame's pairs exceed the capacity
-    __shared__ unsigned s_w[32];
-    const int per = (nb + 1023) / 1024;
-    const int c0 = threadIdx.x * per;
-    unsigned local = 0;
-    for (int k = 0; k < per; ++k)
-        if (c0 + k < nb) local += part[c0 + k];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned incl = local;
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) s_w[warp] = incl;
-    __syncthreads();
-    unsigned wbase = 0;
-    for (int k = 0; k < warp; ++k) wbase += s_w[k];
-    unsigned run = wbase + incl - local;
-    for (int k = 0; k < per; ++k)
-        if (c0 + k < nb) {
-            const unsigned c = part[c0 + k];
-            part[c0 + k] = run;
-            run += c;
-        }
-    if (threadIdx.x == 1023) misc->ps = misc->p_eff ? run : 0u;
-}
-
+// Second half of the rank-order scan: each CTA takes the exclusive prefix of
+// the first kernel's per-CTA sums below it and the grand total (the frame's
+// pairs - of super-tile pairs on the super-tile route - stored by CTA 0 in
+// misc->ps, or 0 if the frame's pairs exceed the capacity) from the sums
+// directly (at most a few loads per thread), then scans its own ranks.
 // With `owner_lo` (super-tile route, G CTAs per pair pass), also records for
 // every chunk c of the pair stream the rank owning its first pair
 // (owner_lo[c]) and its last pair (owner_hi[c]): each rank checks the chunk
 // boundaries inside its own pair range, so no search is needed later.
 __global__ void __launch_bounds__(kSortBlock)
 k_scan_down(int N, const unsigned* __restrict__ cnt_rank, const unsigned* __restrict__ part,
-            unsigned* __restrict__ pair_off, const SortMisc* __restrict__ misc, unsigned G,
+            unsigned* __restrict__ pair_off, SortMisc* __restrict__ misc, unsigned G,
             unsigned* __restrict__ owner_lo, unsigned* __restrict__ owner_hi) {
     pdl_enter();
+    __shared__ unsigned s_pre[kSortBlock / 32], s_tot[kSortBlock / 32];
+    unsigned pre = 0, tot = 0;
+    constexpr int kP = 8;  // partial sums per thread and round, loaded together
+    for (unsigned i0 = 0; i0 < gridDim.x; i0 += kP * kSortBlock) {
+        unsigned pv[kP];
+#pragma unroll
+        for (int k = 0; k < kP; ++k) {
+            const unsigned i = i0 + k * kSortBlock + threadIdx.x;
+            pv[k] = i < gridDim.x ? part[i] : 0u;
+        }
+#pragma unroll
+        for (int k = 0; k < kP; ++k) {
+            tot += pv[k];
+            if (i0 + k * kSortBlock + threadIdx.x < blockIdx.x) pre += pv[k];
+        }
+    }
+    pre = __reduce_add_sync(0xffffffffu, pre);
+    tot = __reduce_add_sync(0xffffffffu, tot);
     // each thread owns kScanItems consecutive ranks
     const int base = blockIdx.x * kScanTile + threadIdx.x * kScanItems;
     unsigned v[kScanItems];
@@ -666,11 +658,23 @@ k_scan_down(int N, const unsigned* __restrict__ cnt_rank, const unsigned* __rest
         if (lane >= o) incl += y;
     }
     if (lane == 31) s_w[warp] = incl;
+    if (lane == 0) {
+        s_pre[warp] = pre;
+        s_tot[warp] = tot;
+    }
     __syncthreads();
+    unsigned cta_pre = 0, total = 0;
+#pragma unroll
+    for (int k = 0; k < kSortBlock / 32; ++k) {
+        cta_pre += s_pre[k];
+        total += s_tot[k];
+    }
+    const unsigned ps = misc->p_eff ? total : 0u;
+    if (blockIdx.x == 0 && threadIdx.x == 0) misc->ps = ps;
     unsigned wbase = 0;
     for (int k = 0; k < warp; ++k) wbase += s_w[k];
-    unsigned run = part[blockIdx.x] + wbase + incl - local;
-    const unsigned P = owner_lo ? misc->ps : 0u;
+    unsigned run = cta_pre + wbase + incl - local;
+    const unsigned P = owner_lo ? ps : 0u;
     const unsigned long long chunk = P ? chunk_size(P, G) : 1ull;
 #pragma unroll
     for (int k = 0; k < kScanItems; ++k) {
@@ -1516,7 +1520,6 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
     const int Gp = (int)((capacity + 2047u) / 2048u) < kSortMaxGrid ? (int)((capacity + 2047u) / 2048u) : kSortMaxGrid;
     launch_pdl(k_scan_partials, nb, kSortBlock, 0, st, N, order, tiles_touched, sup ? rect4 : nullptr, w.cnt_rank,
                                                w.rc_rank, w.sub_rank, w.scan_part, w.misc); note_launch();
-    launch_pdl(k_scan_top, 1, 1024, 0, st, w.scan_part, nb, w.misc); note_launch();
     launch_pdl(k_scan_down, nb, kSortBlock, 0, st, N, w.cnt_rank, w.scan_part, w.pair_off, w.misc,
                                            (unsigned)(Gp < 1 ? 1 : Gp), sup ? w.owner_lo : nullptr, w.owner_hi); note_launch();
     GS_LAUNCH_CHECK();
