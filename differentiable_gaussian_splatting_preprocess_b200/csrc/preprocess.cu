@@ -17,6 +17,7 @@
 #include <math.h>
 
 #include "gs_internal.cuh"
+#include "pdl.cuh"
 
 namespace gs {
 namespace {
@@ -220,6 +221,7 @@ k_preprocess_bwd(gs_camera cam, int N, const float* __restrict__ means, const fl
                  float* __restrict__ dL_dmeans, float* __restrict__ dL_dscales, float4* __restrict__ dL_dquats,
                  float* __restrict__ dL_dopacity, float* __restrict__ dL_dcolors, float* __restrict__ grad2d_accum,
                  unsigned* __restrict__ vis_count) {
+    pdl_enter();
     const int i = blockIdx.x * kPreBlock + threadIdx.x;
     if (i >= N) return;
     // Every load of this Gaussian - inputs and the accumulators read by the
@@ -405,11 +407,12 @@ extern "C" int gs_preprocess_bwd(const gs_camera* cam, int N, const float* means
         !aligned(dL_dquats, 16) || !aligned(dL_dmean2d, 8))
         return GS_ERR_INVALID_ARG;
     const int blocks = (N + kPreBlock - 1) / kPreBlock;
-    k_preprocess_bwd<<<blocks, kPreBlock, 0, (cudaStream_t)stream>>>(
-        *cam, N, means, scales, reinterpret_cast<const float4*>(quats), radius,
-        reinterpret_cast<const float4*>(conic_opacity), reinterpret_cast<const float2*>(dL_dmean2d),
-        reinterpret_cast<const float4*>(dL_dconic_opacity), dL_dcolor2d, dL_dmeans, dL_dscales,
-        reinterpret_cast<float4*>(dL_dquats), dL_dopacity, dL_dcolors, grad2d_accum, vis_count); note_launch();
+    launch_pdl(k_preprocess_bwd, blocks, kPreBlock, 0, (cudaStream_t)stream, *cam, N, means, scales,
+               reinterpret_cast<const float4*>(quats), radius, reinterpret_cast<const float4*>(conic_opacity),
+               reinterpret_cast<const float2*>(dL_dmean2d), reinterpret_cast<const float4*>(dL_dconic_opacity),
+               dL_dcolor2d, dL_dmeans, dL_dscales, reinterpret_cast<float4*>(dL_dquats), dL_dopacity, dL_dcolors,
+               grad2d_accum, vis_count);
+    note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }

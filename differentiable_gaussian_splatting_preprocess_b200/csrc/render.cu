@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 
 #include "gs_internal.cuh"
+#include "pdl.cuh"
 
 namespace gs {
 namespace {
@@ -139,6 +140,7 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
              unsigned* __restrict__ n_contrib, unsigned* __restrict__ cmask, unsigned cmask_words,
              const unsigned* __restrict__ order, unsigned* __restrict__ quad_work,
              unsigned* __restrict__ part_hist) {
+    pdl_enter();
     __shared__ float2 s_xy[kFwdBatch];
     __shared__ float4 s_co[kFwdBatch];
     __shared__ float4 s_col[kFwdBatch];
@@ -521,6 +523,7 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
                   const float* __restrict__ dL_dimage, float* __restrict__ dL_dmean2d,
                   float* __restrict__ dL_dconic_opacity, float* __restrict__ dL_dcolor,
                   const unsigned* __restrict__ order) {
+    pdl_enter();
     __shared__ unsigned s_id[32];
     __shared__ float2 s_xy[32];
     __shared__ float4 s_co[32];
@@ -734,6 +737,7 @@ __device__ __forceinline__ void zero_words(unsigned* __restrict__ a, size_t n, s
 __global__ void __launch_bounds__(kOrderThreads, 1)
 k_fwd_prep(int T, const uint2* __restrict__ ranges, unsigned* __restrict__ tile_order, unsigned* __restrict__ bits,
            size_t n_bits) {
+    pdl_enter();
     if (blockIdx.x == 0) {
         extern __shared__ __align__(16) unsigned char order_smem[];
         order_by_work((unsigned)T, [&](unsigned t) { const uint2 r = ranges[t]; return r.y - r.x; }, tile_order,
@@ -756,6 +760,7 @@ __global__ void __launch_bounds__(kOrderThreads)
 k_bwd_prep(int T, int P, const unsigned* __restrict__ quad_work, const unsigned* __restrict__ part_hist,
            unsigned* __restrict__ quad_order, float* __restrict__ a, size_t na, float* __restrict__ b, size_t nb,
            float* __restrict__ c, size_t nc) {
+    pdl_enter();
     if ((int)blockIdx.x < P) {
         __shared__ unsigned s_cur[kOrderCodes];
         __shared__ unsigned s_w[kOrderCodes / 32];
@@ -893,14 +898,15 @@ extern "C" int gs_render_fwd(const gs_camera* cam, const unsigned* ranges, const
     cudaStream_t st = (cudaStream_t)stream;
     if (contrib_mask) {
         opt_in_smem(k_fwd_prep, sizeof(OrderSmem));
-        k_fwd_prep<<<prep_blocks(m.prep_words), kOrderThreads, sizeof(OrderSmem), st>>>(
-            T, reinterpret_cast<const uint2*>(ranges), m.tile_order, m.part_hist, m.prep_words); note_launch();
+        launch_pdl(k_fwd_prep, prep_blocks(m.prep_words), kOrderThreads, sizeof(OrderSmem), st, T,
+                   reinterpret_cast<const uint2*>(ranges), m.tile_order, m.part_hist, m.prep_words);
+        note_launch();
         GS_LAUNCH_CHECK();
     }
-    k_render_fwd<<<T, kThreads, 0, st>>>(
-        *cam, TX, reinterpret_cast<const uint2*>(ranges), ids, reinterpret_cast<const float2*>(mean2d),
-        reinterpret_cast<const float4*>(conic_opacity), colors, image, final_T, n_contrib, m.bits, m.bits_words,
-        m.tile_order, m.quad_work, m.part_hist); note_launch();
+    launch_pdl(k_render_fwd, T, kThreads, 0, st, *cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
+               reinterpret_cast<const float2*>(mean2d), reinterpret_cast<const float4*>(conic_opacity), colors, image,
+               final_T, n_contrib, m.bits, m.bits_words, m.tile_order, m.quad_work, m.part_hist);
+    note_launch();
     GS_LAUNCH_CHECK();
     return GS_OK;
 }
@@ -924,15 +930,15 @@ extern "C" int gs_render_bwd(const gs_camera* cam, int N, const unsigned* ranges
     if (contrib_mask) {
         const size_t z = (n * 4 + kOrderThreads - 1) / kOrderThreads;
         const int zb = (int)(z < 148 * 2 ? (z ? z : 1) : 148 * 2);
-        k_bwd_prep<<<m.parts + zb, kOrderThreads, 0, st>>>(T, m.parts, m.quad_work, m.part_hist, m.quad_order,
-                                                           dL_dmean2d, n * 2, dL_dconic_opacity, n * 4, dL_dcolor,
-                                                           n * 3); note_launch();
+        launch_pdl(k_bwd_prep, m.parts + zb, kOrderThreads, 0, st, T, m.parts, m.quad_work, m.part_hist,
+                   m.quad_order, dL_dmean2d, n * 2, dL_dconic_opacity, n * 4, dL_dcolor, n * 3);
+        note_launch();
         GS_LAUNCH_CHECK();
-        k_render_bwd_warp<<<4 * T, 32, 0, st>>>(*cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
-                                                  reinterpret_cast<const float2*>(mean2d),
-                                                  reinterpret_cast<const float4*>(conic_opacity), colors, final_T,
-                                                  n_contrib, m.bits, m.bits_words, dL_dimage, dL_dmean2d,
-                                                  dL_dconic_opacity, dL_dcolor, m.quad_order); note_launch();
+        launch_pdl(k_render_bwd_warp, 4 * T, 32, 0, st, *cam, TX, reinterpret_cast<const uint2*>(ranges), ids,
+                   reinterpret_cast<const float2*>(mean2d), reinterpret_cast<const float4*>(conic_opacity), colors,
+                   final_T, n_contrib, m.bits, m.bits_words, dL_dimage, dL_dmean2d, dL_dconic_opacity, dL_dcolor,
+                   m.quad_order);
+        note_launch();
         GS_LAUNCH_CHECK();
         return GS_OK;
     }
