@@ -43,7 +43,7 @@ OPS_BWD_EVAL = 60
 # DRAM bytes per launch from the committed ncu capture of the render backward (k_render_bwd_warp)
 # (dram__bytes_read.sum + dram__bytes_write.sum) and the SHA-1 of the render
 # sources it was taken on; reported only while the sources are unchanged.
-RECORDED_TRAFFIC = {"k_render_bwd": dict(bytes=167509248, sources_sha1="8339ca8f1446b4ffd39383dcd2f97dbf7a61e451")}
+RECORDED_TRAFFIC = {"k_render_bwd": dict(bytes=168287488, sources_sha1="d736dead657ae87b2ef6708cbecb99e83a9436ce")}
 # Algorithmic bytes: per (tile, Gaussian) pair visited, id + mean2d +
 # conic/opacity + colour = 40 B read; the backward adds 36 B of gradient
 # atomics per pair; per pixel the forward writes 20 B (image, T, n_contrib)
@@ -125,7 +125,7 @@ class ClockSampler:
 def _render_sources_sha1() -> str:
     import hashlib
     h = hashlib.sha1()
-    for name in ("render.cu", "gs_internal.cuh"):
+    for name in ("render.cu", "gs_internal.cuh", "pdl.cuh"):
         with open(os.path.join(ROOT, "differentiable_gaussian_splatting_preprocess_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
