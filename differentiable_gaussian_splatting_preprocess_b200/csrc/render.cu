@@ -524,7 +524,6 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
                   float* __restrict__ dL_dconic_opacity, float* __restrict__ dL_dcolor,
                   const unsigned* __restrict__ order) {
     pdl_enter();
-    __shared__ unsigned s_id[32];
     __shared__ float2 s_xy[32];
     __shared__ float4 s_co[32];
     __shared__ float4 s_col[32];
@@ -590,15 +589,15 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
         if (!bits) continue;
         if ((bits >> lane) & 1u) {
             const unsigned j = pos_ok(kb + lane) ? ids[kb + lane] : 0xFFFFFFFFu;
+            // the id rides in the colour's unused fourth lane (as its bits)
             if (id_ok(j)) {
-                s_id[lane] = j;
                 s_xy[lane] = mean2d[j];
                 s_co[lane] = conic_opacity[j];
-                s_col[lane] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], 0.0f);
+                s_col[lane] = make_float4(colors[3 * j], colors[3 * j + 1], colors[3 * j + 2], __uint_as_float(j));
             } else {  // debug build, failed check: an inert entry (zero opacity, id 0)
-                s_id[lane] = 0u;
                 float4 box, thr;
                 stage_inert(s_xy[lane], s_co[lane], s_col[lane], box, thr);
+                s_col[lane].w = __uint_as_float(0u);
             }
         }
         __syncwarp();
@@ -607,14 +606,14 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
             bits &= ~(1u << l);
             const int p = (int)(kb + (unsigned)l - rg.x);
             float v[8], r9;
-            bwd_term<false, true>(q, s_xy[l], s_co[l], s_col[l], p, last0, last1, amax, amin, g0, g1, g2, T, Sg, v,
-                                  r9);
+            const float4 col = s_col[l];
+            bwd_term<false, true>(q, s_xy[l], s_co[l], col, p, last0, last1, amax, amin, g0, g1, g2, T, Sg, v, r9);
             const float r8 = reduce8(v, lane);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
             const float val = (lane == 1 ? r9 : r8) * post;
             // (a zero sum is added too: testing for it costs more than the atomic)
-            if (gbase) atomicAdd(gbase + (size_t)s_id[l] * gstride, val);
+            if (gbase) atomicAdd(gbase + (size_t)__float_as_uint(col.w) * gstride, val);
         }
         __syncwarp();  // the next word reuses this warp's slots
     }
