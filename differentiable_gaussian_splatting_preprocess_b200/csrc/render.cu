@@ -601,19 +601,30 @@ k_render_bwd_warp(gs_camera cam, int TX, const uint2* __restrict__ ranges, const
             }
         }
         __syncwarp();
-        while (bits) {
-            const int l = 31 - __clz(bits);
+        // terms from the back; the next term's staged entry is loaded before
+        // the current one is evaluated
+        int l = 31 - __clz(bits);
+        float2 xy = s_xy[l];
+        float4 co = s_co[l], col = s_col[l];
+        while (true) {
             bits &= ~(1u << l);
+            const int ln = bits ? 31 - __clz(bits) : l;
+            const float2 xy_n = s_xy[ln];
+            const float4 co_n = s_co[ln], col_n = s_col[ln];
             const int p = (int)(kb + (unsigned)l - rg.x);
             float v[8], r9;
-            const float4 col = s_col[l];
-            bwd_term<false, true>(q, s_xy[l], s_co[l], col, p, last0, last1, amax, amin, g0, g1, g2, T, Sg, v, r9);
+            bwd_term<false, true>(q, xy, co, col, p, last0, last1, amax, amin, g0, g1, g2, T, Sg, v, r9);
             const float r8 = reduce8(v, lane);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r9 += __shfl_xor_sync(0xffffffffu, r9, o);
             const float val = (lane == 1 ? r9 : r8) * post;
             // (a zero sum is added too: testing for it costs more than the atomic)
             if (gbase) atomicAdd(gbase + (size_t)__float_as_uint(col.w) * gstride, val);
+            if (!bits) break;
+            l = ln;
+            xy = xy_n;
+            co = co_n;
+            col = col_n;
         }
         __syncwarp();  // the next word reuses this warp's slots
     }
