@@ -158,12 +158,19 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     float2 C0 = make_float2(0.0f, 0.0f), C1 = C0, C2 = C0;
     unsigned last0 = 0, last1 = 0;
     bool done0 = !q.in0, done1 = !q.in1;
+    static_assert(kFwdBatch == kThreads, "one staged entry per thread and batch");
+    // each thread's list entry of the next batch is read one batch ahead, so
+    // that staging a batch waits for one round of loads, not two
+    unsigned j_next = (rg.x + threadIdx.x < rg.y && pos_ok(rg.x + threadIdx.x)) ? ids[rg.x + threadIdx.x] : 0xFFFFFFFFu;
     for (unsigned b = rg.x; b < rg.y; b += kFwdBatch) {
         if (__syncthreads_count(done0 && done1) == kThreads) break;
-        for (int r = threadIdx.x; r < kFwdBatch; r += kThreads) {
+        {
+            const int r = threadIdx.x;
             const unsigned k = b + r;
+            const unsigned j = j_next;
+            const unsigned kn = k + kFwdBatch;
+            j_next = (kn < rg.y && pos_ok(kn)) ? ids[kn] : 0xFFFFFFFFu;
             if (k < rg.y) {
-                const unsigned j = pos_ok(k) ? ids[k] : 0xFFFFFFFFu;
                 if (id_ok(j)) {
                     const float2 xy = mean2d[j];
                     const float4 co = conic_opacity[j];
