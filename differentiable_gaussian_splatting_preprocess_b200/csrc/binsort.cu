@@ -951,34 +951,47 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
     unsigned* s_g = s_off + kGenWin;      // [kGenWin] staged ids
     unsigned* s_rc = s_g + kGenWin;       // [kGenWin] staged packed rectangles
     unsigned char* s_sb = reinterpret_cast<unsigned char*>(s_rc + kGenWin);  // [kGenWin] staged sub_offsets
-    __shared__ unsigned s_r0;
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
     chunk_bases(hist, totals, gtot, radix, sm.base);
     const unsigned P = *n_ptr;
     unsigned lo, hi;
     chunk_of<MAXB>(P, lo, hi);
-    if (threadIdx.x == 0 && lo < hi) s_r0 = owner_lo[blockIdx.x];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // rank data of this thread's slot in the first staging round of the
+    // current tile, loaded while the previous tile was generated and scattered
+    unsigned r0 = lo < hi ? owner_lo[blockIdx.x] : 0u;
+    auto load_rank = [&](unsigned r, unsigned& off, unsigned& g, unsigned& rc, unsigned& sb) {
+        const bool inr = r < (unsigned)N;
+        off = inr ? pair_off[r] : 0xFFFFFFFFu;
+        g = inr ? order[r] : 0u;
+        rc = inr ? rc_rank[r] : 0u;
+        sb = inr ? sub_rank[r] : 0u;
+    };
+    unsigned f_off, f_g, f_rc, f_sb;
+    load_rank(r0 + threadIdx.x, f_off, f_g, f_rc, f_sb);
     for (unsigned base = lo; base < hi; base += C::kTileKeys) {
         const unsigned tile_n = min((unsigned)C::kTileKeys, hi - base);
         const unsigned end = base + tile_n;
-        __syncthreads();  // s_r0 written; the previous tile is finished
-        const unsigned r0 = s_r0;
+        __syncthreads();  // the previous tile is finished with the staging arrays
         // stage the ranks with offsets below `end` (a prefix: offsets of
-        // visible ranks increase strictly, culled ranks sit at P)
+        // visible ranks increase strictly, culled ranks sit at P); every
+        // loaded offset is kept, so the first rank past the tile is known too
         unsigned nr = 0;
         for (int round = 0; round * kSortBlock < kGenWin; ++round) {
             const unsigned idx = round * kSortBlock + threadIdx.x;
-            const unsigned r = r0 + idx;
-            const bool inr = r < (unsigned)N;
-            const unsigned off = inr ? pair_off[r] : 0xFFFFFFFFu;
-            const unsigned g = inr ? order[r] : 0u;
-            const unsigned rc = inr ? rc_rank[r] : 0u;
-            const unsigned sb = inr ? sub_rank[r] : 0u;
+            unsigned off, g, rc, sb;
+            if (round == 0) {
+                off = f_off;
+                g = f_g;
+                rc = f_rc;
+                sb = f_sb;
+            } else {
+                load_rank(r0 + idx, off, g, rc, sb);
+            }
             const bool in = off < end;
+            s_off[idx] = off;
             if (in) {
-                s_off[idx] = off;
                 s_g[idx] = g;
                 s_rc[idx] = rc;
                 s_sb[idx] = (unsigned char)sb;
@@ -987,11 +1000,13 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
             nr += (unsigned)c;
             if (c < kSortBlock) break;
         }
-        // owner of the next tile's first pair: the next rank if it starts there
-        if (threadIdx.x == 0) {
-            const unsigned nx = r0 + nr;
-            s_r0 = (nx < (unsigned)N && pair_off[nx] == end) ? nx : nx - 1;
-        }
+        // owner of the next tile's first pair: the next rank if it starts
+        // there (its offset is staged at nr: nr < kGenWin), else the last one
+        // of this tile; its first staging round is loaded now
+        const unsigned nx = r0 + nr;
+        const unsigned off_nx = nr < (unsigned)kGenWin ? s_off[nr] : (nx < (unsigned)N ? pair_off[nx] : 0xFFFFFFFFu);
+        r0 = (nx < (unsigned)N && off_nx == end) ? nx : nx - 1;
+        if (end < hi) load_rank(r0 + threadIdx.x, f_off, f_g, f_rc, f_sb);
         // generate this thread's slots into the padded key/value arrays
         const unsigned q0 = threadIdx.x * C::kItems;
         if (q0 < tile_n) {
