@@ -208,7 +208,9 @@ __global__ void k_bin_init(int N, int T, const float* __restrict__ depth, const 
     for (int i = tid; i < 2 * T; i += stride) ranges[i] = 0u;
     for (int i = tid; i < kMaxPasses * kRadixMax; i += stride) w.totals[i] = 0u;
     for (int i = tid; i < kMaxPasses * kMaxGroups * kRadixMax; i += stride) w.gtot[i] = 0u;
-    for (int i = tid; i < 2 * w.n_cells; i += stride) w.cell_ranges[i] = 0u;
+    // cell ranges [start, end) are found by atomic min / max in the last
+    // cell pass: starts from above, ends from below (empty: start > end)
+    for (int i = tid; i < 2 * w.n_cells; i += stride) w.cell_ranges[i] = (i & 1) ? 0u : 0xFFFFFFFFu;
     // four items per thread and round, their loads issued together
     constexpr int kU = 4;
     for (long long i0 = tid; i0 < N; i0 += (long long)kU * stride) {
@@ -434,7 +436,8 @@ __device__ __forceinline__ void scatter_tile(const ScatterSmem<MAXB>& sm, const 
                                              const unsigned (&val)[RadixCfg<MAXB>::kItems],
                                              const unsigned (&d)[RadixCfg<MAXB>::kItems], unsigned tile_n, int shift,
                                              int bits, unsigned* __restrict__ keys_out,
-                                             unsigned* __restrict__ vals_out) {
+                                             unsigned* __restrict__ vals_out, unsigned* __restrict__ cell_ranges,
+                                             int SX) {
     using C = RadixCfg<MAXB>;
     const int radix = 1 << bits;
     const unsigned mask = radix - 1;
@@ -514,6 +517,19 @@ __device__ __forceinline__ void scatter_tile(const ScatterSmem<MAXB>& sm, const 
         const unsigned pos = q + sm.tdelta[dq];
         if (keys_out) keys_out[pos] = k2;
         vals_out[pos] = sm.vals[q];
+        if (cell_ranges) {
+            // last cell pass: within its digit's run the tile is in cell
+            // order, so a cell's keys from this tile are one local run; the
+            // first and last keys of each run extend the cell's range
+            const unsigned r0 = sm.tstart[dq], r1 = r0 + sm.tcnt[dq];
+            const bool first = q == r0 || ((sm.keys[q - 1] ^ k2) & kCellBits) != 0u;
+            const bool last = q + 1 == r1 || ((sm.keys[q + 1] ^ k2) & kCellBits) != 0u;
+            if (first || last) {
+                const unsigned c = ((k2 >> 16) & 0xFFu) * (unsigned)SX + (k2 & 0xFFu);
+                if (first) atomicMin(&cell_ranges[2 * c], pos);
+                if (last) atomicMax(&cell_ranges[2 * c + 1], pos + 1);
+            }
+        }
     }
     __syncthreads();  // the next tile reuses every shared array
 }
@@ -525,7 +541,8 @@ __global__ void __launch_bounds__(kSortBlock)
 k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict__ vals_in,
                 unsigned* __restrict__ keys_out, unsigned* __restrict__ vals_out,
                 const unsigned* __restrict__ n_ptr, int shift, int bits, const unsigned* __restrict__ hist,
-                const unsigned* __restrict__ totals, const unsigned* __restrict__ gtot) {
+                const unsigned* __restrict__ totals, const unsigned* __restrict__ gtot,
+                unsigned* __restrict__ cell_ranges, int SX) {
     pdl_enter();
     using C = RadixCfg<MAXB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -548,7 +565,7 @@ k_radix_scatter(const unsigned* __restrict__ keys_in, const unsigned* __restrict
             val[j] = valid ? vals_in[i] : 0u;
             d[j] = valid ? (key[j] >> shift) & mask : kNoDigit;
         }
-        scatter_tile<MAXB>(sm, key, val, d, tile_n, shift, bits, keys_out, vals_out);
+        scatter_tile<MAXB>(sm, key, val, d, tile_n, shift, bits, keys_out, vals_out, cell_ranges, SX);
     }
 }
 
@@ -1060,56 +1077,13 @@ k_gen_scatter(int N, const unsigned* __restrict__ order, const unsigned* __restr
             d[j] = valid ? key[j] & mask : kNoDigit;
         }
         // scatter_tile's first barrier orders these reads before its regroup
-        scatter_tile<MAXB>(sm, key, val, d, tile_n, 0, bits, keys_out, vals_out);
+        scatter_tile<MAXB>(sm, key, val, d, tile_n, 0, bits, keys_out, vals_out, nullptr, 0);
     }
 }
 
 template <int MAXB>
 constexpr size_t gen_scatter_smem() {
     return ScatterSmem<MAXB>::bytes(kPadTile) + 3 * (size_t)kGenWin * sizeof(unsigned) + (size_t)kGenWin;
-}
-
-// Cell ranges of the cell-sorted list by comparing neighbours' cells (the
-// kCellBits of the keys); empty cells keep (0, 0).  Four keys per thread with
-// 16-byte loads, neighbours across lanes by shuffles.
-__global__ void k_cell_ranges(const unsigned* __restrict__ ckeys, const unsigned* __restrict__ n_ptr, int SX,
-                              unsigned* __restrict__ cell_ranges) {
-    pdl_enter();
-    const unsigned n = *n_ptr;
-    const unsigned nq = (n + 3) / 4;
-    const unsigned stride = gridDim.x * blockDim.x;
-    const int lane = threadIdx.x & 31;
-    // every lane of a warp iterates the same number of times (shuffles below)
-    for (unsigned qb = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); qb < nq; qb += stride) {
-        const unsigned qi = qb + lane;
-        const unsigned k0 = qi * 4;
-        unsigned t[4];
-        if (k0 + 3 < n) {
-            const uint4 v = reinterpret_cast<const uint4*>(ckeys)[qi];
-            t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
-        } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) t[j] = k0 + j < n ? ckeys[k0 + j] : 0xFFFFFFFFu;
-        }
-        unsigned prev = __shfl_up_sync(0xffffffffu, t[3], 1);
-        unsigned next = __shfl_down_sync(0xffffffffu, t[0], 1);
-        if (lane == 0) prev = (k0 > 0 && k0 - 1 < n) ? ckeys[k0 - 1] : 0xFFFFFFFFu;
-        if (lane == 31) next = (k0 + 4 < n) ? ckeys[k0 + 4] : 0xFFFFFFFFu;
-        if (qi < nq) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const unsigned k = k0 + j;
-                if (k >= n) break;
-                const unsigned cell = t[j] & kCellBits;
-                const unsigned before = (j == 0 ? prev : t[j - 1]) & kCellBits;
-                const unsigned after =
-                    ((j == 3 || k + 1 == n) ? (k + 1 == n ? 0xFFFFFFFFu : next) : t[j + 1]) & kCellBits;
-                const unsigned c = (cell >> 16) * (unsigned)SX + (cell & 0xFFu);
-                if (k == 0 || before != cell) cell_ranges[2 * c] = k;
-                if (k + 1 == n || after != cell) cell_ranges[2 * c + 1] = k + 1;
-            }
-        }
-    }
 }
 
 // Exclusive scan of one value per thread across a CTA of 1024 threads;
@@ -1141,6 +1115,13 @@ __device__ __forceinline__ unsigned block_exclusive_scan(unsigned x, unsigned* s
     return s_w[warp] + incl - x;
 }
 
+// A cell's range [start, end) of the cell-sorted list as the last cell pass
+// left it (start > end for a cell without pairs: then (0, 0)).
+__device__ __forceinline__ uint2 cell_range(const uint2* __restrict__ rg2, int c) {
+    const uint2 r = rg2[c];
+    return r.x < r.y ? r : make_uint2(0u, 0u);
+}
+
 // Segments of the cell lists (one CTA): cell c gets ceil(len / kSeg)
 // segments, numbered in cell order; cell_seg0[c] is its first.  The ranges
 // and first segments of up to kSegCache cells stay in shared memory for the
@@ -1162,7 +1143,7 @@ k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restric
     for (int k = 0; k < per; ++k) {
         const int c = c0 + k;
         if (c < S) {
-            const uint2 r = rg2[c];
+            const uint2 r = cell_range(rg2, c);
             if (c < kSegCache) s_rg[c] = r;
             local += (r.y - r.x + kSeg - 1) / kSeg;
         }
@@ -1172,7 +1153,7 @@ k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restric
     for (int k = 0; k < per; ++k) {
         const int c = c0 + k;
         if (c < S) {
-            const uint2 r = c < kSegCache ? s_rg[c] : rg2[c];
+            const uint2 r = c < kSegCache ? s_rg[c] : cell_range(rg2, c);
             cell_seg0[c] = run;
             if (c < kSegCache) s_s0[c] = run;
             run += (r.y - r.x + kSeg - 1) / kSeg;
@@ -1186,7 +1167,7 @@ k_seg_table(int S, const unsigned* __restrict__ cell_ranges, unsigned* __restric
     // one warp per cell writes the cell's segments, one lane per segment
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int c = warp; c < S; c += 32) {
-        const uint2 r = c < kSegCache ? s_rg[c] : rg2[c];
+        const uint2 r = c < kSegCache ? s_rg[c] : cell_range(rg2, c);
         const unsigned s0 = c < kSegCache ? s_s0[c] : cell_seg0[c];
         for (unsigned j = lane; r.x + j * kSeg < r.y; j += 32) {
             const unsigned lo = r.x + j * kSeg;
@@ -1441,11 +1422,12 @@ void enable_scatter_smem() {
 
 template <int MAXB>
 void radix_pass(cudaStream_t st, int G, const unsigned* n_ptr, int shift, int bits, const unsigned* ki,
-                const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals, unsigned* gtot) {
+                const unsigned* vi, unsigned* ko, unsigned* vo, unsigned* hist, unsigned* totals, unsigned* gtot,
+                unsigned* cell_ranges = nullptr, int SX = 0) {
     enable_scatter_smem<MAXB>();
     launch_pdl(k_radix_hist<MAXB>, G, kSortBlock, 0, st, ki, n_ptr, shift, bits, hist, totals, gtot); note_launch();
     launch_pdl(k_radix_scatter<MAXB>, G, kSortBlock, RadixCfg<MAXB>::kScatterSmem, st, ki, vi, ko, vo, n_ptr, shift, bits,
-               hist, totals, gtot);
+               hist, totals, gtot, cell_ranges, SX);
     note_launch();
 }
 
@@ -1570,17 +1552,12 @@ extern "C" int gs_bin_sort(const gs_camera* cam, int N, const float* depth, cons
         unsigned* h2 = w.hist + (size_t)5 * kRadixMax * kSortMaxGrid;
         unsigned* t2 = w.totals + (size_t)5 * kRadixMax;
         unsigned* g2 = w.gtot + (size_t)5 * kMaxGroups * kRadixMax;
+        // the cy pass also records each cell's range of the sorted list
         if (by <= 7)
-            radix_pass<7>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2, g2);
+            radix_pass<7>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2, g2, w.cell_ranges, SX);
         else
-            radix_pass<8>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2, g2);
+            radix_pass<8>(st, Gp, ps, 16, by, w.tkeys0, w.tvals0, w.tkeys1, w.tvals1, h2, t2, g2, w.cell_ranges, SX);
         GS_LAUNCH_CHECK();
-        {
-            int blocks = (int)((capacity + 1023u) / 1024u);
-            if (blocks > 148 * 16) blocks = 148 * 16;
-            if (blocks < 1) blocks = 1;
-            launch_pdl(k_cell_ranges, blocks, 256, 0, st, w.tkeys1, ps, SX, w.cell_ranges); note_launch();
-        }
         const int S = SX * SY;
         launch_pdl(k_seg_table, 1, 1024, 0, st, S, w.cell_ranges, w.cell_seg0, w.seg_cell, w.seg_lo, w.seg_hi, w.misc); note_launch();
         const int gseg = (int)(w.max_seg < 148u * 8u ? w.max_seg : 148u * 8u);
