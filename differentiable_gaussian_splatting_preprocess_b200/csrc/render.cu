@@ -141,11 +141,14 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
              const unsigned* __restrict__ order, unsigned* __restrict__ quad_work,
              unsigned* __restrict__ part_hist) {
     pdl_enter();
-    __shared__ float2 s_xy[kFwdBatch];
-    __shared__ float4 s_co[kFwdBatch];
-    __shared__ float4 s_col[kFwdBatch];
-    __shared__ float4 s_box[kFwdBatch];
-    __shared__ float4 s_thr[kFwdBatch];  // threshold, b / c, b / a
+    // two staging buffers: batch k is staged into buffer k & 1 while no warp
+    // can still be reading it (its last readers processed batch k - 2 before
+    // the barrier of batch k - 1), so one block barrier per batch suffices
+    __shared__ float2 s_xy2[2][kFwdBatch];
+    __shared__ float4 s_co2[2][kFwdBatch];
+    __shared__ float4 s_col2[2][kFwdBatch];
+    __shared__ float4 s_box2[2][kFwdBatch];
+    __shared__ float4 s_thr2[2][kFwdBatch];  // threshold, b / c, b / a
     const unsigned tile = order ? order[blockIdx.x] : blockIdx.x;
     if (tile >= gridDim.x) return;  // not a permutation of the tiles: nothing valid to do
     const PixelPair q = pixel_pair(cam, TX, (int)tile);
@@ -162,8 +165,13 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
     // each thread's list entry of the next batch is read one batch ahead, so
     // that staging a batch waits for one round of loads, not two
     unsigned j_next = (rg.x + threadIdx.x < rg.y && pos_ok(rg.x + threadIdx.x)) ? ids[rg.x + threadIdx.x] : 0xFFFFFFFFu;
-    for (unsigned b = rg.x; b < rg.y; b += kFwdBatch) {
-        if (__syncthreads_count(done0 && done1) == kThreads) break;
+    int buf = 0;
+    for (unsigned b = rg.x; b < rg.y; b += kFwdBatch, buf ^= 1) {
+        float2* const s_xy = s_xy2[buf];
+        float4* const s_co = s_co2[buf];
+        float4* const s_col = s_col2[buf];
+        float4* const s_box = s_box2[buf];
+        float4* const s_thr = s_thr2[buf];
         {
             const int r = threadIdx.x;
             const unsigned k = b + r;
@@ -183,7 +191,8 @@ k_render_fwd(gs_camera cam, int TX, const uint2* __restrict__ ranges, const unsi
                 }
             }
         }
-        __syncthreads();
+        // the batch is staged; stop here if every pixel of the tile is done
+        if (__syncthreads_count(done0 && done1) == kThreads) break;
         const int n = min((unsigned)kFwdBatch, rg.y - b);
         bool warp_done = __all_sync(0xffffffffu, done0 && done1);
         // cull against the pixels of this warp that are still compositing
