@@ -405,7 +405,9 @@ __device__ __forceinline__ void chunk_bases(const unsigned* __restrict__ hist, c
 //      tile-local digit starts and advances the running global bases;
 //   3. every key is placed in shared memory at its tile-local sorted position;
 //   4. the regrouped tile is written out in order, so consecutive lanes write
-//      consecutive addresses of one digit's run (coalesced stores).
+//      consecutive addresses of one digit's run (coalesced stores); with
+//      cell_ranges (the last cell pass), the first and last key of each local
+//      run of one cell extend that cell's range by an atomic min / max.
 // keys_out may be null (values only).  Ends with a block barrier.
 template <int MAXB>
 struct ScatterSmem {
