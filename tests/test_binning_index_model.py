@@ -507,3 +507,71 @@ def test_chunk_bases_equal_a_scan_over_chunks(G, radix):
     for c in cs:
         assert np.array_equal(_chunk_bases_model(hist, totals, gtot, c), excl[:, c]), (G, radix, c)
     assert (G - 1) // SCAN_GROUP <= MAX_GROUPS - 1  # every group before the last fits the loop
+
+
+def _stable_pass(keys, digit, G, tile=TILE_KEYS):
+    """One stable radix pass as the scatter kernels run it: chunk c of the
+    input (G chunks of whole tiles) goes, tile by tile, to each digit's
+    region after every earlier chunk's and tile's keys of that digit.
+    Returns the output keys and, per input tile, its regrouped keys with
+    their output positions (the order of the kernel's write-out)."""
+    n = len(keys)
+    chunk = _chunk_size(n, G)
+    counts = {}
+    for k in keys:
+        counts[digit(k)] = counts.get(digit(k), 0) + 1
+    base, run = {}, 0
+    for d in sorted(counts):
+        base[d] = run
+        run += counts[d]
+    out = [None] * n
+    tiles = []
+    for c in range(G):
+        lo, hi = min(c * chunk, n), min(n, c * chunk + chunk)
+        for t0 in range(lo, hi, tile):
+            t = keys[t0:min(hi, t0 + tile)]
+            regrouped = sorted(range(len(t)), key=lambda q: digit(t[q]))  # stable
+            placed = []
+            for q in regrouped:
+                d = digit(t[q])
+                out[base[d]] = t[q]
+                placed.append((t[q], base[d]))
+                base[d] += 1
+            tiles.append(placed)
+    return out, tiles
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_cell_ranges_from_the_last_cell_pass(seed):
+    """The last cell pass (cy digit) records each cell's [start, end) by an
+    atomic min / max at the first and last key of each local run of one cell
+    in a tile's regrouped write-out; that equals boundary detection on the
+    finished cell-sorted list (what a separate pass over it computed)."""
+    rng = np.random.default_rng(seed)
+    SX, SY = int(rng.integers(1, 40)), int(rng.integers(1, 20))
+    n = int(rng.integers(1, 30000))
+    cells = rng.integers(0, SX * SY, size=n)
+    keys0 = [int(c % SX) | int(c // SX) << 16 for c in cells]
+    G = max(1, min((n + 2047) // 2048, SORT_MAX_GRID))
+    by_cx, _ = _stable_pass(keys0, lambda k: k & 0xFF, G)
+    final, tiles = _stable_pass(by_cx, lambda k: (k >> 16) & 0xFF, G)
+    INF = 0xFFFFFFFF
+    rng_min = [INF] * (SX * SY)
+    rng_max = [0] * (SX * SY)
+    for placed in tiles:
+        for q, (k, pos) in enumerate(placed):
+            cell = (k >> 16) * SX + (k & 0xFF)
+            same = lambda j: 0 <= j < len(placed) and placed[j][0] == k and placed[j][1] == pos + (j - q)
+            if not same(q - 1):
+                rng_min[cell] = min(rng_min[cell], pos)
+            if not same(q + 1):
+                rng_max[cell] = max(rng_max[cell], pos + 1)
+    ranges = [(a, b) if a < b else (0, 0) for a, b in zip(rng_min, rng_max)]
+    direct = [(0, 0)] * (SX * SY)
+    for p, k in enumerate(final):
+        cell = (k >> 16) * SX + (k & 0xFF)
+        if p == 0 or final[p - 1] != k:
+            direct[cell] = (p, direct[cell][1])
+        if p + 1 == len(final) or final[p + 1] != k:
+            direct[cell] = (direct[cell][0], p + 1)
+    assert ranges == direct
