@@ -271,6 +271,20 @@ def test_binning_routes(W, H, n, sigma_mult):
     _check_bins(cam, g, pre)
 
 
+def test_rank_scan_over_more_than_2048_blocks():
+    """5M Gaussians: the rank-order scan has 2442 blocks, so each block of
+    its second kernel sums the per-block partials below it in two rounds
+    (2048 per round); the depth sort runs at its maximum grid with several
+    tiles per CTA.  Preprocess and binning against the oracle, bit-exact."""
+    sc = _tiny(n=5_000_000, width=256, height=256, seed=11, distinct_depth_gap=None, scale_log_mean=-4.0)
+    cam = sc.cameras[0]
+    gs = GpuScene(sc)
+    g = frame_np(run_gpu(gs, cam)["frame"])
+    pre = _check_preprocess(sc, cam, g)
+    assert g["num_pairs"] > 0
+    _check_bins(cam, g, pre)
+
+
 def test_no_thresholds_and_large_support():
     """alpha_min = T_min = 0 and a support radius covering the whole image."""
     sc = _tiny(n=24, width=64, height=48, seed=11, sigma_mult=1e3, alpha_min=0.0, T_min=0.0)
